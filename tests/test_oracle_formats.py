@@ -1,0 +1,203 @@
+"""Pins for the oracle's FP4 E2M1 / E4M3 number formats and FP4 quantizer.
+
+The oracle's encoders search the value set by distance; here they are checked
+against an independent implementation (the ml_dtypes format library), against
+closed forms of the formats, and against the invariants that the FP4 scheme
+implies (exact round trips, power-of-two scale shifts, sign symmetry, error
+bounds, 288 bytes per 512-channel token).
+"""
+import os
+from fractions import Fraction
+
+import ml_dtypes
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_e2m1():
+    rows = []
+    for line in open(os.path.join(GOLDEN, "e2m1_values.txt")):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        c, v = line.split()
+        rows.append((int(c), float(v)))
+    return rows
+
+
+def test_e2m1_value_table_matches_golden_and_library():
+    rows = _golden_e2m1()
+    assert [c for c, _ in rows] == list(range(16))
+    lib = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    for c, v in rows:
+        got = oracle.e2m1_value(c)
+        assert got == v and np.signbit(got) == np.signbit(v), (c, got, v)
+        assert got == lib[c] and np.signbit(got) == np.signbit(lib[c])
+    mags = sorted({abs(v) for _, v in rows})
+    assert mags == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_e4m3_decode_all_codes_closed_form_and_library():
+    lib = np.arange(256, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    for c in range(256):
+        v = oracle.e4m3_value(c)
+        if c in (0x7F, 0xFF):
+            assert np.isnan(v) and np.isnan(lib[c])
+            continue
+        assert v == lib[c], (c, v, lib[c])
+        # closed form: sign * 2^(e-7) * (1 + m/8), subnormal m * 2^-9
+        s, e, m = c >> 7, (c >> 3) & 15, c & 7
+        ref = Fraction(m, 512) if e == 0 else Fraction(8 + m, 8) * Fraction(2) ** (e - 7)
+        assert Fraction(abs(v)) == ref
+        assert np.signbit(v) == bool(s)
+    assert oracle.e4m3_value(0x7E) == 448.0
+    assert oracle.e4m3_value(0x01) == 2.0 ** -9
+
+
+def _probe_values():
+    """fp32 probes: every exponent from 2^-30 to 2^12 with a spread of
+    mantissas, plus +-4 ulps around every E2M1 value, every E2M1 tie point and
+    every E4M3 value / tie point, plus zeros, subnormals and huge values."""
+    rng = np.random.default_rng(1234)
+    out = []
+    exps = np.arange(127 - 30, 127 + 13, dtype=np.uint32)
+    mant = np.concatenate([np.arange(0, 1 << 23, 997, dtype=np.uint32),
+                           np.array([0, 1, 2, (1 << 22), (1 << 23) - 1], np.uint32)])
+    bits = (exps[:, None] << 23) | mant[None, :]
+    out.append(bits.ravel().view(np.float32))
+    pts = [0.0, 0.25, 0.5, 0.75, 1.0, 1.25, 1.5, 1.75, 2.0, 2.5, 3.0, 3.5, 4.0, 5.0, 6.0, 7.0]
+    e4 = np.arange(0x7F, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    mids = (e4[1:] + e4[:-1]) / 2
+    pts += list(e4) + list(mids) + [464.0, 480.0]
+    for p in pts:
+        f = np.float32(p)
+        b = np.array([f], np.float32).view(np.uint32)[0]
+        for d in range(-4, 5):
+            if int(b) + d >= 0:
+                out.append(np.array([int(b) + d], np.uint32).view(np.float32))
+    out.append(np.array([0.0, 1e-45, 1e-40, 1.17e-38, 1e-10, 1e6, 1e30, 3.4e38], np.float32))
+    out.append(rng.standard_normal(20000).astype(np.float32) * 3)
+    v = np.concatenate(out).astype(np.float32)
+    return np.concatenate([v, -v])
+
+
+def test_e2m1_encode_matches_library_round_to_nearest_even_saturating():
+    v = _probe_values()
+    got = oracle.e2m1_encode_array(v)
+    ref = v.astype(ml_dtypes.float4_e2m1fn).view(np.uint8)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, [(float(v[i]), int(got[i]), int(ref[i])) for i in bad[:10]]
+
+
+def test_e2m1_tie_and_saturation_cases():
+    # ties go to the even code; above 6 saturates; the sign survives rounding to 0
+    cases = [(0.25, 0), (0.75, 2), (1.25, 2), (1.75, 4), (2.5, 4), (3.5, 6), (5.0, 6), (6.5, 7),
+             (1e9, 7), (0.2500001, 1), (0.2499999, 0), (-0.1, 8), (-0.0, 8), (0.0, 0)]
+    for x, code in cases:
+        assert oracle.e2m1_encode(x) == code, (x, oracle.e2m1_encode(x), code)
+
+
+def test_e4m3_encode_matches_library_in_range_and_saturates_above():
+    v = _probe_values()
+    got = oracle.e4m3_encode_array(v)
+    inr = np.abs(v) < 464.0      # ml_dtypes rounds values >= 464 to NaN (no saturation)
+    ref = v[inr].astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    bad = np.nonzero(got[inr] != ref)[0]
+    assert bad.size == 0, [(float(v[inr][i]), int(got[inr][i]), int(ref[i])) for i in bad[:10]]
+    sat = got[~inr]
+    assert np.all((sat & 0x7F) == 0x7E)
+
+
+def _trunc_bf16(x):
+    """float32 array -> bf16 bit patterns by dropping the low 16 bits."""
+    return (np.ascontiguousarray(x, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _bf16(x):
+    """float32 array -> bf16 bit patterns (x must be exactly representable)."""
+    u = np.asarray(x, np.float32).view(np.uint32)
+    assert np.all((u & 0xFFFF) == 0)
+    return (u >> 16).astype(np.uint16)
+
+
+def test_quantize_exact_round_trip():
+    rng = np.random.default_rng(7)
+    e2m1 = np.array([0, .5, 1, 1.5, 2, 3, 4, 6], np.float64)
+    e4 = np.arange(0x7F, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    for _ in range(200):
+        sc = int(rng.integers(0x08, 0x7F))      # normal-range scale codes
+        s = e4[sc]
+        k = rng.choice(e2m1, 16) * rng.choice([-1, 1], 16)
+        k[rng.integers(16)] = 6.0 * rng.choice([-1, 1])   # amax = 6 s, so amax/6 = s exactly
+        x = (k * s).astype(np.float32)
+        if not np.all((x.view(np.uint32) & 0xFFFF) == 0):
+            continue                                 # not representable in bf16
+        packed, sf = oracle.fp4_quantize(_bf16(x)[None, :])
+        assert sf[0, 0] == sc
+        back = oracle.fp4_dequantize(packed, sf)[0]
+        assert np.array_equal(back, k * s)
+
+
+def test_quantize_power_of_two_scale_shift_and_negation():
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((64, 64)).astype(np.float32)
+    xb = _trunc_bf16(x)
+    base = np.asarray(xb.astype(np.uint32) << 16).view(np.float32)
+    p0, s0 = oracle.fp4_quantize(xb)
+    for e in (-3, -1, 1, 2):
+        p1, s1 = oracle.fp4_quantize(_bf16(base * np.float32(2.0 ** e)))
+        assert np.array_equal(p0, p1)
+        assert np.array_equal(s1.astype(int) - s0.astype(int), np.full(s0.shape, 8 * e))
+    pn, sn = oracle.fp4_quantize(_bf16(-base))
+    assert np.array_equal(sn, s0)
+    # negation flips only the sign bit of each nibble (entries that round to 0 keep
+    # their magnitude code 0 and get the opposite sign bit)
+    assert np.array_equal(pn ^ p0, np.full(p0.shape, 0x88, np.uint8))
+
+
+def test_quantize_error_bound_and_zero_group():
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((256, 128)) * rng.choice([1, 8], 128)).astype(np.float32)
+    xb = _trunc_bf16(x)
+    xv = np.asarray(xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    packed, sf = oracle.fp4_quantize(xb)
+    back = oracle.fp4_dequantize(packed, sf)
+    scale = sf.view(ml_dtypes.float8_e4m3fn).astype(np.float64).repeat(16, axis=1)
+    v = np.abs(xv) / scale
+    err = np.abs(xv - back)
+    # E2M1 spacing: 0.5 below 2, 1 in [2, 4), 2 in [4, 6]; saturation adds at most
+    # (6.4 - 6) s because the E4M3 rounding of amax/6 is within 2^-4 relative.
+    bound = np.where(v < 2, 0.25, np.where(v < 4, 0.5, 1.0)) * scale
+    assert np.all(err <= bound + 1e-12)
+    # all-zero group: scale code 0 and all codes +0
+    z = np.zeros((1, 32), np.uint16)
+    p, s = oracle.fp4_quantize(z)
+    assert np.all(p == 0) and np.all(s == 0)
+    # a group whose amax/6 rounds below the smallest E4M3 subnormal: scale 0, codes +0
+    tiny = _bf16(np.full(16, 2.0 ** -13, np.float32))[None, :]
+    p, s = oracle.fp4_quantize(tiny)
+    assert s[0, 0] == 0 and np.all(p == 0)
+
+
+def test_dequantize_every_code_and_scale_is_exact_product():
+    codes = np.arange(16, dtype=np.uint8)
+    packed = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)
+    for sc in range(0x7F):
+        sf = np.array([[sc]], np.uint8)
+        out = oracle.fp4_dequantize(packed[None, :], sf)[0]
+        s = Fraction(oracle.e4m3_value(sc))
+        for c in range(16):
+            ref = Fraction(float(np.uint8(c).view(ml_dtypes.float4_e2m1fn).astype(np.float64))) * s
+            assert Fraction(out[c]) == ref
+
+
+def test_fp4_row_bytes_match_pages():
+    vals = dict(line.split()[:2] for line in open(os.path.join(GOLDEN, "csa2_layout.txt"))
+                if line.strip() and not line.startswith("#"))
+    assert oracle.fp4_row_bytes(512) == int(vals["fp4_row_bytes_512"]) == 288
+    packed, sf = oracle.fp4_quantize(np.zeros((3, 512), np.uint16))
+    assert packed.shape[1] + sf.shape[1] == 288

@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA2 decode hot path on B200.
+
+Default workload: the full 20-layer decoder attention stack (five groups:
+Full + 3 Reuse, then four Reindex + 3 Reuse), batch 4, context 1,048,576,
+one decode step = append the new token's FP4 KV row, then every layer's
+indexing (scan / pool / top-512 or Reindex rescoring) and sparse attention.
+
+Metric: decode layer-steps/s (layers of the stack / time of one decode step of
+the whole batch), plus the dominant kernel (the Full layer's indexer scan)
+against the HBM roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl csa2|reference]
+
+N > 1 runs one process per GPU (torchrun); each rank decodes its own batch
+(weak scaling, no data-path collective: sequences are independent).
+`--impl reference` times the CPU oracle on a bounded sample of the same
+workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode layer-steps/s at 128K–1M ctx; achieved HBM GB/s vs roofline"
+UNIT = "layer-steps/s"
+DEFAULT_WORKLOAD = "decoder_stack20_b4_ctx1m"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def _scan_traffic(workload: str):
+    """DRAM bytes per scan launch from the committed ncu summary, or None if the
+    scan source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "index_full_scan.traffic.txt")
+    src = os.path.join(ROOT, "sparse_attention_fp4_kv_b200", "csrc", "indexer.cu")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    for line in open(p):
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if kv.get("indexer_cu_sha256") != sha or kv.get("workload") != workload:
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.file.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.file.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _config(wl, name):
+    w = wl.w
+    return {"workload": name, "batch_per_gpu": w.B, "ctx": w.ctx, "layers": w.n_layers,
+            "schedule": "".join("FRU"[m] for m in w.modes), "main_kv": f"fp4 e2m1+e4m3/16, {w.C} ch",
+            "q_heads": w.Hq, "indexer": f"int8 {w.H_idx}x{w.D_idx}", "pool_blocks": 2048,
+            "topk": 512, "n_win": w.n_win,
+            "l2": "inputs larger than L2: every step streams "
+                  f"{w.B * w.ctx * w.H_idx * w.D_idx / 1e9:.2f} GB of indexer keys",
+            "parallelism": "replicas (weak scaling, no collective)"}
+
+
+# ----------------------------------------------------------------------------- oracle timing
+def _oracle_sequence_step(inp):
+    """The oracle's decode step for one sequence of the stack (all layers)."""
+    import oracle
+    modes = inp["modes"]
+    ctx = inp["ctx"]
+    kn, sn, kvb = inp["k_idx"], inp["k_scale"], inp["kv_bf16_rows"]
+    pool = inp.get("pool0")
+    top = None
+    outs = []
+    for l, m in enumerate(modes):
+        if m == 0:
+            r = oracle.full_layer(inp["q_idx"][l], kn, sn, ctx)
+            pool, top = r["pool"], r["top"]
+        elif m == 1:
+            top, _, _ = oracle.reindex_layer(inp["q_idx"][l], kn, sn, pool, ctx)
+        outs.append(oracle.sparse_attention(inp["q"][l], lambda P: kvb(P), top, inp["swa"][l],
+                                            ctx - 1, ctx - inp["swa_rows"], inp["scale"]))
+    return outs
+
+
+def _oracle_inputs_from_device(wl, b):
+    """Host copies of sequence b's inputs (the same buffers the GPU arm uses)."""
+    def bits(t):
+        return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    from sparse_attention_fp4_kv_b200 import synth
+    w = wl.w
+    kv_rows = {}
+
+    def kvb(P):
+        P = np.asarray(P, dtype=np.int64)
+        # re-draw the bf16 rows of the requested positions (seeded, chunked)
+        out = np.empty((P.size, w.C), dtype=np.uint16)
+        for j, p in enumerate(P.tolist()):
+            c = p // 8192
+            if c not in kv_rows:
+                kv_rows[c] = bits(synth.main_kv_bf16(w, b, c * 8192, min(w.ctx, c * 8192 + 8192),
+                                                     wl.device))
+            out[j] = kv_rows[c][p - c * 8192]
+        return out
+
+    inp = dict(modes=list(wl.modes), ctx=w.ctx, k_idx=wl.k_idx[b].cpu().numpy(),
+               k_scale=wl.k_scale[b].cpu().numpy(), kv_bf16_rows=kvb,
+               q_idx={l: q[b, 0].cpu().numpy() for l, q in enumerate(wl.q_idx) if q is not None},
+               q=[bits(q[b, 0]) for q in wl.q], swa=[bits(s[b]) for s in wl.swa],
+               swa_rows=wl.swa_rows, scale=wl.scale)
+    if wl.pool_ready:
+        import oracle
+        inp["pool0"] = oracle.full_layer(wl.pool_q_idx[b, 0].cpu().numpy(), inp["k_idx"],
+                                         inp["k_scale"], w.ctx)["pool"]
+    return inp
+
+
+def _time_oracle(inp, B, n_layers, reps=1):
+    ts = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        _oracle_sequence_step(inp)
+        ts.append(time.perf_counter() - t0)
+    t_seq = statistics.median(ts)
+    # the oracle is single-threaded; a decode step of the batch is B sequences
+    return n_layers / (B * t_seq), t_seq
+
+
+# ----------------------------------------------------------------------------- arms
+def run_reference(args, name):
+    """CPU oracle arm: each step is the oracle's full decode step of one
+    sequence (all layers), a bounded sample of the batch; the rate is scaled to
+    the batch by the number of sequences."""
+    from sparse_attention_fp4_kv_b200 import synth
+    import oracle
+    oracle.build()
+    w = synth.WORKLOADS[name]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    from sparse_attention_fp4_kv_b200.workload import DecodeWorkload
+    wl = DecodeWorkload(w, dev)
+    inp = _oracle_inputs_from_device(wl, 0)
+    cfg = _config(wl, name)
+    del wl
+    if dev == "cuda":
+        torch.cuda.empty_cache()
+    for _ in range(args.warmup):
+        _oracle_sequence_step(inp)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_sequence_step(inp)
+    t_seq = (time.perf_counter() - t0) / args.steps
+    ms = t_seq * w.B * 1e3
+    value = w.n_layers / (ms / 1e3)
+    sample = (f"sequence 0 of {w.B}: Full-layer scan over all {w.ctx} tokens, pool, every "
+              f"layer's top-512 and attention ({w.n_layers} layers); rate scaled x1/{w.B}")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int64/fp64", "data": "synthetic", "config": cfg,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_csa2(args, name, rank, world, local_rank):
+    from sparse_attention_fp4_kv_b200 import synth
+    from sparse_attention_fp4_kv_b200.workload import DecodeWorkload
+    import torch.distributed as dist
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[name]
+    if world > 1:
+        w = synth.scaled(w, seed=w.seed + 1000 * rank)
+    wl = DecodeWorkload(w, dev)
+    stream = torch.cuda.current_stream()
+    K, W = args.steps, args.warmup
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    scan_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+    for a, b in scan_ev:  # materialise the event handles
+        a.record(stream)
+        b.record(stream)
+    for _ in range(W):
+        wl.step()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(dev)
+    time.sleep(0.4)
+    barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(K):
+        wl.stack(stream, scan_events=scan_ev[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_total = t_start.elapsed_time(t_end)
+    scan_ms = statistics.mean(a.elapsed_time(b) for a, b in scan_ev)
+    if world > 1:
+        t = torch.tensor([ms_total, scan_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total, scan_ms = float(t[0]), float(t[1])
+    ms_step = ms_total / K
+    value = world * w.n_layers / (ms_step / 1e3)
+
+    # ---- end to end through the public API with host buffers
+    e2e = _e2e(wl, args, stream, world, local_rank)
+
+    nbytes = wl.step_bytes()
+    peak, peak_kind = _peaks()
+    scan_gbs = nbytes["scan"] / (scan_ms / 1e3) / 1e9
+    traffic = _scan_traffic(name)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8/fp32", "data": "synthetic",
+            "config": _config(wl, name),
+            "roofline": {"bound": "hbm", "kernel": "index_full_kernel (Full-layer indexer scan)",
+                         "achieved": scan_gbs, "peak": peak, "unit": "GB/s",
+                         "frac": scan_gbs / peak, "peak_kind": peak_kind,
+                         "traffic": traffic, "algorithmic_bytes": nbytes["scan"],
+                         "launch_ms": scan_ms},
+            "step_hbm": {"algorithmic_bytes": nbytes["total"],
+                         "achieved_gbs": nbytes["total"] / (ms_step / 1e3) / 1e9,
+                         "frac": nbytes["total"] / (ms_step / 1e3) / 1e9 / peak},
+            "clocks": clk, "e2e": e2e, "gpu_launches": wl.launches_per_step() * K}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inp = _oracle_inputs_from_device(wl, 0)
+        v, t_seq = _time_oracle(inp, w.B, w.n_layers)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "sample": f"sequence 0 of {w.B}, all {w.n_layers} layers "
+                                          f"({t_seq:.1f} s), rate scaled x1/{w.B}"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def _e2e(wl, args, stream, world, local_rank):
+    """Same metric through the public API with pinned host buffers: every step
+    copies that step's inputs host->device (the new KV row, every layer's main Q
+    and indexer Q) and reads every layer's output and top-k indices back."""
+    import torch.distributed as dist
+    dev = wl.device
+    h_in = [(t, torch.empty_like(t, device="cpu").pin_memory())
+            for t in [wl.kv_new] + list(wl.q) + [q for q in wl.q_idx if q is not None]]
+    h_out = [(t, torch.empty_like(t, device="cpu").pin_memory())
+             for t in list(wl.out) + [t for t in wl.topk if t is not None]]
+    for d, h in h_in:
+        h.copy_(d)
+    h2d = sum(h.numel() * h.element_size() for _, h in h_in)
+    d2h = sum(h.numel() * h.element_size() for _, h in h_out)
+    E = max(1, min(args.steps, 200))
+
+    def one():
+        for d, h in h_in:
+            d.copy_(h, non_blocking=True)
+        wl.step(stream)
+        for d, h in h_out:
+            h.copy_(d, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(3):
+        one()
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(E):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / E
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t[0])
+    return {"value": world * wl.w.n_layers / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+            "steps": E, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="csa2", choices=["csa2", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, args.workload)
+        return
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_csa2(args, args.workload, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,153 @@
+// Library-level entry points: status strings, ABI version and the decode step
+// over a CSA2 layer stack.
+//
+// "DeepSeek-V4.1-Flash: 890 Bytes Per Token, 437x Smaller KV Cache", CSA2
+// section: each layer is statically Full, Reindex or Reuse; Full layers build
+// the pool and a fresh top-512, Reindex layers rescore the pool with their own
+// indexer Q, Reuse layers attend the indices of the nearest Full/Reindex
+// layer; every layer attends with its own main Q and SWA KV.
+#include "attention.cuh"
+
+using namespace csa2;
+
+extern "C" const char *csa2_status_string(int status) {
+    switch (status) {
+        case CSA2_OK: return "ok";
+        case CSA2_ERR_NULL: return "a required pointer is NULL";
+        case CSA2_ERR_SHAPE: return "a size is outside the supported range";
+        case CSA2_ERR_ALIGN: return "a pointer or row size breaks the alignment rule";
+        case CSA2_ERR_RANGE: return "a host-side value is out of range";
+        case CSA2_ERR_WORKSPACE: return "workspace missing or too small";
+        case CSA2_ERR_CUDA: return "a CUDA launch failed";
+        default: return "unknown status";
+    }
+}
+
+extern "C" int csa2_abi_version(void) { return CSA2_ABI_VERSION; }
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct StackWs {
+    float *tok;
+    float *blk;
+    int32_t *n_blk;
+    float *pscore;
+    int32_t *ppos;
+    void *attn;
+    size_t attn_bytes;
+    size_t total;
+};
+
+StackWs stack_layout(void *base, int B, int Hq, int C, int64_t cap) {
+    StackWs w{};
+    size_t off = 0;
+    char *p = static_cast<char *>(base);
+    const int64_t nblk = (cap + 7) / 8;
+    const int64_t P8 = (int64_t)kPoolBlocks * kBlockTokens;
+    w.tok = reinterpret_cast<float *>(p + off);
+    off += up(sizeof(float) * (size_t)B * cap);
+    w.blk = reinterpret_cast<float *>(p + off);
+    off += up(sizeof(float) * (size_t)B * nblk);
+    w.n_blk = reinterpret_cast<int32_t *>(p + off);
+    off += up(sizeof(int32_t) * (size_t)B);
+    w.pscore = reinterpret_cast<float *>(p + off);
+    off += up(sizeof(float) * (size_t)B * P8);
+    w.ppos = reinterpret_cast<int32_t *>(p + off);
+    off += up(sizeof(int32_t) * (size_t)B * P8);
+    w.attn = p + off;
+    w.attn_bytes = up(attn_workspace_bytes(B, 1, Hq, C, kTopK, CSA2_N_WIN));
+    off += w.attn_bytes;
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+
+extern "C" size_t csa2_decode_stack_workspace_size(int B, int Hq, int C, int H, int D,
+                                                   int64_t cap) {
+    (void)H;
+    (void)D;
+    if (B < 0 || cap < 1) return 0;
+    return stack_layout(nullptr, B, Hq, C, cap).total;
+}
+
+extern "C" int csa2_decode_stack(const csa2_layer *layers, int n_layers,
+                                 const void *kv_new_bf16, const int8_t *k_idx,
+                                 const float *k_scale, uint8_t *kv_fp4, uint8_t *kv_sf,
+                                 int64_t cap, const int64_t *ctx_len,
+                                 const int64_t *swa_pos0, int swa_rows, int B, int Hq, int C,
+                                 int H, int D, float softmax_scale, int32_t *pool,
+                                 int pool_ready, void *const *scan_events, void *ws,
+                                 size_t ws_bytes, void *stream) {
+    if (!layers || !k_idx || !k_scale || !kv_fp4 || !kv_sf || !ctx_len || !swa_pos0 || !pool)
+        return CSA2_ERR_NULL;
+    if (n_layers < 1 || B < 1 || cap < 1 || C < 32 || C % 32) return CSA2_ERR_SHAPE;
+    if (kv_new_bf16 && !aligned(kv_new_bf16, 16)) return CSA2_ERR_ALIGN;
+    const StackWs w = stack_layout(ws, B, Hq, C, cap);
+    if (!ws || ws_bytes < w.total) return CSA2_ERR_WORKSPACE;
+    // host-side schedule check before anything is launched
+    bool have_pool = pool_ready != 0, have_idx = false;
+    for (int l = 0; l < n_layers; l++) {
+        const csa2_layer &L = layers[l];
+        if (!L.q || !L.out || (swa_rows > 0 && !L.swa)) return CSA2_ERR_NULL;
+        if (L.mode == CSA2_MODE_FULL) {
+            if (!L.q_idx || !L.topk) return CSA2_ERR_NULL;
+            have_pool = have_idx = true;
+        } else if (L.mode == CSA2_MODE_REINDEX) {
+            if (!L.q_idx || !L.topk) return CSA2_ERR_NULL;
+            if (!have_pool) return CSA2_ERR_RANGE;
+            have_idx = true;
+        } else if (L.mode == CSA2_MODE_REUSE) {
+            if (!have_idx) return CSA2_ERR_RANGE;
+        } else {
+            return CSA2_ERR_RANGE;
+        }
+    }
+    const int64_t nblk = (cap + 7) / 8;
+    const int P8 = kPoolBlocks * kBlockTokens;
+    const int32_t *cur = nullptr;
+    bool scan_timed = false;
+    int st;
+    if (kv_new_bf16) {
+        st = launch_kv_append((const uint16_t *)kv_new_bf16, B, 1, C, ctx_len, -1, cap, kv_fp4,
+                              kv_sf, (cudaStream_t)stream);
+        if (st) return st;
+    }
+    for (int l = 0; l < n_layers; l++) {
+        const csa2_layer &L = layers[l];
+        if (L.mode == CSA2_MODE_FULL) {
+            const bool timed = scan_events && !scan_timed;
+            if (timed) cudaEventRecord((cudaEvent_t)scan_events[0], (cudaStream_t)stream);
+            st = csa2_index_full(L.q_idx, k_idx, k_scale, ctx_len, nullptr, B, 1, H, D, cap, w.tok,
+                                 w.blk, w.n_blk, stream);
+            if (st) return st;
+            if (timed) {
+                cudaEventRecord((cudaEvent_t)scan_events[1], (cudaStream_t)stream);
+                scan_timed = true;
+            }
+            st = csa2_topk(w.blk, nullptr, w.n_blk, B, nblk, kPoolBlocks, pool, nullptr, 0, stream);
+            if (st) return st;
+            st = csa2_pool_gather(w.tok, pool, ctx_len, nullptr, B, 1, kPoolBlocks, cap, w.pscore,
+                                  w.ppos, stream);
+            if (st) return st;
+            st = csa2_topk(w.pscore, w.ppos, nullptr, B, P8, kTopK, L.topk, nullptr, 0, stream);
+            if (st) return st;
+            cur = L.topk;
+        } else if (L.mode == CSA2_MODE_REINDEX) {
+            st = csa2_index_reindex(L.q_idx, k_idx, k_scale, pool, ctx_len, nullptr, B, 1, H, D,
+                                    cap, kPoolBlocks, w.pscore, w.ppos, stream);
+            if (st) return st;
+            st = csa2_topk(w.pscore, w.ppos, nullptr, B, P8, kTopK, L.topk, nullptr, 0, stream);
+            if (st) return st;
+            cur = L.topk;
+        }
+        st = csa2_sparse_attn_decode(L.q, kv_fp4, kv_sf, cap, cur, kTopK, L.swa, swa_pos0,
+                                     swa_rows, nullptr, CSA2_N_WIN, B, 1, Hq, C, softmax_scale,
+                                     L.out, w.attn, w.attn_bytes, stream);
+        if (st) return st;
+    }
+    return CSA2_OK;
+}

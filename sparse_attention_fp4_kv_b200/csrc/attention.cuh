@@ -1,0 +1,54 @@
+// Shared definitions of the sparse-attention kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace csa2 {
+
+struct AttnArgs {
+    const void *q;         // bf16 [B][Nq][Hq][C]
+    const uint8_t *kv_fp4; // [B][cap][C/2]
+    const uint8_t *kv_sf;  // [B][cap][C/16]
+    int64_t cap;
+    const int32_t *topk;   // [B][Nq][K]
+    int K;
+    const void *swa;       // bf16 [B][swa_rows][C]
+    const int64_t *swa_pos0;
+    int swa_rows;
+    const int64_t *q_pos;  // [B][Nq] or NULL
+    int n_win;
+    int B, Nq, Hq, C;
+    float scale;
+    float *out;            // fp32 [B][Nq][Hq][C]
+    void *ws;
+};
+
+// Sliding-window rows of query bq: rows [row0, row0 + n) of the SWA tensor,
+// i.e. positions max(0, p - n_win + 1) .. p that the tensor holds.
+struct AttnWindow {
+    int64_t row0;
+    int n;
+};
+
+__device__ __forceinline__ AttnWindow attn_window(const AttnArgs &a, int b, int64_t bq) {
+    AttnWindow w{0, 0};
+    if (a.n_win <= 0 || a.swa_rows <= 0 || !a.swa) return w;
+    const int64_t pos0 = a.swa_pos0 ? a.swa_pos0[b] : 0;
+    const int64_t p = a.q_pos ? a.q_pos[bq] : pos0 + a.swa_rows - 1;
+    int64_t lo = p - a.n_win + 1;
+    if (lo < 0) lo = 0;
+    if (lo < pos0) lo = pos0;
+    int64_t hi = p;
+    if (hi > pos0 + a.swa_rows - 1) hi = pos0 + a.swa_rows - 1;
+    if (hi >= lo) {
+        w.row0 = lo - pos0;
+        w.n = (int)(hi - lo + 1);
+    }
+    return w;
+}
+
+size_t attn_workspace_bytes(int B, int Nq, int Hq, int C, int K, int n_win);
+int launch_attn(const AttnArgs &a, cudaStream_t s);
+int launch_attn_general(const AttnArgs &a, cudaStream_t s);
+
+}  // namespace csa2

@@ -1,0 +1,123 @@
+// Shared helpers of the libcsa2 CUDA sources (sm_100a only).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "csa2.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libcsa2 is written for sm_100a (B200) only"
+#endif
+
+namespace csa2 {
+
+constexpr int kPoolBlocks = CSA2_POOL_BLOCKS;
+constexpr int kBlockTokens = CSA2_BLOCK_TOKENS;
+constexpr int kTopK = CSA2_TOPK;
+constexpr int kWarp = 32;
+
+inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline int launch_status() {
+    return cudaGetLastError() == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+}
+
+inline int num_sms() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+// ---------------------------------------------------------------- bf16 / fp8 / fp4
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// E4M3 code -> fp32 from the format definition (1 sign, 4 exponent bits with
+// bias 7, 3 mantissa bits; exponent field 0 is subnormal m * 2^-9). Exact.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+    uint32_t e = (code >> 3) & 0xF, m = code & 7;
+    float mag = (e == 0) ? (float)m * 0.001953125f                     // m * 2^-9
+                         : __uint_as_float(((e + 120u) << 23) | (m << 20));  // 2^(e-7)(1+m/8)
+    return (code & 0x80) ? -mag : mag;
+}
+
+// E2M1 magnitude code (3 bits) -> fp32: 0, .5, 1, 1.5, 2, 3, 4, 6.
+__device__ __forceinline__ float e2m1_mag(uint32_t c3) {
+    uint32_t e = c3 >> 1, m = c3 & 1;
+    return (e == 0) ? 0.5f * (float)m : __uint_as_float(((e + 126u) << 23) | (m << 22));
+}
+__device__ __forceinline__ float e2m1_to_f32(uint32_t c4) {
+    float v = e2m1_mag(c4 & 7);
+    return (c4 & 8) ? -v : v;
+}
+
+// fp32 -> E4M3 with round-to-nearest-even and saturation to +-448 (PTX cvt).
+__device__ __forceinline__ uint32_t f32_to_e4m3_satfinite(float x) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+    return r & 0xFF;
+}
+
+// Eight fp32 values -> eight E2M1 codes packed in a 32-bit word, value j in
+// nibble j (round-to-nearest-even, saturation to +-6; PTX cvt places its
+// second source in the low nibble of each byte).
+__device__ __forceinline__ uint32_t f32x8_to_e2m1x8(const float *v) {
+    uint32_t r;
+    asm("{\n"
+        ".reg .b8 b0, b1, b2, b3;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n"
+        "mov.b32 %0, {b0, b1, b2, b3};\n"
+        "}"
+        : "=r"(r)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return r;
+}
+
+// ---------------------------------------------------------------- ordering keys
+// fp32 -> uint32 whose unsigned order is the float order (-0 folded onto +0).
+__device__ __forceinline__ uint32_t f32_order_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    if (u == 0x80000000u) u = 0;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// 64-bit rank key: higher key = better candidate (score desc, position asc).
+__device__ __forceinline__ uint64_t rank_key(float score, int32_t pos) {
+    return ((uint64_t)f32_order_key(score) << 32) | (uint32_t)(~(uint32_t)pos);
+}
+__device__ __forceinline__ int32_t rank_key_pos(uint64_t key) { return (int32_t)(~(uint32_t)key); }
+
+// ---------------------------------------------------------------- loads
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// Visible length of query (b, i): the whole context in decode, causal in prefill.
+__device__ __forceinline__ int64_t visible_len(const int64_t *ctx_len, const int64_t *q_pos, int b,
+                                               int i, int Nq) {
+    int64_t v = ctx_len[b];
+    if (q_pos) {
+        int64_t p = q_pos[(int64_t)b * Nq + i] + 1;
+        v = p < v ? p : v;
+    }
+    return v < 0 ? 0 : v;
+}
+
+// FP4 append with positions pos_base[b] + pos_offset + i (kv_append.cu).
+int launch_kv_append(const uint16_t *kv, int B, int n_new, int C, const int64_t *pos_base,
+                     int64_t pos_offset, int64_t cap, uint8_t *fp4, uint8_t *sf, cudaStream_t s);
+
+}  // namespace csa2

@@ -1,0 +1,84 @@
+// FP4 main-KV append: quantize-and-pack new bf16 rows into the cache.
+//
+// "DeepSeek V4.1 Flash KV Cache: 890 Bytes per Token Explained" (FP4 section)
+// and "DeepSeek-V4.1-Flash: 890 Bytes Per Token, 437x Smaller KV Cache" (FP4
+// KV Quantization section): E2M1 elements, one E4M3 scale per 16 channels,
+// the NVFP4 scheme without its global scale.
+//
+// One thread per 16-channel group: two 16-byte loads of bf16, the group's
+// amax, the scale amax/6 rounded to E4M3 (PTX cvt, RNE + saturation), then 16
+// IEEE fp32 divisions by the decoded scale and eight E2M1 pair conversions.
+// A warp covers 512 contiguous channels, so loads (32 B per lane), packed
+// stores (8 B per lane) and scale stores (1 B per lane) are all coalesced.
+// The cost is negligible in decode (one row per sequence) and a few MB of
+// traffic in chunked prefill.
+#include "common.cuh"
+
+namespace csa2 {
+
+__global__ void __launch_bounds__(256) kv_append_fp4_kernel(
+    const uint16_t *__restrict__ kv, int B, int n_new, int C, const int64_t *__restrict__ start_pos,
+    int64_t pos_offset, int64_t cap, uint8_t *__restrict__ fp4, uint8_t *__restrict__ sf) {
+    const int G = C / 16;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t total = (int64_t)B * n_new * G;
+    if (gid >= total) return;
+    const int g = (int)(gid % G);
+    const int64_t row = gid / G;  // b * n_new + i
+    const int i = (int)(row % n_new);
+    const int b = (int)(row / n_new);
+    const int64_t pos = start_pos[b] + pos_offset + i;
+    if (pos < 0 || pos >= cap) return;
+
+    const uint4 *src = reinterpret_cast<const uint4 *>(kv + row * C + (int64_t)g * 16);
+    const uint4 a = src[0], c = src[1];
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+    float x[16];
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        x[2 * j] = bf16_lo(w[j]);
+        x[2 * j + 1] = bf16_hi(w[j]);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; j++) amax = fmaxf(amax, fabsf(x[j]));
+
+    const uint32_t scode = f32_to_e4m3_satfinite(__fdiv_rn(amax, 6.0f));
+    const float s = e4m3_to_f32(scode);
+    uint32_t lo = 0, hi = 0;
+    if (s != 0.0f) {
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; j++) v[j] = __fdiv_rn(x[j], s);
+        lo = f32x8_to_e2m1x8(v);
+        hi = f32x8_to_e2m1x8(v + 8);
+    }
+    const int64_t cell = (int64_t)b * cap + pos;
+    *reinterpret_cast<uint2 *>(fp4 + cell * (C / 2) + (int64_t)g * 8) = make_uint2(lo, hi);
+    sf[cell * G + g] = (uint8_t)scode;
+}
+
+int launch_kv_append(const uint16_t *kv, int B, int n_new, int C, const int64_t *pos_base,
+                     int64_t pos_offset, int64_t cap, uint8_t *fp4, uint8_t *sf, cudaStream_t s) {
+    const int64_t total = (int64_t)B * n_new * (C / 16);
+    if (total == 0) return CSA2_OK;
+    const int threads = 256;
+    const int64_t blocks = (total + threads - 1) / threads;
+    if (blocks > INT32_MAX) return CSA2_ERR_SHAPE;
+    kv_append_fp4_kernel<<<(unsigned)blocks, threads, 0, s>>>(kv, B, n_new, C, pos_base, pos_offset,
+                                                              cap, fp4, sf);
+    return launch_status();
+}
+
+}  // namespace csa2
+
+extern "C" int csa2_kv_append_fp4(const void *kv_bf16, int B, int n_new, int C,
+                                  const int64_t *start_pos, int64_t cap, uint8_t *kv_fp4,
+                                  uint8_t *kv_sf, void *stream) {
+    using namespace csa2;
+    if (!kv_bf16 || !start_pos || !kv_fp4 || !kv_sf) return CSA2_ERR_NULL;
+    if (B < 0 || n_new < 0 || cap < 0 || C < 16 || C > 8192 || C % 16) return CSA2_ERR_SHAPE;
+    if (!aligned(kv_bf16, 16) || !aligned(kv_fp4, 8)) return CSA2_ERR_ALIGN;
+    return launch_kv_append((const uint16_t *)kv_bf16, B, n_new, C, start_pos, 0, cap, kv_fp4,
+                            kv_sf, (cudaStream_t)stream);
+}

@@ -1,0 +1,129 @@
+"""Device-resident decode workloads: the caches, per-layer tensors and output
+buffers of one CSA2 decode step, laid out in HBM for libcsa2.
+
+HBM layout (per workload; B sequences, capacity = context length):
+  k_idx    int8 [B][ctx][H_idx][D_idx]   indexer keys (2 KB per token at 16x128)
+  k_scale  fp32 [B][ctx]
+  kv_fp4   uint8 [B][ctx][C/2]           E2M1 codes, two per byte
+  kv_sf    uint8 [B][ctx][C/16]          E4M3 scales
+  per layer: q bf16 [B][1][Hq][C], swa bf16 [B][128][C], out fp32 [B][1][Hq][C],
+             q_idx int8 [B][1][H_idx][D_idx] and topk int32 [B][512] (Full/Reindex)
+  pool int32 [B][2048], workspace for the decode step.
+The FP4 cache is filled with libcsa2's own append kernel from the seeded bf16
+rows; the last position (ctx - 1) is the token each decode step appends.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from . import binding as csa2
+from . import synth
+
+
+class DecodeWorkload:
+    def __init__(self, w: synth.Workload, device="cuda", keep_kv_bf16: bool = False):
+        self.w = w
+        B, ctx, C, Hq, H, D = w.B, w.ctx, w.C, w.Hq, w.H_idx, w.D_idx
+        dev = torch.device(device)
+        self.device = dev
+        self.cap = ctx
+        self.k_idx = torch.empty((B, ctx, H, D), dtype=torch.int8, device=dev)
+        self.k_scale = torch.empty((B, ctx), dtype=torch.float32, device=dev)
+        for b in range(B):
+            self.k_idx[b] = synth.indexer_keys(w, b, ctx, dev)
+            self.k_scale[b] = synth.indexer_key_scale(w, b, ctx, dev)
+        self.kv_fp4 = torch.empty((B, ctx, C // 2), dtype=torch.uint8, device=dev)
+        self.kv_sf = torch.empty((B, ctx, C // 16), dtype=torch.uint8, device=dev)
+        self.kv_bf16: Optional[torch.Tensor] = None
+        if keep_kv_bf16:
+            self.kv_bf16 = torch.empty((B, ctx, C), dtype=torch.bfloat16, device=dev)
+        zero = torch.zeros(1, dtype=torch.int64, device=dev)
+        chunk = 65536
+        for b in range(B):
+            for t0 in range(0, ctx - 1, chunk):
+                t1 = min(ctx - 1, t0 + chunk)
+                rows = synth.main_kv_bf16(w, b, t0, t1, dev)
+                if self.kv_bf16 is not None:
+                    self.kv_bf16[b, t0:t1] = rows
+                csa2.csa2_kv_append_fp4(rows.unsqueeze(0).contiguous(), zero + t0,
+                                        self.kv_fp4[b:b + 1], self.kv_sf[b:b + 1])
+        # the token this decode step appends (position ctx - 1)
+        self.kv_new = torch.stack([synth.main_kv_bf16(w, b, ctx - 1, ctx, dev)[0] for b in range(B)])
+        if self.kv_bf16 is not None:
+            self.kv_bf16[:, ctx - 1] = self.kv_new
+        self.ctx_len = torch.full((B,), ctx, dtype=torch.int64, device=dev)
+        rows = min(w.n_win, ctx)
+        self.swa_rows = rows
+        self.swa_pos0 = torch.full((B,), ctx - rows, dtype=torch.int64, device=dev)
+        L = w.n_layers
+        self.modes = list(w.modes)
+        self.q = [synth.main_q(w, l, 1, dev) for l in range(L)]
+        self.swa = [synth.swa_kv(w, l, rows, dev) for l in range(L)]
+        self.out = [torch.empty((B, 1, Hq, C), dtype=torch.float32, device=dev) for _ in range(L)]
+        self.q_idx = [synth.indexer_q(w, l, 1, dev) if m != synth.REUSE else None
+                      for l, m in enumerate(self.modes)]
+        self.topk = [torch.empty((B, csa2.TOPK), dtype=torch.int32, device=dev)
+                     if m != synth.REUSE else None for m in self.modes]
+        self.pool = torch.empty((B, csa2.POOL_BLOCKS), dtype=torch.int32, device=dev)
+        self.scale = 1.0 / math.sqrt(C)
+        self.pool_ready = False
+        self.planted = None
+        self.pool_q_idx = None
+        if self.modes[0] == synth.REINDEX:
+            self._build_pool()
+        self.stack = csa2.DecodeStack(self.modes, self.q_idx, self.q, self.swa, self.out,
+                                      self.topk, self.k_idx, self.k_scale, self.kv_fp4, self.kv_sf,
+                                      self.ctx_len, self.swa_pos0, self.pool, self.scale,
+                                      kv_new=self.kv_new, pool_ready=self.pool_ready)
+
+    def _build_pool(self):
+        """A Reindex group starts from the pool of a preceding Full layer: plant
+        the correlated blocks, then run that Full layer once (set-up)."""
+        w = self.w
+        q_r = self.q_idx[0]
+        self.planted = [synth.plant(w, b, self.k_idx[b], q_r[b, 0]) if w.planted_blocks else None
+                        for b in range(w.B)]
+        self.pool_q_idx = synth.pool_builder_q(w, q_r)
+        out = torch.empty_like(self.out[0])
+        topk = torch.empty_like(self.topk[0])
+        setup = csa2.DecodeStack([synth.FULL], [self.pool_q_idx], [self.q[0]], [self.swa[0]],
+                                 [out], [topk], self.k_idx, self.k_scale, self.kv_fp4, self.kv_sf,
+                                 self.ctx_len, self.swa_pos0, self.pool, self.scale,
+                                 kv_new=self.kv_new)
+        setup()
+        torch.cuda.synchronize(self.device)
+        self.pool_ready = True
+
+    def step(self, stream=None):
+        """One decode step: append the new token, then every layer of the stack."""
+        self.stack(stream)
+
+    def launches_per_step(self) -> int:
+        """libcsa2 kernels one step launches: the append, then per Full layer
+        scan + pool top-k + gather + token top-k, per Reindex layer rescoring +
+        top-k, and one attention kernel per layer."""
+        n = 1
+        for m in self.modes:
+            n += {synth.FULL: 4, synth.REINDEX: 2, synth.REUSE: 0}[m] + 1
+        return n
+
+    # ---- algorithmic bytes of one step (what the method must move)
+    def step_bytes(self) -> dict:
+        w = self.w
+        B, ctx, C, Hq = w.B, w.ctx, w.C, w.Hq
+        HD = w.H_idx * w.D_idx
+        scan = attn = reindex = 0
+        nblk = (ctx + 7) // 8
+        for m in self.modes:
+            if m == synth.FULL:
+                scan += B * ctx * (HD + 4) + B * ctx * 4 + B * nblk * 4   # keys+scales, scores
+            elif m == synth.REINDEX:
+                pooled = min(2048, nblk) * 8
+                reindex += B * pooled * (HD + 4)
+            attn += B * (512 * (C // 2 + C // 16) + self.swa_rows * C * 2 + Hq * C * 2 + Hq * C * 4)
+        append = B * (C * 2 + C // 2 + C // 16)
+        return dict(scan=scan, reindex=reindex, attn=attn, append=append,
+                    total=scan + reindex + attn + append)

@@ -1,0 +1,136 @@
+"""GPU parity of whole decode steps (csa2_decode_stack, the call bench.py
+times) against the oracle, on the benchmark workloads at full size and on
+scaled-down variants with ragged shapes.
+
+At full size the oracle recomputes sampled sequences one by one: the Full
+layer's scan over the whole context, the pool, every layer's top-512, and
+every layer's attention for those sequences. Pools and indices must match bit
+for bit; attention within rel-L2 1e-3 / max-abs 5e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_cases import assert_attn_close, bf16_np
+from sparse_attention_fp4_kv_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+NAMES = {synth.FULL: oracle.FULL, synth.REINDEX: oracle.REINDEX, synth.REUSE: oracle.REUSE}
+
+
+def _oracle_sequence(wl, b):
+    """Oracle indices and attention outputs of sequence b for every layer."""
+    w = wl.w
+    ctx = w.ctx
+    kn = wl.k_idx[b].cpu().numpy()
+    sn = wl.k_scale[b].cpu().numpy()
+    kvb = bf16_np(wl.kv_bf16[b])
+    pool = None
+    if wl.pool_ready:
+        pool = oracle.full_layer(wl.pool_q_idx[b, 0].cpu().numpy(), kn, sn, ctx)["pool"]
+    tops, pools, outs = [], [], []
+    top = None
+    for l, m in enumerate(wl.modes):
+        mode = NAMES[m]
+        if mode == oracle.FULL:
+            r = oracle.full_layer(wl.q_idx[l][b, 0].cpu().numpy(), kn, sn, ctx)
+            pool, top = r["pool"], r["top"]
+        elif mode == oracle.REINDEX:
+            top, _, _ = oracle.reindex_layer(wl.q_idx[l][b, 0].cpu().numpy(), kn, sn, pool, ctx)
+        tops.append(top)
+        pools.append(pool)
+        outs.append(oracle.sparse_attention(bf16_np(wl.q[l][b, 0]), lambda P: kvb[P], top,
+                                            bf16_np(wl.swa[l][b]), ctx - 1, ctx - wl.swa_rows,
+                                            wl.scale))
+    return tops, pools, outs
+
+
+def _check(wl, seqs):
+    wl.step()
+    torch.cuda.synchronize()
+    producers = [l for l, m in enumerate(wl.modes) if m != synth.REUSE]
+    for b in seqs:
+        tops, pools, outs = _oracle_sequence(wl, b)
+        assert np.array_equal(wl.pool[b].cpu().numpy(), pools[-1]), f"pool b={b}"
+        for l in range(len(wl.modes)):
+            prod = max(p for p in producers if p <= l)
+            assert np.array_equal(wl.topk[prod][b].cpu().numpy(), tops[l]), f"top-512 b={b} l={l}"
+            assert_attn_close(wl.out[l][b, 0].cpu().numpy(), outs[l], f"attention b={b} l={l}")
+
+
+def _workload(name, **kw):
+    from sparse_attention_fp4_kv_b200.workload import DecodeWorkload
+    w = synth.WORKLOADS[name] if not kw else synth.scaled(synth.WORKLOADS[name], **kw)
+    return DecodeWorkload(w, "cuda", keep_kv_bf16=True)
+
+
+def _free():
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------- scaled variants (ragged)
+@pytest.mark.parametrize("name,kw", [
+    ("decoder_stack20_b4_ctx1m", dict(B=3, ctx=20003)),
+    ("decoder_stack20_b4_ctx1m", dict(B=2, ctx=16389)),
+    ("decoder_group1_b8_ctx128k", dict(B=5, ctx=3001)),
+    ("decoder_group1_b8_ctx128k", dict(B=1, ctx=100)),
+    ("reindex_group_b32_ctx256k", dict(B=3, ctx=50001)),
+    ("full_b1_ctx4k", dict(B=2, ctx=777)),
+])
+def test_scaled_stack(name, kw):
+    wl = _workload(name, **kw)
+    _check(wl, range(wl.w.B))
+    del wl
+    _free()
+
+
+def test_decode_step_is_deterministic():
+    wl = _workload("decoder_stack20_b4_ctx1m", B=2, ctx=30000)
+    wl.step()
+    torch.cuda.synchronize()
+    first = [t.clone() for t in wl.topk if t is not None] + [o.clone() for o in wl.out]
+    for _ in range(2):
+        wl.step()
+        torch.cuda.synchronize()
+        again = [t for t in wl.topk if t is not None] + list(wl.out)
+        for x, y in zip(first, again):
+            assert torch.equal(x, y)
+    del wl
+    _free()
+
+
+# ---------------------------------------------------------------- benchmark workloads, full size
+def test_full_b1_ctx4k():
+    wl = _workload("full_b1_ctx4k")
+    _check(wl, [0])
+    del wl
+    _free()
+
+
+def test_decoder_group1_b8_ctx128k_sampled():
+    wl = _workload("decoder_group1_b8_ctx128k")
+    _check(wl, [0, 7])
+    del wl
+    _free()
+
+
+def test_reindex_group_b32_ctx256k_sampled():
+    wl = _workload("reindex_group_b32_ctx256k")
+    _check(wl, [0, 31])
+    # the planted blocks' tokens are all selected by the Reindex layer
+    for b in (0, 31):
+        top = set(wl.topk[0][b].cpu().tolist())
+        planted = {8 * j + r for j in wl.planted[b].tolist() for r in range(8)}
+        assert planted <= top
+    del wl
+    _free()
+
+
+def test_decoder_stack20_b4_ctx1m_sampled():
+    wl = _workload("decoder_stack20_b4_ctx1m")
+    _check(wl, [0, 3])
+    del wl
+    _free()

@@ -1,0 +1,332 @@
+"""GPU parity of each libcsa2 entry point against the CPU oracle, at sizes the
+oracle finishes in seconds that still span several tiles and a ragged tail.
+
+Bit-exact: packed FP4 bytes, E4M3 scales, token and block scores (fp32 bits),
+block counts, pool and top-k indices. Attention: rel-L2 <= 1e-3 and
+max-abs <= 5e-3 against the fp64 oracle.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_cases import assert_attn_close, bf16_np, f32_bits
+from sparse_attention_fp4_kv_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def B():
+    from sparse_attention_fp4_kv_b200 import binding
+    return binding
+
+
+# ----------------------------------------------------------------------------- a1 append
+def _append_and_compare(B, x_bf16: torch.Tensor, cap_extra=3, start=None):
+    """x_bf16: [Bn, n, C] on device. Appends at start positions and compares
+    every written row with the oracle's quantizer."""
+    Bn, n, C = x_bf16.shape
+    cap = n + cap_extra
+    if start is None:
+        start = torch.arange(Bn, dtype=torch.int64) % (cap_extra + 1)
+    start = start.to(DEV)
+    fp4 = torch.full((Bn, cap, C // 2), 0xAB, dtype=torch.uint8, device=DEV)
+    sf = torch.full((Bn, cap, C // 16), 0xCD, dtype=torch.uint8, device=DEV)
+    B.csa2_kv_append_fp4(x_bf16, start, fp4, sf)
+    torch.cuda.synchronize()
+    xp, xs = oracle.fp4_quantize(bf16_np(x_bf16))
+    g4, gs = fp4.cpu().numpy(), sf.cpu().numpy()
+    for b in range(Bn):
+        s0 = int(start[b])
+        assert np.array_equal(g4[b, s0:s0 + n], xp[b]), f"packed bytes differ (b={b})"
+        assert np.array_equal(gs[b, s0:s0 + n], xs[b]), f"scales differ (b={b})"
+        # rows outside the written range are untouched
+        assert np.all(g4[b, :s0] == 0xAB) and np.all(g4[b, s0 + n:] == 0xAB)
+
+
+def test_append_synthetic_rows(B):
+    w = synth.scaled(synth.WORKLOADS["decoder_group1_b8_ctx128k"], ctx=300)
+    x = torch.stack([synth.main_kv_bf16(w, b, 0, 300, DEV) for b in range(3)])
+    _append_and_compare(B, x)
+
+
+def test_append_random_bit_patterns(B):
+    g = torch.Generator(device=DEV).manual_seed(5)
+    bits = torch.randint(0, 1 << 16, (4, 257, 512), generator=g, device=DEV, dtype=torch.int32)
+    bits = bits.to(torch.int16)
+    x = bits.view(torch.bfloat16)
+    finite = torch.isfinite(x.float())
+    x = torch.where(finite, x, torch.zeros_like(x))
+    _append_and_compare(B, x.contiguous())
+
+
+def test_append_ties_zeros_and_tiny_groups(B):
+    rows = []
+    e4 = [oracle.e4m3_value(c) for c in range(0x01, 0x7F)]
+    mult = np.array([6, .25, .75, 1.25, 1.75, 2.5, 3.5, 5, -.25, -.75, -1.25, -2.5, -5, 0, -0.0, 6.5])
+    for s in e4:
+        rows.append(mult * s)
+    rows.append(np.zeros(16))
+    rows.append(np.full(16, 2.0 ** -13))            # amax/6 below the smallest E4M3 subnormal
+    rows.append(np.full(16, -(2.0 ** -12)))
+    rows.append(np.array([3e38] + [1.0] * 15))       # scale saturates at 448
+    arr = np.concatenate(rows).astype(np.float32)
+    pad = (-arr.size) % 128
+    arr = np.concatenate([arr, np.zeros(pad, np.float32)]).reshape(1, -1, 128)
+    x = torch.from_numpy(arr).to(torch.bfloat16).to(DEV)
+    _append_and_compare(B, x.contiguous(), cap_extra=0)
+
+
+@pytest.mark.parametrize("C", [16, 48, 128, 1024])
+def test_append_channel_counts(B, C):
+    g = torch.Generator(device=DEV).manual_seed(C)
+    x = (torch.randn(2, 33, C, generator=g, device=DEV) * 3).to(torch.bfloat16)
+    _append_and_compare(B, x)
+
+
+def test_append_out_of_range_positions_are_skipped(B):
+    x = torch.ones(2, 4, 32, dtype=torch.bfloat16, device=DEV)
+    fp4 = torch.zeros(2, 4, 16, dtype=torch.uint8, device=DEV)
+    sf = torch.zeros(2, 4, 2, dtype=torch.uint8, device=DEV)
+    start = torch.tensor([2, -3], dtype=torch.int64, device=DEV)
+    B.csa2_kv_append_fp4(x, start, fp4, sf)
+    torch.cuda.synchronize()
+    sfn = sf.cpu().numpy()
+    assert np.all(sfn[0, 2:] != 0) and np.all(sfn[0, :2] == 0)
+    assert np.all(sfn[1, :1] != 0) and np.all(sfn[1, 1:] == 0)
+
+
+# ----------------------------------------------------------------------------- a2/a3 scan
+def _index_inputs(Bn, cap, H, D, seed):
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    k = torch.randint(-127, 128, (Bn, cap, H, D), generator=g, device=DEV, dtype=torch.int8)
+    q = torch.randint(-127, 128, (Bn, 1, H, D), generator=g, device=DEV, dtype=torch.int8)
+    s = 0.5 + torch.rand((Bn, cap), generator=g, device=DEV)
+    return q, k, s
+
+
+@pytest.mark.parametrize("H,D,ctxs", [(16, 128, [4100, 8, 1]), (4, 64, [4096, 3001, 17]),
+                                      (3, 32, [1000, 999, 64]), (8, 128, [2049, 77, 5])])
+def test_index_full_scores_bitexact(B, H, D, ctxs):
+    cap = max(ctxs) + 5
+    Bn = len(ctxs)
+    q, k, s = _index_inputs(Bn, cap, H, D, seed=H * D)
+    ctx = torch.tensor(ctxs, dtype=torch.int64, device=DEV)
+    nb = (cap + 7) // 8
+    blk = torch.full((Bn, 1, nb), -7.0, device=DEV)
+    tok = torch.full((Bn, 1, cap), -7.0, device=DEV)
+    nblk = torch.zeros((Bn, 1), dtype=torch.int32, device=DEV)
+    B.csa2_index_full(q, k, s, ctx, blk, tok, nblk)
+    torch.cuda.synchronize()
+    qn, kn, sn = q.cpu().numpy(), k.cpu().numpy(), s.cpu().numpy()
+    for b, c in enumerate(ctxs):
+        ref_tok = oracle.index_scores(qn[b, 0], kn[b, :c], sn[b, :c])
+        ref_blk = oracle.block_scores(ref_tok, c)
+        assert np.array_equal(f32_bits(tok[b, 0, :c]), f32_bits(ref_tok))
+        assert np.array_equal(f32_bits(blk[b, 0, :ref_blk.size]), f32_bits(ref_blk))
+        assert int(nblk[b, 0]) == ref_blk.size
+        assert np.all(tok[b, 0, c:].cpu().numpy() == -7.0)     # not written beyond ctx
+        assert np.all(blk[b, 0, ref_blk.size:].cpu().numpy() == -7.0)
+
+
+def test_index_full_extreme_values_int32_exact(B):
+    # all +-127 / -128 keys: |S| up to 2048 * 16384; fp32 conversion rounds
+    Bn, cap, H, D = 2, 64, 16, 128
+    q = torch.full((Bn, 1, H, D), -128, dtype=torch.int8, device=DEV)
+    k = torch.full((Bn, cap, H, D), -128, dtype=torch.int8, device=DEV)
+    k[:, 1::2] = 127
+    k[:, 5, :, :7] = -3
+    s = torch.full((Bn, cap), 1.0, device=DEV)
+    s[:, 3] = 0.75
+    ctx = torch.tensor([64, 61], dtype=torch.int64, device=DEV)
+    blk = torch.zeros((Bn, 1, 8), device=DEV)
+    tok = torch.zeros((Bn, 1, cap), device=DEV)
+    B.csa2_index_full(q, k, s, ctx, blk, tok)
+    torch.cuda.synchronize()
+    for b, c in enumerate([64, 61]):
+        ref = oracle.index_scores(q[b, 0].cpu().numpy(), k[b, :c].cpu().numpy(), s[b, :c].cpu().numpy())
+        assert np.array_equal(f32_bits(tok[b, 0, :c]), f32_bits(ref))
+
+
+def test_index_full_causal_multi_query(B):
+    Bn, cap, H, D, Nq = 2, 3000, 4, 64, 5
+    g = torch.Generator(device=DEV).manual_seed(9)
+    k = torch.randint(-127, 128, (Bn, cap, H, D), generator=g, device=DEV, dtype=torch.int8)
+    q = torch.randint(-127, 128, (Bn, Nq, H, D), generator=g, device=DEV, dtype=torch.int8)
+    s = 0.5 + torch.rand((Bn, cap), generator=g, device=DEV)
+    ctx = torch.tensor([3000, 2500], dtype=torch.int64, device=DEV)
+    qpos = torch.tensor([[0, 7, 8, 1234, 2999], [100, 2499, 2600, 9, 10]], dtype=torch.int64,
+                        device=DEV)
+    nb = (cap + 7) // 8
+    blk = torch.zeros((Bn, Nq, nb), device=DEV)
+    tok = torch.zeros((Bn, Nq, cap), device=DEV)
+    nblk = torch.zeros((Bn, Nq), dtype=torch.int32, device=DEV)
+    B.csa2_index_full(q, k, s, ctx, blk, tok, nblk, q_pos=qpos)
+    torch.cuda.synchronize()
+    for b in range(Bn):
+        for i in range(Nq):
+            V = min(int(qpos[b, i]) + 1, int(ctx[b]))
+            ref = oracle.index_scores(q[b, i].cpu().numpy(), k[b, :V].cpu().numpy(), s[b, :V].cpu().numpy())
+            rb = oracle.block_scores(ref, V)
+            assert np.array_equal(f32_bits(tok[b, i, :V]), f32_bits(ref))
+            assert np.array_equal(f32_bits(blk[b, i, :rb.size]), f32_bits(rb))
+            assert int(nblk[b, i]) == rb.size
+
+
+# ----------------------------------------------------------------------------- a4/a5 top-k
+def _topk_ref(score, pos, valid, k):
+    sel = pos >= 0
+    if valid is not None:
+        sel &= np.arange(score.size) < valid
+    return oracle.topk(score[sel], pos[sel], k)
+
+
+@pytest.mark.parametrize("n,k,levels", [(131072, 2048, None), (20000, 512, 7), (16384, 512, None),
+                                        (5000, 512, 1), (300, 512, None), (70000, 2048, 3),
+                                        (9000, 4096, None), (1, 1, None)])
+def test_topk_bitexact(B, n, k, levels):
+    R = 3
+    g = torch.Generator(device=DEV).manual_seed(n + k)
+    if levels is None:
+        score = torch.randn((R, n), generator=g, device=DEV) * 1e5
+    else:
+        score = torch.randint(0, levels, (R, n), generator=g, device=DEV).float() - 1.0
+    score[0, : n // 3] = -0.0 if levels == 1 else score[0, : n // 3]
+    out = torch.empty((R, k), dtype=torch.int32, device=DEV)
+    nv = torch.tensor([n, max(n // 2, 1), max(n - 17, 1)], dtype=torch.int32, device=DEV)
+    B.csa2_topk(score, k, out, n_valid=nv)
+    torch.cuda.synchronize()
+    sc = score.cpu().numpy()
+    for r in range(R):
+        ref = _topk_ref(sc[r], np.arange(n), int(nv[r]), k)
+        assert np.array_equal(out[r].cpu().numpy(), ref), f"row {r}"
+
+
+def test_topk_with_candidate_positions(B):
+    R, n, k = 4, 16384, 512
+    g = torch.Generator(device=DEV).manual_seed(77)
+    score = torch.randint(-50, 50, (R, n), generator=g, device=DEV).float()
+    pos = torch.randperm(10 * n, generator=g, device=DEV)[: R * n].view(R, n).to(torch.int32)
+    pos[:, ::5] = -1
+    out = torch.empty((R, k), dtype=torch.int32, device=DEV)
+    B.csa2_topk(score, k, out, cand_pos=pos)
+    torch.cuda.synchronize()
+    for r in range(R):
+        ref = _topk_ref(score[r].cpu().numpy(), pos[r].cpu().numpy().astype(np.int64), None, k)
+        assert np.array_equal(out[r].cpu().numpy(), ref)
+
+
+# ----------------------------------------------------------------------------- Full / Reindex
+def _full_layer_gpu(B, q, k, s, ctx):
+    Bn, cap = s.shape
+    nb = (cap + 7) // 8
+    tok = torch.empty((Bn, 1, cap), device=DEV)
+    blk = torch.empty((Bn, 1, nb), device=DEV)
+    nblk = torch.empty((Bn, 1), dtype=torch.int32, device=DEV)
+    B.csa2_index_full(q, k, s, ctx, blk, tok, nblk)
+    pool = torch.empty((Bn, 1, 2048), dtype=torch.int32, device=DEV)
+    B.csa2_topk(blk.view(Bn, nb), 2048, pool.view(Bn, 2048), n_valid=nblk.view(Bn))
+    ps = torch.empty((Bn, 1, 16384), device=DEV)
+    pp = torch.empty((Bn, 1, 16384), dtype=torch.int32, device=DEV)
+    B.csa2_pool_gather(tok, pool, ctx, ps, pp)
+    top = torch.empty((Bn, 1, 512), dtype=torch.int32, device=DEV)
+    B.csa2_topk(ps.view(Bn, -1), 512, top.view(Bn, 512), cand_pos=pp.view(Bn, -1))
+    torch.cuda.synchronize()
+    return pool, top
+
+
+@pytest.mark.parametrize("ctxs", [[20003, 4096, 100], [40000, 16384, 16385], [600, 7, 1]])
+def test_full_layer_pool_and_topk_bitexact(B, ctxs):
+    H, D = 16, 128
+    cap = max(ctxs)
+    q, k, s = _index_inputs(len(ctxs), cap, H, D, seed=sum(ctxs))
+    ctx = torch.tensor(ctxs, dtype=torch.int64, device=DEV)
+    pool, top = _full_layer_gpu(B, q, k, s, ctx)
+    for b, c in enumerate(ctxs):
+        r = oracle.full_layer(q[b, 0].cpu().numpy(), k[b].cpu().numpy(), s[b].cpu().numpy(), c)
+        assert np.array_equal(pool[b, 0].cpu().numpy(), r["pool"])
+        assert np.array_equal(top[b, 0].cpu().numpy(), r["top"])
+
+
+def test_reindex_bitexact(B):
+    ctxs = [30000, 20001, 9000]
+    H, D = 16, 128
+    cap = max(ctxs)
+    q, k, s = _index_inputs(len(ctxs), cap, H, D, seed=3)
+    q2 = torch.randint(-127, 128, q.shape, device=DEV, dtype=torch.int8,
+                       generator=torch.Generator(device=DEV).manual_seed(4))
+    ctx = torch.tensor(ctxs, dtype=torch.int64, device=DEV)
+    kn, sn = k.cpu().numpy(), s.cpu().numpy()
+    # the oracle's own pool (oracle output -> GPU input is allowed; not the reverse)
+    pools = [oracle.full_layer(q[b, 0].cpu().numpy(), kn[b], sn[b], c)["pool"] for b, c in enumerate(ctxs)]
+    pool = torch.from_numpy(np.stack(pools).astype(np.int32)).view(len(ctxs), 1, 2048).to(DEV)
+    ps = torch.empty((len(ctxs), 1, 16384), device=DEV)
+    pp = torch.empty((len(ctxs), 1, 16384), dtype=torch.int32, device=DEV)
+    B.csa2_index_reindex(q2, k, s, pool, ctx, ps, pp)
+    top = torch.empty((len(ctxs), 512), dtype=torch.int32, device=DEV)
+    B.csa2_topk(ps.view(len(ctxs), -1), 512, top, cand_pos=pp.view(len(ctxs), -1))
+    torch.cuda.synchronize()
+    for b, c in enumerate(ctxs):
+        ref_top, ppos, psc = oracle.reindex_layer(q2[b, 0].cpu().numpy(), kn[b], sn[b], pools[b], c)
+        g_pos = pp[b, 0].cpu().numpy()
+        valid = g_pos >= 0
+        assert np.array_equal(g_pos[valid], ppos)
+        assert np.array_equal(f32_bits(ps[b, 0].cpu().numpy()[valid]), f32_bits(psc))
+        assert np.array_equal(top[b].cpu().numpy(), ref_top)
+
+
+# ----------------------------------------------------------------------------- a8 attention
+def _attention_case(B, Bn, ctx, C, Hq, K, n_win, seed, q_pos=None, Nq=1, drop=0):
+    w = synth.scaled(synth.WORKLOADS["decoder_group1_b8_ctx128k"], B=Bn, ctx=ctx, C=C, Hq=Hq,
+                     seed=seed)
+    kv = torch.stack([synth.main_kv_bf16(w, b, 0, ctx, DEV) for b in range(Bn)])
+    fp4 = torch.empty((Bn, ctx, C // 2), dtype=torch.uint8, device=DEV)
+    sf = torch.empty((Bn, ctx, C // 16), dtype=torch.uint8, device=DEV)
+    B.csa2_kv_append_fp4(kv, torch.zeros(Bn, dtype=torch.int64, device=DEV), fp4, sf)
+    q = synth.main_q(w, 0, Nq, DEV)
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    kk = min(K, ctx)
+    top = torch.stack([torch.stack([torch.randperm(ctx, generator=g, device=DEV)[:kk].sort().values
+                                    for _ in range(Nq)]) for _ in range(Bn)]).to(torch.int32)
+    if kk < K:
+        top = torch.cat([top, torch.full((Bn, Nq, K - kk), -1, dtype=torch.int32, device=DEV)], 2)
+    if drop:
+        top[:, :, ::drop] = -1
+    rows = min(n_win, ctx) if q_pos is None else ctx
+    swa = synth.swa_kv(w, 0, rows, DEV)
+    pos0 = torch.full((Bn,), ctx - rows, dtype=torch.int64, device=DEV)
+    out = torch.empty((Bn, Nq, Hq, C), device=DEV)
+    scale = 1.0 / math.sqrt(C)
+    B.csa2_sparse_attn_decode(q, fp4, sf, top.contiguous(), swa, pos0, out, scale, q_pos=q_pos,
+                              n_win=n_win)
+    torch.cuda.synchronize()
+    kvn, qn, topn, swan = bf16_np(kv), bf16_np(q), top.cpu().numpy(), bf16_np(swa)
+    for b in range(Bn):
+        for i in range(Nq):
+            p = (ctx - 1) if q_pos is None else int(q_pos[b, i])
+            ref = oracle.sparse_attention(qn[b, i], lambda P: kvn[b][P], topn[b, i], swan[b], p,
+                                          ctx - rows, scale, n_win)
+            assert_attn_close(out[b, i].cpu().numpy(), ref, f"b={b} i={i}")
+
+
+@pytest.mark.parametrize("Bn,ctx,C,Hq,K", [(3, 5000, 512, 64, 512), (2, 3000, 128, 8, 512),
+                                           (1, 300, 512, 64, 512), (2, 100, 256, 16, 512),
+                                           (1, 2000, 64, 3, 100)])
+def test_sparse_attention_matches_oracle(B, Bn, ctx, C, Hq, K):
+    _attention_case(B, Bn, ctx, C, Hq, K, 128, seed=ctx + C)
+
+
+def test_sparse_attention_skips_negative_indices_and_short_window(B):
+    _attention_case(B, 2, 2500, 512, 64, 512, 128, seed=1, drop=3)
+    _attention_case(B, 1, 50, 512, 64, 512, 128, seed=2)
+
+
+def test_sparse_attention_prefill_positions(B):
+    ctx = 1200
+    q_pos = torch.tensor([[1199, 1100, 600, 130]], dtype=torch.int64, device=DEV)
+    _attention_case(B, 1, ctx, 512, 64, 512, 128, seed=3, q_pos=q_pos, Nq=4)

@@ -11,8 +11,8 @@
 // General kernel: one CTA per (query, head). Warps compute one logit per key
 // (lane = C/32 channels, dequantized in registers, fp32 dot, shuffle reduce),
 // the CTA does the softmax in shared memory, and each thread then accumulates
-// its channels over all keys. Used for every shape; the tensor-core kernel in
-// attention_tc.cu takes over where its shape constraints hold.
+// its channels over all keys. Used for shapes outside the tensor-core
+// kernel's constraints (attention_tc.cu).
 #include <cfloat>
 
 #include "attention.cuh"
@@ -171,6 +171,11 @@ size_t attn_workspace_bytes(int B, int Nq, int Hq, int C, int K, int n_win) {
     return 0;
 }
 
-int launch_attn(const AttnArgs &a, cudaStream_t s) { return launch_attn_general(a, s); }
+// Tensor-core kernel where its shape constraints hold (64 heads, 512 channels,
+// at most 640 keys per query), the general kernel otherwise.
+int launch_attn(const AttnArgs &a, cudaStream_t s) {
+    if (attn_tc_supported(a)) return launch_attn_tc(a, s);
+    return launch_attn_general(a, s);
+}
 
 }  // namespace csa2

@@ -1,0 +1,515 @@
+// Tensor-core sparse attention for the pages' decoder shape: 64 main-Q heads,
+// 512-channel shared KV head, up to 512 selected FP4 rows + 128 window rows.
+//
+// "890 bytes per token: how DeepSeek V4.1-Flash's KV cache works", mechanism
+// 4: attention runs only over the selected candidates. "DeepSeek-V4.1-Flash:
+// 890 Bytes Per Token, 437x Smaller KV Cache", CSA2 and CED sections: each
+// layer has its own main Q and SWA KV; the window is the last 128 tokens.
+// FP4 section of both pages: E2M1 elements with one E4M3 scale per 16 channels.
+//
+// One thread-block cluster of 8 CTAs per query; CTA r takes keys
+// [80 r, 80 r + 80) of the query's key list (selected rows, then window rows).
+//  1. cp.async stages the query's 64 x 512 bf16 Q and the CTA's window rows
+//     into 128-byte-swizzled K-major tiles; the FP4 rows are loaded with 8-byte
+//     vector loads and dequantized in registers (e2m1 * e4m3 is exact in bf16).
+//  2. One thread issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32):
+//     S = Q K^T with M = 64 heads, N = 80 keys, K = 512, accumulated in TMEM.
+//  3. Each of the 4 warps reads its 16 heads' logits from TMEM (two threads per
+//     head), does a chunk-local softmax in fp32 and writes P to shared memory
+//     as bf16 hi + lo parts (P = hi + lo to ~16 bits, so the P V product keeps
+//     fp32-level accuracy with bf16 operands).
+//  4. O = P_hi V + P_lo V: M = 64, N = 256 (two halves of 512 channels), K = 80,
+//     the same shared-memory KV tile read as an MN-major operand.
+//  5. The unnormalized O, the row maxima and the row sums go to shared memory;
+//     after a cluster barrier each CTA combines 64 channels of all 64 heads over
+//     the 8 CTAs through distributed shared memory and writes the output.
+// TMEM: O uses columns 0..511 of lanes 0-15 of each 32-lane subpartition
+// (the M = 64 accumulator layout); S uses lanes 16-31 of columns 0..79.
+// No global scratch; one launch per layer.
+#include <cuda_bf16.h>
+
+#include "attention.cuh"
+
+namespace csa2 {
+namespace tc {
+
+constexpr int HQ = 64;
+constexpr int CH = 512;
+constexpr int T = 80;        // keys per CTA
+constexpr int CL = 8;        // CTAs per query (cluster size)
+constexpr int THREADS = 128;
+constexpr int KEYS_MAX = T * CL;
+
+constexpr int Q_CHUNK = HQ * 128;  // one 64-channel column of Q: 64 rows x 128 B
+constexpr int Q_BYTES = HQ * CH * 2;
+constexpr int K_CHUNK = T * 128;   // one 64-channel column of the KV tile
+constexpr int K_BYTES = T * CH * 2;
+constexpr int P_ATOM = HQ * 128;   // 64 tokens of P for 64 heads
+constexpr int P_BYTES = 2 * P_ATOM;
+
+constexpr int Q_OFF = 0;
+constexpr int K_OFF = Q_OFF + Q_BYTES;
+constexpr int PHI_OFF = K_OFF + K_BYTES;
+constexpr int PLO_OFF = PHI_OFF + P_BYTES;
+constexpr int M_OFF = PLO_OFF + P_BYTES;  // fp32 row max (log2 domain) [64]
+constexpr int L_OFF = M_OFF + HQ * 4;     // fp32 row sum [64]
+constexpr int SLOT_OFF = L_OFF + HQ * 4;  // int64 source offset per key slot [T]
+constexpr int KIND_OFF = SLOT_OFF + T * 8;
+constexpr int BAR_OFF = (KIND_OFF + T + 15) / 16 * 16;
+constexpr int TADDR_OFF = BAR_OFF + 16;
+constexpr int SMEM_USED = TADDR_OFF + 16;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
+// Partial-O staging ([64][512 + 4] fp32) reuses the Q and KV tiles.
+constexpr int STG_STRIDE = CH + 4;
+static_assert(HQ * STG_STRIDE * 4 <= Q_BYTES + K_BYTES, "staging must fit in Q + KV tiles");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr long WAIT_LIMIT = 1L << 24;
+
+__device__ int g_attn_error = 0;
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t a, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+// Bounded wait on an mbarrier phase; returns false if the limit ran out.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase) {
+    for (long it = 0; it < WAIT_LIMIT; it++) {
+        uint32_t done;
+        asm volatile(
+            "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+            "selp.u32 %0, 1, 0, p;\n}"
+            : "=r"(done)
+            : "r"(bar), "r"(phase)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// Shared-memory matrix descriptor: 128-byte swizzle, sm_100 descriptor version.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t acc) {
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+
+// 16 lanes x 32-bit, 32 columns per half-warp: threads 0-15 read columns
+// [col, col + 32) of lanes base..base+15, threads 16-31 read [col + 32, col + 64).
+__device__ __forceinline__ void tmem_ld_16x32x2_32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+        "%30, %31}, [%32], 32;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
+}
+// Same with 8 columns per half-warp.
+__device__ __forceinline__ void tmem_ld_16x32x2_8(uint32_t taddr, float (&v)[8]) {
+    uint32_t r[8];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8], 8;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 8; i++) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+__device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+// Byte offset of 16-byte piece p (0..7) of row r inside a 128B-swizzled,
+// 8-row-atom column (rows at 128 B, atoms at 1024 B).
+__device__ __forceinline__ uint32_t sw128(int r, int p) {
+    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((p ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// ---------------------------------------------------------------- kernel
+__global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *sm = smem_raw + (base - raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t rank = cluster_rank();
+    const int64_t bq = blockIdx.y;
+    const int b = (int)(bq / a.Nq);
+    const AttnWindow w = attn_window(a, b, bq);
+
+    float *m_s = reinterpret_cast<float *>(sm + M_OFF);
+    float *l_s = reinterpret_cast<float *>(sm + L_OFF);
+    int64_t *slot_src = reinterpret_cast<int64_t *>(sm + SLOT_OFF);
+    uint8_t *slot_kind = sm + KIND_OFF;
+    const uint32_t bar = base + BAR_OFF;
+    uint32_t *taddr_s = reinterpret_cast<uint32_t *>(sm + TADDR_OFF);
+
+    // ---- set-up: mbarrier, TMEM, key slots
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) tmem_alloc(base + TADDR_OFF, 512);
+    if (tid < T) {
+        const int kidx = (int)rank * T + tid;
+        uint8_t kind = 0;
+        int64_t src = 0;
+        if (kidx < a.K) {
+            const int32_t pos = a.topk[bq * a.K + kidx];
+            if (pos >= 0 && pos < a.cap) {
+                kind = 1;
+                src = (int64_t)b * a.cap + pos;
+            }
+        } else if (kidx - a.K < w.n) {
+            kind = 2;
+            src = (int64_t)b * a.swa_rows + w.row0 + (kidx - a.K);
+        }
+        slot_kind[tid] = kind;
+        slot_src[tid] = src;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *taddr_s;
+
+    // ---- stage Q and the window rows (cp.async), dequantize FP4 rows
+    const uint8_t *qg = reinterpret_cast<const uint8_t *>(a.q) + bq * (int64_t)HQ * CH * 2;
+    for (int i = tid; i < HQ * 64; i += THREADS) {
+        const int r = i >> 6, pg = i & 63;
+        cp_async16(base + Q_OFF + (pg >> 3) * Q_CHUNK + sw128(r, pg & 7), qg + r * 1024 + pg * 16);
+    }
+    const uint8_t *swa = reinterpret_cast<const uint8_t *>(a.swa);
+    for (int i = tid; i < T * 64; i += THREADS) {
+        const int j = i >> 6, pg = i & 63;
+        const uint32_t dst = base + K_OFF + (pg >> 3) * K_CHUNK + sw128(j, pg & 7);
+        const uint8_t kind = slot_kind[j];
+        if (kind == 2)
+            cp_async16(dst, swa + slot_src[j] * 1024 + pg * 16);
+        else if (kind == 0)
+            st_shared_v4(dst, make_uint4(0, 0, 0, 0));
+    }
+    for (int i = tid; i < T * 32; i += THREADS) {  // (slot, 16-channel group)
+        const int j = i >> 5, g = i & 31;
+        if (slot_kind[j] != 1) continue;
+        const int64_t cell = slot_src[j];
+        const uint2 codes = *reinterpret_cast<const uint2 *>(a.kv_fp4 + cell * 256 + g * 8);
+        const float s = e4m3_to_f32(a.kv_sf[cell * 32 + g]);
+        uint32_t wds[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            const uint32_t byte = ((u < 4 ? codes.x : codes.y) >> (8 * (u & 3))) & 0xFF;
+            wds[u] = pack_bf16x2(e2m1_to_f32(byte & 0xF) * s, e2m1_to_f32(byte >> 4) * s);
+        }
+        const int pg = g * 2;  // two 16-byte pieces
+        const uint32_t d0 = base + K_OFF + (pg >> 3) * K_CHUNK + sw128(j, pg & 7);
+        const uint32_t d1 = base + K_OFF + ((pg + 1) >> 3) * K_CHUNK + sw128(j, (pg + 1) & 7);
+        st_shared_v4(d0, make_uint4(wds[0], wds[1], wds[2], wds[3]));
+        st_shared_v4(d1, make_uint4(wds[4], wds[5], wds[6], wds[7]));
+    }
+    cp_async_wait_all();
+    fence_proxy_async();
+    __syncthreads();
+
+    bool ok = true;
+    // ---- S = Q K^T  (M = 64, N = 80, K = 512) into TMEM lanes 16..31
+    const uint32_t s_tmem = tmem + (16u << 16);
+    if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t id_s = idesc_bf16(HQ, T, false);
+#pragma unroll 1
+        for (int kk = 0; kk < CH / 16; kk++) {
+            const uint32_t off = (kk & 3) * 32;
+            const uint64_t ad = sdesc(base + Q_OFF + (kk >> 2) * Q_CHUNK + off, 16, 1024);
+            const uint64_t bd = sdesc(base + K_OFF + (kk >> 2) * K_CHUNK + off, 16, 1024);
+            mma_bf16(s_tmem, ad, bd, id_s, kk > 0);
+        }
+        mma_commit(bar);
+    }
+    ok = mbar_wait(bar, 0);
+    tc_fence_after();
+
+    // ---- softmax over this CTA's keys; two threads per head
+    const int h = warp * 16 + (lane & 15);
+    const int half = lane >> 4;
+    const float sl2 = a.scale * LOG2E;
+    float p[40];
+    {
+        float v32[32], v8[8];
+        const uint32_t row_addr = s_tmem + ((uint32_t)(warp * 32) << 16);
+        tmem_ld_16x32x2_32(row_addr + 0, v32);
+        tmem_ld_16x32x2_8(row_addr + 64, v8);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+            const int j = half * 32 + i;
+            p[i] = (ok && slot_kind[j] != 0) ? v32[i] * sl2 : -INFINITY;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const int j = 64 + half * 8 + i;
+            p[32 + i] = (ok && slot_kind[j] != 0) ? v8[i] * sl2 : -INFINITY;
+        }
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 40; i++) mx = fmaxf(mx, p[i]);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    float sum = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 40; i++) {
+        p[i] = (p[i] == -INFINITY) ? 0.0f : ex2(p[i] - mx);
+        sum += p[i];
+    }
+    sum += __shfl_xor_sync(0xffffffffu, sum, 16);
+    if (half == 0) {
+        m_s[h] = mx;
+        l_s[h] = sum;
+    }
+    // P = hi + lo (bf16), K-major 128B-swizzled tiles: tokens 0..63 in the
+    // first atom column, 64..79 in the second.
+#pragma unroll
+    for (int piece = 0; piece < 5; piece++) {
+        const int tok0 = piece < 4 ? half * 32 + piece * 8 : 64 + half * 8;
+        const float *pp = p + piece * 8;
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const __nv_bfloat162 hb = __floats2bfloat162_rn(pp[2 * u], pp[2 * u + 1]);
+            const float2 hf = __bfloat1622float2(hb);
+            hi[u] = *reinterpret_cast<const uint32_t *>(&hb);
+            lo[u] = pack_bf16x2(pp[2 * u] - hf.x, pp[2 * u + 1] - hf.y);
+        }
+        const uint32_t off = (tok0 >> 6) * P_ATOM + sw128(h, (tok0 & 63) >> 3);
+        st_shared_v4(base + PHI_OFF + off, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+        st_shared_v4(base + PLO_OFF + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- O = P_hi V + P_lo V  (M = 64, N = 256 per half, K = 80)
+    if (tid == 0 && ok) {
+        tc_fence_after();
+        constexpr uint32_t id_o = idesc_bf16(HQ, 256, true);
+#pragma unroll 1
+        for (int hf = 0; hf < 2; hf++) {
+#pragma unroll 1
+            for (int kk = 0; kk < T / 16; kk++) {
+                const uint32_t poff = (kk >> 2) * P_ATOM + (kk & 3) * 32;
+                const uint64_t vd =
+                    sdesc(base + K_OFF + hf * 4 * K_CHUNK + kk * 2048, K_CHUNK, 1024);
+                mma_bf16(tmem + hf * 256, sdesc(base + PHI_OFF + poff, 16, 1024), vd, id_o, kk > 0);
+                mma_bf16(tmem + hf * 256, sdesc(base + PLO_OFF + poff, 16, 1024), vd, id_o, 1);
+            }
+        }
+        mma_commit(bar);
+    }
+    if (ok) ok = mbar_wait(bar, 1);
+    tc_fence_after();
+
+    // ---- unnormalized O -> shared staging [64][516] fp32 (reuses Q and KV tiles)
+    float *stg = reinterpret_cast<float *>(sm + Q_OFF);
+    {
+        const uint32_t row_addr = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll 1
+        for (int c0 = 0; c0 < CH; c0 += 64) {
+            float v[32];
+            tmem_ld_16x32x2_32(row_addr + c0, v);
+            tmem_ld_wait();
+            float *dst = stg + h * STG_STRIDE + c0 + half * 32;
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                const float4 f = ok ? make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3])
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4 *>(dst + 4 * u) = f;
+            }
+        }
+    }
+    if (!ok && tid == 0) atomicExch(&g_attn_error, 1);
+    tc_fence_before();
+    cluster_sync();  // staging of every CTA in the cluster is complete
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+
+    // ---- combine: this CTA owns channels [64 rank, 64 rank + 64) of all heads
+    {
+        const int hh = tid >> 1;           // head
+        const int c0 = (int)rank * 64 + (tid & 1) * 32;
+        float mr[CL], M = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < CL; r++) {
+            mr[r] = ld_dsmem_f32(map_rank(base + M_OFF + hh * 4, r));
+            M = fmaxf(M, mr[r]);
+        }
+        float acc[32];
+#pragma unroll
+        for (int i = 0; i < 32; i++) acc[i] = 0.0f;
+        float den = 0.0f;
+        if (M != -INFINITY) {
+#pragma unroll 1
+            for (int r = 0; r < CL; r++) {
+                if (mr[r] == -INFINITY) continue;
+                const float wgt = ex2(mr[r] - M);
+                den += wgt * ld_dsmem_f32(map_rank(base + L_OFF + hh * 4, r));
+                const uint32_t src =
+                    map_rank(base + Q_OFF + (uint32_t)(hh * STG_STRIDE + c0) * 4, r);
+#pragma unroll
+                for (int u = 0; u < 8; u++) {
+                    const float4 f = ld_dsmem_v4(src + 16 * u);
+                    acc[4 * u] += wgt * f.x;
+                    acc[4 * u + 1] += wgt * f.y;
+                    acc[4 * u + 2] += wgt * f.z;
+                    acc[4 * u + 3] += wgt * f.w;
+                }
+            }
+        }
+        const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+        float *out = a.out + (bq * HQ + hh) * (int64_t)CH + c0;
+#pragma unroll
+        for (int u = 0; u < 8; u++)
+            *reinterpret_cast<float4 *>(out + 4 * u) =
+                make_float4(acc[4 * u] * inv, acc[4 * u + 1] * inv, acc[4 * u + 2] * inv,
+                            acc[4 * u + 3] * inv);
+    }
+    cluster_sync();  // peers may still be reading this CTA's staging
+}
+
+}  // namespace tc
+
+bool attn_tc_supported(const AttnArgs &a) {
+    const int nwin = a.n_win < a.swa_rows ? a.n_win : a.swa_rows;
+    return a.C == tc::CH && a.Hq == tc::HQ && a.K + (nwin > 0 ? nwin : 0) <= tc::KEYS_MAX &&
+           aligned(a.q, 16) && (a.swa == nullptr || aligned(a.swa, 16)) && aligned(a.kv_fp4, 8);
+}
+
+int launch_attn_tc(const AttnArgs &a, cudaStream_t s) {
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::SMEM_BYTES) != cudaSuccess)
+            return CSA2_ERR_CUDA;
+        attr = true;
+    }
+    const int64_t rows = (int64_t)a.B * a.Nq;
+    if (rows > 65535) return CSA2_ERR_SHAPE;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(tc::CL, (unsigned)rows, 1);
+    cfg.blockDim = dim3(tc::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = tc::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr_cl[1];
+    attr_cl[0].id = cudaLaunchAttributeClusterDimension;
+    attr_cl[0].val.clusterDim.x = tc::CL;
+    attr_cl[0].val.clusterDim.y = 1;
+    attr_cl[0].val.clusterDim.z = 1;
+    cfg.attrs = attr_cl;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel, a) != cudaSuccess) return CSA2_ERR_CUDA;
+    return launch_status();
+}
+
+}  // namespace csa2

@@ -96,7 +96,8 @@ _T_KV, _T_KIDX, _T_KSCALE, _T_Q, _T_SWA, _T_QIDX, _T_OUTL, _T_PLANT, _T_PLANTU, 
 
 def _gen(w: Workload, tensor: int, a: int = 0, b: int = 0, device="cpu") -> torch.Generator:
     g = torch.Generator(device=device)
-    g.manual_seed(((w.seed * 1_000_003 + tensor) * 1_000_033 + a) * 1_000_037 + b)
+    key = ((w.seed * 1_000_003 + tensor) * 1_000_033 + a) * 1_000_037 + b
+    g.manual_seed(key % (1 << 63))
     return g
 
 

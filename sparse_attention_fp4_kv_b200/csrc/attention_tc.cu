@@ -10,8 +10,9 @@
 // One thread-block cluster of 8 CTAs per query; CTA r takes keys
 // [80 r, 80 r + 80) of the query's key list (selected rows, then window rows).
 //  1. cp.async stages the query's 64 x 512 bf16 Q and the CTA's window rows
-//     into 128-byte-swizzled K-major tiles; the FP4 rows are loaded with 8-byte
-//     vector loads and dequantized in registers (e2m1 * e4m3 is exact in bf16).
+//     into 128-byte-swizzled K-major tiles, and the raw FP4 rows (codes and
+//     scales) into a staging area, all in flight at once; the FP4 rows are then
+//     dequantized from shared memory (e2m1 * e4m3 is exact in bf16).
 //  2. One thread issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32):
 //     S = Q K^T with M = 64 heads, N = 80 keys, K = 512, accumulated in TMEM.
 //  3. Each of the 4 warps reads its 16 heads' logits from TMEM (two threads per
@@ -55,6 +56,8 @@ constexpr int M_OFF = PLO_OFF + P_BYTES;  // fp32 row max (log2 domain) [64]
 constexpr int L_OFF = M_OFF + HQ * 4;     // fp32 row sum [64]
 constexpr int SLOT_OFF = L_OFF + HQ * 4;  // int64 source offset per key slot [T]
 constexpr int KIND_OFF = SLOT_OFF + T * 8;
+constexpr int FP4_STAGE_OFF = PHI_OFF;    // raw FP4 rows [T][288], before P is written
+static_assert(T * 288 <= 2 * P_BYTES, "FP4 staging must fit in the P buffers");
 constexpr int BAR_OFF = (KIND_OFF + T + 15) / 16 * 16;
 constexpr int TADDR_OFF = BAR_OFF + 16;
 constexpr int SMEM_USED = TADDR_OFF + 16;
@@ -274,7 +277,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
     tc_fence_after();
     const uint32_t tmem = *taddr_s;
 
-    // ---- stage Q and the window rows (cp.async), dequantize FP4 rows
+    // ---- stage Q, the window rows and the raw FP4 rows with cp.async (all in
+    // flight together), then dequantize the FP4 rows from shared memory
     const uint8_t *qg = reinterpret_cast<const uint8_t *>(a.q) + bq * (int64_t)HQ * CH * 2;
     for (int i = tid; i < HQ * 64; i += THREADS) {
         const int r = i >> 6, pg = i & 63;
@@ -290,12 +294,23 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
         else if (kind == 0)
             st_shared_v4(dst, make_uint4(0, 0, 0, 0));
     }
+    // raw FP4 rows: 16 pieces of codes + 2 pieces of scales per row, staged in
+    // the (not yet used) P buffers as [T][288] bytes
+    for (int i = tid; i < T * 18; i += THREADS) {
+        const int j = i / 18, pc = i - j * 18;
+        if (slot_kind[j] != 1) continue;
+        const int64_t cell = slot_src[j];
+        const uint8_t *src = pc < 16 ? a.kv_fp4 + cell * 256 + pc * 16 : a.kv_sf + cell * 32 + (pc - 16) * 16;
+        cp_async16(base + FP4_STAGE_OFF + j * 288 + pc * 16, src);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    const uint8_t *stage = sm + FP4_STAGE_OFF;
     for (int i = tid; i < T * 32; i += THREADS) {  // (slot, 16-channel group)
         const int j = i >> 5, g = i & 31;
         if (slot_kind[j] != 1) continue;
-        const int64_t cell = slot_src[j];
-        const uint2 codes = *reinterpret_cast<const uint2 *>(a.kv_fp4 + cell * 256 + g * 8);
-        const float s = e4m3_to_f32(a.kv_sf[cell * 32 + g]);
+        const uint2 codes = *reinterpret_cast<const uint2 *>(stage + j * 288 + g * 8);
+        const float s = e4m3_to_f32(stage[j * 288 + 256 + g]);
         uint32_t wds[8];
 #pragma unroll
         for (int u = 0; u < 8; u++) {
@@ -308,7 +323,6 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
         st_shared_v4(d0, make_uint4(wds[0], wds[1], wds[2], wds[3]));
         st_shared_v4(d1, make_uint4(wds[4], wds[5], wds[6], wds[7]));
     }
-    cp_async_wait_all();
     fence_proxy_async();
     __syncthreads();
 
@@ -437,43 +451,48 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
 
     // ---- combine: this CTA owns channels [64 rank, 64 rank + 64) of all heads
     {
-        const int hh = tid >> 1;           // head
+        const int hh = tid >> 1;  // head
         const int c0 = (int)rank * 64 + (tid & 1) * 32;
-        float mr[CL], M = -INFINITY;
+        float mr[CL], lr[CL], M = -INFINITY;
 #pragma unroll
         for (int r = 0; r < CL; r++) {
             mr[r] = ld_dsmem_f32(map_rank(base + M_OFF + hh * 4, r));
-            M = fmaxf(M, mr[r]);
+            lr[r] = ld_dsmem_f32(map_rank(base + L_OFF + hh * 4, r));
         }
-        float acc[32];
 #pragma unroll
-        for (int i = 0; i < 32; i++) acc[i] = 0.0f;
-        float den = 0.0f;
-        if (M != -INFINITY) {
-#pragma unroll 1
-            for (int r = 0; r < CL; r++) {
-                if (mr[r] == -INFINITY) continue;
-                const float wgt = ex2(mr[r] - M);
-                den += wgt * ld_dsmem_f32(map_rank(base + L_OFF + hh * 4, r));
-                const uint32_t src =
-                    map_rank(base + Q_OFF + (uint32_t)(hh * STG_STRIDE + c0) * 4, r);
+        for (int r = 0; r < CL; r++) M = fmaxf(M, mr[r]);
+        float wgt[CL], den = 0.0f;
 #pragma unroll
-                for (int u = 0; u < 8; u++) {
-                    const float4 f = ld_dsmem_v4(src + 16 * u);
-                    acc[4 * u] += wgt * f.x;
-                    acc[4 * u + 1] += wgt * f.y;
-                    acc[4 * u + 2] += wgt * f.z;
-                    acc[4 * u + 3] += wgt * f.w;
-                }
-            }
+        for (int r = 0; r < CL; r++) {
+            wgt[r] = (M == -INFINITY || mr[r] == -INFINITY) ? 0.0f : ex2(mr[r] - M);
+            den += wgt[r] * lr[r];
         }
         const float inv = den > 0.0f ? 1.0f / den : 0.0f;
         float *out = a.out + (bq * HQ + hh) * (int64_t)CH + c0;
+#pragma unroll 1
+        for (int part = 0; part < 2; part++) {  // 16 channels per part
+            float4 f[CL][4];
 #pragma unroll
-        for (int u = 0; u < 8; u++)
-            *reinterpret_cast<float4 *>(out + 4 * u) =
-                make_float4(acc[4 * u] * inv, acc[4 * u + 1] * inv, acc[4 * u + 2] * inv,
-                            acc[4 * u + 3] * inv);
+            for (int r = 0; r < CL; r++) {
+                const uint32_t src = map_rank(
+                    base + Q_OFF + (uint32_t)(hh * STG_STRIDE + c0 + part * 16) * 4, r);
+#pragma unroll
+                for (int u = 0; u < 4; u++) f[r][u] = ld_dsmem_v4(src + 16 * u);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int r = 0; r < CL; r++) {
+                    acc.x += wgt[r] * f[r][u].x;
+                    acc.y += wgt[r] * f[r][u].y;
+                    acc.z += wgt[r] * f[r][u].z;
+                    acc.w += wgt[r] * f[r][u].w;
+                }
+                *reinterpret_cast<float4 *>(out + part * 16 + 4 * u) =
+                    make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+            }
+        }
     }
     cluster_sync();  // peers may still be reading this CTA's staging
 }
@@ -483,7 +502,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
 bool attn_tc_supported(const AttnArgs &a) {
     const int nwin = a.n_win < a.swa_rows ? a.n_win : a.swa_rows;
     return a.C == tc::CH && a.Hq == tc::HQ && a.K + (nwin > 0 ? nwin : 0) <= tc::KEYS_MAX &&
-           aligned(a.q, 16) && (a.swa == nullptr || aligned(a.swa, 16)) && aligned(a.kv_fp4, 8);
+           aligned(a.q, 16) && (a.swa == nullptr || aligned(a.swa, 16)) && aligned(a.kv_fp4, 16) &&
+           aligned(a.kv_sf, 16);
 }
 
 int launch_attn_tc(const AttnArgs &a, cudaStream_t s) {

@@ -36,6 +36,10 @@ struct TopkArgs {
     int32_t *out;
 };
 
+__device__ __forceinline__ bool aligned16(const void *p) {
+    return (reinterpret_cast<uintptr_t>(p) & 15) == 0;
+}
+
 struct TopkShared {
     uint32_t *hist;
     uint64_t *buf;
@@ -99,27 +103,61 @@ __device__ __forceinline__ bool load_cand(const TopkArgs &a, int64_t r, int64_t 
     return pos >= 0;
 }
 
-constexpr int TK_UNROLL = 8;
+constexpr int TK_UNROLL = 4;  // 16-byte loads in flight per thread
+
+// Four consecutive candidates i0..i0+3 (i0 % 4 == 0) with 16-byte loads when the
+// row is 16-byte aligned, else element by element.
+__device__ __forceinline__ void load_cand4(const TopkArgs &a, int64_t r, int64_t i0, int64_t nv,
+                                           bool vec, uint64_t (&key)[4], bool (&ok)[4]) {
+    if (vec && i0 + 3 < nv) {
+        const float4 s = *reinterpret_cast<const float4 *>(a.score + r * a.n + i0);
+        int4 p = make_int4((int)i0, (int)i0 + 1, (int)i0 + 2, (int)i0 + 3);
+        if (a.cand_pos) p = *reinterpret_cast<const int4 *>(a.cand_pos + r * a.n + i0);
+        key[0] = rank_key(s.x, p.x);
+        key[1] = rank_key(s.y, p.y);
+        key[2] = rank_key(s.z, p.z);
+        key[3] = rank_key(s.w, p.w);
+        ok[0] = p.x >= 0;
+        ok[1] = p.y >= 0;
+        ok[2] = p.z >= 0;
+        ok[3] = p.w >= 0;
+    } else {
+#pragma unroll
+        for (int u = 0; u < 4; u++) ok[u] = (i0 + u < nv) && load_cand(a, r, i0 + u, key[u]);
+    }
+}
+
+// Calls f(key) for every candidate of row r (i < nv), TK_UNROLL x 4 per thread
+// per iteration.
+template <typename F>
+__device__ __forceinline__ void for_each_cand(const TopkArgs &a, int64_t r, int64_t nv, bool vec,
+                                              F f) {
+    const int64_t step = (int64_t)TK_THREADS * 4 * TK_UNROLL;
+    for (int64_t b0 = 0; b0 < nv; b0 += step) {
+        uint64_t key[TK_UNROLL][4];
+        bool ok[TK_UNROLL][4];
+#pragma unroll
+        for (int u = 0; u < TK_UNROLL; u++)
+            load_cand4(a, r, b0 + ((int64_t)u * TK_THREADS + threadIdx.x) * 4, nv, vec, key[u],
+                       ok[u]);
+#pragma unroll
+        for (int u = 0; u < TK_UNROLL; u++)
+#pragma unroll
+            for (int v = 0; v < 4; v++)
+                if (ok[u][v]) f(key[u][v]);
+    }
+}
 
 // One digit histogram pass over the global row: keys whose masked bits equal
 // the prefix are binned by (key >> shift) & (NB - 1).
-__device__ void global_hist_pass(const TopkArgs &a, int64_t r, int64_t nv, uint32_t *hist, int NB,
-                                 int shift, uint64_t prefix, uint64_t mask) {
+__device__ void global_hist_pass(const TopkArgs &a, int64_t r, int64_t nv, bool vec,
+                                 uint32_t *hist, int NB, int shift, uint64_t prefix,
+                                 uint64_t mask) {
     for (int b = threadIdx.x; b < NB; b += TK_THREADS) hist[b] = 0;
     __syncthreads();
-    for (int64_t i0 = 0; i0 < nv; i0 += (int64_t)TK_THREADS * TK_UNROLL) {
-        uint64_t key[TK_UNROLL];
-        bool ok[TK_UNROLL];
-#pragma unroll
-        for (int u = 0; u < TK_UNROLL; u++) {
-            const int64_t i = i0 + (int64_t)u * TK_THREADS + threadIdx.x;
-            ok[u] = (i < nv) && load_cand(a, r, i, key[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < TK_UNROLL; u++)
-            if (ok[u] && (key[u] & mask) == prefix)
-                atomicAdd(&hist[(key[u] >> shift) & (uint64_t)(NB - 1)], 1u);
-    }
+    for_each_cand(a, r, nv, vec, [&](uint64_t key) {
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (uint64_t)(NB - 1)], 1u);
+    });
     __syncthreads();
 }
 
@@ -169,6 +207,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
         const int64_t v = a.n_valid[r];
         nv = v < 0 ? 0 : (v < a.n ? v : a.n);
     }
+    const bool vec = ((r * a.n) % 4 == 0) && aligned16(a.score) &&
+                     (a.cand_pos == nullptr || aligned16(a.cand_pos));
     if (threadIdx.x == 0) {
         st.prefix = 0;
         st.mask = 0;
@@ -182,7 +222,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
     int shift = 52, NB = TK_HIST;
     bool all_selected = false, exact = false;
     while (true) {
-        global_hist_pass(a, r, nv, sh.hist, NB, shift, st.prefix, st.mask);
+        global_hist_pass(a, r, nv, vec, sh.hist, NB, shift, st.prefix, st.mask);
         if (shift == 52) {
             find_digit(sh.hist, NB, st.kk, st);
             if (st.total <= (uint32_t)a.k) {  // every candidate is selected
@@ -210,27 +250,16 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
 
     const uint64_t gprefix = st.prefix, gmask = st.mask;
     // ---- one pass: select everything above the prefix group; keep the group
-    for (int64_t i0 = 0; i0 < nv; i0 += (int64_t)TK_THREADS * TK_UNROLL) {
-        uint64_t key[TK_UNROLL];
-        bool ok[TK_UNROLL];
-#pragma unroll
-        for (int u = 0; u < TK_UNROLL; u++) {
-            const int64_t i = i0 + (int64_t)u * TK_THREADS + threadIdx.x;
-            ok[u] = (i < nv) && load_cand(a, r, i, key[u]);
+    for_each_cand(a, r, nv, vec, [&](uint64_t key) {
+        const uint64_t km = key & gmask;
+        if (all_selected || km > gprefix || (exact && km == gprefix)) {
+            const int s = atomicAdd(&st.nsel, 1);
+            if (s < TK_MAXK) sh.sel[s] = rank_key_pos(key);
+        } else if (km == gprefix) {
+            const int s = atomicAdd(&st.nbuf, 1);
+            if (s < TK_BUF) sh.buf[s] = key;
         }
-#pragma unroll
-        for (int u = 0; u < TK_UNROLL; u++) {
-            if (!ok[u]) continue;
-            const uint64_t km = key[u] & gmask;
-            if (all_selected || km > gprefix || (exact && km == gprefix)) {
-                const int s = atomicAdd(&st.nsel, 1);
-                if (s < TK_MAXK) sh.sel[s] = rank_key_pos(key[u]);
-            } else if (km == gprefix) {
-                const int s = atomicAdd(&st.nbuf, 1);
-                if (s < TK_BUF) sh.buf[s] = key[u];
-            }
-        }
-    }
+    });
     __syncthreads();
 
     // ---- remaining digits inside shared memory

@@ -1,0 +1,108 @@
+"""CPU tests of the C ABI: the library loads, exports every function that
+include/csa2.h declares, and rejects bad arguments on the host with the
+documented status codes (no kernel is launched on those paths, so no GPU is
+needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa2.h")
+LIB = os.path.join(ROOT, "sparse_attention_fp4_kv_b200", "libcsa2.so")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(csa2_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_attention_fp4_kv_b200 import build
+    build.build()
+    return ctypes.CDLL(LIB)
+
+
+def test_every_declared_function_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 12
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (csa2_\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        getattr(lib, n)
+
+
+def test_binding_covers_the_header():
+    from sparse_attention_fp4_kv_b200 import binding
+    assert set(binding.exported_symbols()) == set(_declared())
+    assert binding.lib.csa2_abi_version() == 1
+
+
+def test_status_strings():
+    from sparse_attention_fp4_kv_b200 import binding as B
+    for st in (0, -1, -2, -3, -4, -5, -6):
+        assert B.status_string(st) and B.status_string(st) != "unknown status"
+    assert B.status_string(-99) == "unknown status"
+
+
+def test_host_validation_codes():
+    from sparse_attention_fp4_kv_b200 import binding as B
+    L = B.lib
+    P = ctypes.c_void_p
+    good = P(4096)        # any 16-byte aligned non-null value; never dereferenced
+    odd = P(4096 + 8)
+    # NULL pointers
+    assert L.csa2_kv_append_fp4(None, 1, 1, 512, good, 10, good, good, None) == -1
+    assert L.csa2_index_full(None, good, good, good, None, 1, 1, 16, 128, 10, None, good, None,
+                             None) == -1
+    assert L.csa2_topk(None, None, None, 1, 10, 5, good, None, 0, None) == -1
+    # shapes
+    assert L.csa2_kv_append_fp4(good, 1, 1, 40, good, 10, good, good, None) == -2
+    assert L.csa2_index_full(good, good, good, good, None, 1, 1, 3, 5, 10, None, good, None,
+                             None) == -2
+    assert L.csa2_topk(good, None, None, 1, 10, 5000, good, None, 0, None) == -2
+    assert L.csa2_topk(good, None, None, 1, 0, 5, good, None, 0, None) == -2
+    assert L.csa2_sparse_attn_decode(good, good, good, 10, good, 512, good, good, 128, None, 128,
+                                     1, 1, 64, 48, ctypes.c_float(0.1), good, None, 0,
+                                     None) == -2
+    # alignment
+    assert L.csa2_kv_append_fp4(odd, 1, 1, 512, good, 10, good, good, None) == -3
+    assert L.csa2_index_full(odd, good, good, good, None, 1, 1, 16, 128, 10, None, good, None,
+                             None) == -3
+    # empty work is a no-op
+    assert L.csa2_kv_append_fp4(good, 0, 1, 512, good, 10, good, good, None) == 0
+    assert L.csa2_index_full(good, good, good, good, None, 0, 1, 16, 128, 10, None, good, None,
+                             None) == 0
+    assert L.csa2_topk(good, None, None, 0, 10, 5, good, None, 0, None) == 0
+
+
+def test_decode_stack_schedule_checks():
+    from sparse_attention_fp4_kv_b200 import binding as B
+    P = ctypes.c_void_p
+    good = P(4096)
+    layers = (B.csa2_layer * 2)()
+    layers[0] = B.csa2_layer(B.MODE_REUSE, None, good, good, good, None)
+    layers[1] = B.csa2_layer(B.MODE_FULL, good, good, good, good, good)
+    ws_need = B.lib.csa2_decode_stack_workspace_size(2, 64, 512, 16, 128, 1000)
+    assert ws_need > 0
+    args = [good, good, good, good, 1000, good, good, 128, 2, 64, 512, 16, 128, ctypes.c_float(0.04),
+            good, 0, None, good, ws_need, None]
+    # a Reuse layer with no producer before it
+    assert B.lib.csa2_decode_stack(layers, 2, None, *args) == -4
+    # a Reindex layer with no pool
+    layers[0] = B.csa2_layer(B.MODE_REINDEX, good, good, good, good, good)
+    assert B.lib.csa2_decode_stack(layers, 2, None, *args) == -4
+    # workspace too small
+    layers[0] = B.csa2_layer(B.MODE_FULL, good, good, good, good, good)
+    small = list(args)
+    small[-2] = ws_need - 1
+    assert B.lib.csa2_decode_stack(layers, 2, None, *small) == -5
+    # unknown mode
+    layers[1] = B.csa2_layer(7, good, good, good, good, good)
+    assert B.lib.csa2_decode_stack(layers, 2, None, *args) == -4

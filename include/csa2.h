@@ -250,6 +250,40 @@ int csa2_decode_stack(const csa2_layer *layers, int n_layers, const void *kv_new
                       int pool_ready, void *const *scan_events, void *ws, size_t ws_bytes,
                       void *stream);
 
+/* ------------------------------------------------------------------------
+ * csa2_decode_stack_noalloc: csa2_decode_stack for callers that cannot
+ * allocate device memory. The pages have no counterpart; this is a service of
+ * this library.
+ *
+ * Who needs it: code that runs while a stream is being captured into a CUDA
+ * graph (allocation is not allowed there), plugin hosts that pass a kernel only
+ * its input and output buffers and own every allocation, and latency-critical
+ * loops that cannot pay for the device-wide synchronisation cudaMalloc/cudaFree
+ * may cause. They cannot provide the workspace csa2_decode_stack asks for.
+ *
+ * Arguments and results: as csa2_decode_stack, minus scan_events, ws and
+ * ws_bytes. The scratch space is a file-scope device array of
+ * CSA2_NOALLOC_SCRATCH_BYTES inside the library. Every GPU that loads the
+ * library holds it until the process exits. The call allocates nothing.
+ * Limit: problems whose csa2_decode_stack_workspace_size exceeds
+ * CSA2_NOALLOC_SCRATCH_BYTES are rejected with CSA2_ERR_WORKSPACE before
+ * anything is launched. (B = 4 sequences of 1,048,576 tokens need 18.5 MiB.)
+ * Set-up: the first call on each device, with that device current, looks up
+ * the array's device address (cudaGetSymbolAddress) and keeps it. Make that
+ * first call before any stream capture. A failed look-up returns CSA2_ERR_CUDA.
+ * Sharing: every call uses the same array, which keeps the last call's
+ * contents. Calls that overlap on the GPU (other streams, other host threads)
+ * race and must be serialised by the caller. No part of the array has to
+ * start at zero.
+ * ------------------------------------------------------------------------ */
+#define CSA2_NOALLOC_SCRATCH_BYTES (24u << 20)
+int csa2_decode_stack_noalloc(const csa2_layer *layers, int n_layers, const void *kv_new_bf16,
+                              const int8_t *k_idx, const float *k_scale, uint8_t *kv_fp4,
+                              uint8_t *kv_sf, int64_t cap, const int64_t *ctx_len,
+                              const int64_t *swa_pos0, int swa_rows, int B, int Hq, int C, int H,
+                              int D, float softmax_scale, int32_t *pool, int pool_ready,
+                              void *stream);
+
 #ifdef __cplusplus
 }
 #endif

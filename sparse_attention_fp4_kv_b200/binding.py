@@ -61,6 +61,8 @@ _SIGS = {
     "csa2_decode_stack_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I64]),
     "csa2_decode_stack": (_I, [ctypes.POINTER(csa2_layer), _I, _P, _P, _P, _P, _P, _I64, _P, _P,
                                _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _P, _SZ, _P]),
+    "csa2_decode_stack_noalloc": (_I, [ctypes.POINTER(csa2_layer), _I, _P, _P, _P, _P, _P, _I64,
+                                       _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -235,6 +237,12 @@ class DecodeStack:
                      _ptr(ctx_len), _ptr(swa_pos0), swa[0].shape[1], B, Hq, C, H, D,
                      float(softmax_scale), _ptr(pool), int(bool(pool_ready)))
         self.ws_args = (_ptr(ws), ws.numel())
+
+    def call_noalloc(self, stream=None) -> int:
+        """The same decode step through csa2_decode_stack_noalloc, which uses
+        the library's own scratch array instead of self.ws (for callers that
+        cannot allocate). Returns the C status code."""
+        return lib.csa2_decode_stack_noalloc(*self.args, _stream(stream))
 
     def __call__(self, stream=None, scan_events=None) -> None:
         """One decode step. scan_events: optional (start, end) torch.cuda.Event

@@ -235,6 +235,69 @@ def run_reference(args, name):
     print(json.dumps(line), flush=True)
 
 
+def run_prefill(args, name, rank, world, local_rank):
+    """Chunked-prefill workload (one Full layer, n_new causal queries): tokens
+    (queries) per second, and the tensor-core indexer against the int8 roofline."""
+    from sparse_attention_fp4_kv_b200 import synth
+    from sparse_attention_fp4_kv_b200.workload import PrefillWorkload
+    import torch.distributed as dist
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[name]
+    pw = PrefillWorkload(w, dev)
+    stream = torch.cuda.current_stream()
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        pw.step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    clocks = ClockSampler(dev)
+    time.sleep(0.4)
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(K):
+        pw.step(scan_events=ev[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1) / K
+    scan_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    if world > 1:
+        t = torch.tensor([ms, scan_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, scan_ms = float(t[0]), float(t[1])
+    peaks = {}
+    pth = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pth):
+        peaks = json.load(open(pth))
+    bf16 = float(peaks.get("bf16_tflops", 1590.0))
+    # int8 dense is twice the bf16 dense rate (nominal 4.5 vs 2.25 PFLOP/s)
+    int8_peak = 2.0 * bf16
+    ops = pw.index_ops()
+    tops = ops / (scan_ms / 1e3) / 1e12
+    tokens = world * w.B * w.n_new
+    line = {"metric": "CSA2 chunked-prefill tokens/s (Full layer: append, causal indexer, "
+                      "pool, top-512, attention)", "value": tokens / (ms / 1e3),
+            "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8/fp32", "data": "synthetic",
+            "config": {"workload": name, "batch_per_gpu": w.B, "ctx": w.ctx, "new_tokens": w.n_new,
+                       "indexer": f"int8 {w.H_idx}x{w.D_idx}", "q_heads": w.Hq, "C": w.C},
+            "roofline": {"bound": "tensor", "kernel": "index_mma_kernel (tcgen05 kind::i8)",
+                         "achieved": tops, "peak": int8_peak, "unit": "TOPS",
+                         "frac": tops / int8_peak,
+                         "peak_kind": "measured bf16 burst x 2 (nominal int8/bf16 ratio)"
+                         if peaks else "fallback bf16 x 2",
+                         "traffic": None, "algorithmic_ops": ops, "launch_ms": scan_ms},
+            "clocks": clk, "gpu_launches": pw.launches_per_step() * K}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_csa2(args, name, rank, world, local_rank):
     from sparse_attention_fp4_kv_b200 import synth
     from sparse_attention_fp4_kv_b200.workload import DecodeWorkload
@@ -378,7 +441,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
-        run_csa2(args, args.workload, rank, world, local_rank)
+        if args.workload.startswith("prefill"):
+            run_prefill(args, args.workload, rank, world, local_rank)
+        else:
+            run_csa2(args, args.workload, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

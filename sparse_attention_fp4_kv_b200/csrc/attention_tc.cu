@@ -7,12 +7,15 @@
 // layer has its own main Q and SWA KV; the window is the last 128 tokens.
 // FP4 section of both pages: E2M1 elements with one E4M3 scale per 16 channels.
 //
-// One thread-block cluster of 8 CTAs per query; CTA r takes keys
-// [80 r, 80 r + 80) of the query's key list (selected rows, then window rows).
-//  1. cp.async stages the query's 64 x 512 bf16 Q and the CTA's window rows
-//     into 128-byte-swizzled K-major tiles, and the raw FP4 rows (codes and
-//     scales) into a staging area, all in flight at once; the FP4 rows are then
-//     dequantized from shared memory (e2m1 * e4m3 is exact in bf16).
+// One thread-block cluster of 8 CTAs (256 threads each) per query; CTA r takes
+// keys [80 r, 80 r + 80) of the query's key list (selected rows, then window
+// rows).
+//  1. One thread issues TMA copies of the query's 64 x 512 bf16 Q and of the
+//     CTA's window rows straight into 128-byte-swizzled K-major tiles; one warp
+//     issues a 1-D bulk copy per selected FP4 row (256 B of codes, 32 B of
+//     scales) into a staging area. All copies complete on one mbarrier. The
+//     FP4 rows are then dequantized from shared memory by all 8 warps
+//     (hardware E2M1 -> f16 conversion, times the E4M3 scale; exact in bf16).
 //  2. One thread issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32):
 //     S = Q K^T with M = 64 heads, N = 80 keys, K = 512, accumulated in TMEM.
 //  3. Each of the 4 warps reads its 16 heads' logits from TMEM (two threads per
@@ -28,8 +31,10 @@
 // (the M = 64 accumulator layout); S uses lanes 16-31 of columns 0..79.
 // No global scratch; one launch per layer.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "attention.cuh"
+#include "tma.cuh"
 
 namespace csa2 {
 namespace tc {
@@ -38,7 +43,8 @@ constexpr int HQ = 64;
 constexpr int CH = 512;
 constexpr int T = 80;        // keys per CTA
 constexpr int CL = 8;        // CTAs per query (cluster size)
-constexpr int THREADS = 128;
+constexpr int THREADS = 256;
+constexpr int SWA_BOX = 16;  // window rows per TMA box
 constexpr int KEYS_MAX = T * CL;
 
 constexpr int Q_CHUNK = HQ * 128;  // one 64-channel column of Q: 64 rows x 128 B
@@ -58,8 +64,9 @@ constexpr int SLOT_OFF = L_OFF + HQ * 4;  // int64 source offset per key slot [T
 constexpr int KIND_OFF = SLOT_OFF + T * 8;
 constexpr int FP4_STAGE_OFF = PHI_OFF;    // raw FP4 rows [T][288], before P is written
 static_assert(T * 288 <= 2 * P_BYTES, "FP4 staging must fit in the P buffers");
-constexpr int BAR_OFF = (KIND_OFF + T + 15) / 16 * 16;
+constexpr int BAR_OFF = (KIND_OFF + T + 15) / 16 * 16;  // [0] loads, [1] MMAs
 constexpr int TADDR_OFF = BAR_OFF + 16;
+constexpr int NTX_OFF = TADDR_OFF + 4;  // expected bytes of the load phase
 constexpr int SMEM_USED = TADDR_OFF + 16;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 // Partial-O staging ([64][512 + 4] fp32) reuses the Q and KV tiles.
@@ -77,12 +84,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
-}
 __device__ __forceinline__ void st_shared_v4(uint32_t a, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
                  "r"(v.w)
@@ -231,7 +232,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // ---------------------------------------------------------------- kernel
-__global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
+// E2M1 pair (one byte: low nibble first) -> two fp32 values, via the hardware
+// E2M1 -> f16 conversion (exact).
+__device__ __forceinline__ float2 e2m1x2_to_f32x2(uint32_t byte) {
+    uint32_t h2;
+    asm("{\n.reg .b8 b0, b1, b2, b3;\nmov.b32 {b0, b1, b2, b3}, %1;\n"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n}"
+        : "=r"(h2)
+        : "r"(byte));
+    const __half2 h = *reinterpret_cast<const __half2 *>(&h2);
+    return __half22float2(h);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tswa,
+                   AttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -246,17 +261,31 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
     float *l_s = reinterpret_cast<float *>(sm + L_OFF);
     int64_t *slot_src = reinterpret_cast<int64_t *>(sm + SLOT_OFF);
     uint8_t *slot_kind = sm + KIND_OFF;
-    const uint32_t bar = base + BAR_OFF;
+    const uint32_t bar_ld = base + BAR_OFF, bar = base + BAR_OFF + 8;
     uint32_t *taddr_s = reinterpret_cast<uint32_t *>(sm + TADDR_OFF);
+    uint32_t *ntx_s = reinterpret_cast<uint32_t *>(sm + NTX_OFF);
 
-    // ---- set-up: mbarrier, TMEM, key slots
+    // Window slots of this CTA: [js, je) are window keys; TMA copies them in
+    // boxes of SWA_BOX rows starting at js (a multiple of 16).
+    const int k0 = (int)rank * T;
+    int js = a.K - k0;
+    js = js < 0 ? 0 : (js > T ? T : js);
+    int je = a.K + w.n - k0;
+    je = je < js ? js : (je > T ? T : je);
+    const int nbox = (je - js + SWA_BOX - 1) / SWA_BOX;
+    const int cover_end = js + nbox * SWA_BOX;  // slots written by the window boxes
+
+    // ---- set-up: mbarriers, TMEM, key slots
     if (tid == 0) {
+        mbar_init(bar_ld, 1);
         mbar_init(bar, 1);
+        *ntx_s = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) tmem_alloc(base + TADDR_OFF, 512);
+    __syncthreads();
     if (tid < T) {
-        const int kidx = (int)rank * T + tid;
+        const int kidx = k0 + tid;
         uint8_t kind = 0;
         int64_t src = 0;
         if (kidx < a.K) {
@@ -264,10 +293,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
             if (pos >= 0 && pos < a.cap) {
                 kind = 1;
                 src = (int64_t)b * a.cap + pos;
+                atomicAdd(ntx_s, 288u);
             }
         } else if (kidx - a.K < w.n) {
             kind = 2;
-            src = (int64_t)b * a.swa_rows + w.row0 + (kidx - a.K);
         }
         slot_kind[tid] = kind;
         slot_src[tid] = src;
@@ -277,34 +306,41 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
     tc_fence_after();
     const uint32_t tmem = *taddr_s;
 
-    // ---- stage Q, the window rows and the raw FP4 rows with cp.async (all in
-    // flight together), then dequantize the FP4 rows from shared memory
-    const uint8_t *qg = reinterpret_cast<const uint8_t *>(a.q) + bq * (int64_t)HQ * CH * 2;
-    for (int i = tid; i < HQ * 64; i += THREADS) {
-        const int r = i >> 6, pg = i & 63;
-        cp_async16(base + Q_OFF + (pg >> 3) * Q_CHUNK + sw128(r, pg & 7), qg + r * 1024 + pg * 16);
+    // ---- load phase: Q and window rows by TMA, FP4 rows by bulk copies
+    if (tid == 0) {
+        const uint32_t bytes = (uint32_t)Q_BYTES + (uint32_t)nbox * 8u * SWA_BOX * 128u + *ntx_s;
+        mbar_expect_tx(bar_ld, bytes);
     }
-    const uint8_t *swa = reinterpret_cast<const uint8_t *>(a.swa);
+    // slots that no copy writes (invalid keys outside the window boxes) are zeroed
     for (int i = tid; i < T * 64; i += THREADS) {
         const int j = i >> 6, pg = i & 63;
-        const uint32_t dst = base + K_OFF + (pg >> 3) * K_CHUNK + sw128(j, pg & 7);
-        const uint8_t kind = slot_kind[j];
-        if (kind == 2)
-            cp_async16(dst, swa + slot_src[j] * 1024 + pg * 16);
-        else if (kind == 0)
-            st_shared_v4(dst, make_uint4(0, 0, 0, 0));
+        if (slot_kind[j] == 0 && (j < js || j >= cover_end))
+            st_shared_v4(base + K_OFF + (pg >> 3) * K_CHUNK + sw128(j, pg & 7),
+                         make_uint4(0, 0, 0, 0));
     }
-    // raw FP4 rows: 16 pieces of codes + 2 pieces of scales per row, staged in
-    // the (not yet used) P buffers as [T][288] bytes
-    for (int i = tid; i < T * 18; i += THREADS) {
-        const int j = i / 18, pc = i - j * 18;
-        if (slot_kind[j] != 1) continue;
-        const int64_t cell = slot_src[j];
-        const uint8_t *src = pc < 16 ? a.kv_fp4 + cell * 256 + pc * 16 : a.kv_sf + cell * 32 + (pc - 16) * 16;
-        cp_async16(base + FP4_STAGE_OFF + j * 288 + pc * 16, src);
+    __syncthreads();  // the expected byte count is registered before any copy lands
+    if (tid == 0) {
+        const int qrow = (int)(bq * HQ);
+#pragma unroll
+        for (int cc = 0; cc < 8; cc++) tma_load_2d(base + Q_OFF + cc * Q_CHUNK, &tq, cc * 64, qrow, bar_ld);
+        const int wrow0 = (int)((int64_t)b * a.swa_rows + w.row0 + (k0 + js - a.K));
+        for (int bx = 0; bx < nbox; bx++)
+#pragma unroll
+            for (int cc = 0; cc < 8; cc++)
+                tma_load_2d(base + K_OFF + cc * K_CHUNK + (js + bx * SWA_BOX) * 128, &tswa, cc * 64,
+                            wrow0 + bx * SWA_BOX, bar_ld);
     }
-    cp_async_wait_all();
-    __syncthreads();
+    if (warp == 1) {
+        for (int j = lane; j < T; j += 32) {
+            if (slot_kind[j] != 1) continue;
+            const int64_t cell = slot_src[j];
+            bulk_load(base + FP4_STAGE_OFF + j * 288, a.kv_fp4 + cell * 256, 256, bar_ld);
+            bulk_load(base + FP4_STAGE_OFF + j * 288 + 256, a.kv_sf + cell * 32, 32, bar_ld);
+        }
+    }
+    bool ok = mbar_wait(bar_ld, 0);
+
+    // ---- dequantize the FP4 rows into the KV tile
     const uint8_t *stage = sm + FP4_STAGE_OFF;
     for (int i = tid; i < T * 32; i += THREADS) {  // (slot, 16-channel group)
         const int j = i >> 5, g = i & 31;
@@ -315,7 +351,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
 #pragma unroll
         for (int u = 0; u < 8; u++) {
             const uint32_t byte = ((u < 4 ? codes.x : codes.y) >> (8 * (u & 3))) & 0xFF;
-            wds[u] = pack_bf16x2(e2m1_to_f32(byte & 0xF) * s, e2m1_to_f32(byte >> 4) * s);
+            const float2 f = e2m1x2_to_f32x2(byte);
+            wds[u] = pack_bf16x2(f.x * s, f.y * s);
         }
         const int pg = g * 2;  // two 16-byte pieces
         const uint32_t d0 = base + K_OFF + (pg >> 3) * K_CHUNK + sw128(j, pg & 7);
@@ -326,10 +363,9 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
     fence_proxy_async();
     __syncthreads();
 
-    bool ok = true;
     // ---- S = Q K^T  (M = 64, N = 80, K = 512) into TMEM lanes 16..31
     const uint32_t s_tmem = tmem + (16u << 16);
-    if (tid == 0) {
+    if (tid == 0 && ok) {
         tc_fence_after();
         constexpr uint32_t id_s = idesc_bf16(HQ, T, false);
 #pragma unroll 1
@@ -341,63 +377,65 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
         }
         mma_commit(bar);
     }
-    ok = mbar_wait(bar, 0);
+    if (ok) ok = mbar_wait(bar, 0);
     tc_fence_after();
 
-    // ---- softmax over this CTA's keys; two threads per head
-    const int h = warp * 16 + (lane & 15);
+    // ---- softmax over this CTA's keys (warps 0-3; two threads per head)
+    const int h = (warp & 3) * 16 + (lane & 15);
     const int half = lane >> 4;
-    const float sl2 = a.scale * LOG2E;
-    float p[40];
-    {
-        float v32[32], v8[8];
-        const uint32_t row_addr = s_tmem + ((uint32_t)(warp * 32) << 16);
-        tmem_ld_16x32x2_32(row_addr + 0, v32);
-        tmem_ld_16x32x2_8(row_addr + 64, v8);
-        tmem_ld_wait();
+    if (warp < 4) {
+        const float sl2 = a.scale * LOG2E;
+        float p[40];
+        {
+            float v32[32], v8[8];
+            const uint32_t row_addr = s_tmem + ((uint32_t)(warp * 32) << 16);
+            tmem_ld_16x32x2_32(row_addr + 0, v32);
+            tmem_ld_16x32x2_8(row_addr + 64, v8);
+            tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; i++) {
-            const int j = half * 32 + i;
-            p[i] = (ok && slot_kind[j] != 0) ? v32[i] * sl2 : -INFINITY;
+            for (int i = 0; i < 32; i++) {
+                const int j = half * 32 + i;
+                p[i] = (ok && slot_kind[j] != 0) ? v32[i] * sl2 : -INFINITY;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const int j = 64 + half * 8 + i;
+                p[32 + i] = (ok && slot_kind[j] != 0) ? v8[i] * sl2 : -INFINITY;
+            }
         }
+        float mx = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
-            const int j = 64 + half * 8 + i;
-            p[32 + i] = (ok && slot_kind[j] != 0) ? v8[i] * sl2 : -INFINITY;
+        for (int i = 0; i < 40; i++) mx = fmaxf(mx, p[i]);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        float sum = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 40; i++) {
+            p[i] = (p[i] == -INFINITY) ? 0.0f : ex2(p[i] - mx);
+            sum += p[i];
         }
-    }
-    float mx = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < 40; i++) mx = fmaxf(mx, p[i]);
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    float sum = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 40; i++) {
-        p[i] = (p[i] == -INFINITY) ? 0.0f : ex2(p[i] - mx);
-        sum += p[i];
-    }
-    sum += __shfl_xor_sync(0xffffffffu, sum, 16);
-    if (half == 0) {
-        m_s[h] = mx;
-        l_s[h] = sum;
-    }
-    // P = hi + lo (bf16), K-major 128B-swizzled tiles: tokens 0..63 in the
-    // first atom column, 64..79 in the second.
-#pragma unroll
-    for (int piece = 0; piece < 5; piece++) {
-        const int tok0 = piece < 4 ? half * 32 + piece * 8 : 64 + half * 8;
-        const float *pp = p + piece * 8;
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int u = 0; u < 4; u++) {
-            const __nv_bfloat162 hb = __floats2bfloat162_rn(pp[2 * u], pp[2 * u + 1]);
-            const float2 hf = __bfloat1622float2(hb);
-            hi[u] = *reinterpret_cast<const uint32_t *>(&hb);
-            lo[u] = pack_bf16x2(pp[2 * u] - hf.x, pp[2 * u + 1] - hf.y);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 16);
+        if (half == 0) {
+            m_s[h] = mx;
+            l_s[h] = sum;
         }
-        const uint32_t off = (tok0 >> 6) * P_ATOM + sw128(h, (tok0 & 63) >> 3);
-        st_shared_v4(base + PHI_OFF + off, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-        st_shared_v4(base + PLO_OFF + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+        // P = hi + lo (bf16), K-major 128B-swizzled tiles: tokens 0..63 in the
+        // first atom column, 64..79 in the second.
+#pragma unroll
+        for (int piece = 0; piece < 5; piece++) {
+            const int tok0 = piece < 4 ? half * 32 + piece * 8 : 64 + half * 8;
+            const float *pp = p + piece * 8;
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const __nv_bfloat162 hb = __floats2bfloat162_rn(pp[2 * u], pp[2 * u + 1]);
+                const float2 hf = __bfloat1622float2(hb);
+                hi[u] = *reinterpret_cast<const uint32_t *>(&hb);
+                lo[u] = pack_bf16x2(pp[2 * u] - hf.x, pp[2 * u + 1] - hf.y);
+            }
+            const uint32_t off = (tok0 >> 6) * P_ATOM + sw128(h, (tok0 & 63) >> 3);
+            st_shared_v4(base + PHI_OFF + off, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+            st_shared_v4(base + PLO_OFF + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+        }
     }
     fence_proxy_async();
     tc_fence_before();
@@ -423,12 +461,14 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
     if (ok) ok = mbar_wait(bar, 1);
     tc_fence_after();
 
-    // ---- unnormalized O -> shared staging [64][516] fp32 (reuses Q and KV tiles)
+    // ---- unnormalized O -> shared staging [64][516] fp32 (reuses Q and KV
+    // tiles); warps w and w + 4 share a TMEM lane quadrant and split the columns
     float *stg = reinterpret_cast<float *>(sm + Q_OFF);
     {
-        const uint32_t row_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        const uint32_t row_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const int cbeg = (warp >> 2) * 256;
 #pragma unroll 1
-        for (int c0 = 0; c0 < CH; c0 += 64) {
+        for (int c0 = cbeg; c0 < cbeg + 256; c0 += 64) {
             float v[32];
             tmem_ld_16x32x2_32(row_addr + c0, v);
             tmem_ld_wait();
@@ -449,10 +489,11 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
         tmem_dealloc(tmem, 512);
     }
 
-    // ---- combine: this CTA owns channels [64 rank, 64 rank + 64) of all heads
+    // ---- combine: this CTA owns channels [64 rank, 64 rank + 64) of all heads;
+    // thread = (head, 16 channels)
     {
-        const int hh = tid >> 1;  // head
-        const int c0 = (int)rank * 64 + (tid & 1) * 32;
+        const int hh = tid >> 2;
+        const int c0 = (int)rank * 64 + (tid & 3) * 16;
         float mr[CL], lr[CL], M = -INFINITY;
 #pragma unroll
         for (int r = 0; r < CL; r++) {
@@ -468,30 +509,26 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
             den += wgt[r] * lr[r];
         }
         const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+        float4 f[CL][4];
+#pragma unroll
+        for (int r = 0; r < CL; r++) {
+            const uint32_t src = map_rank(base + Q_OFF + (uint32_t)(hh * STG_STRIDE + c0) * 4, r);
+#pragma unroll
+            for (int u = 0; u < 4; u++) f[r][u] = ld_dsmem_v4(src + 16 * u);
+        }
         float *out = a.out + (bq * HQ + hh) * (int64_t)CH + c0;
-#pragma unroll 1
-        for (int part = 0; part < 2; part++) {  // 16 channels per part
-            float4 f[CL][4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int r = 0; r < CL; r++) {
-                const uint32_t src = map_rank(
-                    base + Q_OFF + (uint32_t)(hh * STG_STRIDE + c0 + part * 16) * 4, r);
-#pragma unroll
-                for (int u = 0; u < 4; u++) f[r][u] = ld_dsmem_v4(src + 16 * u);
+                acc.x += wgt[r] * f[r][u].x;
+                acc.y += wgt[r] * f[r][u].y;
+                acc.z += wgt[r] * f[r][u].z;
+                acc.w += wgt[r] * f[r][u].w;
             }
-#pragma unroll
-            for (int u = 0; u < 4; u++) {
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int r = 0; r < CL; r++) {
-                    acc.x += wgt[r] * f[r][u].x;
-                    acc.y += wgt[r] * f[r][u].y;
-                    acc.z += wgt[r] * f[r][u].z;
-                    acc.w += wgt[r] * f[r][u].w;
-                }
-                *reinterpret_cast<float4 *>(out + part * 16 + 4 * u) =
-                    make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-            }
+            *reinterpret_cast<float4 *>(out + 4 * u) =
+                make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
         }
     }
     cluster_sync();  // peers may still be reading this CTA's staging
@@ -501,9 +538,11 @@ __global__ void __launch_bounds__(THREADS, 1) attn_tc_kernel(AttnArgs a) {
 
 bool attn_tc_supported(const AttnArgs &a) {
     const int nwin = a.n_win < a.swa_rows ? a.n_win : a.swa_rows;
+    const bool has_win = nwin > 0 && a.swa != nullptr;
     return a.C == tc::CH && a.Hq == tc::HQ && a.K + (nwin > 0 ? nwin : 0) <= tc::KEYS_MAX &&
-           aligned(a.q, 16) && (a.swa == nullptr || aligned(a.swa, 16)) && aligned(a.kv_fp4, 16) &&
-           aligned(a.kv_sf, 16);
+           a.K % 16 == 0 && aligned(a.q, 16) && aligned(a.kv_fp4, 16) && aligned(a.kv_sf, 16) &&
+           (!has_win || (aligned(a.swa, 16) && (int64_t)a.B * a.swa_rows >= tc::SWA_BOX)) &&
+           (int64_t)a.B * a.Nq * tc::HQ < INT32_MAX && (int64_t)a.B * a.swa_rows < INT32_MAX;
 }
 
 int launch_attn_tc(const AttnArgs &a, cudaStream_t s) {
@@ -516,6 +555,16 @@ int launch_attn_tc(const AttnArgs &a, cudaStream_t s) {
     }
     const int64_t rows = (int64_t)a.B * a.Nq;
     if (rows > 65535) return CSA2_ERR_SHAPE;
+    CUtensorMap tq, tswa;
+    if (!make_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.q, tc::CH, (uint64_t)rows * tc::HQ,
+                      tc::CH * 2, 64, 64))
+        return CSA2_ERR_CUDA;
+    const bool has_win = a.swa != nullptr && a.swa_rows > 0 && a.n_win > 0;
+    // without a window the map is never used; describe the Q tensor instead
+    if (!make_tmap_2d(&tswa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, has_win ? a.swa : a.q, tc::CH,
+                      has_win ? (uint64_t)a.B * a.swa_rows : (uint64_t)rows * tc::HQ, tc::CH * 2, 64,
+                      tc::SWA_BOX))
+        return CSA2_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(tc::CL, (unsigned)rows, 1);
     cfg.blockDim = dim3(tc::THREADS, 1, 1);
@@ -528,7 +577,8 @@ int launch_attn_tc(const AttnArgs &a, cudaStream_t s) {
     attr_cl[0].val.clusterDim.z = 1;
     cfg.attrs = attr_cl;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel, a) != cudaSuccess) return CSA2_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel, tq, tswa, a) != cudaSuccess)
+        return CSA2_ERR_CUDA;
     return launch_status();
 }
 

@@ -120,4 +120,10 @@ __device__ __forceinline__ int64_t visible_len(const int64_t *ctx_len, const int
 int launch_kv_append(const uint16_t *kv, int B, int n_new, int C, const int64_t *pos_base,
                      int64_t pos_offset, int64_t cap, uint8_t *fp4, uint8_t *sf, cudaStream_t s);
 
+// Multi-query indexer scan on tensor cores (index_mma.cu).
+bool index_mma_supported(int Nq, int HD, int64_t cap, int B);
+int launch_index_mma(const int8_t *q, const int8_t *k, const float *kscale, const int64_t *ctx_len,
+                     const int64_t *q_pos, int B, int Nq, int HD, int64_t cap, float *tok,
+                     float *blk, int32_t *n_blk, cudaStream_t s);
+
 }  // namespace csa2

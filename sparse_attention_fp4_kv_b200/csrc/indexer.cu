@@ -86,7 +86,8 @@ __device__ __forceinline__ void load_qfrag(const int8_t *q, uint4 (&qf)[RowShape
 
 // Exact int32 dot products of the block's ntok (1..8) tokens with the query;
 // returns the sum for token reduce_token_of_lane(lane) (0 for t >= ntok).
-template <int HD>
+// GROUP = 16-byte loads each lane has in flight before it uses them.
+template <int HD, int GROUP = 8>
 __device__ __forceinline__ int block_dots(const int8_t *kblk, const uint4 (&qf)[RowShape<HD>::QV],
                                           int lane, int ntok) {
     using RS = RowShape<HD>;
@@ -94,7 +95,6 @@ __device__ __forceinline__ int block_dots(const int8_t *kblk, const uint4 (&qf)[
     int part[8];
 #pragma unroll
     for (int t = 0; t < 8; t++) part[t] = 0;
-    constexpr int GROUP = 8;  // loads in flight per lane before use
 #pragma unroll
     for (int i0 = 0; i0 < RS::VPL; i0 += GROUP) {
         uint4 k[GROUP];
@@ -250,43 +250,40 @@ __device__ __forceinline__ int64_t reindex_block(const ReindexArgs &a, int64_t b
     return t0;
 }
 
+// One warp per pooled block (no persistence: the kernel is short, so a grid
+// of one warp per item hides the ramp-up and tail better), 16 loads per lane
+// in flight.
 template <int HD>
 __global__ void __launch_bounds__(256) index_reindex_kernel(ReindexArgs a) {
     using RS = RowShape<HD>;
     const int lane = threadIdx.x & 31;
-    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t items = (int64_t)a.B * a.Nq * a.P;
+    if (it >= items) return;
     const int my_tok = reduce_token_of_lane(lane);
-    int64_t cur_bq = -1, V = 0;
+    const int64_t bq = it / a.P;
+    const int s = (int)(it - bq * a.P);
+    const int b = (int)(bq / a.Nq), i = (int)(bq % a.Nq);
+    int64_t V = visible_len(a.ctx_len, a.q_pos, b, i, a.Nq);
+    if (V > a.cap) V = a.cap;
+    int ntok;
+    const int64_t t0 = reindex_block(a, bq, s, V, ntok);
+    const int64_t slot = bq * 8 * (int64_t)a.P + 8 * (int64_t)s;
+    if (t0 < 0) {
+        if (lane < 8) {
+            a.ppos[slot + lane] = -1;
+            a.pscore[slot + lane] = 0.0f;
+        }
+        return;
+    }
     uint4 qf[RS::QV];
-    for (int64_t it = warp; it < items; it += nwarps) {
-        const int64_t bq = it / a.P;
-        const int s = (int)(it - bq * a.P);
-        const int b = (int)(bq / a.Nq), i = (int)(bq % a.Nq);
-        if (bq != cur_bq) {
-            cur_bq = bq;
-            V = visible_len(a.ctx_len, a.q_pos, b, i, a.Nq);
-            if (V > a.cap) V = a.cap;
-            load_qfrag<HD>(a.q + bq * HD, qf, lane);
-        }
-        int ntok;
-        const int64_t t0 = reindex_block(a, bq, s, V, ntok);
-        const int64_t slot = bq * 8 * (int64_t)a.P + 8 * (int64_t)s;
-        if (t0 < 0) {
-            if (lane < 8) {
-                a.ppos[slot + lane] = -1;
-                a.pscore[slot + lane] = 0.0f;
-            }
-            continue;
-        }
-        const int64_t row0 = (int64_t)b * a.cap + t0;
-        const int S = block_dots<HD>(a.k + row0 * HD, qf, lane, ntok);
-        const float sc = lane_score(S, a.kscale + row0, my_tok, ntok);
-        if ((lane & 3) == 0) {
-            a.ppos[slot + my_tok] = my_tok < ntok ? (int32_t)(t0 + my_tok) : -1;
-            a.pscore[slot + my_tok] = my_tok < ntok ? sc : 0.0f;
-        }
+    load_qfrag<HD>(a.q + bq * HD, qf, lane);
+    const int64_t row0 = (int64_t)b * a.cap + t0;
+    const int S = block_dots<HD, 16>(a.k + row0 * HD, qf, lane, ntok);
+    const float sc = lane_score(S, a.kscale + row0, my_tok, ntok);
+    if ((lane & 3) == 0) {
+        a.ppos[slot + my_tok] = my_tok < ntok ? (int32_t)(t0 + my_tok) : -1;
+        a.pscore[slot + my_tok] = my_tok < ntok ? sc : 0.0f;
     }
 }
 
@@ -351,8 +348,6 @@ __global__ void __launch_bounds__(256) pool_gather_kernel(const float *__restric
 
 template <typename K>
 static int persistent_grid(K kernel, int threads, int64_t items_warps) {
-    static int occ_cache[8] = {0};
-    (void)occ_cache;
     int occ = 0;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, 0);
     if (occ <= 0) occ = 1;
@@ -383,6 +378,9 @@ extern "C" int csa2_index_full(const int8_t *q_idx, const int8_t *k_idx, const f
     if (st) return st;
     if (!blk_score) return CSA2_ERR_NULL;
     if ((int64_t)B * Nq == 0) return CSA2_OK;
+    if (index_mma_supported(Nq, H * D, cap, B))
+        return launch_index_mma(q_idx, k_idx, k_scale, ctx_len, q_pos, B, Nq, H * D, cap,
+                                tok_score, blk_score, n_blk, (cudaStream_t)stream);
     ScanArgs a{q_idx, k_idx, k_scale, ctx_len, q_pos, B, Nq, H * D, cap, (cap + 7) / 8,
                tok_score, blk_score, n_blk};
     const int64_t items = (int64_t)B * Nq * a.nblk_cap;
@@ -427,8 +425,9 @@ extern "C" int csa2_index_reindex(const int8_t *q_idx, const int8_t *k_idx, cons
     switch (a.HD) {
 #define CSA2_RI_CASE(HDV)                                                               \
     case HDV: {                                                                         \
-        int g = persistent_grid(index_reindex_kernel<HDV>, T, items);                   \
-        index_reindex_kernel<HDV><<<g, T, 0, s>>>(a);                                   \
+        const int64_t g = (items + T / 32 - 1) / (T / 32);                              \
+        if (g > INT32_MAX) return CSA2_ERR_SHAPE;                                       \
+        index_reindex_kernel<HDV><<<(unsigned)g, T, 0, s>>>(a);                         \
         break;                                                                          \
     }
         CSA2_RI_CASE(128)

@@ -127,3 +127,94 @@ class DecodeWorkload:
         append = B * (C * 2 + C // 2 + C // 16)
         return dict(scan=scan, reindex=reindex, attn=attn, append=append,
                     total=scan + reindex + attn + append)
+
+
+class PrefillWorkload:
+    """Chunked prefill of one Full layer: n_new tokens appended to a context
+    of ctx - n_new, each new token a query that sees positions <= its own.
+
+    One step = FP4 append of the n_new rows, causal indexer scoring of every
+    query against every visible key (tensor-core kernel), per-query pool of
+    2048 blocks and top-512, then attention of each query over its 512 rows
+    plus its own 128-token window. Buffers per sequence: token scores
+    [n_new][ctx] fp32 (1.1 GB at 4096 x 69632), block scores, pools, pooled
+    scores/positions, indices and outputs [n_new][64][512] fp32."""
+
+    def __init__(self, w: synth.Workload, device="cuda", keep_kv_bf16: bool = False):
+        self.w = w
+        B, cap, C, Hq, H, D, n = w.B, w.ctx, w.C, w.Hq, w.H_idx, w.D_idx, w.n_new
+        dev = torch.device(device)
+        self.device = dev
+        self.ctx0 = cap - n
+        self.k_idx = torch.empty((B, cap, H, D), dtype=torch.int8, device=dev)
+        self.k_scale = torch.empty((B, cap), dtype=torch.float32, device=dev)
+        for b in range(B):
+            self.k_idx[b] = synth.indexer_keys(w, b, cap, dev)
+            self.k_scale[b] = synth.indexer_key_scale(w, b, cap, dev)
+        self.kv_fp4 = torch.zeros((B, cap, C // 2), dtype=torch.uint8, device=dev)
+        self.kv_sf = torch.zeros((B, cap, C // 16), dtype=torch.uint8, device=dev)
+        self.kv_bf16 = (torch.empty((B, cap, C), dtype=torch.bfloat16, device=dev)
+                        if keep_kv_bf16 else None)
+        zero = torch.zeros(1, dtype=torch.int64, device=dev)
+        chunk = 65536
+        for b in range(B):
+            for t0 in range(0, self.ctx0, chunk):
+                t1 = min(self.ctx0, t0 + chunk)
+                rows = synth.main_kv_bf16(w, b, t0, t1, dev)
+                if self.kv_bf16 is not None:
+                    self.kv_bf16[b, t0:t1] = rows
+                csa2.csa2_kv_append_fp4(rows.unsqueeze(0).contiguous(), zero + t0,
+                                        self.kv_fp4[b:b + 1], self.kv_sf[b:b + 1])
+        self.kv_new = torch.stack([synth.main_kv_bf16(w, b, self.ctx0, cap, dev) for b in range(B)])
+        if self.kv_bf16 is not None:
+            self.kv_bf16[:, self.ctx0:] = self.kv_new
+        self.start = torch.full((B,), self.ctx0, dtype=torch.int64, device=dev)
+        self.ctx_len = torch.full((B,), cap, dtype=torch.int64, device=dev)
+        self.q_pos = (self.ctx0 + torch.arange(n, device=dev, dtype=torch.int64)).repeat(B, 1).contiguous()
+        self.q_idx = synth.indexer_q(w, 0, n, dev)
+        self.q = synth.main_q(w, 0, n, dev)
+        lo = max(0, self.ctx0 - (w.n_win - 1))
+        self.swa_rows = cap - lo
+        self.swa = synth.swa_kv(w, 0, self.swa_rows, dev)
+        self.swa_pos0 = torch.full((B,), lo, dtype=torch.int64, device=dev)
+        nb = (cap + 7) // 8
+        self.tok = torch.empty((B, n, cap), dtype=torch.float32, device=dev)
+        self.blk = torch.empty((B, n, nb), dtype=torch.float32, device=dev)
+        self.nblk = torch.empty((B, n), dtype=torch.int32, device=dev)
+        self.pool = torch.empty((B, n, csa2.POOL_BLOCKS), dtype=torch.int32, device=dev)
+        P8 = csa2.POOL_BLOCKS * csa2.BLOCK_TOKENS
+        self.pscore = torch.empty((B, n, P8), dtype=torch.float32, device=dev)
+        self.ppos = torch.empty((B, n, P8), dtype=torch.int32, device=dev)
+        self.top = torch.empty((B, n, csa2.TOPK), dtype=torch.int32, device=dev)
+        self.out = torch.empty((B, n, Hq, C), dtype=torch.float32, device=dev)
+        self.scale = 1.0 / math.sqrt(C)
+
+    def step(self, stream=None, scan_events=None):
+        w = self.w
+        B, n = w.B, w.n_new
+        csa2.csa2_kv_append_fp4(self.kv_new, self.start, self.kv_fp4, self.kv_sf, stream=stream)
+        if scan_events is not None:
+            scan_events[0].record(stream or torch.cuda.current_stream())
+        csa2.csa2_index_full(self.q_idx, self.k_idx, self.k_scale, self.ctx_len, self.blk, self.tok,
+                             self.nblk, q_pos=self.q_pos, stream=stream)
+        if scan_events is not None:
+            scan_events[1].record(stream or torch.cuda.current_stream())
+        csa2.csa2_topk(self.blk.view(B * n, -1), csa2.POOL_BLOCKS, self.pool.view(B * n, -1),
+                       n_valid=self.nblk.view(-1), stream=stream)
+        csa2.csa2_pool_gather(self.tok, self.pool, self.ctx_len, self.pscore, self.ppos,
+                              q_pos=self.q_pos, stream=stream)
+        csa2.csa2_topk(self.pscore.view(B * n, -1), csa2.TOPK, self.top.view(B * n, -1),
+                       cand_pos=self.ppos.view(B * n, -1), stream=stream)
+        csa2.csa2_sparse_attn_decode(self.q, self.kv_fp4, self.kv_sf, self.top, self.swa,
+                                     self.swa_pos0, self.out, self.scale, q_pos=self.q_pos,
+                                     stream=stream)
+
+    def launches_per_step(self) -> int:
+        return 6
+
+    def index_ops(self) -> int:
+        """int8 multiply-adds x 2 of the causal scoring (every query x every
+        visible key x H*D)."""
+        w = self.w
+        vis = sum(min(self.ctx0 + i + 1, w.ctx) for i in range(w.n_new))
+        return 2 * w.B * vis * w.H_idx * w.D_idx

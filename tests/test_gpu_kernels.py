@@ -330,3 +330,52 @@ def test_sparse_attention_prefill_positions(B):
     ctx = 1200
     q_pos = torch.tensor([[1199, 1100, 600, 130]], dtype=torch.int64, device=DEV)
     _attention_case(B, 1, ctx, 512, 64, 512, 128, seed=3, q_pos=q_pos, Nq=4)
+
+
+# ----------------------------------------------------------------------------- a9 prefill scan
+@pytest.mark.parametrize("Nq,ctx0,H,D", [(300, 5000, 16, 128), (129, 2048, 8, 128), (40, 777, 4, 64)])
+def test_index_full_multi_query_tensor_core_path(B, Nq, ctx0, H, D):
+    """Nq >= 16 runs the tcgen05 kind::i8 kernel: causal scores and block maxima
+    must equal the oracle bit for bit, and equal the per-query dp4a scan."""
+    Bn = 2
+    cap = ctx0 + Nq
+    g = torch.Generator(device=DEV).manual_seed(Nq + ctx0)
+    k = torch.randint(-127, 128, (Bn, cap, H, D), generator=g, device=DEV, dtype=torch.int8)
+    q = torch.randint(-127, 128, (Bn, Nq, H, D), generator=g, device=DEV, dtype=torch.int8)
+    s = 0.5 + torch.rand((Bn, cap), generator=g, device=DEV)
+    ctx = torch.tensor([cap, cap - 3], dtype=torch.int64, device=DEV)
+    qpos = (ctx0 + torch.arange(Nq, device=DEV)).repeat(Bn, 1).contiguous()
+    nb = (cap + 7) // 8
+    blk = torch.full((Bn, Nq, nb), -7.0, device=DEV)
+    tok = torch.full((Bn, Nq, cap), -7.0, device=DEV)
+    nblk = torch.zeros((Bn, Nq), dtype=torch.int32, device=DEV)
+    B.csa2_index_full(q, k, s, ctx, blk, tok, nblk, q_pos=qpos)
+    # the same queries one at a time (Nq = 1 runs the dp4a scan kernel)
+    blk1 = torch.full_like(blk, -7.0)
+    tok1 = torch.full_like(tok, -7.0)
+    nblk1 = torch.zeros_like(nblk)
+    for i in range(Nq):
+        b1 = torch.empty((Bn, 1, nb), device=DEV)
+        t1 = torch.empty((Bn, 1, cap), device=DEV)
+        n1 = torch.empty((Bn, 1), dtype=torch.int32, device=DEV)
+        B.csa2_index_full(q[:, i:i + 1].contiguous(), k, s, ctx, b1, t1, n1,
+                          q_pos=qpos[:, i:i + 1].contiguous())
+        blk1[:, i] = b1[:, 0]
+        tok1[:, i] = t1[:, 0]
+        nblk1[:, i] = n1[:, 0]
+    torch.cuda.synchronize()
+    for b in range(Bn):
+        for i in range(Nq):
+            V = min(int(qpos[b, i]) + 1, int(ctx[b]))
+            nv = (V + 7) // 8
+            assert int(nblk[b, i]) == nv == int(nblk1[b, i])
+            assert torch.equal(tok[b, i, :V], tok1[b, i, :V]), f"tok b={b} i={i}"
+            assert torch.equal(blk[b, i, :nv], blk1[b, i, :nv]), f"blk b={b} i={i}"
+            assert bool((tok[b, i, V:] == -7.0).all()) and bool((blk[b, i, nv:] == -7.0).all())
+    kn, sn, qn = k.cpu().numpy(), s.cpu().numpy(), q.cpu().numpy()
+    for b in range(Bn):
+        for i in sorted({0, 1, Nq // 2, Nq - 1}):
+            V = min(int(qpos[b, i]) + 1, int(ctx[b]))
+            ref = oracle.index_scores(qn[b, i], kn[b, :V], sn[b, :V])
+            assert np.array_equal(f32_bits(tok[b, i, :V]), f32_bits(ref))
+            assert np.array_equal(f32_bits(blk[b, i, :(V + 7) // 8]), f32_bits(oracle.block_scores(ref, V)))

@@ -243,7 +243,8 @@ def run_prefill(args, name, rank, world, local_rank):
     import torch.distributed as dist
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = synth.WORKLOADS[name]
+    from sparse_attention_fp4_kv_b200 import replicas
+    w = replicas.rank_workload(synth.WORKLOADS[name], rank, world)
     pw = PrefillWorkload(w, dev)
     stream = torch.cuda.current_stream()
     K, W = args.steps, args.warmup
@@ -266,10 +267,8 @@ def run_prefill(args, name, rank, world, local_rank):
     clk = clocks.stop()
     ms = t0.elapsed_time(t1) / K
     scan_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    if world > 1:
-        t = torch.tensor([ms, scan_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, scan_ms = float(t[0]), float(t[1])
+    from sparse_attention_fp4_kv_b200 import replicas
+    ms, scan_ms = replicas.slowest([ms, scan_ms], dev)
     peaks = {}
     pth = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(pth):
@@ -304,9 +303,8 @@ def run_csa2(args, name, rank, world, local_rank):
     import torch.distributed as dist
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = synth.WORKLOADS[name]
-    if world > 1:
-        w = synth.scaled(w, seed=w.seed + 1000 * rank)
+    from sparse_attention_fp4_kv_b200 import replicas
+    w = replicas.rank_workload(synth.WORKLOADS[name], rank, world)
     wl = DecodeWorkload(w, dev)
     stream = torch.cuda.current_stream()
     K, W = args.steps, args.warmup
@@ -338,12 +336,9 @@ def run_csa2(args, name, rank, world, local_rank):
     clk = clocks.stop()
     ms_total = t_start.elapsed_time(t_end)
     scan_ms = statistics.mean(a.elapsed_time(b) for a, b in scan_ev)
-    if world > 1:
-        t = torch.tensor([ms_total, scan_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total, scan_ms = float(t[0]), float(t[1])
+    ms_total, scan_ms = replicas.slowest([ms_total, scan_ms], dev)
     ms_step = ms_total / K
-    value = world * w.n_layers / (ms_step / 1e3)
+    value = replicas.aggregate_rate(w.n_layers, world, ms_step)
 
     # ---- end to end through the public API with host buffers
     e2e = _e2e(wl, args, stream, world, local_rank)
@@ -410,11 +405,9 @@ def _e2e(wl, args, stream, world, local_rank):
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / E
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t[0])
-    return {"value": world * wl.w.n_layers / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+    from sparse_attention_fp4_kv_b200 import replicas
+    ms = replicas.slowest([ms], dev)[0]
+    return {"value": replicas.aggregate_rate(wl.w.n_layers, world, ms), "unit": UNIT, "ms_per_step": ms,
             "steps": E, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 

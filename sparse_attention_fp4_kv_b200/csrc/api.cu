@@ -27,6 +27,8 @@ extern "C" int csa2_abi_version(void) { return CSA2_ABI_VERSION; }
 
 namespace {
 
+uint32_t *topk_hist_ptr_of(void *ws) { return static_cast<uint32_t *>(ws); }
+
 constexpr size_t kAlign = 256;
 inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -36,6 +38,9 @@ struct StackWs {
     int32_t *n_blk;
     float *pscore;
     int32_t *ppos;
+    void *sel_blk;     // histogram-fed top-k workspace of the pool selection
+    void *sel_tok;     // ... and of the token top-512
+    size_t hist_bytes; // leading bytes of each that must be zero before a step
     void *attn;
     size_t attn_bytes;
     size_t total;
@@ -57,6 +62,11 @@ StackWs stack_layout(void *base, int B, int Hq, int C, int64_t cap) {
     off += up(sizeof(float) * (size_t)B * P8);
     w.ppos = reinterpret_cast<int32_t *>(p + off);
     off += up(sizeof(int32_t) * (size_t)B * P8);
+    w.sel_blk = p + off;
+    off += up(topk_hist_ws_bytes(B, kPoolBlocks));
+    w.sel_tok = p + off;
+    off += up(topk_hist_ws_bytes(B, kTopK));
+    w.hist_bytes = up((size_t)B * kHistBins * 4) + up((size_t)B * 2 * 4);
     w.attn = p + off;
     w.attn_bytes = up(attn_workspace_bytes(B, 1, Hq, C, kTopK, CSA2_N_WIN));
     off += w.attn_bytes;
@@ -111,36 +121,47 @@ extern "C" int csa2_decode_stack(const csa2_layer *layers, int n_layers,
     const int32_t *cur = nullptr;
     bool scan_timed = false;
     int st;
+    cudaStream_t s = (cudaStream_t)stream;
     if (kv_new_bf16) {
         st = launch_kv_append((const uint16_t *)kv_new_bf16, B, 1, C, ctx_len, -1, cap, kv_fp4,
-                              kv_sf, (cudaStream_t)stream);
+                              kv_sf, s);
         if (st) return st;
     }
+    // the selection histograms and counters start the step at zero (every
+    // finishing top-k kernel leaves its rows clear for the next producer)
+    if (cudaMemsetAsync(w.sel_blk, 0, w.hist_bytes, s) != cudaSuccess ||
+        cudaMemsetAsync(w.sel_tok, 0, w.hist_bytes, s) != cudaSuccess)
+        return CSA2_ERR_CUDA;
+    uint32_t *hist_blk = topk_hist_ptr_of(w.sel_blk);
+    uint32_t *hist_tok = topk_hist_ptr_of(w.sel_tok);
     for (int l = 0; l < n_layers; l++) {
         const csa2_layer &L = layers[l];
         if (L.mode == CSA2_MODE_FULL) {
             const bool timed = scan_events && !scan_timed;
             if (timed) cudaEventRecord((cudaEvent_t)scan_events[0], (cudaStream_t)stream);
-            st = csa2_index_full(L.q_idx, k_idx, k_scale, ctx_len, nullptr, B, 1, H, D, cap, w.tok,
-                                 w.blk, w.n_blk, stream);
+            st = launch_index_full_hist(L.q_idx, k_idx, k_scale, ctx_len, B, H, D, cap, w.tok, w.blk,
+                                        w.n_blk, hist_blk, s);
             if (st) return st;
             if (timed) {
                 cudaEventRecord((cudaEvent_t)scan_events[1], (cudaStream_t)stream);
                 scan_timed = true;
             }
-            st = csa2_topk(w.blk, nullptr, w.n_blk, B, nblk, kPoolBlocks, pool, nullptr, 0, stream);
+            st = launch_topk_from_hist(w.blk, nullptr, w.n_blk, B, nblk, kPoolBlocks, pool,
+                                       w.sel_blk, s);
             if (st) return st;
-            st = csa2_pool_gather(w.tok, pool, ctx_len, nullptr, B, 1, kPoolBlocks, cap, w.pscore,
-                                  w.ppos, stream);
+            st = launch_pool_gather_hist(w.tok, pool, ctx_len, B, kPoolBlocks, cap, w.pscore, w.ppos,
+                                         hist_tok, s);
             if (st) return st;
-            st = csa2_topk(w.pscore, w.ppos, nullptr, B, P8, kTopK, L.topk, nullptr, 0, stream);
+            st = launch_topk_from_hist(w.pscore, w.ppos, nullptr, B, P8, kTopK, L.topk, w.sel_tok,
+                                       s);
             if (st) return st;
             cur = L.topk;
         } else if (L.mode == CSA2_MODE_REINDEX) {
-            st = csa2_index_reindex(L.q_idx, k_idx, k_scale, pool, ctx_len, nullptr, B, 1, H, D,
-                                    cap, kPoolBlocks, w.pscore, w.ppos, stream);
+            st = launch_reindex_hist(L.q_idx, k_idx, k_scale, pool, ctx_len, B, H, D, cap,
+                                     kPoolBlocks, w.pscore, w.ppos, hist_tok, s);
             if (st) return st;
-            st = csa2_topk(w.pscore, w.ppos, nullptr, B, P8, kTopK, L.topk, nullptr, 0, stream);
+            st = launch_topk_from_hist(w.pscore, w.ppos, nullptr, B, P8, kTopK, L.topk, w.sel_tok,
+                                       s);
             if (st) return st;
             cur = L.topk;
         }

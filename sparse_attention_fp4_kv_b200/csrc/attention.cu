@@ -161,13 +161,12 @@ extern "C" int csa2_sparse_attn_decode(const void *q_bf16, const uint8_t *kv_fp4
 
 namespace csa2 {
 
+// The tensor-core kernel exchanges per-CTA partial results through the
+// workspace; the general kernel needs none. The size covers the tensor-core
+// path whenever its shape constraints could hold.
 size_t attn_workspace_bytes(int B, int Nq, int Hq, int C, int K, int n_win) {
-    (void)B;
-    (void)Nq;
-    (void)Hq;
-    (void)C;
-    (void)K;
-    (void)n_win;
+    if (C == 512 && Hq == 64 && K % 16 == 0 && K + (n_win > 0 ? n_win : 0) <= 640)
+        return attn_tc_workspace_bytes(B, Nq);
     return 0;
 }
 

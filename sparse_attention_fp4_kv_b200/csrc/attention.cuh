@@ -51,6 +51,7 @@ size_t attn_workspace_bytes(int B, int Nq, int Hq, int C, int K, int n_win);
 int launch_attn(const AttnArgs &a, cudaStream_t s);
 int launch_attn_general(const AttnArgs &a, cudaStream_t s);
 bool attn_tc_supported(const AttnArgs &a);
+size_t attn_tc_workspace_bytes(int B, int Nq);
 int launch_attn_tc(const AttnArgs &a, cudaStream_t s);
 
 }  // namespace csa2

@@ -11,10 +11,10 @@
 // keys [80 r, 80 r + 80) of the query's key list (selected rows, then window
 // rows).
 //  1. One thread issues TMA copies of the query's 64 x 512 bf16 Q and of the
-//     CTA's window rows straight into 128-byte-swizzled K-major tiles; one warp
-//     issues a 1-D bulk copy per selected FP4 row (256 B of codes, 32 B of
-//     scales) into a staging area. All copies complete on one mbarrier. The
-//     FP4 rows are then dequantized from shared memory by all 8 warps
+//     CTA's window rows straight into 128-byte-swizzled K-major tiles (they
+//     complete on an mbarrier); all threads gather the selected FP4 rows (256 B
+//     of codes, 32 B of scales each) with 16-byte cp.async into a staging area.
+//     The FP4 rows are then dequantized from shared memory by all 8 warps
 //     (hardware E2M1 -> f16 conversion, times the E4M3 scale; exact in bf16).
 //  2. One thread issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32):
 //     S = Q K^T with M = 64 heads, N = 80 keys, K = 512, accumulated in TMEM.
@@ -24,12 +24,16 @@
 //     fp32-level accuracy with bf16 operands).
 //  4. O = P_hi V + P_lo V: M = 64, N = 256 (two halves of 512 channels), K = 80,
 //     the same shared-memory KV tile read as an MN-major operand.
-//  5. The unnormalized O, the row maxima and the row sums go to shared memory;
-//     after a cluster barrier each CTA combines 64 channels of all 64 heads over
-//     the 8 CTAs through distributed shared memory and writes the output.
+//  5. Each CTA writes its unnormalized O (from TMEM), row maxima and sums into
+//     its cluster's exchange slot in the workspace (L2 resident); after a
+//     cluster barrier each CTA combines its 64 channels of all 64 heads over the
+//     8 partial results and writes the output. (Moving the 1 MB of partials of a
+//     cluster through L2 measured about 4x faster than through distributed
+//     shared memory.) Clusters are persistent over query rows (at most 18, one
+//     wave on 148 SMs), so the workspace is 18 slots at most.
 // TMEM: O uses columns 0..511 of lanes 0-15 of each 32-lane subpartition
 // (the M = 64 accumulator layout); S uses lanes 16-31 of columns 0..79.
-// No global scratch; one launch per layer.
+// One launch per layer; scratch: one exchange slot (1.05 MB) per cluster.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -66,12 +70,17 @@ constexpr int FP4_STAGE_OFF = PHI_OFF;    // raw FP4 rows [T][288], before P is 
 static_assert(T * 288 <= 2 * P_BYTES, "FP4 staging must fit in the P buffers");
 constexpr int BAR_OFF = (KIND_OFF + T + 15) / 16 * 16;  // [0] loads, [1] MMAs
 constexpr int TADDR_OFF = BAR_OFF + 16;
-constexpr int NTX_OFF = TADDR_OFF + 4;  // expected bytes of the load phase
+
 constexpr int SMEM_USED = TADDR_OFF + 16;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
-// Partial-O staging ([64][512 + 4] fp32) reuses the Q and KV tiles.
-constexpr int STG_STRIDE = CH + 4;
-static_assert(HQ * STG_STRIDE * 4 <= Q_BYTES + K_BYTES, "staging must fit in Q + KV tiles");
+// Exchange slot of one cluster in the workspace: partial O [8 sources][8
+// slices][64 heads][64 channels] fp32, row maxima [8][64] and row sums [8][64].
+constexpr int SLICE_BYTES = HQ * 64 * 4;  // 16 KB
+constexpr int STG_OFF = Q_OFF;            // staging of the partial O (128 KB)
+static_assert(CL * SLICE_BYTES <= Q_BYTES + K_BYTES, "staging must fit in the Q + KV tiles");
+constexpr int64_t XSLOT_FLOATS = (int64_t)CL * HQ * CH + 2 * CL * HQ;
+// Clusters resident at once (148 SMs / 8); each walks query rows with this stride.
+constexpr int MAX_CLUSTERS = 18;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
 constexpr float LOG2E = 1.4426950408889634f;
@@ -206,6 +215,20 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
     return r;
 }
+__device__ __forceinline__ void st_dsmem_v4(uint32_t addr, float4 v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x),
+                 "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ void st_dsmem_f32(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
 __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
     float v;
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
@@ -253,9 +276,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t *sm = smem_raw + (base - raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t rank = cluster_rank();
-    const int64_t bq = blockIdx.y;
-    const int b = (int)(bq / a.Nq);
-    const AttnWindow w = attn_window(a, b, bq);
 
     float *m_s = reinterpret_cast<float *>(sm + M_OFF);
     float *l_s = reinterpret_cast<float *>(sm + L_OFF);
@@ -263,275 +283,319 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t *slot_kind = sm + KIND_OFF;
     const uint32_t bar_ld = base + BAR_OFF, bar = base + BAR_OFF + 8;
     uint32_t *taddr_s = reinterpret_cast<uint32_t *>(sm + TADDR_OFF);
-    uint32_t *ntx_s = reinterpret_cast<uint32_t *>(sm + NTX_OFF);
+    // this cluster's exchange slot in the workspace
+    float *xo = reinterpret_cast<float *>(a.ws) + (int64_t)blockIdx.y * XSLOT_FLOATS;
+    float *xm = xo + CL * HQ * CH;
+    float *xl = xm + CL * HQ;
 
-    // Window slots of this CTA: [js, je) are window keys; TMA copies them in
-    // boxes of SWA_BOX rows starting at js (a multiple of 16).
-    const int k0 = (int)rank * T;
-    int js = a.K - k0;
-    js = js < 0 ? 0 : (js > T ? T : js);
-    int je = a.K + w.n - k0;
-    je = je < js ? js : (je > T ? T : je);
-    const int nbox = (je - js + SWA_BOX - 1) / SWA_BOX;
-    const int cover_end = js + nbox * SWA_BOX;  // slots written by the window boxes
-
-    // ---- set-up: mbarriers, TMEM, key slots
+    // ---- once per CTA: mbarriers and TMEM
     if (tid == 0) {
         mbar_init(bar_ld, 1);
         mbar_init(bar, 1);
-        *ntx_s = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) tmem_alloc(base + TADDR_OFF, 512);
-    __syncthreads();
-    if (tid < T) {
-        const int kidx = k0 + tid;
-        uint8_t kind = 0;
-        int64_t src = 0;
-        if (kidx < a.K) {
-            const int32_t pos = a.topk[bq * a.K + kidx];
-            if (pos >= 0 && pos < a.cap) {
-                kind = 1;
-                src = (int64_t)b * a.cap + pos;
-                atomicAdd(ntx_s, 288u);
-            }
-        } else if (kidx - a.K < w.n) {
-            kind = 2;
-        }
-        slot_kind[tid] = kind;
-        slot_src[tid] = src;
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *taddr_s;
+    const int64_t rows = (int64_t)a.B * a.Nq;
+    uint32_t ld_phase = 0;
+    bool ok = true;
 
-    // ---- load phase: Q and window rows by TMA, FP4 rows by bulk copies
-    if (tid == 0) {
-        const uint32_t bytes = (uint32_t)Q_BYTES + (uint32_t)nbox * 8u * SWA_BOX * 128u + *ntx_s;
-        mbar_expect_tx(bar_ld, bytes);
-    }
-    // slots that no copy writes (invalid keys outside the window boxes) are zeroed
-    for (int i = tid; i < T * 64; i += THREADS) {
-        const int j = i >> 6, pg = i & 63;
-        if (slot_kind[j] == 0 && (j < js || j >= cover_end))
-            st_shared_v4(base + K_OFF + (pg >> 3) * K_CHUNK + sw128(j, pg & 7),
-                         make_uint4(0, 0, 0, 0));
-    }
-    __syncthreads();  // the expected byte count is registered before any copy lands
-    if (tid == 0) {
-        const int qrow = (int)(bq * HQ);
-#pragma unroll
-        for (int cc = 0; cc < 8; cc++) tma_load_2d(base + Q_OFF + cc * Q_CHUNK, &tq, cc * 64, qrow, bar_ld);
-        const int wrow0 = (int)((int64_t)b * a.swa_rows + w.row0 + (k0 + js - a.K));
-        for (int bx = 0; bx < nbox; bx++)
+    // The cluster walks query rows blockIdx.y, blockIdx.y + gridDim.y, ...
+    for (int64_t bq = blockIdx.y; bq < rows; bq += gridDim.y) {
+        const int b = (int)(bq / a.Nq);
+        const AttnWindow w = attn_window(a, b, bq);
+        // Window slots of this CTA: [js, je) are window keys; TMA copies them in
+        // boxes of SWA_BOX rows starting at js (a multiple of 16).
+        const int k0 = (int)rank * T;
+        int js = a.K - k0;
+        js = js < 0 ? 0 : (js > T ? T : js);
+        int je = a.K + w.n - k0;
+        je = je < js ? js : (je > T ? T : je);
+        const int nbox = (je - js + SWA_BOX - 1) / SWA_BOX;
+        const int cover_end = js + nbox * SWA_BOX;  // slots written by the window boxes
+
+        if (tid < T) {
+            const int kidx = k0 + tid;
+            uint8_t kind = 0;
+            int64_t src = 0;
+            if (kidx < a.K) {
+                const int32_t pos = a.topk[bq * a.K + kidx];
+                if (pos >= 0 && pos < a.cap) {
+                    kind = 1;
+                    src = (int64_t)b * a.cap + pos;
+                }
+            } else if (kidx - a.K < w.n) {
+                kind = 2;
+            }
+            slot_kind[tid] = kind;
+            slot_src[tid] = src;
+        }
+        if (tid == 0)
+            mbar_expect_tx(bar_ld, (uint32_t)Q_BYTES + (uint32_t)nbox * 8u * SWA_BOX * 128u);
+        __syncthreads();
+
+        // ---- load phase: Q and window rows by TMA, FP4 rows by cp.async
+        // slots that no copy writes (invalid keys outside the window boxes) are zeroed
+        for (int i = tid; i < T * 64; i += THREADS) {
+            const int j = i >> 6, pg = i & 63;
+            if (slot_kind[j] == 0 && (j < js || j >= cover_end))
+                st_shared_v4(base + K_OFF + (pg >> 3) * K_CHUNK + sw128(j, pg & 7),
+                             make_uint4(0, 0, 0, 0));
+        }
+        if (tid == 0) {
+            const int qrow = (int)(bq * HQ);
 #pragma unroll
             for (int cc = 0; cc < 8; cc++)
-                tma_load_2d(base + K_OFF + cc * K_CHUNK + (js + bx * SWA_BOX) * 128, &tswa, cc * 64,
-                            wrow0 + bx * SWA_BOX, bar_ld);
-    }
-    if (warp == 1) {
-        for (int j = lane; j < T; j += 32) {
+                tma_load_2d(base + Q_OFF + cc * Q_CHUNK, &tq, cc * 64, qrow, bar_ld);
+            const int wrow0 = (int)((int64_t)b * a.swa_rows + w.row0 + (k0 + js - a.K));
+            for (int bx = 0; bx < nbox; bx++)
+#pragma unroll
+                for (int cc = 0; cc < 8; cc++)
+                    tma_load_2d(base + K_OFF + cc * K_CHUNK + (js + bx * SWA_BOX) * 128, &tswa,
+                                cc * 64, wrow0 + bx * SWA_BOX, bar_ld);
+        }
+        for (int i = tid; i < T * 18; i += THREADS) {  // (slot, 16-byte piece of its 288 B)
+            const int j = i / 18, pc = i - j * 18;
             if (slot_kind[j] != 1) continue;
             const int64_t cell = slot_src[j];
-            bulk_load(base + FP4_STAGE_OFF + j * 288, a.kv_fp4 + cell * 256, 256, bar_ld);
-            bulk_load(base + FP4_STAGE_OFF + j * 288 + 256, a.kv_sf + cell * 32, 32, bar_ld);
+            const uint8_t *src =
+                pc < 16 ? a.kv_fp4 + cell * 256 + pc * 16 : a.kv_sf + cell * 32 + (pc - 16) * 16;
+            cp_async16(base + FP4_STAGE_OFF + j * 288 + pc * 16, src);
         }
-    }
-    bool ok = mbar_wait(bar_ld, 0);
+        cp_async_wait_all();
+        if (ok) ok = mbar_wait(bar_ld, ld_phase);
+        ld_phase ^= 1;
+        __syncthreads();
 
-    // ---- dequantize the FP4 rows into the KV tile
-    const uint8_t *stage = sm + FP4_STAGE_OFF;
-    for (int i = tid; i < T * 32; i += THREADS) {  // (slot, 16-channel group)
-        const int j = i >> 5, g = i & 31;
-        if (slot_kind[j] != 1) continue;
-        const uint2 codes = *reinterpret_cast<const uint2 *>(stage + j * 288 + g * 8);
-        const float s = e4m3_to_f32(stage[j * 288 + 256 + g]);
-        uint32_t wds[8];
-#pragma unroll
-        for (int u = 0; u < 8; u++) {
-            const uint32_t byte = ((u < 4 ? codes.x : codes.y) >> (8 * (u & 3))) & 0xFF;
-            const float2 f = e2m1x2_to_f32x2(byte);
-            wds[u] = pack_bf16x2(f.x * s, f.y * s);
-        }
-        const int pg = g * 2;  // two 16-byte pieces
-        const uint32_t d0 = base + K_OFF + (pg >> 3) * K_CHUNK + sw128(j, pg & 7);
-        const uint32_t d1 = base + K_OFF + ((pg + 1) >> 3) * K_CHUNK + sw128(j, (pg + 1) & 7);
-        st_shared_v4(d0, make_uint4(wds[0], wds[1], wds[2], wds[3]));
-        st_shared_v4(d1, make_uint4(wds[4], wds[5], wds[6], wds[7]));
-    }
-    fence_proxy_async();
-    __syncthreads();
-
-    // ---- S = Q K^T  (M = 64, N = 80, K = 512) into TMEM lanes 16..31
-    const uint32_t s_tmem = tmem + (16u << 16);
-    if (tid == 0 && ok) {
-        tc_fence_after();
-        constexpr uint32_t id_s = idesc_bf16(HQ, T, false);
-#pragma unroll 1
-        for (int kk = 0; kk < CH / 16; kk++) {
-            const uint32_t off = (kk & 3) * 32;
-            const uint64_t ad = sdesc(base + Q_OFF + (kk >> 2) * Q_CHUNK + off, 16, 1024);
-            const uint64_t bd = sdesc(base + K_OFF + (kk >> 2) * K_CHUNK + off, 16, 1024);
-            mma_bf16(s_tmem, ad, bd, id_s, kk > 0);
-        }
-        mma_commit(bar);
-    }
-    if (ok) ok = mbar_wait(bar, 0);
-    tc_fence_after();
-
-    // ---- softmax over this CTA's keys (warps 0-3; two threads per head)
-    const int h = (warp & 3) * 16 + (lane & 15);
-    const int half = lane >> 4;
-    if (warp < 4) {
-        const float sl2 = a.scale * LOG2E;
-        float p[40];
-        {
-            float v32[32], v8[8];
-            const uint32_t row_addr = s_tmem + ((uint32_t)(warp * 32) << 16);
-            tmem_ld_16x32x2_32(row_addr + 0, v32);
-            tmem_ld_16x32x2_8(row_addr + 64, v8);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; i++) {
-                const int j = half * 32 + i;
-                p[i] = (ok && slot_kind[j] != 0) ? v32[i] * sl2 : -INFINITY;
-            }
-#pragma unroll
-            for (int i = 0; i < 8; i++) {
-                const int j = 64 + half * 8 + i;
-                p[32 + i] = (ok && slot_kind[j] != 0) ? v8[i] * sl2 : -INFINITY;
-            }
-        }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 40; i++) mx = fmaxf(mx, p[i]);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        float sum = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 40; i++) {
-            p[i] = (p[i] == -INFINITY) ? 0.0f : ex2(p[i] - mx);
-            sum += p[i];
-        }
-        sum += __shfl_xor_sync(0xffffffffu, sum, 16);
-        if (half == 0) {
-            m_s[h] = mx;
-            l_s[h] = sum;
-        }
-        // P = hi + lo (bf16), K-major 128B-swizzled tiles: tokens 0..63 in the
-        // first atom column, 64..79 in the second.
-#pragma unroll
-        for (int piece = 0; piece < 5; piece++) {
-            const int tok0 = piece < 4 ? half * 32 + piece * 8 : 64 + half * 8;
-            const float *pp = p + piece * 8;
-            uint32_t hi[4], lo[4];
-#pragma unroll
-            for (int u = 0; u < 4; u++) {
-                const __nv_bfloat162 hb = __floats2bfloat162_rn(pp[2 * u], pp[2 * u + 1]);
-                const float2 hf = __bfloat1622float2(hb);
-                hi[u] = *reinterpret_cast<const uint32_t *>(&hb);
-                lo[u] = pack_bf16x2(pp[2 * u] - hf.x, pp[2 * u + 1] - hf.y);
-            }
-            const uint32_t off = (tok0 >> 6) * P_ATOM + sw128(h, (tok0 & 63) >> 3);
-            st_shared_v4(base + PHI_OFF + off, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-            st_shared_v4(base + PLO_OFF + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
-        }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- O = P_hi V + P_lo V  (M = 64, N = 256 per half, K = 80)
-    if (tid == 0 && ok) {
-        tc_fence_after();
-        constexpr uint32_t id_o = idesc_bf16(HQ, 256, true);
-#pragma unroll 1
-        for (int hf = 0; hf < 2; hf++) {
-#pragma unroll 1
-            for (int kk = 0; kk < T / 16; kk++) {
-                const uint32_t poff = (kk >> 2) * P_ATOM + (kk & 3) * 32;
-                const uint64_t vd =
-                    sdesc(base + K_OFF + hf * 4 * K_CHUNK + kk * 2048, K_CHUNK, 1024);
-                mma_bf16(tmem + hf * 256, sdesc(base + PHI_OFF + poff, 16, 1024), vd, id_o, kk > 0);
-                mma_bf16(tmem + hf * 256, sdesc(base + PLO_OFF + poff, 16, 1024), vd, id_o, 1);
-            }
-        }
-        mma_commit(bar);
-    }
-    if (ok) ok = mbar_wait(bar, 1);
-    tc_fence_after();
-
-    // ---- unnormalized O -> shared staging [64][516] fp32 (reuses Q and KV
-    // tiles); warps w and w + 4 share a TMEM lane quadrant and split the columns
-    float *stg = reinterpret_cast<float *>(sm + Q_OFF);
-    {
-        const uint32_t row_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        const int cbeg = (warp >> 2) * 256;
-#pragma unroll 1
-        for (int c0 = cbeg; c0 < cbeg + 256; c0 += 64) {
-            float v[32];
-            tmem_ld_16x32x2_32(row_addr + c0, v);
-            tmem_ld_wait();
-            float *dst = stg + h * STG_STRIDE + c0 + half * 32;
+        // ---- dequantize the FP4 rows into the KV tile
+        const uint8_t *stage = sm + FP4_STAGE_OFF;
+        for (int i = tid; i < T * 32; i += THREADS) {  // (slot, 16-channel group)
+            const int j = i >> 5, g = i & 31;
+            if (slot_kind[j] != 1) continue;
+            const uint2 codes = *reinterpret_cast<const uint2 *>(stage + j * 288 + g * 8);
+            const float s = e4m3_to_f32(stage[j * 288 + 256 + g]);
+            uint32_t wds[8];
 #pragma unroll
             for (int u = 0; u < 8; u++) {
-                const float4 f = ok ? make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3])
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-                *reinterpret_cast<float4 *>(dst + 4 * u) = f;
+                const uint32_t byte = ((u < 4 ? codes.x : codes.y) >> (8 * (u & 3))) & 0xFF;
+                const float2 f = e2m1x2_to_f32x2(byte);
+                wds[u] = pack_bf16x2(f.x * s, f.y * s);
+            }
+            const int pg = g * 2;  // two 16-byte pieces
+            const uint32_t d0 = base + K_OFF + (pg >> 3) * K_CHUNK + sw128(j, pg & 7);
+            const uint32_t d1 = base + K_OFF + ((pg + 1) >> 3) * K_CHUNK + sw128(j, (pg + 1) & 7);
+            st_shared_v4(d0, make_uint4(wds[0], wds[1], wds[2], wds[3]));
+            st_shared_v4(d1, make_uint4(wds[4], wds[5], wds[6], wds[7]));
+        }
+        fence_proxy_async();
+        __syncthreads();
+
+        // ---- S = Q K^T  (M = 64, N = 80, K = 512) into TMEM lanes 16..31
+        const uint32_t s_tmem = tmem + (16u << 16);
+        if (tid == 0 && ok) {
+            tc_fence_after();
+            constexpr uint32_t id_s = idesc_bf16(HQ, T, false);
+#pragma unroll 1
+            for (int kk = 0; kk < CH / 16; kk++) {
+                const uint32_t off = (kk & 3) * 32;
+                const uint64_t ad = sdesc(base + Q_OFF + (kk >> 2) * Q_CHUNK + off, 16, 1024);
+                const uint64_t bd = sdesc(base + K_OFF + (kk >> 2) * K_CHUNK + off, 16, 1024);
+                mma_bf16(s_tmem, ad, bd, id_s, kk > 0);
+            }
+            mma_commit(bar);
+        }
+        if (ok) ok = mbar_wait(bar, 0);
+        tc_fence_after();
+
+        // ---- softmax over this CTA's keys (warps 0-3; two threads per head)
+        const int h = (warp & 3) * 16 + (lane & 15);
+        const int half = lane >> 4;
+        if (warp < 4) {
+            const float sl2 = a.scale * LOG2E;
+            float p[40];
+            {
+                float v32[32], v8[8];
+                const uint32_t row_addr = s_tmem + ((uint32_t)(warp * 32) << 16);
+                tmem_ld_16x32x2_32(row_addr + 0, v32);
+                tmem_ld_16x32x2_8(row_addr + 64, v8);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; i++) {
+                    const int j = half * 32 + i;
+                    p[i] = (ok && slot_kind[j] != 0) ? v32[i] * sl2 : -INFINITY;
+                }
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const int j = 64 + half * 8 + i;
+                    p[32 + i] = (ok && slot_kind[j] != 0) ? v8[i] * sl2 : -INFINITY;
+                }
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 40; i++) mx = fmaxf(mx, p[i]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            float sum = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 40; i++) {
+                p[i] = (p[i] == -INFINITY) ? 0.0f : ex2(p[i] - mx);
+                sum += p[i];
+            }
+            sum += __shfl_xor_sync(0xffffffffu, sum, 16);
+            if (half == 0) {
+                m_s[h] = mx;
+                l_s[h] = sum;
+            }
+            // P = hi + lo (bf16), K-major 128B-swizzled tiles: tokens 0..63 in the
+            // first atom column, 64..79 in the second.
+#pragma unroll
+            for (int piece = 0; piece < 5; piece++) {
+                const int tok0 = piece < 4 ? half * 32 + piece * 8 : 64 + half * 8;
+                const float *pp = p + piece * 8;
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                    const __nv_bfloat162 hb = __floats2bfloat162_rn(pp[2 * u], pp[2 * u + 1]);
+                    const float2 hf = __bfloat1622float2(hb);
+                    hi[u] = *reinterpret_cast<const uint32_t *>(&hb);
+                    lo[u] = pack_bf16x2(pp[2 * u] - hf.x, pp[2 * u + 1] - hf.y);
+                }
+                const uint32_t off = (tok0 >> 6) * P_ATOM + sw128(h, (tok0 & 63) >> 3);
+                st_shared_v4(base + PHI_OFF + off, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+                st_shared_v4(base + PLO_OFF + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
             }
         }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- O = P_hi V + P_lo V  (M = 64, N = 256 per half, K = 80)
+        if (tid == 0 && ok) {
+            tc_fence_after();
+            constexpr uint32_t id_o = idesc_bf16(HQ, 256, true);
+#pragma unroll 1
+            for (int hf = 0; hf < 2; hf++) {
+#pragma unroll 1
+                for (int kk = 0; kk < T / 16; kk++) {
+                    const uint32_t poff = (kk >> 2) * P_ATOM + (kk & 3) * 32;
+                    const uint64_t vd =
+                        sdesc(base + K_OFF + hf * 4 * K_CHUNK + kk * 2048, K_CHUNK, 1024);
+                    mma_bf16(tmem + hf * 256, sdesc(base + PHI_OFF + poff, 16, 1024), vd, id_o,
+                             kk > 0);
+                    mma_bf16(tmem + hf * 256, sdesc(base + PLO_OFF + poff, 16, 1024), vd, id_o, 1);
+                }
+            }
+            mma_commit(bar);
+        }
+        if (ok) ok = mbar_wait(bar, 1);
+        tc_fence_after();
+
+        // ---- publish this CTA's unnormalized O, row maxima and sums in the
+        // cluster's exchange slot (L2). O is first staged in shared memory
+        // slice-major ([8 slices of 64 channels][64 heads][64 channels]) over the
+        // now idle Q and KV tiles, then copied out as 8 contiguous 16 KB bulk
+        // stores; warps w and w + 4 split the TMEM columns.
+        {
+            const uint32_t row_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+            const int cbeg = (warp >> 2) * 256;
+#pragma unroll 1
+            for (int c0 = cbeg; c0 < cbeg + 256; c0 += 64) {
+                float v[32];
+                tmem_ld_16x32x2_32(row_addr + c0, v);
+                tmem_ld_wait();
+                const uint32_t dst = base + STG_OFF + (uint32_t)(((c0 >> 6) * HQ + h) * 64 + half * 32) * 4;
+                // rotate the 8 pieces by lane so that a warp's stores spread over the banks
+#pragma unroll
+                for (int u0 = 0; u0 < 8; u0++) {
+                    const int u = (u0 + (lane & 7)) & 7;
+                    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int q = 0; q < 8; q++)
+                        if (q == u && ok) f = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    st_shared_v4(dst + 16 * u, make_uint4(__float_as_uint(f.x), __float_as_uint(f.y),
+                                                          __float_as_uint(f.z), __float_as_uint(f.w)));
+                }
+            }
+            if (warp < 4 && half == 0) {
+                xm[rank * HQ + h] = ok ? m_s[h] : -INFINITY;
+                xl[rank * HQ + h] = ok ? l_s[h] : 0.0f;
+            }
+        }
+        fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) {
+#pragma unroll
+            for (int c = 0; c < CL; c++)
+                bulk_store(xo + ((int64_t)rank * CL + c) * (HQ * 64), base + STG_OFF + c * SLICE_BYTES,
+                           SLICE_BYTES);
+            bulk_store_wait();
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
+        __syncthreads();
+        __threadfence();
+        tc_fence_before();
+        cluster_sync();  // all partial results of this row are in the slot
+
+        // ---- combine: this CTA owns channels [64 rank, 64 rank + 64); the slice
+        // of source r is contiguous at xo[r][rank]. Thread t takes elements
+        // e = 4 (t + 256 u), u = 0..3, of the [64 heads][64 channels] slice.
+        {
+            float *wts = reinterpret_cast<float *>(sm + PHI_OFF);  // [64 heads][8] weight / den
+            if (tid < HQ) {
+                float mr[CL], lr[CL];
+#pragma unroll
+                for (int r = 0; r < CL; r++) {
+                    mr[r] = __ldcg(xm + r * HQ + tid);
+                    lr[r] = __ldcg(xl + r * HQ + tid);
+                }
+                float M = -INFINITY;
+#pragma unroll
+                for (int r = 0; r < CL; r++) M = fmaxf(M, mr[r]);
+                float den = 0.0f, wg[CL];
+#pragma unroll
+                for (int r = 0; r < CL; r++) {
+                    wg[r] = (M == -INFINITY || mr[r] == -INFINITY) ? 0.0f : ex2(mr[r] - M);
+                    den += wg[r] * lr[r];
+                }
+                const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+#pragma unroll
+                for (int r = 0; r < CL; r++) wts[tid * CL + r] = wg[r] * inv;
+            }
+            float4 f[4][CL];
+#pragma unroll
+            for (int u = 0; u < 4; u++)
+#pragma unroll
+                for (int r = 0; r < CL; r++)
+                    f[u][r] = __ldcg(reinterpret_cast<const float4 *>(
+                                         xo + ((int64_t)r * CL + rank) * (HQ * 64)) +
+                                     tid + 256 * u);
+            __syncthreads();  // weights ready
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const int e = 4 * (tid + 256 * u);
+                const int hh = e >> 6, ch = e & 63;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int r = 0; r < CL; r++) {
+                    const float wr = wts[hh * CL + r];
+                    acc.x += wr * f[u][r].x;
+                    acc.y += wr * f[u][r].y;
+                    acc.z += wr * f[u][r].z;
+                    acc.w += wr * f[u][r].w;
+                }
+                *reinterpret_cast<float4 *>(a.out + (bq * HQ + hh) * (int64_t)CH + (int)rank * 64 + ch) =
+                    acc;
+            }
+        }
+        cluster_sync();  // the slot, the tiles and TMEM are free for the next row
     }
     if (!ok && tid == 0) atomicExch(&g_attn_error, 1);
-    tc_fence_before();
-    cluster_sync();  // staging of every CTA in the cluster is complete
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
-
-    // ---- combine: this CTA owns channels [64 rank, 64 rank + 64) of all heads;
-    // thread = (head, 16 channels)
-    {
-        const int hh = tid >> 2;
-        const int c0 = (int)rank * 64 + (tid & 3) * 16;
-        float mr[CL], lr[CL], M = -INFINITY;
-#pragma unroll
-        for (int r = 0; r < CL; r++) {
-            mr[r] = ld_dsmem_f32(map_rank(base + M_OFF + hh * 4, r));
-            lr[r] = ld_dsmem_f32(map_rank(base + L_OFF + hh * 4, r));
-        }
-#pragma unroll
-        for (int r = 0; r < CL; r++) M = fmaxf(M, mr[r]);
-        float wgt[CL], den = 0.0f;
-#pragma unroll
-        for (int r = 0; r < CL; r++) {
-            wgt[r] = (M == -INFINITY || mr[r] == -INFINITY) ? 0.0f : ex2(mr[r] - M);
-            den += wgt[r] * lr[r];
-        }
-        const float inv = den > 0.0f ? 1.0f / den : 0.0f;
-        float4 f[CL][4];
-#pragma unroll
-        for (int r = 0; r < CL; r++) {
-            const uint32_t src = map_rank(base + Q_OFF + (uint32_t)(hh * STG_STRIDE + c0) * 4, r);
-#pragma unroll
-            for (int u = 0; u < 4; u++) f[r][u] = ld_dsmem_v4(src + 16 * u);
-        }
-        float *out = a.out + (bq * HQ + hh) * (int64_t)CH + c0;
-#pragma unroll
-        for (int u = 0; u < 4; u++) {
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int r = 0; r < CL; r++) {
-                acc.x += wgt[r] * f[r][u].x;
-                acc.y += wgt[r] * f[r][u].y;
-                acc.z += wgt[r] * f[r][u].z;
-                acc.w += wgt[r] * f[r][u].w;
-            }
-            *reinterpret_cast<float4 *>(out + 4 * u) =
-                make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-        }
-    }
-    cluster_sync();  // peers may still be reading this CTA's staging
 }
 
 }  // namespace tc
@@ -554,7 +618,7 @@ int launch_attn_tc(const AttnArgs &a, cudaStream_t s) {
         attr = true;
     }
     const int64_t rows = (int64_t)a.B * a.Nq;
-    if (rows > 65535) return CSA2_ERR_SHAPE;
+    if (a.ws == nullptr) return CSA2_ERR_WORKSPACE;
     CUtensorMap tq, tswa;
     if (!make_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.q, tc::CH, (uint64_t)rows * tc::HQ,
                       tc::CH * 2, 64, 64))
@@ -566,7 +630,8 @@ int launch_attn_tc(const AttnArgs &a, cudaStream_t s) {
                       tc::SWA_BOX))
         return CSA2_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(tc::CL, (unsigned)rows, 1);
+    const int64_t clusters = rows < tc::MAX_CLUSTERS ? rows : tc::MAX_CLUSTERS;
+    cfg.gridDim = dim3(tc::CL, (unsigned)clusters, 1);
     cfg.blockDim = dim3(tc::THREADS, 1, 1);
     cfg.dynamicSmemBytes = tc::SMEM_BYTES;
     cfg.stream = s;
@@ -580,6 +645,16 @@ int launch_attn_tc(const AttnArgs &a, cudaStream_t s) {
     if (cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel, tq, tswa, a) != cudaSuccess)
         return CSA2_ERR_CUDA;
     return launch_status();
+}
+
+}  // namespace csa2
+
+namespace csa2 {
+
+size_t attn_tc_workspace_bytes(int B, int Nq) {
+    const int64_t rows = (int64_t)B * Nq;
+    const int64_t clusters = rows < tc::MAX_CLUSTERS ? rows : tc::MAX_CLUSTERS;
+    return (size_t)clusters * tc::XSLOT_FLOATS * sizeof(float);
 }
 
 }  // namespace csa2

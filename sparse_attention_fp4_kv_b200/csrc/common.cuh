@@ -120,6 +120,30 @@ __device__ __forceinline__ int64_t visible_len(const int64_t *ctx_len, const int
 int launch_kv_append(const uint16_t *kv, int B, int n_new, int C, const int64_t *pos_base,
                      int64_t pos_offset, int64_t cap, uint8_t *fp4, uint8_t *sf, cudaStream_t s);
 
+// First-digit histogram bin of a score (top 12 bits of its order-preserving
+// key), shared by the score producers and the histogram-fed top-k.
+constexpr int kHistBins = 4096;
+__device__ __forceinline__ uint32_t hist_bin(float score) { return f32_order_key(score) >> 20; }
+
+// Histogram-fed top-k (topk.cu): the workspace starts with hist[R][4096] and
+// two counters per row, all zero before the producer runs.
+size_t topk_hist_ws_bytes(int R, int k);
+int launch_topk_from_hist(const float *score, const int32_t *cand_pos, const int32_t *n_valid,
+                          int R, int64_t n, int k, int32_t *out, void *ws, cudaStream_t s);
+
+// Score producers with an optional histogram output (indexer.cu).
+int launch_index_full_hist(const int8_t *q_idx, const int8_t *k_idx, const float *k_scale,
+                           const int64_t *ctx_len, int B, int H, int D, int64_t cap,
+                           float *tok_score, float *blk_score, int32_t *n_blk, uint32_t *hist,
+                           cudaStream_t s);
+int launch_pool_gather_hist(const float *tok_score, const int32_t *pool, const int64_t *ctx_len,
+                            int B, int P, int64_t cap, float *pool_score, int32_t *pool_pos,
+                            uint32_t *hist, cudaStream_t s);
+int launch_reindex_hist(const int8_t *q_idx, const int8_t *k_idx, const float *k_scale,
+                        const int32_t *pool, const int64_t *ctx_len, int B, int H, int D,
+                        int64_t cap, int P, float *pool_score, int32_t *pool_pos, uint32_t *hist,
+                        cudaStream_t s);
+
 // Multi-query indexer scan on tensor cores (index_mma.cu).
 bool index_mma_supported(int Nq, int HD, int64_t cap, int B);
 int launch_index_mma(const int8_t *q, const int8_t *k, const float *kscale, const int64_t *ctx_len,

@@ -166,6 +166,7 @@ struct ScanArgs {
     float *tok;
     float *blk;
     int32_t *n_blk;
+    uint32_t *hist;  // optional [B*Nq][4096] counts of block scores by first digit
 };
 
 template <int HD>
@@ -197,7 +198,10 @@ __global__ void __launch_bounds__(256) index_full_kernel(ScanArgs a) {
         const float sc = lane_score(S, a.kscale + t0, my_tok, ntok);
         const float m = warp_block_max(sc);
         if (a.tok && (lane & 3) == 0 && my_tok < ntok) a.tok[bq * a.cap + 8 * j + my_tok] = sc;
-        if (lane == 0) a.blk[bq * a.nblk_cap + j] = m;
+        if (lane == 0) {
+            a.blk[bq * a.nblk_cap + j] = m;
+            if (a.hist) atomicAdd(&a.hist[bq * kHistBins + hist_bin(m)], 1u);
+        }
     }
 }
 
@@ -221,7 +225,10 @@ __global__ void __launch_bounds__(256) index_full_generic_kernel(ScanArgs a) {
         const float sc = lane_score(S, a.kscale + t0, my_tok, ntok);
         const float m = warp_block_max(sc);
         if (a.tok && (lane & 3) == 0 && my_tok < ntok) a.tok[bq * a.cap + 8 * j + my_tok] = sc;
-        if (lane == 0) a.blk[bq * a.nblk_cap + j] = m;
+        if (lane == 0) {
+            a.blk[bq * a.nblk_cap + j] = m;
+            if (a.hist) atomicAdd(&a.hist[bq * kHistBins + hist_bin(m)], 1u);
+        }
     }
 }
 
@@ -237,6 +244,7 @@ struct ReindexArgs {
     int64_t cap;
     float *pscore;
     int32_t *ppos;
+    uint32_t *hist;  // optional [B*Nq][4096] counts of pooled scores by first digit
 };
 
 __device__ __forceinline__ int64_t reindex_block(const ReindexArgs &a, int64_t bq, int s, int64_t V,
@@ -284,6 +292,7 @@ __global__ void __launch_bounds__(256) index_reindex_kernel(ReindexArgs a) {
     if ((lane & 3) == 0) {
         a.ppos[slot + my_tok] = my_tok < ntok ? (int32_t)(t0 + my_tok) : -1;
         a.pscore[slot + my_tok] = my_tok < ntok ? sc : 0.0f;
+        if (a.hist && my_tok < ntok) atomicAdd(&a.hist[bq * kHistBins + hist_bin(sc)], 1u);
     }
 }
 
@@ -315,6 +324,7 @@ __global__ void __launch_bounds__(256) index_reindex_generic_kernel(ReindexArgs 
         if ((lane & 3) == 0) {
             a.ppos[slot + my_tok] = my_tok < ntok ? (int32_t)(t0 + my_tok) : -1;
             a.pscore[slot + my_tok] = my_tok < ntok ? sc : 0.0f;
+            if (a.hist && my_tok < ntok) atomicAdd(&a.hist[bq * kHistBins + hist_bin(sc)], 1u);
         }
     }
 }
@@ -325,7 +335,7 @@ __global__ void __launch_bounds__(256) pool_gather_kernel(const float *__restric
                                                           const int64_t *ctx_len,
                                                           const int64_t *q_pos, int B, int Nq,
                                                           int P, int64_t cap, float *pscore,
-                                                          int32_t *ppos) {
+                                                          int32_t *ppos, uint32_t *hist) {
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t total = (int64_t)B * Nq * P * 8;
     if (idx >= total) return;
@@ -338,8 +348,10 @@ __global__ void __launch_bounds__(256) pool_gather_kernel(const float *__restric
     const int32_t blkid = pool[s_all];
     const int64_t p = 8 * (int64_t)blkid + r;
     if (blkid >= 0 && p < V) {
+        const float sc = tok[bq * cap + p];
         ppos[idx] = (int32_t)p;
-        pscore[idx] = tok[bq * cap + p];
+        pscore[idx] = sc;
+        if (hist) atomicAdd(&hist[bq * kHistBins + hist_bin(sc)], 1u);
     } else {
         ppos[idx] = -1;
         pscore[idx] = 0.0f;
@@ -360,31 +372,8 @@ static int persistent_grid(K kernel, int threads, int64_t items_warps) {
 
 using namespace csa2;
 
-static int check_indexer_common(const int8_t *q_idx, const int8_t *k_idx, const float *k_scale,
-                                const int64_t *ctx_len, int B, int Nq, int H, int D, int64_t cap) {
-    if (!q_idx || !k_idx || !k_scale || !ctx_len) return CSA2_ERR_NULL;
-    if (B < 0 || Nq < 0 || H <= 0 || D <= 0 || cap < 1) return CSA2_ERR_SHAPE;
-    const int64_t HD = (int64_t)H * D;
-    if (HD % 16 || HD > 65536) return CSA2_ERR_SHAPE;
-    if (!aligned(q_idx, 16) || !aligned(k_idx, 16)) return CSA2_ERR_ALIGN;
-    return CSA2_OK;
-}
-
-extern "C" int csa2_index_full(const int8_t *q_idx, const int8_t *k_idx, const float *k_scale,
-                               const int64_t *ctx_len, const int64_t *q_pos, int B, int Nq, int H,
-                               int D, int64_t cap, float *tok_score, float *blk_score,
-                               int32_t *n_blk, void *stream) {
-    int st = check_indexer_common(q_idx, k_idx, k_scale, ctx_len, B, Nq, H, D, cap);
-    if (st) return st;
-    if (!blk_score) return CSA2_ERR_NULL;
-    if ((int64_t)B * Nq == 0) return CSA2_OK;
-    if (index_mma_supported(Nq, H * D, cap, B))
-        return launch_index_mma(q_idx, k_idx, k_scale, ctx_len, q_pos, B, Nq, H * D, cap,
-                                tok_score, blk_score, n_blk, (cudaStream_t)stream);
-    ScanArgs a{q_idx, k_idx, k_scale, ctx_len, q_pos, B, Nq, H * D, cap, (cap + 7) / 8,
-               tok_score, blk_score, n_blk};
-    const int64_t items = (int64_t)B * Nq * a.nblk_cap;
-    cudaStream_t s = (cudaStream_t)stream;
+static int dispatch_scan(const ScanArgs &a, cudaStream_t s) {
+    const int64_t items = (int64_t)a.B * a.Nq * a.nblk_cap;
     const int T = 256;
     switch (a.HD) {
 #define CSA2_SCAN_CASE(HDV)                                                             \
@@ -408,19 +397,8 @@ extern "C" int csa2_index_full(const int8_t *q_idx, const int8_t *k_idx, const f
     return launch_status();
 }
 
-extern "C" int csa2_index_reindex(const int8_t *q_idx, const int8_t *k_idx, const float *k_scale,
-                                  const int32_t *pool, const int64_t *ctx_len,
-                                  const int64_t *q_pos, int B, int Nq, int H, int D, int64_t cap,
-                                  int P, float *pool_score, int32_t *pool_pos, void *stream) {
-    int st = check_indexer_common(q_idx, k_idx, k_scale, ctx_len, B, Nq, H, D, cap);
-    if (st) return st;
-    if (!pool || !pool_score || !pool_pos) return CSA2_ERR_NULL;
-    if (P < 0 || P > (1 << 24)) return CSA2_ERR_SHAPE;
-    if ((int64_t)B * Nq * P == 0) return CSA2_OK;
-    ReindexArgs a{q_idx, k_idx, k_scale, pool, ctx_len, q_pos, B, Nq, H * D, P, cap,
-                  pool_score, pool_pos};
-    const int64_t items = (int64_t)B * Nq * P;
-    cudaStream_t s = (cudaStream_t)stream;
+static int dispatch_reindex(const ReindexArgs &a, cudaStream_t s) {
+    const int64_t items = (int64_t)a.B * a.Nq * a.P;
     const int T = 256;
     switch (a.HD) {
 #define CSA2_RI_CASE(HDV)                                                               \
@@ -445,6 +423,46 @@ extern "C" int csa2_index_reindex(const int8_t *q_idx, const int8_t *k_idx, cons
     return launch_status();
 }
 
+static int check_indexer_common(const int8_t *q_idx, const int8_t *k_idx, const float *k_scale,
+                                const int64_t *ctx_len, int B, int Nq, int H, int D, int64_t cap) {
+    if (!q_idx || !k_idx || !k_scale || !ctx_len) return CSA2_ERR_NULL;
+    if (B < 0 || Nq < 0 || H <= 0 || D <= 0 || cap < 1) return CSA2_ERR_SHAPE;
+    const int64_t HD = (int64_t)H * D;
+    if (HD % 16 || HD > 65536) return CSA2_ERR_SHAPE;
+    if (!aligned(q_idx, 16) || !aligned(k_idx, 16)) return CSA2_ERR_ALIGN;
+    return CSA2_OK;
+}
+
+extern "C" int csa2_index_full(const int8_t *q_idx, const int8_t *k_idx, const float *k_scale,
+                               const int64_t *ctx_len, const int64_t *q_pos, int B, int Nq, int H,
+                               int D, int64_t cap, float *tok_score, float *blk_score,
+                               int32_t *n_blk, void *stream) {
+    int st = check_indexer_common(q_idx, k_idx, k_scale, ctx_len, B, Nq, H, D, cap);
+    if (st) return st;
+    if (!blk_score) return CSA2_ERR_NULL;
+    if ((int64_t)B * Nq == 0) return CSA2_OK;
+    if (index_mma_supported(Nq, H * D, cap, B))
+        return launch_index_mma(q_idx, k_idx, k_scale, ctx_len, q_pos, B, Nq, H * D, cap,
+                                tok_score, blk_score, n_blk, (cudaStream_t)stream);
+    ScanArgs a{q_idx, k_idx, k_scale, ctx_len, q_pos, B, Nq, H * D, cap, (cap + 7) / 8,
+               tok_score, blk_score, n_blk, nullptr};
+    return dispatch_scan(a, (cudaStream_t)stream);
+}
+
+extern "C" int csa2_index_reindex(const int8_t *q_idx, const int8_t *k_idx, const float *k_scale,
+                                  const int32_t *pool, const int64_t *ctx_len,
+                                  const int64_t *q_pos, int B, int Nq, int H, int D, int64_t cap,
+                                  int P, float *pool_score, int32_t *pool_pos, void *stream) {
+    int st = check_indexer_common(q_idx, k_idx, k_scale, ctx_len, B, Nq, H, D, cap);
+    if (st) return st;
+    if (!pool || !pool_score || !pool_pos) return CSA2_ERR_NULL;
+    if (P < 0 || P > (1 << 24)) return CSA2_ERR_SHAPE;
+    if ((int64_t)B * Nq * P == 0) return CSA2_OK;
+    ReindexArgs a{q_idx, k_idx, k_scale, pool, ctx_len, q_pos, B, Nq, H * D, P, cap,
+                  pool_score, pool_pos, nullptr};
+    return dispatch_reindex(a, (cudaStream_t)stream);
+}
+
 extern "C" int csa2_pool_gather(const float *tok_score, const int32_t *pool,
                                 const int64_t *ctx_len, const int64_t *q_pos, int B, int Nq, int P,
                                 int64_t cap, float *pool_score, int32_t *pool_pos, void *stream) {
@@ -457,6 +475,39 @@ extern "C" int csa2_pool_gather(const float *tok_score, const int32_t *pool,
     if (g > INT32_MAX) return CSA2_ERR_SHAPE;
     pool_gather_kernel<<<(unsigned)g, T, 0, (cudaStream_t)stream>>>(tok_score, pool, ctx_len, q_pos,
                                                                    B, Nq, P, cap, pool_score,
-                                                                   pool_pos);
+                                                                   pool_pos, nullptr);
     return launch_status();
 }
+
+namespace csa2 {
+
+int launch_index_full_hist(const int8_t *q_idx, const int8_t *k_idx, const float *k_scale,
+                           const int64_t *ctx_len, int B, int H, int D, int64_t cap,
+                           float *tok_score, float *blk_score, int32_t *n_blk, uint32_t *hist,
+                           cudaStream_t s) {
+    ScanArgs a{q_idx, k_idx, k_scale, ctx_len, nullptr, B, 1, H * D, cap, (cap + 7) / 8,
+               tok_score, blk_score, n_blk, hist};
+    return dispatch_scan(a, s);
+}
+
+int launch_pool_gather_hist(const float *tok_score, const int32_t *pool, const int64_t *ctx_len,
+                            int B, int P, int64_t cap, float *pool_score, int32_t *pool_pos,
+                            uint32_t *hist, cudaStream_t s) {
+    const int64_t total = (int64_t)B * P * 8;
+    if (total == 0) return CSA2_OK;
+    const int T = 256;
+    pool_gather_kernel<<<(unsigned)((total + T - 1) / T), T, 0, s>>>(
+        tok_score, pool, ctx_len, nullptr, B, 1, P, cap, pool_score, pool_pos, hist);
+    return launch_status();
+}
+
+int launch_reindex_hist(const int8_t *q_idx, const int8_t *k_idx, const float *k_scale,
+                        const int32_t *pool, const int64_t *ctx_len, int B, int H, int D,
+                        int64_t cap, int P, float *pool_score, int32_t *pool_pos, uint32_t *hist,
+                        cudaStream_t s) {
+    ReindexArgs a{q_idx, k_idx, k_scale, pool, ctx_len, nullptr, B, 1, H * D, P, cap,
+                  pool_score, pool_pos, hist};
+    return dispatch_reindex(a, s);
+}
+
+}  // namespace csa2

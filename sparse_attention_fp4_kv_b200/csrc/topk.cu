@@ -57,11 +57,12 @@ struct TopkState {
     uint32_t wsum[32];
 };
 
-// Block-wide: given hist[0..NB), find the bin d where the count of keys at or
-// above it first reaches kk (scanning from the top bin down).
+// Block-wide (NT threads): given hist[0..NB), find the bin d where the count
+// of keys at or above it first reaches kk (scanning from the top bin down).
+template <int NT = TK_THREADS>
 __device__ void find_digit(const uint32_t *hist, int NB, int kk, TopkState &st) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int BPT = (NB + TK_THREADS - 1) / TK_THREADS;
+    const int BPT = (NB + NT - 1) / NT;
     const int b0 = tid * BPT;
     uint32_t local = 0;
     for (int j = 0; j < BPT; j++)
@@ -76,7 +77,7 @@ __device__ void find_digit(const uint32_t *hist, int NB, int kk, TopkState &st) 
     if (lane == 0) st.wsum[warp] = x;
     __syncthreads();
     uint32_t warps_above = 0, all = 0;
-    for (int w = 0; w < TK_THREADS / 32; w++) {
+    for (int w = 0; w < NT / 32; w++) {
         all += st.wsum[w];
         if (w > warp) warps_above += st.wsum[w];
     }
@@ -195,13 +196,14 @@ __device__ void bitonic_sort_asc(int32_t *v, int n) {
     }
 }
 
-__global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    __shared__ TopkState st;
-    TopkShared sh{reinterpret_cast<uint32_t *>(smem_raw),
-                  reinterpret_cast<uint64_t *>(smem_raw + TK_HIST * 4),
-                  reinterpret_cast<int32_t *>(smem_raw + TK_HIST * 4 + TK_BUF * 8)};
-    const int64_t r = blockIdx.x;
+__device__ __forceinline__ TopkShared topk_shared(uint8_t *smem_raw) {
+    return TopkShared{reinterpret_cast<uint32_t *>(smem_raw),
+                      reinterpret_cast<uint64_t *>(smem_raw + TK_HIST * 4),
+                      reinterpret_cast<int32_t *>(smem_raw + TK_HIST * 4 + TK_BUF * 8)};
+}
+
+// The whole selection of row r by one CTA of TK_THREADS threads.
+__device__ void topk_row_full(const TopkArgs &a, int64_t r, TopkShared sh, TopkState &st) {
     int64_t nv = a.n;
     if (a.n_valid) {
         const int64_t v = a.n_valid[r];
@@ -296,9 +298,299 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
     for (int i = threadIdx.x; i < a.k; i += TK_THREADS) out[i] = i < nsel ? sh.sel[i] : -1;
 }
 
+__global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __shared__ TopkState st;
+    topk_row_full(a, blockIdx.x, topk_shared(smem_raw), st);
+}
+
+// ------------------------------------------------------------------ histogram-fed selection
+// Used inside the decode step, where every candidate list is in ascending
+// position order (block ids, or the pool's blocks expanded to tokens): there,
+// "lower position" equals "lower candidate index", so the ranking key can
+// carry the index instead of the position, and the output (ascending
+// positions) is the selected indices in index order.
+//
+// The producer of the scores (scan, pool gather, Reindex) has already counted
+// every candidate of row r into hist[r][top 12 bits of its key]. From the
+// histogram, the compaction kernel (many CTAs per row) sends the index of
+// every candidate above the threshold bin straight to the selection and the
+// threshold bin's keys to a tie list (one atomic per warp per list); the
+// finish kernel (one CTA per row) resolves the tie list in shared memory,
+// marks the selected indices in a bitmap and writes them in index order via a
+// block-wide prefix count, and clears the row's histogram and counters for the
+// next producer. A tie list longer than its buffer falls back to the whole
+// single-CTA selection of the row.
+constexpr int TC_THREADS = 256;
+constexpr int TC_SLICE = 4096;  // candidates per compaction CTA
+constexpr int TC_PER = TC_SLICE / TC_THREADS;
+constexpr int64_t TF_MAX_N = (int64_t)TK_BUF * 2 * 32;  // bitmap capacity of the finish
+
+struct TopkHistWs {
+    uint32_t *hist;  // [R][4096]
+    int *cnt;        // [R][2]: selected, ties
+    int32_t *sel;    // [R][k] candidate indices
+    uint64_t *tie;   // [R][TK_BUF] keys
+};
+
+// Copy a 4096-bin histogram row from global to shared memory with 16-byte
+// loads issued together (one round trip), NT threads.
+template <int NT>
+__device__ __forceinline__ void load_hist(uint32_t *dst, const uint32_t *src) {
+    constexpr int PER = TK_HIST / 4 / NT;
+    uint4 v[PER];
+#pragma unroll
+    for (int u = 0; u < PER; u++) v[u] = reinterpret_cast<const uint4 *>(src)[u * NT + threadIdx.x];
+#pragma unroll
+    for (int u = 0; u < PER; u++) reinterpret_cast<uint4 *>(dst)[u * NT + threadIdx.x] = v[u];
+}
+
+// Copy n elements of T from global to shared memory, 8 loads in flight per thread.
+template <typename T>
+__device__ __forceinline__ void load_batched(T *dst, const T *src, int n) {
+    for (int i0 = 0; i0 < n; i0 += 8 * TK_THREADS) {
+        T v[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            const int i = i0 + u * TK_THREADS + threadIdx.x;
+            if (i < n) v[u] = src[i];
+        }
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            const int i = i0 + u * TK_THREADS + threadIdx.x;
+            if (i < n) dst[i] = v[u];
+        }
+    }
+}
+
+__device__ __forceinline__ int warp_incl_scan(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+    }
+    return v;
+}
+
+__global__ void __launch_bounds__(TC_THREADS) topk_compact_kernel(TopkArgs a, TopkHistWs ws) {
+    __shared__ uint32_t hist[TK_HIST];
+    __shared__ TopkState st;
+    const int64_t r = blockIdx.y;
+    int64_t nv = a.n;
+    if (a.n_valid) {
+        const int64_t v = a.n_valid[r];
+        nv = v < 0 ? 0 : (v < a.n ? v : a.n);
+    }
+    const int64_t i_beg = (int64_t)blockIdx.x * TC_SLICE;
+    if (i_beg >= nv) return;
+    load_hist<TC_THREADS>(hist, ws.hist + r * TK_HIST);
+    __syncthreads();
+    find_digit<TC_THREADS>(hist, TK_HIST, a.k, st);
+    const bool all = st.total <= (uint32_t)a.k;
+    const uint64_t d = (uint64_t)st.digit;
+    const bool vec = ((r * a.n) % 4 == 0) && aligned16(a.score) &&
+                     (a.cand_pos == nullptr || aligned16(a.cand_pos));
+    uint64_t key[TC_PER];
+    uint32_t selm = 0, tiem = 0;
+#pragma unroll
+    for (int u = 0; u < TC_PER / 4; u++) {
+        const int64_t i0 = i_beg + 4 * ((int64_t)u * TC_THREADS + threadIdx.x);
+        uint64_t pk[4];
+        bool ok[4];
+        load_cand4(a, r, i0, nv, vec, pk, ok);
+#pragma unroll
+        for (int v = 0; v < 4; v++) {
+            const int j = 4 * u + v;
+            // index-keyed: the ordered score bits above the inverted index
+            key[j] = (pk[v] & 0xFFFFFFFF00000000ull) | (uint32_t)(~(uint32_t)(i0 + v));
+            const uint64_t bin = key[j] >> 52;
+            if (ok[v] && (all || bin > d)) selm |= 1u << j;
+            else if (ok[v] && bin == d) tiem |= 1u << j;
+        }
+    }
+    const int ns = __popc(selm), nt = __popc(tiem);
+    const int is = warp_incl_scan(ns), it = warp_incl_scan(nt);
+    const int lane = threadIdx.x & 31;
+    int bs = 0, bt = 0;
+    if (lane == 31) {
+        if (is) bs = atomicAdd(ws.cnt + 2 * r, is);
+        if (it) bt = atomicAdd(ws.cnt + 2 * r + 1, it);
+    }
+    bs = __shfl_sync(0xffffffffu, bs, 31) + is - ns;
+    bt = __shfl_sync(0xffffffffu, bt, 31) + it - nt;
+#pragma unroll
+    for (int j = 0; j < TC_PER; j++) {
+        if (selm & (1u << j)) {
+            if (bs < a.k) ws.sel[r * a.k + bs] = (int32_t)(~(uint32_t)key[j]);
+            bs++;
+        } else if (tiem & (1u << j)) {
+            if (bt < TK_BUF) ws.tie[r * TK_BUF + bt] = key[j];
+            bt++;
+        }
+    }
+}
+
+// Block-wide exclusive prefix sum of v over TK_THREADS threads.
+__device__ __forceinline__ int block_excl_scan(int v, TopkState &st) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int incl = warp_incl_scan(v);
+    if (lane == 31) st.wsum[warp] = (uint32_t)incl;
+    __syncthreads();
+    int off = 0;
+    for (int w = 0; w < warp; w++) off += (int)st.wsum[w];
+    __syncthreads();
+    return off + incl - v;
+}
+
+__global__ void __launch_bounds__(TK_THREADS, 1) topk_finish_kernel(TopkArgs a, TopkHistWs ws) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __shared__ TopkState st;
+    TopkShared sh = topk_shared(smem_raw);
+    const int64_t r = blockIdx.x;
+    load_hist<TK_THREADS>(sh.hist, ws.hist + r * TK_HIST);
+    const int nsel0 = min(ws.cnt[2 * r], a.k);
+    const int ntie = ws.cnt[2 * r + 1];
+    if (threadIdx.x == 0) {
+        st.prefix = 0;
+        st.mask = 0;
+        st.nsel = 0;
+        st.nbuf = 0;
+    }
+    __syncthreads();
+    find_digit(sh.hist, TK_HIST, a.k, st);
+    const bool all = st.total <= (uint32_t)a.k;
+    int32_t *out = a.out + r * a.k;
+    if ((!all && ntie > TK_BUF) || a.n > TF_MAX_N) {
+        __syncthreads();
+        topk_row_full(a, r, sh, st);  // rare: the tie list or the bitmap does not fit
+    } else {
+        load_batched(sh.sel, ws.sel + r * a.k, nsel0);
+        if (threadIdx.x == 0) st.nsel = nsel0;
+        if (!all) {
+            const int nbuf = ntie;
+            load_batched(sh.buf, ws.tie + r * TK_BUF, nbuf);
+            if (threadIdx.x == 0) {
+                st.kk = a.k - (int)st.above;
+                st.prefix = (uint64_t)st.digit << 52;
+                st.mask = (uint64_t)(TK_HIST - 1) << 52;
+            }
+            __syncthreads();
+            if (st.match != (uint32_t)st.kk) {
+                // remaining digits: 10 + 10 bits finish the score, then the index bytes
+                const int widths[6] = {10, 10, 8, 8, 8, 8};
+                int shift = 52;
+                for (int wi = 0; wi < 6; wi++) {
+                    shift -= widths[wi];
+                    const int NB = 1 << widths[wi];
+                    smem_hist_pass(sh.buf, nbuf, sh.hist, NB, shift, st.prefix, st.mask);
+                    find_digit(sh.hist, NB, st.kk, st);
+                    if (threadIdx.x == 0) {
+                        st.kk -= (int)st.above;
+                        st.prefix |= (uint64_t)st.digit << shift;
+                        st.mask |= (uint64_t)(NB - 1) << shift;
+                    }
+                    __syncthreads();
+                    if (st.match == (uint32_t)st.kk) break;
+                }
+            }
+            const uint64_t p = st.prefix, m = st.mask;
+            for (int i = threadIdx.x; i < nbuf; i += TK_THREADS) {
+                const uint64_t key = sh.buf[i];
+                if ((key & m) >= p) {
+                    const int s2 = atomicAdd(&st.nsel, 1);
+                    if (s2 < TK_MAXK) sh.sel[s2] = (int32_t)(~(uint32_t)key);
+                }
+            }
+        }
+        __syncthreads();
+        const int nsel = min(st.nsel, a.k);
+        // emit in index order: bitmap over [0, n), block prefix count of set bits
+        uint32_t *bm = reinterpret_cast<uint32_t *>(sh.buf);
+        const int nwords = (int)((a.n + 31) / 32);
+        for (int i = threadIdx.x; i < nwords; i += TK_THREADS) bm[i] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < nsel; i += TK_THREADS) {
+            const int idx = sh.sel[i];
+            atomicOr(&bm[idx >> 5], 1u << (idx & 31));
+        }
+        __syncthreads();
+        const int per = (nwords + TK_THREADS - 1) / TK_THREADS;
+        const int w0 = threadIdx.x * per;
+        int c = 0;
+        for (int i = 0; i < per; i++)
+            if (w0 + i < nwords) c += __popc(bm[w0 + i]);
+        int rank = block_excl_scan(c, st);
+        for (int i = 0; i < per; i++) {
+            if (w0 + i >= nwords) break;
+            uint32_t bits = bm[w0 + i];
+            while (bits) {
+                const int b = __ffs(bits) - 1;
+                bits &= bits - 1;
+                const int64_t idx = (int64_t)(w0 + i) * 32 + b;
+                if (rank < a.k) out[rank] = a.cand_pos ? a.cand_pos[r * a.n + idx] : (int32_t)idx;
+                rank++;
+            }
+        }
+        for (int i = nsel + threadIdx.x; i < a.k; i += TK_THREADS) out[i] = -1;
+    }
+    // leave the histogram and counters of this row clear for the next producer
+    __syncthreads();
+    for (int b = threadIdx.x; b < TK_HIST; b += TK_THREADS) ws.hist[r * TK_HIST + b] = 0;
+    if (threadIdx.x < 2) ws.cnt[2 * r + threadIdx.x] = 0;
+}
+
 }  // namespace csa2
 
 using namespace csa2;
+
+namespace csa2 {
+
+size_t topk_hist_ws_bytes(int R, int k) {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    return up((size_t)R * TK_HIST * 4) + up((size_t)R * 2 * 4) + up((size_t)R * k * 4) +
+           up((size_t)R * TK_BUF * 8);
+}
+
+static TopkHistWs topk_hist_ws(void *base, int R, int k) {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    char *p = static_cast<char *>(base);
+    TopkHistWs w;
+    w.hist = reinterpret_cast<uint32_t *>(p);
+    p += up((size_t)R * TK_HIST * 4);
+    w.cnt = reinterpret_cast<int *>(p);
+    p += up((size_t)R * 2 * 4);
+    w.sel = reinterpret_cast<int32_t *>(p);
+    p += up((size_t)R * k * 4);
+    w.tie = reinterpret_cast<uint64_t *>(p);
+    return w;
+}
+
+
+// Selection of rows whose histogram (hist[r][4096], counters zero) the score
+// producer has filled: compaction over many CTAs, then one finishing CTA per row.
+int launch_topk_from_hist(const float *score, const int32_t *cand_pos, const int32_t *n_valid,
+                          int R, int64_t n, int k, int32_t *out, void *ws, cudaStream_t s) {
+    if (R == 0) return CSA2_OK;
+    if (R > 65535) return CSA2_ERR_SHAPE;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)TK_SMEM) != cudaSuccess ||
+            cudaFuncSetAttribute(topk_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)TK_SMEM) != cudaSuccess)
+            return CSA2_ERR_CUDA;
+        attr = true;
+    }
+    TopkArgs a{score, cand_pos, n_valid, R, n, k, out};
+    TopkHistWs w = topk_hist_ws(ws, R, k);
+    const int64_t slices = (n + TC_SLICE - 1) / TC_SLICE;
+    topk_compact_kernel<<<dim3((unsigned)slices, (unsigned)R), TC_THREADS, 0, s>>>(a, w);
+    topk_finish_kernel<<<R, TK_THREADS, TK_SMEM, s>>>(a, w);
+    return launch_status();
+}
+
+}  // namespace csa2
 
 extern "C" size_t csa2_topk_workspace_size(int R, int64_t n, int k) {
     (void)R;

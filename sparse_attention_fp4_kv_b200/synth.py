@@ -22,6 +22,8 @@ FULL, REINDEX, REUSE = 0, 1, 2
 # Reuse, the other four 1 Reindex + 3 Reuse ("DeepSeek-V4.1-Flash: 890 Bytes
 # Per Token, 437x Smaller KV Cache", CSA2 section).
 DECODER_MODES = [FULL, REUSE, REUSE, REUSE] + [REINDEX, REUSE, REUSE, REUSE] * 4
+# Encoder CSA2 layers: three groups of six, each 1 Full + 5 Reuse (same section).
+ENCODER_MODES = ([FULL] + [REUSE] * 5) * 3
 
 
 @dataclass
@@ -73,6 +75,10 @@ WORKLOADS = {
     "decoder_stack20_b4_ctx1m": Workload("decoder_stack20_b4_ctx1m", B=4, ctx=1048576, C=512,
                                          Hq=64, H_idx=16, D_idx=128, modes=list(DECODER_MODES),
                                          outlier_frac=0.01, outlier_mult=16.0, seed=3),
+    # The 18 CSA2 encoder layers of a decode step, batch 4, 1M context.
+    "encoder_stack18_b4_ctx1m": Workload("encoder_stack18_b4_ctx1m", B=4, ctx=1048576, C=512,
+                                         Hq=64, H_idx=16, D_idx=128, modes=list(ENCODER_MODES),
+                                         outlier_frac=0.01, outlier_mult=16.0, seed=5),
     # Chunked prefill: 4096 new tokens appended to a 65536-token context.
     "prefill_4096_at_64k": Workload("prefill_4096_at_64k", B=1, ctx=65536 + 4096, C=512, Hq=64,
                                     H_idx=16, D_idx=128, modes=[FULL], outlier_frac=0.01,

@@ -103,11 +103,13 @@ class DecodeWorkload:
 
     def launches_per_step(self) -> int:
         """libcsa2 kernels one step launches: the append, then per Full layer
-        scan + pool top-k + gather + token top-k, per Reindex layer rescoring +
-        top-k, and one attention kernel per layer."""
+        the scan, pool selection (compaction + finish), gather and token
+        selection (compaction + finish); per Reindex layer the rescoring and
+        token selection (compaction + finish); one attention kernel per layer.
+        (The per-step histogram clear is a memset, not counted.)"""
         n = 1
         for m in self.modes:
-            n += {synth.FULL: 4, synth.REINDEX: 2, synth.REUSE: 0}[m] + 1
+            n += {synth.FULL: 6, synth.REINDEX: 3, synth.REUSE: 0}[m] + 1
         return n
 
     # ---- algorithmic bytes of one step (what the method must move)

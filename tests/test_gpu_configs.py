@@ -78,6 +78,7 @@ def _free():
     ("decoder_group1_b8_ctx128k", dict(B=5, ctx=3001)),
     ("decoder_group1_b8_ctx128k", dict(B=1, ctx=100)),
     ("reindex_group_b32_ctx256k", dict(B=3, ctx=50001)),
+    ("encoder_stack18_b4_ctx1m", dict(B=2, ctx=40007)),
     ("full_b1_ctx4k", dict(B=2, ctx=777)),
 ])
 def test_scaled_stack(name, kw):

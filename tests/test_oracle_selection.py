@@ -41,6 +41,11 @@ def test_schedules_match_pages():
     name = {"F": oracle.FULL, "Ri": oracle.REINDEX, "U": oracle.REUSE}
     assert oracle.decoder_schedule() == [name[m] for m in L["decoder"]]
     assert oracle.encoder_schedule() == [name[m] for m in L["encoder"]]
+    # the benchmark workloads use the same schedules
+    from sparse_attention_fp4_kv_b200 import synth
+    code = {synth.FULL: oracle.FULL, synth.REINDEX: oracle.REINDEX, synth.REUSE: oracle.REUSE}
+    assert [code[m] for m in synth.DECODER_MODES] == oracle.decoder_schedule()
+    assert [code[m] for m in synth.ENCODER_MODES] == oracle.encoder_schedule()
     assert len(oracle.decoder_schedule()) == 20 and len(oracle.encoder_schedule()) == 18
 
 

@@ -20,6 +20,9 @@ POOL_BLOCKS = 2048
 BLOCK_TOKENS = 8
 TOPK = 512
 N_WIN = 128
+# Rows of at most this many candidates are selected by one single-CTA kernel
+# inside the decode step; longer rows take a compaction and a finishing kernel.
+TOPK_SHORT_ROW = 65536
 MODE_FULL, MODE_REINDEX, MODE_REUSE = 0, 1, 2
 
 

@@ -505,17 +505,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                 float v[32];
                 tmem_ld_16x32x2_32(row_addr + c0, v);
                 tmem_ld_wait();
-                const uint32_t dst = base + STG_OFF + (uint32_t)(((c0 >> 6) * HQ + h) * 64 + half * 32) * 4;
-                // rotate the 8 pieces by lane so that a warp's stores spread over the banks
+                // 16-byte chunk j of a head's 256-byte row sits at position j ^ (h & 7):
+                // lanes 0-7 of a warp hold 8 consecutive heads, so each store of
+                // the warp covers all 8 bank groups
+                const uint32_t row = base + STG_OFF + (uint32_t)(((c0 >> 6) * HQ + h) * 256);
 #pragma unroll
-                for (int u0 = 0; u0 < 8; u0++) {
-                    const int u = (u0 + (lane & 7)) & 7;
-                    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                    for (int q = 0; q < 8; q++)
-                        if (q == u && ok) f = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                    st_shared_v4(dst + 16 * u, make_uint4(__float_as_uint(f.x), __float_as_uint(f.y),
-                                                          __float_as_uint(f.z), __float_as_uint(f.w)));
+                for (int u = 0; u < 8; u++) {
+                    const int j = (half * 8 + u) ^ (h & 7);
+                    const uint4 w = ok ? make_uint4(__float_as_uint(v[4 * u]), __float_as_uint(v[4 * u + 1]),
+                                                    __float_as_uint(v[4 * u + 2]), __float_as_uint(v[4 * u + 3]))
+                                       : make_uint4(0u, 0u, 0u, 0u);
+                    st_shared_v4(row + 16 * j, w);
                 }
             }
             if (warp < 4 && half == 0) {
@@ -539,8 +539,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         cluster_sync();  // all partial results of this row are in the slot
 
         // ---- combine: this CTA owns channels [64 rank, 64 rank + 64); the slice
-        // of source r is contiguous at xo[r][rank]. Thread t takes elements
-        // e = 4 (t + 256 u), u = 0..3, of the [64 heads][64 channels] slice.
+        // of source r is contiguous at xo[r][rank]. Thread t takes the 16-byte
+        // chunks e = 4 (t + 256 u), u = 0..3, of the [64 heads][64 channels]
+        // slice; chunk position p of head hh holds channels 4 (p ^ (hh & 7)).
         {
             float *wts = reinterpret_cast<float *>(sm + PHI_OFF);  // [64 heads][8] weight / den
             if (tid < HQ) {
@@ -575,7 +576,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int u = 0; u < 4; u++) {
                 const int e = 4 * (tid + 256 * u);
-                const int hh = e >> 6, ch = e & 63;
+                const int hh = e >> 6, ch = 4 * (((e & 63) >> 2) ^ (hh & 7));
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int r = 0; r < CL; r++) {
@@ -589,7 +590,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                     acc;
             }
         }
-        cluster_sync();  // the slot, the tiles and TMEM are free for the next row
+        // the slot, the tiles and TMEM are free for the next row (after the last
+        // row nothing is shared any more: the exchange went through global memory)
+        if (bq + (int64_t)gridDim.y < rows) cluster_sync();
     }
     if (!ok && tid == 0) atomicExch(&g_attn_error, 1);
     if (warp == 0) {

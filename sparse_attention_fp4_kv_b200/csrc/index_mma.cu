@@ -14,9 +14,13 @@
 //               and K (256 keys x 128 B) into a 4-stage shared-memory ring;
 //   warp 1      TMEM owner and MMA issuer: 4 MMAs (M = 128, N = 256, K = 32)
 //               per stage into one of two 256-column int32 accumulators;
-//   warps 2-5   epilogue: one query row per thread; int32 -> fp32 (RNE) times the
-//               key scale, causal mask (t <= query position), token scores and
-//               8-token block maxima written straight to global memory.
+//   warps 2-5   epilogue: one query row per thread, 32 key columns at a time
+//               (the next TMEM load in flight while the current chunk is
+//               stored); int32 -> fp32 (RNE) times the key scale (staged once
+//               per tile in shared memory), causal mask (t <= query position),
+//               8-token block maxima as 16-byte stores, token scores
+//               transposed through shared memory so that every warp store
+//               writes whole 128-byte row segments.
 // Tiles are ordered query-tile fastest, so the CTAs working at the same time
 // share key tiles in L2 and every key tile is read from HBM about once.
 // All mbarrier waits are bounded; on timeout the kernel records an error flag
@@ -34,7 +38,13 @@ constexpr int A_STAGE = BM * BK;
 constexpr int B_STAGE = BN * BK;
 constexpr int THREADS = 192;
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE) + BAR_BYTES + 1024;
+// per epilogue warp: a [32 rows][36] fp32 transpose tile (rows padded by 16 B so
+// that both its row-wise and column-wise 16-byte accesses are conflict-free)
+// and the tile's 256 key scales
+constexpr int STG_LD = 36;
+constexpr int EPI_WARP = 32 * STG_LD * 4 + BN * 4;
+constexpr int EPI_OFF = STAGES * (A_STAGE + B_STAGE) + BAR_BYTES;
+constexpr int SMEM_BYTES = EPI_OFF + 4 * EPI_WARP + 1024;
 constexpr long WAIT_LIMIT = 1L << 26;
 
 __device__ int g_imma_error = 0;
@@ -50,7 +60,8 @@ struct Args {
     int32_t *n_blk;
     int m_tiles, n_tiles;
     int64_t tiles;
-    bool vec;  // token rows and key scales are 16-byte aligned
+    bool vec;      // token rows and key scales are 16-byte aligned
+    bool vec_blk;  // block-score rows are 16-byte aligned
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -102,6 +113,8 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
                      bar)
                  : "memory");
 }
+// 32 consecutive columns of this warp's 32 TMEM lanes; the registers are valid
+// after tmem_ld_wait(v), which names them so that no use moves above the wait.
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, int (&v)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
@@ -113,7 +126,17 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, int (&v)[32])
           "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
           "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
         : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait(int (&v)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                   "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                   "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]), "+r"(v[16]), "+r"(v[17]),
+                   "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]), "+r"(v[22]), "+r"(v[23]),
+                   "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]), "+r"(v[29]),
+                   "+r"(v[30]), "+r"(v[31])
+                 :
+                 : "memory");
 }
 
 struct Tile {
@@ -222,10 +245,32 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ---------------- epilogue: thread = query row of the tile
         const int ew = warp & 3;  // TMEM lane quadrant this warp may access
         const int mrow = ew * 32 + lane;
+        float *stg = reinterpret_cast<float *>(sm + EPI_OFF + ew * EPI_WARP);  // [32][STG_LD]
+        float *scs = stg + 32 * STG_LD;                                        // [BN]
         int buf = 0;
         uint32_t tphase = 0;
         for (int64_t t = blockIdx.x; t < a.tiles; t += gridDim.x) {
             const Tile tl = tile_of(a, t);
+            {
+                // the tile's key scales (the same for every row), 8 per lane
+                __syncwarp();  // every lane is done with the previous tile's scales
+                const int64_t k0 = (int64_t)tl.n0 + 8 * lane;
+                const float *src = a.kscale + (int64_t)tl.b * a.cap + k0;
+                float4 s0, s1;
+                if (a.vec && k0 + 8 <= a.cap) {
+                    s0 = __ldg(reinterpret_cast<const float4 *>(src));
+                    s1 = __ldg(reinterpret_cast<const float4 *>(src) + 1);
+                } else {
+                    float e[8];
+#pragma unroll
+                    for (int j = 0; j < 8; j++) e[j] = k0 + j < a.cap ? __ldg(src + j) : 0.0f;
+                    s0 = make_float4(e[0], e[1], e[2], e[3]);
+                    s1 = make_float4(e[4], e[5], e[6], e[7]);
+                }
+                reinterpret_cast<float4 *>(scs)[2 * lane] = s0;
+                reinterpret_cast<float4 *>(scs)[2 * lane + 1] = s1;
+                __syncwarp();
+            }
             if (!mbar_wait(tfull + 8 * buf, tphase)) break;
             tc_fence_after();
             const int m = tl.m0 + mrow;
@@ -236,62 +281,84 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (V > a.cap) V = a.cap;
             }
             const int64_t bq = (int64_t)tl.b * a.Nq + m;
-            const float *ks = a.kscale + (int64_t)tl.b * a.cap;
+            const int64_t bq0 = (int64_t)tl.b * a.Nq + tl.m0 + ew * 32;  // row of lane 0
+            const uint32_t trow = tmem + ((uint32_t)(ew * 32) << 16) + buf * BN;
+            int S[32];
+            tmem_ld_32x32b_x32(trow, S);
 #pragma unroll 1
             for (int c = 0; c < BN / 32; c++) {
-                int S[32];
-                // warp-synchronous TMEM load first; the per-row work below is predicated
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(ew * 32) << 16) + buf * BN + c * 32, S);
+                tmem_ld_wait(S);
                 const int64_t t0 = (int64_t)tl.n0 + c * 32;
+                float v[32];
+#pragma unroll
+                for (int u = 0; u < 8; u++) {
+                    const float4 sc = reinterpret_cast<const float4 *>(scs + c * 32)[u];
+                    v[4 * u] = (t0 + 4 * u < V) ? __fmul_rn(__int2float_rn(S[4 * u]), sc.x) : -INFINITY;
+                    v[4 * u + 1] =
+                        (t0 + 4 * u + 1 < V) ? __fmul_rn(__int2float_rn(S[4 * u + 1]), sc.y) : -INFINITY;
+                    v[4 * u + 2] =
+                        (t0 + 4 * u + 2 < V) ? __fmul_rn(__int2float_rn(S[4 * u + 2]), sc.z) : -INFINITY;
+                    v[4 * u + 3] =
+                        (t0 + 4 * u + 3 < V) ? __fmul_rn(__int2float_rn(S[4 * u + 3]), sc.w) : -INFINITY;
+                }
+                if (c + 1 < BN / 32) {
+                    tmem_ld_32x32b_x32(trow + (c + 1) * 32, S);  // overlaps the stores below
+                } else {
+                    // every column of this accumulator has been read: hand it back
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(tempty + 8 * buf);
+                }
                 if (row_ok && t0 < V) {
-                    float sc[32];
-                    if (a.vec && t0 + 32 <= a.cap) {
-#pragma unroll
-                        for (int u = 0; u < 8; u++) {
-                            const float4 f = __ldg(reinterpret_cast<const float4 *>(ks + t0) + u);
-                            sc[4 * u] = f.x;
-                            sc[4 * u + 1] = f.y;
-                            sc[4 * u + 2] = f.z;
-                            sc[4 * u + 3] = f.w;
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; j++)
-                            sc[j] = (t0 + j < a.cap) ? __ldg(ks + t0 + j) : 0.0f;
-                    }
-                    float v[32];
-#pragma unroll
-                    for (int j = 0; j < 32; j++)
-                        v[j] = (t0 + j < V) ? __fmul_rn(__int2float_rn(S[j]), sc[j]) : -INFINITY;
-                    if (a.tok) {
-                        float *dst = a.tok + bq * a.cap + t0;
-                        if (a.vec && t0 + 32 <= V) {
-#pragma unroll
-                            for (int u = 0; u < 8; u++)
-                                reinterpret_cast<float4 *>(dst)[u] =
-                                    make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-                        } else {
-                            for (int j = 0; j < 32; j++)
-                                if (t0 + j < V) dst[j] = v[j];
-                        }
-                    }
+                    // maxima of the four 8-token blocks of this row in the chunk
+                    float mx[4];
 #pragma unroll
                     for (int q = 0; q < 4; q++) {
-                        const int64_t j0 = t0 + 8 * q;
-                        if (j0 < V) {
-                            float mx = v[8 * q];
+                        mx[q] = v[8 * q];
 #pragma unroll
-                            for (int u = 1; u < 8; u++) mx = fmaxf(mx, v[8 * q + u]);
-                            a.blk[bq * a.nblk_cap + j0 / 8] = mx;
-                        }
+                        for (int u = 1; u < 8; u++) mx[q] = fmaxf(mx[q], v[8 * q + u]);
+                    }
+                    float *bd = a.blk + bq * a.nblk_cap + t0 / 8;
+                    if (a.vec_blk && t0 + 32 <= V) {
+                        *reinterpret_cast<float4 *>(bd) = make_float4(mx[0], mx[1], mx[2], mx[3]);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; q++)
+                            if (t0 + 8 * q < V) bd[q] = mx[q];
                     }
                 }
-                __syncwarp();
+                if (a.tok) {
+                    // transpose through shared memory: each warp store then covers
+                    // 4 rows x 128 contiguous bytes
+#pragma unroll
+                    for (int u = 0; u < 8; u++)
+                        reinterpret_cast<float4 *>(stg + lane * STG_LD)[u] =
+                            make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                    __syncwarp();
+                    const int64_t rem = row_ok ? V - t0 : 0;
+                    const int nv_l = rem <= 0 ? 0 : (rem >= 32 ? 32 : (int)rem);
+                    const int q = lane & 7;
+#pragma unroll
+                    for (int i = 0; i < 8; i++) {
+                        const int rr = 4 * i + (lane >> 3);
+                        const int nvr = __shfl_sync(0xffffffffu, nv_l, rr);
+                        if (4 * q < nvr) {
+                            const float4 f = reinterpret_cast<const float4 *>(stg + rr * STG_LD)[q];
+                            float *dst = a.tok + (bq0 + rr) * a.cap + t0 + 4 * q;
+                            if (a.vec && 4 * q + 4 <= nvr) {
+                                *reinterpret_cast<float4 *>(dst) = f;
+                            } else {
+                                dst[0] = f.x;
+                                if (4 * q + 1 < nvr) dst[1] = f.y;
+                                if (4 * q + 2 < nvr) dst[2] = f.z;
+                                if (4 * q + 3 < nvr) dst[3] = f.w;
+                            }
+                        }
+                    }
+                    __syncwarp();
+                }
             }
             if (row_ok && tl.n0 == 0 && a.n_blk) a.n_blk[bq] = (int32_t)((V + 7) / 8);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tempty + 8 * buf);
             if (++buf == 2) {
                 buf = 0;
                 tphase ^= 1;
@@ -347,6 +414,7 @@ int launch_index_mma(const int8_t *q, const int8_t *k, const float *kscale, cons
     a.n_tiles = (int)((cap + BN - 1) / BN);
     a.tiles = (int64_t)B * a.m_tiles * a.n_tiles;
     a.vec = (cap % 4 == 0) && aligned(kscale, 16) && (tok == nullptr || aligned(tok, 16));
+    a.vec_blk = (a.nblk_cap % 4 == 0) && aligned(blk, 16);
     const int64_t grid = a.tiles < num_sms() ? a.tiles : num_sms();
     index_mma_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, s>>>(mq, mk, a);
     return launch_status();

@@ -162,11 +162,12 @@ __device__ void global_hist_pass(const TopkArgs &a, int64_t r, int64_t nv, bool 
     __syncthreads();
 }
 
+template <int NT = TK_THREADS>
 __device__ void smem_hist_pass(const uint64_t *buf, int nbuf, uint32_t *hist, int NB, int shift,
                                uint64_t prefix, uint64_t mask) {
-    for (int b = threadIdx.x; b < NB; b += TK_THREADS) hist[b] = 0;
+    for (int b = threadIdx.x; b < NB; b += NT) hist[b] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < nbuf; i += TK_THREADS) {
+    for (int i = threadIdx.x; i < nbuf; i += NT) {
         const uint64_t key = buf[i];
         if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (uint64_t)(NB - 1)], 1u);
     }
@@ -431,7 +432,7 @@ __global__ void __launch_bounds__(TC_THREADS) topk_compact_kernel(TopkArgs a, To
     }
 }
 
-// Block-wide exclusive prefix sum of v over TK_THREADS threads.
+// Block-wide exclusive prefix sum of v over the CTA's threads.
 __device__ __forceinline__ int block_excl_scan(int v, TopkState &st) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int incl = warp_incl_scan(v);
@@ -441,6 +442,81 @@ __device__ __forceinline__ int block_excl_scan(int v, TopkState &st) {
     for (int w = 0; w < warp; w++) off += (int)st.wsum[w];
     __syncthreads();
     return off + incl - v;
+}
+
+// Resolves the threshold bin's tie list (nbuf keys in sh.buf, all inside bin
+// st.digit of the first 12-bit digit): the remaining digits run over the list
+// and the tie keys at or above the k-th are appended to sh.sel as indices.
+// st.above and st.match come from find_digit over the first-digit histogram.
+__device__ void resolve_ties(TopkShared sh, TopkState &st, int nbuf, int k) {
+    if (threadIdx.x == 0) {
+        st.kk = k - (int)st.above;
+        st.prefix = (uint64_t)st.digit << 52;
+        st.mask = (uint64_t)(TK_HIST - 1) << 52;
+    }
+    __syncthreads();
+    if (st.match != (uint32_t)st.kk) {
+        // remaining digits: 10 + 10 bits finish the score, then the index bytes
+        const int widths[6] = {10, 10, 8, 8, 8, 8};
+        int shift = 52;
+        for (int wi = 0; wi < 6; wi++) {
+            shift -= widths[wi];
+            const int NB = 1 << widths[wi];
+            smem_hist_pass(sh.buf, nbuf, sh.hist, NB, shift, st.prefix, st.mask);
+            find_digit(sh.hist, NB, st.kk, st);
+            if (threadIdx.x == 0) {
+                st.kk -= (int)st.above;
+                st.prefix |= (uint64_t)st.digit << shift;
+                st.mask |= (uint64_t)(NB - 1) << shift;
+            }
+            __syncthreads();
+            if (st.match == (uint32_t)st.kk) break;
+        }
+    }
+    const uint64_t p = st.prefix, m = st.mask;
+    for (int i = threadIdx.x; i < nbuf; i += TK_THREADS) {
+        const uint64_t key = sh.buf[i];
+        if ((key & m) >= p) {
+            const int s2 = atomicAdd(&st.nsel, 1);
+            if (s2 < TK_MAXK) sh.sel[s2] = (int32_t)(~(uint32_t)key);
+        }
+    }
+}
+
+// Writes the selected candidate indices sh.sel[0..nsel) of row r in index
+// order (their positions, or the indices themselves without cand_pos), then
+// -1 up to k: a bitmap over [0, n) in sh.buf and a block prefix count of its
+// set bits give every selected index its output slot.
+__device__ void emit_in_index_order(const TopkArgs &a, int64_t r, TopkShared sh, TopkState &st,
+                                    int nsel) {
+    int32_t *out = a.out + r * a.k;
+    uint32_t *bm = reinterpret_cast<uint32_t *>(sh.buf);
+    const int nwords = (int)((a.n + 31) / 32);
+    for (int i = threadIdx.x; i < nwords; i += TK_THREADS) bm[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < nsel; i += TK_THREADS) {
+        const int idx = sh.sel[i];
+        atomicOr(&bm[idx >> 5], 1u << (idx & 31));
+    }
+    __syncthreads();
+    const int per = (nwords + TK_THREADS - 1) / TK_THREADS;
+    const int w0 = threadIdx.x * per;
+    int c = 0;
+    for (int i = 0; i < per; i++)
+        if (w0 + i < nwords) c += __popc(bm[w0 + i]);
+    int rank = block_excl_scan(c, st);
+    for (int i = 0; i < per; i++) {
+        if (w0 + i >= nwords) break;
+        uint32_t bits = bm[w0 + i];
+        while (bits) {
+            const int b = __ffs(bits) - 1;
+            bits &= bits - 1;
+            const int64_t idx = (int64_t)(w0 + i) * 32 + b;
+            if (rank < a.k) out[rank] = a.cand_pos ? a.cand_pos[r * a.n + idx] : (int32_t)idx;
+            rank++;
+        }
+    }
+    for (int i = nsel + threadIdx.x; i < a.k; i += TK_THREADS) out[i] = -1;
 }
 
 __global__ void __launch_bounds__(TK_THREADS, 1) topk_finish_kernel(TopkArgs a, TopkHistWs ws) {
@@ -460,7 +536,6 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_finish_kernel(TopkArgs a, 
     __syncthreads();
     find_digit(sh.hist, TK_HIST, a.k, st);
     const bool all = st.total <= (uint32_t)a.k;
-    int32_t *out = a.out + r * a.k;
     if ((!all && ntie > TK_BUF) || a.n > TF_MAX_N) {
         __syncthreads();
         topk_row_full(a, r, sh, st);  // rare: the tie list or the bitmap does not fit
@@ -468,76 +543,101 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_finish_kernel(TopkArgs a, 
         load_batched(sh.sel, ws.sel + r * a.k, nsel0);
         if (threadIdx.x == 0) st.nsel = nsel0;
         if (!all) {
-            const int nbuf = ntie;
-            load_batched(sh.buf, ws.tie + r * TK_BUF, nbuf);
-            if (threadIdx.x == 0) {
-                st.kk = a.k - (int)st.above;
-                st.prefix = (uint64_t)st.digit << 52;
-                st.mask = (uint64_t)(TK_HIST - 1) << 52;
-            }
-            __syncthreads();
-            if (st.match != (uint32_t)st.kk) {
-                // remaining digits: 10 + 10 bits finish the score, then the index bytes
-                const int widths[6] = {10, 10, 8, 8, 8, 8};
-                int shift = 52;
-                for (int wi = 0; wi < 6; wi++) {
-                    shift -= widths[wi];
-                    const int NB = 1 << widths[wi];
-                    smem_hist_pass(sh.buf, nbuf, sh.hist, NB, shift, st.prefix, st.mask);
-                    find_digit(sh.hist, NB, st.kk, st);
-                    if (threadIdx.x == 0) {
-                        st.kk -= (int)st.above;
-                        st.prefix |= (uint64_t)st.digit << shift;
-                        st.mask |= (uint64_t)(NB - 1) << shift;
-                    }
-                    __syncthreads();
-                    if (st.match == (uint32_t)st.kk) break;
-                }
-            }
-            const uint64_t p = st.prefix, m = st.mask;
-            for (int i = threadIdx.x; i < nbuf; i += TK_THREADS) {
-                const uint64_t key = sh.buf[i];
-                if ((key & m) >= p) {
-                    const int s2 = atomicAdd(&st.nsel, 1);
-                    if (s2 < TK_MAXK) sh.sel[s2] = (int32_t)(~(uint32_t)key);
-                }
-            }
+            load_batched(sh.buf, ws.tie + r * TK_BUF, ntie);
+            resolve_ties(sh, st, ntie, a.k);
         }
         __syncthreads();
-        const int nsel = min(st.nsel, a.k);
-        // emit in index order: bitmap over [0, n), block prefix count of set bits
-        uint32_t *bm = reinterpret_cast<uint32_t *>(sh.buf);
-        const int nwords = (int)((a.n + 31) / 32);
-        for (int i = threadIdx.x; i < nwords; i += TK_THREADS) bm[i] = 0;
-        __syncthreads();
-        for (int i = threadIdx.x; i < nsel; i += TK_THREADS) {
-            const int idx = sh.sel[i];
-            atomicOr(&bm[idx >> 5], 1u << (idx & 31));
-        }
-        __syncthreads();
-        const int per = (nwords + TK_THREADS - 1) / TK_THREADS;
-        const int w0 = threadIdx.x * per;
-        int c = 0;
-        for (int i = 0; i < per; i++)
-            if (w0 + i < nwords) c += __popc(bm[w0 + i]);
-        int rank = block_excl_scan(c, st);
-        for (int i = 0; i < per; i++) {
-            if (w0 + i >= nwords) break;
-            uint32_t bits = bm[w0 + i];
-            while (bits) {
-                const int b = __ffs(bits) - 1;
-                bits &= bits - 1;
-                const int64_t idx = (int64_t)(w0 + i) * 32 + b;
-                if (rank < a.k) out[rank] = a.cand_pos ? a.cand_pos[r * a.n + idx] : (int32_t)idx;
-                rank++;
-            }
-        }
-        for (int i = nsel + threadIdx.x; i < a.k; i += TK_THREADS) out[i] = -1;
+        emit_in_index_order(a, r, sh, st, min(st.nsel, a.k));
     }
     // leave the histogram and counters of this row clear for the next producer
     __syncthreads();
     for (int b = threadIdx.x; b < TK_HIST; b += TK_THREADS) ws.hist[r * TK_HIST + b] = 0;
     if (threadIdx.x < 2) ws.cnt[2 * r + threadIdx.x] = 0;
+}
+
+// Rows of at most TS_MAX_N candidates skip the global lists: one CTA per row
+// takes the threshold bin from the producer's histogram, reads its candidates
+// once (16 per thread per pass, one shared atomic per warp per list), keeps
+// the indices above the bin and the bin's keys in shared memory, resolves the
+// ties and emits in index order. A tie list longer than its buffer falls back
+// to the whole single-CTA selection. Clears the row's histogram.
+constexpr int64_t TS_MAX_N = 65536;
+constexpr int TS_PER = 16;
+
+__global__ void __launch_bounds__(TK_THREADS, 1) topk_row_hist_kernel(TopkArgs a, uint32_t *ghist) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __shared__ TopkState st;
+    TopkShared sh = topk_shared(smem_raw);
+    const int64_t r = blockIdx.x;
+    const int lane = threadIdx.x & 31;
+    int64_t nv = a.n;
+    if (a.n_valid) {
+        const int64_t v = a.n_valid[r];
+        nv = v < 0 ? 0 : (v < a.n ? v : a.n);
+    }
+    load_hist<TK_THREADS>(sh.hist, ghist + r * TK_HIST);
+    if (threadIdx.x == 0) {
+        st.prefix = 0;
+        st.mask = 0;
+        st.nsel = 0;
+        st.nbuf = 0;
+    }
+    __syncthreads();
+    find_digit(sh.hist, TK_HIST, a.k, st);
+    const bool all = st.total <= (uint32_t)a.k;
+    const uint32_t d = (uint32_t)st.digit;
+    const bool vec = ((r * a.n) % 4 == 0) && aligned16(a.score) &&
+                     (a.cand_pos == nullptr || aligned16(a.cand_pos));
+    for (int64_t b0 = 0; b0 < nv; b0 += (int64_t)TK_THREADS * TS_PER) {
+        uint32_t ob[TS_PER];  // order-preserving score bits
+        uint32_t selm = 0, tiem = 0;
+#pragma unroll
+        for (int u = 0; u < TS_PER / 4; u++) {
+            const int64_t i0 = b0 + 4 * ((int64_t)u * TK_THREADS + threadIdx.x);
+            uint64_t pk[4];
+            bool ok[4];
+            load_cand4(a, r, i0, nv, vec, pk, ok);
+#pragma unroll
+            for (int v = 0; v < 4; v++) {
+                const int j = 4 * u + v;
+                ob[j] = (uint32_t)(pk[v] >> 32);
+                const uint32_t bin = ob[j] >> 20;
+                if (ok[v] && (all || bin > d)) selm |= 1u << j;
+                else if (ok[v] && bin == d) tiem |= 1u << j;
+            }
+        }
+        const int ns = __popc(selm), nt = __popc(tiem);
+        const int is = warp_incl_scan(ns), it = warp_incl_scan(nt);
+        int bs = 0, bt = 0;
+        if (lane == 31) {
+            if (is) bs = atomicAdd(&st.nsel, is);
+            if (it) bt = atomicAdd(&st.nbuf, it);
+        }
+        bs = __shfl_sync(0xffffffffu, bs, 31) + is - ns;
+        bt = __shfl_sync(0xffffffffu, bt, 31) + it - nt;
+#pragma unroll
+        for (int j = 0; j < TS_PER; j++) {
+            const uint32_t i = (uint32_t)(b0 + 4 * ((j >> 2) * TK_THREADS + threadIdx.x) + (j & 3));
+            if (selm & (1u << j)) {
+                if (bs < TK_MAXK) sh.sel[bs] = (int32_t)i;
+                bs++;
+            } else if (tiem & (1u << j)) {
+                if (bt < TK_BUF) sh.buf[bt] = ((uint64_t)ob[j] << 32) | (uint32_t)~i;
+                bt++;
+            }
+        }
+    }
+    __syncthreads();
+    if (!all && st.nbuf > TK_BUF) {
+        __syncthreads();
+        topk_row_full(a, r, sh, st);  // rare: the tie list does not fit
+    } else {
+        if (!all) resolve_ties(sh, st, st.nbuf, a.k);
+        __syncthreads();
+        emit_in_index_order(a, r, sh, st, min(st.nsel, a.k));
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b < TK_HIST; b += TK_THREADS) ghist[r * TK_HIST + b] = 0;
 }
 
 }  // namespace csa2
@@ -568,7 +668,8 @@ static TopkHistWs topk_hist_ws(void *base, int R, int k) {
 
 
 // Selection of rows whose histogram (hist[r][4096], counters zero) the score
-// producer has filled: compaction over many CTAs, then one finishing CTA per row.
+// producer has filled: one CTA per row for short rows, else compaction over
+// many CTAs, then one finishing CTA per row.
 int launch_topk_from_hist(const float *score, const int32_t *cand_pos, const int32_t *n_valid,
                           int R, int64_t n, int k, int32_t *out, void *ws, cudaStream_t s) {
     if (R == 0) return CSA2_OK;
@@ -578,12 +679,18 @@ int launch_topk_from_hist(const float *score, const int32_t *cand_pos, const int
         if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)TK_SMEM) != cudaSuccess ||
             cudaFuncSetAttribute(topk_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)TK_SMEM) != cudaSuccess ||
+            cudaFuncSetAttribute(topk_row_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)TK_SMEM) != cudaSuccess)
             return CSA2_ERR_CUDA;
         attr = true;
     }
     TopkArgs a{score, cand_pos, n_valid, R, n, k, out};
     TopkHistWs w = topk_hist_ws(ws, R, k);
+    if (n <= TS_MAX_N) {
+        topk_row_hist_kernel<<<R, TK_THREADS, TK_SMEM, s>>>(a, w.hist);
+        return launch_status();
+    }
     const int64_t slices = (n + TC_SLICE - 1) / TC_SLICE;
     topk_compact_kernel<<<dim3((unsigned)slices, (unsigned)R), TC_THREADS, 0, s>>>(a, w);
     topk_finish_kernel<<<R, TK_THREADS, TK_SMEM, s>>>(a, w);

@@ -103,13 +103,19 @@ class DecodeWorkload:
 
     def launches_per_step(self) -> int:
         """libcsa2 kernels one step launches: the append, then per Full layer
-        the scan, pool selection (compaction + finish), gather and token
-        selection (compaction + finish); per Reindex layer the rescoring and
-        token selection (compaction + finish); one attention kernel per layer.
-        (The per-step histogram clear is a memset, not counted.)"""
+        the scan, the pool selection, the gather and the token selection; per
+        Reindex layer the rescoring and the token selection; one attention
+        kernel per layer. A selection is one kernel for rows of at most
+        TOPK_SHORT_ROW candidates, else two (compaction + finish). (The
+        per-step histogram clear is a memset, not counted.)"""
+        def sel(n):
+            return 1 if n <= csa2.TOPK_SHORT_ROW else 2
+        nblk = (self.kv_fp4.shape[1] + 7) // 8
+        pooled = csa2.POOL_BLOCKS * csa2.BLOCK_TOKENS
         n = 1
         for m in self.modes:
-            n += {synth.FULL: 6, synth.REINDEX: 3, synth.REUSE: 0}[m] + 1
+            n += {synth.FULL: 2 + sel(nblk) + sel(pooled), synth.REINDEX: 1 + sel(pooled),
+                  synth.REUSE: 0}[m] + 1
         return n
 
     # ---- algorithmic bytes of one step (what the method must move)

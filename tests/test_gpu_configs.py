@@ -88,6 +88,40 @@ def test_scaled_stack(name, kw):
     _free()
 
 
+@pytest.mark.parametrize("levels", [1, 3])
+def test_stack_tie_heavy_keys(levels):
+    """Coarse indexer keys give many equal scores: with levels=1 every score is
+    zero (the whole candidate list ties and the order falls to positions); with
+    levels=3 the threshold bins hold long runs of equal scores."""
+    wl = _workload("decoder_stack20_b4_ctx1m", B=2, ctx=30011)
+    g = torch.Generator(device="cuda").manual_seed(levels)
+    wl.k_idx.copy_(torch.randint(0, levels, wl.k_idx.shape, generator=g, device="cuda",
+                                 dtype=torch.int8))
+    wl.k_scale.fill_(1.0)
+    _check(wl, range(wl.w.B))
+    del wl
+    _free()
+
+
+@pytest.mark.parametrize("ctx", [30000, 600000])
+def test_launches_per_step_matches_profiler(ctx):
+    """The kernel count the benchmark reports equals the libcsa2 kernels the
+    CUDA profiler sees in one step (600K tokens: the pool selection's rows are
+    long enough to take two kernels)."""
+    wl = _workload("decoder_stack20_b4_ctx1m", B=1, ctx=ctx)
+    wl.step()
+    torch.cuda.synchronize()
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        wl.step()
+        torch.cuda.synchronize()
+    names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+    ours = [n for n in names if "csa2::" in n]
+    assert len(ours) == wl.launches_per_step(), sorted(set(ours))
+    del wl
+    _free()
+
+
 def test_decode_step_is_deterministic():
     wl = _workload("decoder_stack20_b4_ctx1m", B=2, ctx=30000)
     wl.step()

@@ -333,7 +333,8 @@ def test_sparse_attention_prefill_positions(B):
 
 
 # ----------------------------------------------------------------------------- a9 prefill scan
-@pytest.mark.parametrize("Nq,ctx0,H,D", [(300, 5000, 16, 128), (129, 2048, 8, 128), (40, 777, 4, 64)])
+@pytest.mark.parametrize("Nq,ctx0,H,D", [(300, 5000, 16, 128), (129, 2048, 8, 128), (40, 777, 4, 64),
+                                         (256, 7936, 16, 128)])
 def test_index_full_multi_query_tensor_core_path(B, Nq, ctx0, H, D):
     """Nq >= 16 runs the tcgen05 kind::i8 kernel: causal scores and block maxima
     must equal the oracle bit for bit, and equal the per-query dp4a scan."""

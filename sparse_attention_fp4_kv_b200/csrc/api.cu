@@ -124,7 +124,7 @@ extern "C" int csa2_decode_stack(const csa2_layer *layers, int n_layers,
     cudaStream_t s = (cudaStream_t)stream;
     if (kv_new_bf16) {
         st = launch_kv_append((const uint16_t *)kv_new_bf16, B, 1, C, ctx_len, -1, cap, kv_fp4,
-                              kv_sf, s);
+                              kv_sf, s, true);
         if (st) return st;
     }
     // the selection histograms and counters start the step at zero (every
@@ -165,9 +165,15 @@ extern "C" int csa2_decode_stack(const csa2_layer *layers, int n_layers,
             if (st) return st;
             cur = L.topk;
         }
-        st = csa2_sparse_attn_decode(L.q, kv_fp4, kv_sf, cap, cur, kTopK, L.swa, swa_pos0,
-                                     swa_rows, nullptr, CSA2_N_WIN, B, 1, Hq, C, softmax_scale,
-                                     L.out, w.attn, w.attn_bytes, stream);
+        // Every kernel of the step is launched with programmatic stream
+        // serialization. A Reuse layer's attention follows the previous layer's
+        // attention, and its indices come from an earlier selection kernel, so
+        // it gathers and dequantizes its rows before waiting for that kernel;
+        // Q and the window rows (the layer's own inputs) are read after the wait.
+        AttnArgs aa{L.q, kv_fp4, kv_sf, cap, cur, kTopK, L.swa, swa_pos0, swa_rows, nullptr,
+                    CSA2_N_WIN, B, 1, Hq, C, softmax_scale, L.out, w.attn, true,
+                    L.mode == CSA2_MODE_REUSE};
+        st = attn_checked_launch(aa, w.attn_bytes, s);
         if (st) return st;
     }
     return CSA2_OK;

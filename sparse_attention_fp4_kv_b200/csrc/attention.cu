@@ -20,6 +20,8 @@
 namespace csa2 {
 
 __global__ void __launch_bounds__(256) attn_general_kernel(AttnArgs a) {
+    grid_dep_wait();
+    grid_dep_launch();
     extern __shared__ float sm[];
     const int C = a.C;
     float *qs = sm;            // [C]
@@ -125,8 +127,7 @@ int launch_attn_general(const AttnArgs &a, cudaStream_t s) {
     }
     const int64_t grid = (int64_t)a.B * a.Nq * a.Hq;
     if (grid > INT32_MAX) return CSA2_ERR_SHAPE;
-    attn_general_kernel<<<(unsigned)grid, 256, smem, s>>>(a);
-    return launch_status();
+    return launch_kernel(a.pdl, attn_general_kernel, dim3((unsigned)grid), dim3(256), smem, s, a);
 }
 
 }  // namespace csa2
@@ -143,23 +144,28 @@ extern "C" int csa2_sparse_attn_decode(const void *q_bf16, const uint8_t *kv_fp4
                                        int swa_rows, const int64_t *q_pos, int n_win, int B,
                                        int Nq, int Hq, int C, float softmax_scale, float *out,
                                        void *ws, size_t ws_bytes, void *stream) {
-    if (!q_bf16 || !kv_fp4 || !kv_sf || !out) return CSA2_ERR_NULL;
-    if (K > 0 && !topk) return CSA2_ERR_NULL;
-    if (n_win > 0 && swa_rows > 0 && (!swa_bf16 || !swa_pos0)) return CSA2_ERR_NULL;
-    if (!q_pos && !swa_pos0) return CSA2_ERR_NULL;
-    if (B < 0 || Nq < 0 || cap < 1 || C < 32 || C > 1024 || C % 32 || Hq < 1 || Hq > 256 ||
-        K < 0 || K > 4096 || n_win < 0 || n_win > 4096 || swa_rows < 0)
-        return CSA2_ERR_SHAPE;
-    if (!aligned(q_bf16, 16) || (swa_bf16 && !aligned(swa_bf16, 16)) || !aligned(kv_fp4, 8))
-        return CSA2_ERR_ALIGN;
-    if (ws_bytes < attn_workspace_bytes(B, Nq, Hq, C, K, n_win)) return CSA2_ERR_WORKSPACE;
-    if ((int64_t)B * Nq == 0) return CSA2_OK;
     AttnArgs a{q_bf16, kv_fp4, kv_sf, cap, topk, K, swa_bf16, swa_pos0, swa_rows, q_pos,
-               n_win, B, Nq, Hq, C, softmax_scale, out, ws};
-    return launch_attn(a, (cudaStream_t)stream);
+               n_win, B, Nq, Hq, C, softmax_scale, out, ws, false, false};
+    return attn_checked_launch(a, ws_bytes, (cudaStream_t)stream);
 }
 
 namespace csa2 {
+
+int attn_checked_launch(const AttnArgs &a, size_t ws_bytes, cudaStream_t s) {
+    if (!a.q || !a.kv_fp4 || !a.kv_sf || !a.out) return CSA2_ERR_NULL;
+    if (a.K > 0 && !a.topk) return CSA2_ERR_NULL;
+    if (a.n_win > 0 && a.swa_rows > 0 && (!a.swa || !a.swa_pos0)) return CSA2_ERR_NULL;
+    if (!a.q_pos && !a.swa_pos0) return CSA2_ERR_NULL;
+    if (a.B < 0 || a.Nq < 0 || a.cap < 1 || a.C < 32 || a.C > 1024 || a.C % 32 || a.Hq < 1 ||
+        a.Hq > 256 || a.K < 0 || a.K > 4096 || a.n_win < 0 || a.n_win > 4096 || a.swa_rows < 0)
+        return CSA2_ERR_SHAPE;
+    if (!aligned(a.q, 16) || (a.swa && !aligned(a.swa, 16)) || !aligned(a.kv_fp4, 8))
+        return CSA2_ERR_ALIGN;
+    if (ws_bytes < attn_workspace_bytes(a.B, a.Nq, a.Hq, a.C, a.K, a.n_win))
+        return CSA2_ERR_WORKSPACE;
+    if ((int64_t)a.B * a.Nq == 0) return CSA2_OK;
+    return launch_attn(a, s);
+}
 
 // The tensor-core kernel exchanges per-CTA partial results through the
 // workspace; the general kernel needs none. The size covers the tensor-core

@@ -21,6 +21,14 @@ struct AttnArgs {
     float scale;
     float *out;            // fp32 [B][Nq][Hq][C]
     void *ws;
+    // Launch with programmatic stream serialization (the kernel may start
+    // while the previous kernel on the stream runs; it waits for that grid
+    // before reading Q or the window rows and before writing anything).
+    bool pdl;
+    // With pdl: topk, kv_fp4/kv_sf and swa_pos0 were written two or more
+    // kernels earlier, so the selected rows may be gathered and dequantized
+    // before the wait.
+    bool prefetch;
 };
 
 // Sliding-window rows of query bq: rows [row0, row0 + n) of the SWA tensor,
@@ -48,6 +56,9 @@ __device__ __forceinline__ AttnWindow attn_window(const AttnArgs &a, int b, int6
 }
 
 size_t attn_workspace_bytes(int B, int Nq, int Hq, int C, int K, int n_win);
+// Validates the arguments of a sparse-attention call (status codes of
+// csa2_sparse_attn_decode) and launches it.
+int attn_checked_launch(const AttnArgs &a, size_t ws_bytes, cudaStream_t s);
 int launch_attn(const AttnArgs &a, cudaStream_t s);
 int launch_attn_general(const AttnArgs &a, cudaStream_t s);
 bool attn_tc_supported(const AttnArgs &a);

@@ -302,6 +302,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int64_t rows = (int64_t)a.B * a.Nq;
     uint32_t ld_phase = 0;
     bool ok = true;
+    // dependency on the previous kernel of the stream: at once, or (prefetch)
+    // after the first row's selected FP4 rows are gathered and dequantized
+    bool waited = !a.prefetch;
+    if (waited) {
+        grid_dep_wait();
+        grid_dep_launch();
+    }
 
     // The cluster walks query rows blockIdx.y, blockIdx.y + gridDim.y, ...
     for (int64_t bq = blockIdx.y; bq < rows; bq += gridDim.y) {
@@ -345,7 +352,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 st_shared_v4(base + K_OFF + (pg >> 3) * K_CHUNK + sw128(j, pg & 7),
                              make_uint4(0, 0, 0, 0));
         }
-        if (tid == 0) {
+        // Q and this CTA's window rows by TMA (one thread)
+        auto issue_q_swa = [&]() {
             const int qrow = (int)(bq * HQ);
 #pragma unroll
             for (int cc = 0; cc < 8; cc++)
@@ -356,7 +364,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int cc = 0; cc < 8; cc++)
                     tma_load_2d(base + K_OFF + cc * K_CHUNK + (js + bx * SWA_BOX) * 128, &tswa,
                                 cc * 64, wrow0 + bx * SWA_BOX, bar_ld);
-        }
+        };
+        if (waited && tid == 0) issue_q_swa();
         for (int i = tid; i < T * 18; i += THREADS) {  // (slot, 16-byte piece of its 288 B)
             const int j = i / 18, pc = i - j * 18;
             if (slot_kind[j] != 1) continue;
@@ -366,11 +375,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             cp_async16(base + FP4_STAGE_OFF + j * 288 + pc * 16, src);
         }
         cp_async_wait_all();
-        if (ok) ok = mbar_wait(bar_ld, ld_phase);
-        ld_phase ^= 1;
         __syncthreads();
 
-        // ---- dequantize the FP4 rows into the KV tile
+        // ---- dequantize the FP4 rows into the KV tile (slots of kind 1; the
+        // TMA copies write only window slots, so this need not wait for them)
         const uint8_t *stage = sm + FP4_STAGE_OFF;
         for (int i = tid; i < T * 32; i += THREADS) {  // (slot, 16-channel group)
             const int j = i >> 5, g = i & 31;
@@ -391,6 +399,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             st_shared_v4(d1, make_uint4(wds[4], wds[5], wds[6], wds[7]));
         }
         fence_proxy_async();
+        if (!waited) {
+            grid_dep_wait();
+            grid_dep_launch();
+            waited = true;
+            if (tid == 0) issue_q_swa();
+        }
+        if (ok) ok = mbar_wait(bar_ld, ld_phase);
+        ld_phase ^= 1;
         __syncthreads();
 
         // ---- S = Q K^T  (M = 64, N = 80, K = 512) into TMEM lanes 16..31
@@ -638,13 +654,15 @@ int launch_attn_tc(const AttnArgs &a, cudaStream_t s) {
     cfg.blockDim = dim3(tc::THREADS, 1, 1);
     cfg.dynamicSmemBytes = tc::SMEM_BYTES;
     cfg.stream = s;
-    cudaLaunchAttribute attr_cl[1];
+    cudaLaunchAttribute attr_cl[2];
     attr_cl[0].id = cudaLaunchAttributeClusterDimension;
     attr_cl[0].val.clusterDim.x = tc::CL;
     attr_cl[0].val.clusterDim.y = 1;
     attr_cl[0].val.clusterDim.z = 1;
+    attr_cl[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr_cl[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr_cl;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = a.pdl ? 2 : 1;
     if (cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel, tq, tswa, a) != cudaSuccess)
         return CSA2_ERR_CUDA;
     return launch_status();

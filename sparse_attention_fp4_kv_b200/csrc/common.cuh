@@ -23,6 +23,40 @@ inline int launch_status() {
     return cudaGetLastError() == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- dependent launches
+// Kernels of one decode step may be launched with programmatic stream
+// serialization: the next kernel's CTAs can be scheduled while the previous
+// kernel on the stream is still running. Every kernel therefore calls
+// grid_dep_wait() before its first access to memory that the previous kernel
+// may read or write (the wait returns once that grid has completed and its
+// writes are visible), and grid_dep_launch() right after it, so that a
+// kernel which starts early can rely on everything launched two or more
+// kernels before it being complete. Both are no-ops in a kernel launched
+// without the attribute.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch `kernel`, with programmatic stream serialization when pdl is true.
+template <typename... KArgs, typename... Args>
+inline int launch_kernel(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                         cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) != cudaSuccess)
+        return CSA2_ERR_CUDA;
+    return launch_status();
+}
+
 inline int num_sms() {
     static int n = 0;
     if (n == 0) {
@@ -118,7 +152,8 @@ __device__ __forceinline__ int64_t visible_len(const int64_t *ctx_len, const int
 
 // FP4 append with positions pos_base[b] + pos_offset + i (kv_append.cu).
 int launch_kv_append(const uint16_t *kv, int B, int n_new, int C, const int64_t *pos_base,
-                     int64_t pos_offset, int64_t cap, uint8_t *fp4, uint8_t *sf, cudaStream_t s);
+                     int64_t pos_offset, int64_t cap, uint8_t *fp4, uint8_t *sf, cudaStream_t s,
+                     bool pdl = false);
 
 // First-digit histogram bin of a score (top 12 bits of its order-preserving
 // key), shared by the score producers and the histogram-fed top-k.
@@ -126,7 +161,9 @@ constexpr int kHistBins = 4096;
 __device__ __forceinline__ uint32_t hist_bin(float score) { return f32_order_key(score) >> 20; }
 
 // Histogram-fed top-k (topk.cu): the workspace starts with hist[R][4096] and
-// two counters per row, all zero before the producer runs.
+// two counters per row, all zero before the producer runs. This launcher and
+// the three score producers below serve the decode step only and launch with
+// programmatic stream serialization.
 size_t topk_hist_ws_bytes(int R, int k);
 int launch_topk_from_hist(const float *score, const int32_t *cand_pos, const int32_t *n_valid,
                           int R, int64_t n, int k, int32_t *out, void *ws, cudaStream_t s);

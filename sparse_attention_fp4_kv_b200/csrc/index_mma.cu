@@ -155,6 +155,8 @@ __device__ __forceinline__ Tile tile_of(const Args &a, int64_t t) {
 __global__ void __launch_bounds__(THREADS, 1)
     index_mma_kernel(const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_k, Args a) {
+    grid_dep_wait();
+    grid_dep_launch();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;

@@ -171,6 +171,8 @@ struct ScanArgs {
 
 template <int HD>
 __global__ void __launch_bounds__(256) index_full_kernel(ScanArgs a) {
+    grid_dep_wait();
+    grid_dep_launch();
     using RS = RowShape<HD>;
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -206,6 +208,8 @@ __global__ void __launch_bounds__(256) index_full_kernel(ScanArgs a) {
 }
 
 __global__ void __launch_bounds__(256) index_full_generic_kernel(ScanArgs a) {
+    grid_dep_wait();
+    grid_dep_launch();
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -263,6 +267,8 @@ __device__ __forceinline__ int64_t reindex_block(const ReindexArgs &a, int64_t b
 // in flight.
 template <int HD>
 __global__ void __launch_bounds__(256) index_reindex_kernel(ReindexArgs a) {
+    grid_dep_wait();
+    grid_dep_launch();
     using RS = RowShape<HD>;
     const int lane = threadIdx.x & 31;
     const int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -297,6 +303,8 @@ __global__ void __launch_bounds__(256) index_reindex_kernel(ReindexArgs a) {
 }
 
 __global__ void __launch_bounds__(256) index_reindex_generic_kernel(ReindexArgs a) {
+    grid_dep_wait();
+    grid_dep_launch();
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -336,6 +344,8 @@ __global__ void __launch_bounds__(256) pool_gather_kernel(const float *__restric
                                                           const int64_t *q_pos, int B, int Nq,
                                                           int P, int64_t cap, float *pscore,
                                                           int32_t *ppos, uint32_t *hist) {
+    grid_dep_wait();
+    grid_dep_launch();
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t total = (int64_t)B * Nq * P * 8;
     if (idx >= total) return;
@@ -372,15 +382,14 @@ static int persistent_grid(K kernel, int threads, int64_t items_warps) {
 
 using namespace csa2;
 
-static int dispatch_scan(const ScanArgs &a, cudaStream_t s) {
+static int dispatch_scan(const ScanArgs &a, cudaStream_t s, bool pdl) {
     const int64_t items = (int64_t)a.B * a.Nq * a.nblk_cap;
     const int T = 256;
     switch (a.HD) {
 #define CSA2_SCAN_CASE(HDV)                                                             \
     case HDV: {                                                                         \
         int g = persistent_grid(index_full_kernel<HDV>, T, items);                      \
-        index_full_kernel<HDV><<<g, T, 0, s>>>(a);                                      \
-        break;                                                                          \
+        return launch_kernel(pdl, index_full_kernel<HDV>, dim3(g), dim3(T), 0, s, a);  \
     }
         CSA2_SCAN_CASE(128)
         CSA2_SCAN_CASE(256)
@@ -391,13 +400,12 @@ static int dispatch_scan(const ScanArgs &a, cudaStream_t s) {
 #undef CSA2_SCAN_CASE
         default: {
             int g = persistent_grid(index_full_generic_kernel, T, items);
-            index_full_generic_kernel<<<g, T, 0, s>>>(a);
+            return launch_kernel(pdl, index_full_generic_kernel, dim3(g), dim3(T), 0, s, a);
         }
     }
-    return launch_status();
 }
 
-static int dispatch_reindex(const ReindexArgs &a, cudaStream_t s) {
+static int dispatch_reindex(const ReindexArgs &a, cudaStream_t s, bool pdl) {
     const int64_t items = (int64_t)a.B * a.Nq * a.P;
     const int T = 256;
     switch (a.HD) {
@@ -405,8 +413,8 @@ static int dispatch_reindex(const ReindexArgs &a, cudaStream_t s) {
     case HDV: {                                                                         \
         const int64_t g = (items + T / 32 - 1) / (T / 32);                              \
         if (g > INT32_MAX) return CSA2_ERR_SHAPE;                                       \
-        index_reindex_kernel<HDV><<<(unsigned)g, T, 0, s>>>(a);                         \
-        break;                                                                          \
+        return launch_kernel(pdl, index_reindex_kernel<HDV>, dim3((unsigned)g), dim3(T), 0, s, \
+                             a);                                                        \
     }
         CSA2_RI_CASE(128)
         CSA2_RI_CASE(256)
@@ -417,10 +425,9 @@ static int dispatch_reindex(const ReindexArgs &a, cudaStream_t s) {
 #undef CSA2_RI_CASE
         default: {
             int g = persistent_grid(index_reindex_generic_kernel, T, items);
-            index_reindex_generic_kernel<<<g, T, 0, s>>>(a);
+            return launch_kernel(pdl, index_reindex_generic_kernel, dim3(g), dim3(T), 0, s, a);
         }
     }
-    return launch_status();
 }
 
 static int check_indexer_common(const int8_t *q_idx, const int8_t *k_idx, const float *k_scale,
@@ -446,7 +453,7 @@ extern "C" int csa2_index_full(const int8_t *q_idx, const int8_t *k_idx, const f
                                 tok_score, blk_score, n_blk, (cudaStream_t)stream);
     ScanArgs a{q_idx, k_idx, k_scale, ctx_len, q_pos, B, Nq, H * D, cap, (cap + 7) / 8,
                tok_score, blk_score, n_blk, nullptr};
-    return dispatch_scan(a, (cudaStream_t)stream);
+    return dispatch_scan(a, (cudaStream_t)stream, false);
 }
 
 extern "C" int csa2_index_reindex(const int8_t *q_idx, const int8_t *k_idx, const float *k_scale,
@@ -460,7 +467,7 @@ extern "C" int csa2_index_reindex(const int8_t *q_idx, const int8_t *k_idx, cons
     if ((int64_t)B * Nq * P == 0) return CSA2_OK;
     ReindexArgs a{q_idx, k_idx, k_scale, pool, ctx_len, q_pos, B, Nq, H * D, P, cap,
                   pool_score, pool_pos, nullptr};
-    return dispatch_reindex(a, (cudaStream_t)stream);
+    return dispatch_reindex(a, (cudaStream_t)stream, false);
 }
 
 extern "C" int csa2_pool_gather(const float *tok_score, const int32_t *pool,
@@ -487,7 +494,7 @@ int launch_index_full_hist(const int8_t *q_idx, const int8_t *k_idx, const float
                            cudaStream_t s) {
     ScanArgs a{q_idx, k_idx, k_scale, ctx_len, nullptr, B, 1, H * D, cap, (cap + 7) / 8,
                tok_score, blk_score, n_blk, hist};
-    return dispatch_scan(a, s);
+    return dispatch_scan(a, s, true);
 }
 
 int launch_pool_gather_hist(const float *tok_score, const int32_t *pool, const int64_t *ctx_len,
@@ -496,9 +503,9 @@ int launch_pool_gather_hist(const float *tok_score, const int32_t *pool, const i
     const int64_t total = (int64_t)B * P * 8;
     if (total == 0) return CSA2_OK;
     const int T = 256;
-    pool_gather_kernel<<<(unsigned)((total + T - 1) / T), T, 0, s>>>(
-        tok_score, pool, ctx_len, nullptr, B, 1, P, cap, pool_score, pool_pos, hist);
-    return launch_status();
+    return launch_kernel(true, pool_gather_kernel, dim3((unsigned)((total + T - 1) / T)), dim3(T), 0,
+                         s, tok_score, pool, ctx_len, nullptr, B, 1, P, cap, pool_score, pool_pos,
+                         hist);
 }
 
 int launch_reindex_hist(const int8_t *q_idx, const int8_t *k_idx, const float *k_scale,
@@ -507,7 +514,7 @@ int launch_reindex_hist(const int8_t *q_idx, const int8_t *k_idx, const float *k
                         cudaStream_t s) {
     ReindexArgs a{q_idx, k_idx, k_scale, pool, ctx_len, nullptr, B, 1, H * D, P, cap,
                   pool_score, pool_pos, hist};
-    return dispatch_reindex(a, s);
+    return dispatch_reindex(a, s, true);
 }
 
 }  // namespace csa2

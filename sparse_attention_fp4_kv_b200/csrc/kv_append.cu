@@ -19,6 +19,8 @@ namespace csa2 {
 __global__ void __launch_bounds__(256) kv_append_fp4_kernel(
     const uint16_t *__restrict__ kv, int B, int n_new, int C, const int64_t *__restrict__ start_pos,
     int64_t pos_offset, int64_t cap, uint8_t *__restrict__ fp4, uint8_t *__restrict__ sf) {
+    grid_dep_wait();
+    grid_dep_launch();
     const int G = C / 16;
     const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t total = (int64_t)B * n_new * G;
@@ -59,15 +61,15 @@ __global__ void __launch_bounds__(256) kv_append_fp4_kernel(
 }
 
 int launch_kv_append(const uint16_t *kv, int B, int n_new, int C, const int64_t *pos_base,
-                     int64_t pos_offset, int64_t cap, uint8_t *fp4, uint8_t *sf, cudaStream_t s) {
+                     int64_t pos_offset, int64_t cap, uint8_t *fp4, uint8_t *sf, cudaStream_t s,
+                     bool pdl) {
     const int64_t total = (int64_t)B * n_new * (C / 16);
     if (total == 0) return CSA2_OK;
     const int threads = 256;
     const int64_t blocks = (total + threads - 1) / threads;
     if (blocks > INT32_MAX) return CSA2_ERR_SHAPE;
-    kv_append_fp4_kernel<<<(unsigned)blocks, threads, 0, s>>>(kv, B, n_new, C, pos_base, pos_offset,
-                                                              cap, fp4, sf);
-    return launch_status();
+    return launch_kernel(pdl, kv_append_fp4_kernel, dim3((unsigned)blocks), dim3(threads), 0, s, kv,
+                         B, n_new, C, pos_base, pos_offset, cap, fp4, sf);
 }
 
 }  // namespace csa2

@@ -300,6 +300,8 @@ __device__ void topk_row_full(const TopkArgs &a, int64_t r, TopkShared sh, TopkS
 }
 
 __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a) {
+    grid_dep_wait();
+    grid_dep_launch();
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ TopkState st;
     topk_row_full(a, blockIdx.x, topk_shared(smem_raw), st);
@@ -375,6 +377,8 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
 }
 
 __global__ void __launch_bounds__(TC_THREADS) topk_compact_kernel(TopkArgs a, TopkHistWs ws) {
+    grid_dep_wait();
+    grid_dep_launch();
     __shared__ uint32_t hist[TK_HIST];
     __shared__ TopkState st;
     const int64_t r = blockIdx.y;
@@ -520,6 +524,8 @@ __device__ void emit_in_index_order(const TopkArgs &a, int64_t r, TopkShared sh,
 }
 
 __global__ void __launch_bounds__(TK_THREADS, 1) topk_finish_kernel(TopkArgs a, TopkHistWs ws) {
+    grid_dep_wait();
+    grid_dep_launch();
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ TopkState st;
     TopkShared sh = topk_shared(smem_raw);
@@ -565,6 +571,8 @@ constexpr int64_t TS_MAX_N = 65536;
 constexpr int TS_PER = 16;
 
 __global__ void __launch_bounds__(TK_THREADS, 1) topk_row_hist_kernel(TopkArgs a, uint32_t *ghist) {
+    grid_dep_wait();
+    grid_dep_launch();
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ TopkState st;
     TopkShared sh = topk_shared(smem_raw);
@@ -687,14 +695,14 @@ int launch_topk_from_hist(const float *score, const int32_t *cand_pos, const int
     }
     TopkArgs a{score, cand_pos, n_valid, R, n, k, out};
     TopkHistWs w = topk_hist_ws(ws, R, k);
-    if (n <= TS_MAX_N) {
-        topk_row_hist_kernel<<<R, TK_THREADS, TK_SMEM, s>>>(a, w.hist);
-        return launch_status();
-    }
+    if (n <= TS_MAX_N)
+        return launch_kernel(true, topk_row_hist_kernel, dim3(R), dim3(TK_THREADS), TK_SMEM, s, a,
+                             w.hist);
     const int64_t slices = (n + TC_SLICE - 1) / TC_SLICE;
-    topk_compact_kernel<<<dim3((unsigned)slices, (unsigned)R), TC_THREADS, 0, s>>>(a, w);
-    topk_finish_kernel<<<R, TK_THREADS, TK_SMEM, s>>>(a, w);
-    return launch_status();
+    const int st = launch_kernel(true, topk_compact_kernel, dim3((unsigned)slices, (unsigned)R),
+                                 dim3(TC_THREADS), 0, s, a, w);
+    if (st) return st;
+    return launch_kernel(true, topk_finish_kernel, dim3(R), dim3(TK_THREADS), TK_SMEM, s, a, w);
 }
 
 }  // namespace csa2

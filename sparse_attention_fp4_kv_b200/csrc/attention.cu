@@ -176,9 +176,14 @@ size_t attn_workspace_bytes(int B, int Nq, int Hq, int C, int K, int n_win) {
     return 0;
 }
 
-// Tensor-core kernel where its shape constraints hold (64 heads, 512 channels,
-// at most 640 keys per query), the general kernel otherwise.
+// Tensor-core kernels where their shape constraints hold (64 heads, 512
+// channels): one CTA per row when there are more rows than the split-key
+// kernel's clusters cover in one wave (and for more than 640 keys per row),
+// the split-key cluster kernel otherwise; the general kernel for other shapes.
 int launch_attn(const AttnArgs &a, cudaStream_t s) {
+    const int64_t rows = (int64_t)a.B * a.Nq;
+    const bool rows_ok = attn_rows_supported(a);
+    if (rows_ok && (rows >= kAttnRowsMin || !attn_tc_supported(a))) return launch_attn_rows(a, s);
     if (attn_tc_supported(a)) return launch_attn_tc(a, s);
     return launch_attn_general(a, s);
 }

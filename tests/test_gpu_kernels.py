@@ -332,6 +332,23 @@ def test_sparse_attention_prefill_positions(B):
     _attention_case(B, 1, ctx, 512, 64, 512, 128, seed=3, q_pos=q_pos, Nq=4)
 
 
+# One CTA per query row: calls with 19 or more rows (and any call with more than
+# 640 keys per row) take the per-row kernel; its window tiles, masked slots and
+# online-softmax rescaling are covered here.
+@pytest.mark.parametrize("Bn,Nq,K,n_win,drop", [(20, 1, 512, 128, 0), (24, 1, 512, 128, 5),
+                                                (2, 1, 1024, 128, 0), (20, 1, 512, 0, 0),
+                                                (3, 8, 576, 64, 7)])
+def test_sparse_attention_one_cta_per_row(B, Bn, Nq, K, n_win, drop):
+    _attention_case(B, Bn, 3000, 512, 64, K, n_win, seed=7 * Bn + K + n_win, Nq=Nq, drop=drop)
+
+
+def test_sparse_attention_one_cta_per_row_causal_positions(B):
+    ctx = 1500
+    pos = [1499, 1400, 900, 200, 127, 126, 64, 63, 5, 0] + list(range(1000, 1030))
+    q_pos = torch.tensor([pos], dtype=torch.int64, device=DEV)
+    _attention_case(B, 1, ctx, 512, 64, 512, 128, seed=11, q_pos=q_pos, Nq=len(pos))
+
+
 # ----------------------------------------------------------------------------- a9 prefill scan
 @pytest.mark.parametrize("Nq,ctx0,H,D", [(300, 5000, 16, 128), (129, 2048, 8, 128), (40, 777, 4, 64),
                                          (256, 7936, 16, 128)])

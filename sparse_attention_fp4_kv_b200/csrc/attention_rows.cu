@@ -25,8 +25,8 @@
 //              scales) straight into registers, issued before the KV tile is
 //              free, then dequantized into it (exact in bf16); the next tile's
 //              indices prefetched meanwhile; window rows by TMA;
-//   warp 8     one thread issues the MMAs: S of the first tile, then P V of
-//              each tile followed by S of the next.
+//   warp 8     one thread issues the MMAs: P V of the oldest tile whose P is
+//              ready, or S of the next tile (up to two tiles ahead).
 // The KV tile is double-buffered; S uses two TMEM buffers; P and O^T one.
 // The reference maximum m of a head only moves when a tile's maximum exceeds
 // it by more than 2^8 (then O^T is rescaled in TMEM); otherwise P may reach
@@ -45,7 +45,8 @@ namespace tr {
 constexpr int HQ = 64;
 constexpr int CH = 512;
 constexpr int TK = 64;  // keys per tile
-constexpr int NSOFT = 128, NLOAD = 128;
+constexpr int NSOFT = 128, NLOAD = 256;
+constexpr int LROWS = TK / (NLOAD / 32);  // rows of a KV tile per load warp
 constexpr int THREADS = NSOFT + NLOAD + 32;
 constexpr int MMA_WARP = (NSOFT + NLOAD) / 32;
 constexpr int BAR_SOFT = 1, BAR_LOAD = 2;  // named barriers of the two groups
@@ -58,14 +59,13 @@ constexpr int P_BYTES = HQ * TK * 2;  // one part (hi or lo) of P: 64 heads x 64
 
 constexpr int Q_OFF = 0;
 constexpr int K_OFF = Q_OFF + Q_BYTES;  // two KV tiles
-constexpr int PHI_OFF = K_OFF + 2 * KT_BYTES;
-constexpr int PLO_OFF = PHI_OFF + P_BYTES;
-constexpr int KIND_OFF = PLO_OFF + P_BYTES;  // uint8 [2][TK]: 0 none, 1 selected, 2 window
+constexpr int P_OFF = K_OFF + 2 * KT_BYTES;  // two P buffers, each hi then lo
+constexpr int KIND_OFF = P_OFF + 4 * P_BYTES;  // uint8 [2][TK]: 0 none, 1 selected, 2 window
 constexpr int ALPHA_OFF = KIND_OFF + 2 * TK; // fp32 [HQ]: rescale factor of O^T
 constexpr int INVL_OFF = ALPHA_OFF + HQ * 4; // fp32 [HQ]: 1 / row sum
 constexpr int BAR_OFF = INVL_OFF + HQ * 4;
 enum { B_QFULL, B_QFREE, B_KFULL0, B_KFULL1, B_KFREE0, B_KFREE1, B_SFULL0, B_SFULL1, B_SFREE0,
-       B_SFREE1, B_PFULL, B_PFREE, B_OFULL, B_OFREE, NBARS };
+       B_SFREE1, B_PFULL0, B_PFULL1, B_PFREE0, B_PFREE1, B_OFULL, B_OFREE, NBARS };
 constexpr int TADDR_OFF = BAR_OFF + NBARS * 8;
 constexpr int ABORT_OFF = TADDR_OFF + 4;
 constexpr int SMEM_USED = ABORT_OFF + 4;
@@ -101,6 +101,18 @@ __device__ __forceinline__ bool try_wait(uint32_t bar, uint32_t parity) {
         "selp.u32 %0, 1, 0, p;\n}"
         : "=r"(done)
         : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+// try_wait with a suspend-time hint (ns): returns at the phase completion or
+// after about the hint.
+__device__ __forceinline__ bool try_wait_hint(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        "selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity), "r"(ns)
         : "memory");
     return done != 0;
 }
@@ -156,8 +168,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(bar(B_SFULL0 + i), 1);
             mbar_init(bar(B_SFREE0 + i), 4);  // one arrival per softmax warp
         }
-        mbar_init(bar(B_PFULL), 1);
-        mbar_init(bar(B_PFREE), 1);
+        for (int i = 0; i < 2; i++) {
+            mbar_init(bar(B_PFULL0 + i), 1);
+            mbar_init(bar(B_PFREE0 + i), 1);
+        }
         mbar_init(bar(B_OFULL), 1);
         mbar_init(bar(B_OFREE), 4);  // one arrival per epilogue warp
         *abort = 0;
@@ -206,8 +220,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const float m_new = (m_ref == -INFINITY || need) ? mt : m_ref;
                 const float alpha = need ? ex2(m_ref - m_new) : 1.0f;
                 const bool any = named_bar_or(BAR_SOFT, NSOFT, need);
-                // P and O^T are free once the previous tile's P V has completed
-                ok = wait_bar(bar(B_PFREE), (g & 1) ^ 1, abort) && ok;
+                // P buffer g & 1 is free once P V of tile g - 2 has completed
+                const uint32_t pb = g & 1;
+                ok = wait_bar(bar(B_PFREE0 + pb), ((g >> 1) & 1) ^ 1, abort) && ok;
+                if (any && g > 0) {
+                    // O^T may change only after P V of tile g - 1 has completed
+                    ok = wait_bar(bar(B_PFREE0 + (pb ^ 1)), ((g - 1) >> 1) & 1, abort) && ok;
+                }
                 if (any) {
                     if (half == 0) alpha_s[h] = alpha;
                     named_bar_sync(BAR_SOFT, NSOFT);
@@ -250,13 +269,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                         lo[u] = pack_bf16x2(p0 - hf.x, p1 - hf.y);
                     }
                     const uint32_t off = sw128(h, half * 4 + q);
-                    st_shared_v4(base + PHI_OFF + off, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-                    st_shared_v4(base + PLO_OFF + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+                    const uint32_t pbase = base + P_OFF + pb * 2 * P_BYTES;
+                    st_shared_v4(pbase + off, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+                    st_shared_v4(pbase + P_BYTES + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
                 }
                 fence_proxy_async();
                 tc_fence_before();
                 named_bar_sync(BAR_SOFT, NSOFT);
-                if (tid == 0) mbar_arrive(bar(B_PFULL));
+                if (tid == 0) mbar_arrive(bar(B_PFULL0 + pb));
             }
             // ---- epilogue of row bq: O = (O^T)^T / l
             if (half == 0) invl_s[h] = l > 0.0f ? 1.0f / l : 0.0f;
@@ -285,13 +305,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int lt = tid - NSOFT, wl = lt >> 5;
         bool ok = true;
         uint32_t g = 0, qi = 0;
-        int32_t pos_next[16];
+        int32_t pos_next[LROWS];
         for (int64_t bq = blockIdx.x; bq < rows; bq += gridDim.x, qi++) {
             const int b = (int)(bq / a.Nq);
             const AttnWindow w = attn_window(a, b, bq);
             if (n_sel_tiles > 0) {
 #pragma unroll
-                for (int u = 0; u < 16; u++) pos_next[u] = __ldg(a.topk + bq * a.K + wl + 4 * u);
+                for (int u = 0; u < LROWS; u++)
+                    pos_next[u] = __ldg(a.topk + bq * a.K + wl + (NLOAD / 32) * u);
             }
             if (lt == 0) {
                 ok = wait_bar(bar(B_QFREE), (qi & 1) ^ 1, abort) && ok;
@@ -307,13 +328,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t gb = g & 1, gp = (g >> 1) & 1;
                 const uint32_t kt = base + K_OFF + gb * KT_BYTES;
                 if (t < n_sel_tiles) {
-                    // FP4 rows of this tile into registers: warp wl takes rows wl + 4 u,
+                    // FP4 rows of this tile into registers: warp wl takes rows wl + 8 u,
                     // lane = 16-channel group (one 256-byte code row per warp load)
-                    uint2 codes[16];
-                    uint32_t scl[4] = {0, 0, 0, 0};
-                    bool vrow[16];
+                    uint2 codes[LROWS];
+                    uint32_t scl[LROWS / 4] = {};
+                    bool vrow[LROWS];
 #pragma unroll
-                    for (int u = 0; u < 16; u++) {
+                    for (int u = 0; u < LROWS; u++) {
                         const int32_t pos = pos_next[u];
                         vrow[u] = pos >= 0 && pos < a.cap;
                         const int64_t src = (int64_t)b * a.cap + pos;
@@ -325,21 +346,23 @@ __global__ void __launch_bounds__(THREADS, 1)
                     // indices of the next selected tile, while these loads are in flight
                     if (t + 1 < n_sel_tiles) {
 #pragma unroll
-                        for (int u = 0; u < 16; u++)
-                            pos_next[u] = __ldg(a.topk + bq * a.K + (t + 1) * TK + wl + 4 * u);
+                        for (int u = 0; u < LROWS; u++)
+                            pos_next[u] =
+                                __ldg(a.topk + bq * a.K + (t + 1) * TK + wl + (NLOAD / 32) * u);
                     }
                     ok = wait_bar(bar(B_KFREE0 + gb), gp ^ 1, abort) && ok;
                     if (lane == 0) {
 #pragma unroll
-                        for (int u = 0; u < 16; u++) kinds[gb * TK + wl + 4 * u] = vrow[u] ? 1 : 0;
+                        for (int u = 0; u < LROWS; u++)
+                            kinds[gb * TK + wl + (NLOAD / 32) * u] = vrow[u] ? 1 : 0;
                     }
                     // even and odd channel blocks store their two 16-byte halves in
                     // opposite order, so each warp store covers all 8 bank groups
                     const int pg = 2 * lane;
                     const bool swap = ((pg >> 3) & 1) != 0;
 #pragma unroll
-                    for (int u = 0; u < 16; u++) {
-                        const int j = wl + 4 * u;
+                    for (int u = 0; u < LROWS; u++) {
+                        const int j = wl + (NLOAD / 32) * u;
                         const float s = e4m3_to_f32((scl[u >> 2] >> (8 * (u & 3))) & 0xFF);
                         uint32_t wds[8];
 #pragma unroll
@@ -380,61 +403,78 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
     } else if (lane == 0) {
-        // ------------------------------------------------ MMA issue: S(0), then
-        // P V of each tile followed by S of the next (P of a tile is normally
-        // ready before the next tile is dequantized)
+        // ------------------------------------------------ MMA issue: P V of the
+        // oldest tile whose P is ready, or S of the next tile once its KV tile and
+        // S buffer are (S may run up to two tiles ahead of P V)
         constexpr uint32_t id_s = idesc_bf16(HQ, TK, false);
         constexpr uint32_t id_o = idesc_bf16(128, HQ, false, true);
+        // descriptors of the tile bases; an address offset adds (offset >> 4)
+        const uint64_t dq = sdesc(base + Q_OFF, 16, 1024);
+        const uint64_t dk0 = sdesc(base + K_OFF, 16, 1024);
+        const uint64_t dv0 = sdesc(base + K_OFF, KT_CHUNK, 1024);
+        const uint64_t dp0 = sdesc(base + P_OFF, 16, 1024);
         const int64_t nrows = rows > blockIdx.x ? (rows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
         const int64_t total = nrows * NT;
-        bool ok = true;
-        auto issue_s = [&](int64_t g) {
-            const int ts = (int)(g % NT);
-            const uint32_t qs = (uint32_t)(g / NT);
-            const uint32_t gb = (uint32_t)(g & 1), gp = (uint32_t)((g >> 1) & 1);
-            if (ts == 0) ok = wait_bar(bar(B_QFULL), qs & 1, abort) && ok;
-            ok = wait_bar(bar(B_KFULL0 + gb), gp, abort) && ok;
-            ok = wait_bar(bar(B_SFREE0 + gb), gp ^ 1, abort) && ok;
-            tc_fence_after();
-            if (ok) {
-                const uint32_t kt = base + K_OFF + gb * KT_BYTES;
-                const uint32_t sd = tmem + ((16u * gb) << 16) + S_COL;
-#pragma unroll 4
-                for (int kk = 0; kk < CH / 16; kk++) {
-                    const uint32_t off = (kk & 3) * 32;
-                    mma_bf16(sd, sdesc(base + Q_OFF + (kk >> 2) * Q_CHUNK + off, 16, 1024),
-                             sdesc(kt + (kk >> 2) * KT_CHUNK + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+        int64_t s_next = 0, p_next = 0;
+        uint64_t last = globaltimer_ns();
+        while (p_next < total && !*abort) {
+            bool progressed = false;
+            const bool s_cand = s_next < total && s_next < p_next + 2;
+            if (p_next < s_next) {
+                const int tp = (int)(p_next % NT);
+                const uint32_t qp = (uint32_t)(p_next / NT);
+                const uint32_t pb = (uint32_t)(p_next & 1), pp = (uint32_t)((p_next >> 1) & 1);
+                // suspend here briefly only when no S is waiting to be issued
+                const bool pready = s_cand ? test_wait(bar(B_PFULL0 + pb), pp)
+                                           : try_wait_hint(bar(B_PFULL0 + pb), pp, 1000);
+                if (pready && (tp != 0 || test_wait(bar(B_OFREE), (qp & 1) ^ 1))) {
+                    tc_fence_after();
+                    const uint64_t dv = dv0 + (uint64_t)((pb * KT_BYTES) >> 4);
+                    const uint64_t dphi = dp0 + (uint64_t)((pb * 2 * P_BYTES) >> 4);
+                    const uint64_t dplo = dphi + (uint64_t)(P_BYTES >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < TK / 16; kk++)
+#pragma unroll
+                        for (int c = 0; c < 4; c++) {
+                            const uint64_t vd = dv + (uint64_t)((2 * c * KT_CHUNK + kk * 2048) >> 4);
+                            mma_bf16(tmem + 64 * c, vd, dphi + (uint64_t)(kk * 2), id_o,
+                                     (tp > 0 || kk > 0) ? 1u : 0u);
+                            mma_bf16(tmem + 64 * c, vd, dplo + (uint64_t)(kk * 2), id_o, 1u);
+                        }
+                    mma_commit(bar(B_KFREE0 + pb));
+                    mma_commit(bar(B_PFREE0 + pb));
+                    if (tp == NT - 1) mma_commit(bar(B_OFULL));
+                    p_next++;
+                    progressed = true;
                 }
             }
-            mma_commit(bar(B_SFULL0 + gb));
-            if (ts == NT - 1) mma_commit(bar(B_QFREE));
-        };
-        auto issue_pv = [&](int64_t g) {
-            const int tp = (int)(g % NT);
-            const uint32_t qp = (uint32_t)(g / NT);
-            ok = wait_bar(bar(B_PFULL), (uint32_t)(g & 1), abort) && ok;
-            if (tp == 0) ok = wait_bar(bar(B_OFREE), (qp & 1) ^ 1, abort) && ok;
-            tc_fence_after();
-            if (ok) {
-                const uint32_t kt = base + K_OFF + (uint32_t)(g & 1) * KT_BYTES;
-#pragma unroll 1
-                for (int c = 0; c < 4; c++)
+            if (!progressed && s_cand) {
+                const int ts = (int)(s_next % NT);
+                const uint32_t qs = (uint32_t)(s_next / NT);
+                const uint32_t gb = (uint32_t)(s_next & 1), gp = (uint32_t)((s_next >> 1) & 1);
+                // the KV tile is usually the last to be ready: suspend on it
+                if ((ts != 0 || test_wait(bar(B_QFULL), qs & 1)) &&
+                    test_wait(bar(B_SFREE0 + gb), gp ^ 1) &&
+                    try_wait_hint(bar(B_KFULL0 + gb), gp, p_next < s_next ? 200 : 1000)) {
+                    tc_fence_after();
+                    const uint64_t dk = dk0 + (uint64_t)((gb * KT_BYTES) >> 4);
+                    const uint32_t sd = tmem + ((16u * gb) << 16) + S_COL;
 #pragma unroll
-                    for (int kk = 0; kk < TK / 16; kk++) {
-                        const uint64_t vd = sdesc(kt + 2 * c * KT_CHUNK + kk * 2048, KT_CHUNK, 1024);
-                        mma_bf16(tmem + 64 * c, vd, sdesc(base + PHI_OFF + kk * 32, 16, 1024), id_o,
-                                 (tp > 0 || kk > 0) ? 1u : 0u);
-                        mma_bf16(tmem + 64 * c, vd, sdesc(base + PLO_OFF + kk * 32, 16, 1024), id_o, 1u);
+                    for (int kk = 0; kk < CH / 16; kk++) {
+                        const uint32_t off = (uint32_t)((kk >> 2) * Q_CHUNK + (kk & 3) * 32) >> 4;
+                        mma_bf16(sd, dq + off, dk + off, id_s, kk > 0 ? 1u : 0u);
                     }
+                    mma_commit(bar(B_SFULL0 + gb));
+                    if (ts == NT - 1) mma_commit(bar(B_QFREE));
+                    s_next++;
+                    progressed = true;
+                }
             }
-            mma_commit(bar(B_KFREE0 + (uint32_t)(g & 1)));
-            mma_commit(bar(B_PFREE));
-            if (tp == NT - 1) mma_commit(bar(B_OFULL));
-        };
-        if (total > 0) issue_s(0);
-        for (int64_t g = 0; g < total; g++) {
-            issue_pv(g);
-            if (g + 1 < total) issue_s(g + 1);
+            if (progressed) {
+                last = globaltimer_ns();
+            } else if (globaltimer_ns() - last > WAIT_NS) {
+                raise_abort(abort);
+            }
         }
     }
     __syncthreads();

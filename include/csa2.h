@@ -155,6 +155,32 @@ int csa2_pool_gather(const float *tok_score, const int32_t *pool, const int64_t 
                      int32_t *pool_pos, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Full-layer selection in one call: the pool and the top-K of each query from
+ * the scan's outputs ([G] indexer section: the pool keeps the best 2,048
+ * blocks of 8 tokens and each query its best 512 candidates of the pool;
+ * [N] CSA2 section: a Full layer builds the pool and selects a fresh top-512).
+ * For query (b, i), with V = V(b, i) as in csa2_index_full and
+ * nb = clamp(n_blk[b][i], 0, ceil(cap/8)):
+ *   pool[b][i] = the best min(P, nb) of blk_score[b][i][0..nb) by (score desc,
+ *                block id asc), block ids ascending, then -1;
+ *   top[b][i]  = the best min(K, #) positions p = 8 j + r with j in the pool
+ *                and p < V, by (tok_score[b][i][p] desc, p asc), ascending,
+ *                then -1.
+ * The result equals csa2_topk (k = P, n_valid = n_blk), csa2_pool_gather and
+ * csa2_topk (k = K) in sequence, bit for bit; no intermediate buffer is
+ * needed. One CTA per query holds a row in shared memory, hence the limits.
+ *  blk_score [B][Nq][ceil(cap/8)] fp32, n_blk [B][Nq] int32
+ *  tok_score [B][Nq][cap] fp32 (no NaN)
+ *  ctx_len   [B] int64 (device); q_pos [B][Nq] int64 (device) or NULL
+ *  pool      [B][Nq][P] int32, top [B][Nq][K] int32
+ *  1 <= P <= 2048, 1 <= K <= 8 P, ceil(cap/8) <= 16384 and 8 P <= 16384;
+ *  CSA2_ERR_SHAPE otherwise (the three calls have no such limits).
+ * ------------------------------------------------------------------------ */
+int csa2_full_select(const float *blk_score, const int32_t *n_blk, const float *tok_score,
+                     const int64_t *ctx_len, const int64_t *q_pos, int B, int Nq, int64_t cap,
+                     int P, int K, int32_t *pool, int32_t *top, void *stream);
+
+/* ------------------------------------------------------------------------
  * Reindex rescoring ([N] CSA2 section: a Reindex layer reuses the main KV and
  * indexer K of the preceding Full layer and rescores the candidate pool with
  * its own indexer Q; [G] indexer section: later layers search only the pool).

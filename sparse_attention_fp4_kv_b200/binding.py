@@ -23,6 +23,9 @@ N_WIN = 128
 # Rows of at most this many candidates are selected by one single-CTA kernel
 # inside the decode step; longer rows take a compaction and a finishing kernel.
 TOPK_SHORT_ROW = 65536
+# csa2_full_select holds a row of block scores (and of pooled token scores) in
+# shared memory: at most this many of each.
+FULL_SELECT_MAX = 16384
 MODE_FULL, MODE_REINDEX, MODE_REUSE = 0, 1, 2
 
 
@@ -57,6 +60,7 @@ _SIGS = {
     "csa2_topk_workspace_size": (_SZ, [_I, _I64, _I]),
     "csa2_topk": (_I, [_P, _P, _P, _I, _I64, _I, _P, _P, _SZ, _P]),
     "csa2_pool_gather": (_I, [_P, _P, _P, _P, _I, _I, _I, _I64, _P, _P, _P]),
+    "csa2_full_select": (_I, [_P, _P, _P, _P, _P, _I, _I, _I64, _I, _I, _P, _P, _P]),
     "csa2_index_reindex": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _P, _P, _P]),
     "csa2_sparse_attn_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "csa2_sparse_attn_decode": (_I, [_P, _P, _P, _I64, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I,
@@ -167,6 +171,22 @@ def csa2_pool_gather(tok_score, pool, ctx_len, pool_score, pool_pos, q_pos=None,
     _check("csa2_pool_gather", lib.csa2_pool_gather(
         _ptr(tok_score), _ptr(pool), _ptr(ctx_len), _ptr(q_pos), B, Nq, P, cap,
         _ptr(pool_score), _ptr(pool_pos), _stream(stream)))
+
+
+def csa2_full_select(blk_score, n_blk, tok_score, ctx_len, pool, top, q_pos=None,
+                     stream=None) -> None:
+    """blk_score [B][Nq][ceil(cap/8)] fp32; n_blk [B][Nq] int32; tok_score [B][Nq][cap] fp32;
+    pool [B][Nq][P] int32; top [B][Nq][K] int32."""
+    _want(blk_score, torch.float32, "blk_score")
+    _want(tok_score, torch.float32, "tok_score")
+    _want(n_blk, torch.int32, "n_blk")
+    B, Nq, cap = tok_score.shape
+    P, K = pool.shape[2], top.shape[2]
+    assert blk_score.shape == (B, Nq, (cap + 7) // 8) and n_blk.shape == (B, Nq)
+    assert pool.shape[:2] == (B, Nq) and top.shape[:2] == (B, Nq)
+    _check("csa2_full_select", lib.csa2_full_select(
+        _ptr(blk_score), _ptr(n_blk), _ptr(tok_score), _ptr(ctx_len), _ptr(q_pos), B, Nq, cap, P, K,
+        _ptr(pool), _ptr(top), _stream(stream)))
 
 
 def csa2_index_reindex(q_idx, k_idx, k_scale, pool, ctx_len, pool_score, pool_pos, q_pos=None,

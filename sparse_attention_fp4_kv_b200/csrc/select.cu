@@ -1,0 +1,277 @@
+// Full-layer selection of one query in one CTA: the pool of blocks and the
+// top-k tokens of the pool, from the scan's block and token scores.
+//
+// "DeepSeek V4.1 Flash KV Cache: 890 Bytes per Token Explained", indexer
+// section: the pool keeps the best 2,048 blocks of 8 tokens and each query
+// keeps its best 512 candidates. "DeepSeek-V4.1-Flash: 890 Bytes Per Token,
+// 437x Smaller KV Cache", CSA2 section: a Full layer builds the pool and
+// selects a fresh top-512.
+//
+// The same result as three calls (block top-k, pool gather, token top-k) with
+// nothing written to global memory between them: for rows that fit in shared
+// memory (at most 16,384 blocks and 16,384 pooled tokens), one CTA per query
+//   1. loads the block scores as 32-bit order keys and selects the best P by
+//      (score desc, block asc) with three radix digits (12, 10, 10 bits) and a
+//      tie rank in index order; writes the pool (ascending block ids);
+//   2. gathers the pooled blocks' token scores (positions below the query's
+//      visible length) into the same key array, in position order;
+//   3. selects the best K tokens the same way and writes their positions
+//      ascending.
+// Key 0 marks a slot that holds no candidate (no finite score maps to 0).
+// Emission walks each warp's contiguous range with ballots, so the output is
+// in index order without a sort.
+#include "common.cuh"
+
+namespace csa2 {
+
+constexpr int FS_THREADS = 512;
+constexpr int FS_WARPS = FS_THREADS / 32;
+constexpr int FS_MAXN = 16384;  // keys held in shared memory
+constexpr int FS_HIST = 4096;
+
+struct FsState {
+    uint32_t wsum[32];
+    int digit;
+    uint32_t above, match, total;
+    uint32_t wcnt[FS_WARPS];  // packed (greater << 16 | equal) counts per warp
+};
+
+// Bin d where the count of keys in bins >= d first reaches kk (scanning from
+// the top bin); st.above = keys in bins above d, st.match = keys in d,
+// st.total = all counted keys.
+__device__ void fs_find_digit(const uint32_t *hist, int NB, int kk, FsState &st) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int BPT = (NB + FS_THREADS - 1) / FS_THREADS;
+    const int b0 = tid * BPT;
+    uint32_t local = 0;
+    for (int j = 0; j < BPT; j++)
+        if (b0 + j < NB) local += hist[b0 + j];
+    uint32_t x = local;  // inclusive suffix sum within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
+        if (lane + o < 32) x += y;
+    }
+    if (lane == 0) st.wsum[warp] = x;
+    __syncthreads();
+    uint32_t warps_above = 0, all = 0;
+    for (int w = 0; w < FS_WARPS; w++) {
+        all += st.wsum[w];
+        if (w > warp) warps_above += st.wsum[w];
+    }
+    uint32_t above = (x - local) + warps_above;
+    for (int j = BPT - 1; j >= 0; j--) {
+        const int bin = b0 + j;
+        if (bin >= NB) continue;
+        const uint32_t h = hist[bin];
+        if (above < (uint32_t)kk && above + h >= (uint32_t)kk) {
+            st.digit = bin;
+            st.above = above;
+            st.match = h;
+        }
+        above += h;
+    }
+    if (tid == 0) st.total = all;
+    __syncthreads();
+}
+
+// The k best of keys[0..n) by (key desc, index asc), as a threshold: every
+// key > T is selected, and of the keys == T the first `take` in index order.
+// T = 0 (take = 0) when all candidates are selected. Returns the number
+// selected.
+__device__ int fs_select(const uint32_t *keys, int n, int k, uint32_t *hist, FsState &st,
+                         uint32_t &T, int &take) {
+    const int tid = threadIdx.x;
+    for (int b = tid; b < FS_HIST; b += FS_THREADS) hist[b] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += FS_THREADS) {
+        const uint32_t key = keys[i];
+        if (key) atomicAdd(&hist[key >> 20], 1u);
+    }
+    __syncthreads();
+    fs_find_digit(hist, FS_HIST, k, st);
+    const uint32_t total = st.total;
+    if (total <= (uint32_t)k) {
+        T = 0;
+        take = 0;
+        return (int)total;
+    }
+    uint32_t prefix = (uint32_t)st.digit;  // digits found so far
+    int kk = k - (int)st.above;
+    // two more digits of 10 bits among the keys that share the prefix
+#pragma unroll 1
+    for (int shift = 10; shift >= 0; shift -= 10) {
+        __syncthreads();
+        for (int b = tid; b < 1024; b += FS_THREADS) hist[b] = 0;
+        __syncthreads();
+        const int pshift = shift + 10;
+        for (int i = tid; i < n; i += FS_THREADS) {
+            const uint32_t key = keys[i];
+            if (key && (key >> pshift) == prefix) atomicAdd(&hist[(key >> shift) & 1023u], 1u);
+        }
+        __syncthreads();
+        fs_find_digit(hist, 1024, kk, st);
+        prefix = (prefix << 10) | (uint32_t)st.digit;
+        kk -= (int)st.above;
+    }
+    T = prefix;
+    take = kk;
+    return k;
+}
+
+// Calls f(out_slot, index) for the selected keys in ascending index order.
+// Warp w walks the contiguous range [w R, w R + R), 32 keys per step.
+template <typename F>
+__device__ void fs_emit(const uint32_t *keys, int n, uint32_t T, int take, FsState &st, F f) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int R = ((n + FS_WARPS * 32 - 1) / (FS_WARPS * 32)) * 32;
+    const int i0 = warp * R;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    uint32_t gt = 0, eq = 0;
+    for (int j = i0; j < i0 + R && j < n; j += 32) {
+        const int i = j + lane;
+        const uint32_t key = i < n ? keys[i] : 0u;
+        gt += __popc(__ballot_sync(0xffffffffu, key > T));
+        eq += __popc(__ballot_sync(0xffffffffu, key != 0 && key == T));
+    }
+    if (lane == 0) st.wcnt[warp] = (gt << 16) | eq;
+    __syncthreads();
+    uint32_t gt_base = 0, eq_base = 0;
+    for (int w = 0; w < warp; w++) {
+        gt_base += st.wcnt[w] >> 16;
+        eq_base += st.wcnt[w] & 0xFFFFu;
+    }
+    for (int j = i0; j < i0 + R && j < n; j += 32) {
+        const int i = j + lane;
+        const uint32_t key = i < n ? keys[i] : 0u;
+        const bool g = key > T;
+        const bool e = key != 0 && key == T;
+        const uint32_t bg = __ballot_sync(0xffffffffu, g);
+        const uint32_t be = __ballot_sync(0xffffffffu, e);
+        const uint32_t erank = eq_base + __popc(be & lt_mask);
+        const bool sel = g || (e && erank < (uint32_t)take);
+        // ties taken before this lane: min(take, eq rank) over the eq keys so far
+        const uint32_t eq_taken_before =
+            min((uint32_t)take, eq_base + __popc(be & lt_mask));
+        if (sel) f((int)(gt_base + __popc(bg & lt_mask) + eq_taken_before), i);
+        gt_base += __popc(bg);
+        eq_base += __popc(be);
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(FS_THREADS) full_select_kernel(
+    const float *__restrict__ blk, const int32_t *__restrict__ n_blk, const float *__restrict__ tok,
+    const int64_t *ctx_len, const int64_t *q_pos, int B, int Nq, int64_t cap, int P, int K,
+    int32_t *__restrict__ pool, int32_t *__restrict__ top) {
+    grid_dep_wait();
+    grid_dep_launch();
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw);  // [FS_MAXN]
+    uint32_t *hist = keys + FS_MAXN;                           // [FS_HIST]
+    int32_t *pool_s = reinterpret_cast<int32_t *>(hist + FS_HIST);  // [P]
+    __shared__ FsState st;
+    const int tid = threadIdx.x;
+    const int64_t row = blockIdx.x;
+    const int b = (int)(row / Nq), qi = (int)(row % Nq);
+    const int64_t nblk_cap = (cap + 7) / 8;
+    int64_t V = visible_len(ctx_len, q_pos, b, qi, Nq);
+    if (V > cap) V = cap;
+    int nb = n_blk[row];
+    nb = nb < 0 ? 0 : (nb > nblk_cap ? (int)nblk_cap : nb);
+
+    // ---- 1. pool: the best P blocks
+    const float *brow = blk + row * nblk_cap;
+    for (int i0 = 0; i0 < nb; i0 += FS_THREADS * 8) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            const int i = i0 + u * FS_THREADS + tid;
+            v[u] = i < nb ? __ldg(brow + i) : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            const int i = i0 + u * FS_THREADS + tid;
+            if (i < nb) keys[i] = f32_order_key(v[u]);
+        }
+    }
+    __syncthreads();
+    uint32_t T;
+    int take;
+    const int npool = fs_select(keys, nb, P, hist, st, T, take);
+    fs_emit(keys, nb, T, take, st, [&](int slot, int i) { pool_s[slot] = i; });
+    int32_t *prow = pool + row * P;
+    for (int s = tid; s < P; s += FS_THREADS) {
+        if (s >= npool) pool_s[s] = -1;
+        prow[s] = pool_s[s];
+    }
+    __syncthreads();
+
+    // ---- 2. token scores of the pooled blocks, in position order
+    const float *trow = tok + row * cap;
+    const int n2 = 8 * P;
+    for (int i0 = 0; i0 < n2; i0 += FS_THREADS * 8) {
+        float v[8];
+        bool ok[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            const int i = i0 + u * FS_THREADS + tid;
+            const int32_t j = i < n2 ? pool_s[i >> 3] : -1;
+            const int64_t p = 8 * (int64_t)j + (i & 7);
+            ok[u] = j >= 0 && p < V;
+            v[u] = ok[u] ? __ldg(trow + p) : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            const int i = i0 + u * FS_THREADS + tid;
+            if (i < n2) keys[i] = ok[u] ? f32_order_key(v[u]) : 0u;
+        }
+    }
+    __syncthreads();
+
+    // ---- 3. the best K tokens, positions ascending
+    const int ntop = fs_select(keys, n2, K, hist, st, T, take);
+    int32_t *trow_out = top + row * K;
+    fs_emit(keys, n2, T, take, st,
+            [&](int slot, int i) { trow_out[slot] = 8 * pool_s[i >> 3] + (i & 7); });
+    for (int s = ntop + tid; s < K; s += FS_THREADS) trow_out[s] = -1;
+}
+
+size_t full_select_smem(int P) { return (size_t)(FS_MAXN + FS_HIST) * 4 + (size_t)P * 4; }
+
+bool full_select_supported(int64_t cap, int P, int K) {
+    return (cap + 7) / 8 <= FS_MAXN && P >= 1 && 8 * (int64_t)P <= FS_MAXN && K >= 1 && K <= 8 * P;
+}
+
+int launch_full_select(const float *blk, const int32_t *n_blk, const float *tok,
+                       const int64_t *ctx_len, const int64_t *q_pos, int B, int Nq, int64_t cap,
+                       int P, int K, int32_t *pool, int32_t *top, cudaStream_t s, bool pdl) {
+    const int64_t rows = (int64_t)B * Nq;
+    if (rows == 0) return CSA2_OK;
+    if (rows > INT32_MAX) return CSA2_ERR_SHAPE;
+    const size_t smem = full_select_smem(P);
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(full_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)full_select_smem(kPoolBlocks)) != cudaSuccess)
+            return CSA2_ERR_CUDA;
+        attr = true;
+    }
+    return launch_kernel(pdl, full_select_kernel, dim3((unsigned)rows), dim3(FS_THREADS), smem, s,
+                         blk, n_blk, tok, ctx_len, q_pos, B, Nq, cap, P, K, pool, top);
+}
+
+}  // namespace csa2
+
+using namespace csa2;
+
+extern "C" int csa2_full_select(const float *blk_score, const int32_t *n_blk,
+                                const float *tok_score, const int64_t *ctx_len,
+                                const int64_t *q_pos, int B, int Nq, int64_t cap, int P, int K,
+                                int32_t *pool, int32_t *top, void *stream) {
+    if (!blk_score || !n_blk || !tok_score || !ctx_len || !pool || !top) return CSA2_ERR_NULL;
+    if (B < 0 || Nq < 0 || cap < 1) return CSA2_ERR_SHAPE;
+    if (P < 1 || P > kPoolBlocks || !full_select_supported(cap, P, K)) return CSA2_ERR_SHAPE;
+    return launch_full_select(blk_score, n_blk, tok_score, ctx_len, q_pos, B, Nq, cap, P, K, pool,
+                              top, (cudaStream_t)stream, false);
+}

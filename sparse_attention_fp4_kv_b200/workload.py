@@ -191,8 +191,12 @@ class PrefillWorkload:
         self.nblk = torch.empty((B, n), dtype=torch.int32, device=dev)
         self.pool = torch.empty((B, n, csa2.POOL_BLOCKS), dtype=torch.int32, device=dev)
         P8 = csa2.POOL_BLOCKS * csa2.BLOCK_TOKENS
-        self.pscore = torch.empty((B, n, P8), dtype=torch.float32, device=dev)
-        self.ppos = torch.empty((B, n, P8), dtype=torch.int32, device=dev)
+        # one fused selection kernel when a row fits in shared memory, else
+        # block top-k, pool gather and token top-k
+        self.fused_select = nb <= csa2.FULL_SELECT_MAX
+        if not self.fused_select:
+            self.pscore = torch.empty((B, n, P8), dtype=torch.float32, device=dev)
+            self.ppos = torch.empty((B, n, P8), dtype=torch.int32, device=dev)
         self.top = torch.empty((B, n, csa2.TOPK), dtype=torch.int32, device=dev)
         self.out = torch.empty((B, n, Hq, C), dtype=torch.float32, device=dev)
         self.scale = 1.0 / math.sqrt(C)
@@ -207,18 +211,23 @@ class PrefillWorkload:
                              self.nblk, q_pos=self.q_pos, stream=stream)
         if scan_events is not None:
             scan_events[1].record(stream or torch.cuda.current_stream())
-        csa2.csa2_topk(self.blk.view(B * n, -1), csa2.POOL_BLOCKS, self.pool.view(B * n, -1),
-                       n_valid=self.nblk.view(-1), stream=stream)
-        csa2.csa2_pool_gather(self.tok, self.pool, self.ctx_len, self.pscore, self.ppos,
-                              q_pos=self.q_pos, stream=stream)
-        csa2.csa2_topk(self.pscore.view(B * n, -1), csa2.TOPK, self.top.view(B * n, -1),
-                       cand_pos=self.ppos.view(B * n, -1), stream=stream)
+        if self.fused_select:
+            csa2.csa2_full_select(self.blk, self.nblk, self.tok, self.ctx_len, self.pool, self.top,
+                                  q_pos=self.q_pos, stream=stream)
+        else:
+            csa2.csa2_topk(self.blk.view(B * n, -1), csa2.POOL_BLOCKS, self.pool.view(B * n, -1),
+                           n_valid=self.nblk.view(-1), stream=stream)
+            csa2.csa2_pool_gather(self.tok, self.pool, self.ctx_len, self.pscore, self.ppos,
+                                  q_pos=self.q_pos, stream=stream)
+            csa2.csa2_topk(self.pscore.view(B * n, -1), csa2.TOPK, self.top.view(B * n, -1),
+                           cand_pos=self.ppos.view(B * n, -1), stream=stream)
         csa2.csa2_sparse_attn_decode(self.q, self.kv_fp4, self.kv_sf, self.top, self.swa,
                                      self.swa_pos0, self.out, self.scale, q_pos=self.q_pos,
                                      stream=stream)
 
     def launches_per_step(self) -> int:
-        return 6
+        """append, scan, selection (one fused kernel, or three), attention."""
+        return 4 if self.fused_select else 6
 
     def index_ops(self) -> int:
         """int8 multiply-adds x 2 of the causal scoring (every query x every

@@ -80,6 +80,14 @@ def test_host_validation_codes():
     assert L.csa2_index_full(good, good, good, good, None, 0, 1, 16, 128, 10, None, good, None,
                              None) == 0
     assert L.csa2_topk(good, None, None, 0, 10, 5, good, None, 0, None) == 0
+    # fused Full-layer selection: NULL, the shared-memory row limits, empty work
+    fs = L.csa2_full_select
+    assert fs(None, good, good, good, None, 1, 1, 4096, 2048, 512, good, good, None) == -1
+    assert fs(good, good, good, good, None, 1, 1, 8 * 16384 + 8, 2048, 512, good, good, None) == -2
+    assert fs(good, good, good, good, None, 1, 1, 4096, 4096, 512, good, good, None) == -2
+    assert fs(good, good, good, good, None, 1, 1, 4096, 64, 600, good, good, None) == -2
+    assert fs(good, good, good, good, None, 1, 1, 4096, 2048, 0, good, good, None) == -2
+    assert fs(good, good, good, good, None, 0, 1, 4096, 2048, 512, good, good, None) == 0
 
 
 def test_decode_stack_schedule_checks():

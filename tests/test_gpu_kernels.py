@@ -253,6 +253,90 @@ def test_full_layer_pool_and_topk_bitexact(B, ctxs):
         assert np.array_equal(top[b, 0].cpu().numpy(), r["top"])
 
 
+# ----------------------------------------------------------------------------- fused Full-layer selection
+def _full_select_check(B, q, k, s, ctx, q_pos=None, P=2048, K=512, oracle_rows=()):
+    """csa2_full_select against csa2_topk -> csa2_pool_gather -> csa2_topk on the
+    same scan outputs (bit for bit), and against the oracle on sampled rows."""
+    Bn, Nq = q.shape[0], q.shape[1]
+    cap = s.shape[1]
+    nb = (cap + 7) // 8
+    tok = torch.full((Bn, Nq, cap), -7.0, device=DEV)
+    blk = torch.full((Bn, Nq, nb), -7.0, device=DEV)
+    nblk = torch.zeros((Bn, Nq), dtype=torch.int32, device=DEV)
+    B.csa2_index_full(q, k, s, ctx, blk, tok, nblk, q_pos=q_pos)
+    pool_f = torch.full((Bn, Nq, P), -9, dtype=torch.int32, device=DEV)
+    top_f = torch.full((Bn, Nq, K), -9, dtype=torch.int32, device=DEV)
+    B.csa2_full_select(blk, nblk, tok, ctx, pool_f, top_f, q_pos=q_pos)
+    pool_c = torch.empty((Bn, Nq, P), dtype=torch.int32, device=DEV)
+    B.csa2_topk(blk.view(Bn * Nq, nb), P, pool_c.view(Bn * Nq, P), n_valid=nblk.view(-1))
+    ps = torch.empty((Bn, Nq, 8 * P), device=DEV)
+    pp = torch.empty((Bn, Nq, 8 * P), dtype=torch.int32, device=DEV)
+    B.csa2_pool_gather(tok, pool_c, ctx, ps, pp, q_pos=q_pos)
+    top_c = torch.empty((Bn, Nq, K), dtype=torch.int32, device=DEV)
+    B.csa2_topk(ps.view(Bn * Nq, -1), K, top_c.view(Bn * Nq, K), cand_pos=pp.view(Bn * Nq, -1))
+    torch.cuda.synchronize()
+    assert torch.equal(pool_f, pool_c), "pool differs from the three-call composition"
+    assert torch.equal(top_f, top_c), "top-k differs from the three-call composition"
+    kn, sn, qn = k.cpu().numpy(), s.cpu().numpy(), q.cpu().numpy()
+    for b, i in oracle_rows:
+        V = int(ctx[b]) if q_pos is None else min(int(q_pos[b, i]) + 1, int(ctx[b]))
+        r = oracle.full_layer(qn[b, i], kn[b], sn[b], V)
+        if P == 2048 and K == 512:
+            assert np.array_equal(pool_f[b, i].cpu().numpy(), r["pool"]), f"pool b={b} i={i}"
+            assert np.array_equal(top_f[b, i].cpu().numpy(), r["top"]), f"top b={b} i={i}"
+
+
+@pytest.mark.parametrize("ctxs,H,D", [([20003, 4096, 100, 1], 16, 128), ([16385, 16384, 7], 4, 64)])
+def test_full_select_decode_rows(B, ctxs, H, D):
+    cap = max(ctxs)
+    q, k, s = _index_inputs(len(ctxs), cap, H, D, seed=sum(ctxs))
+    ctx = torch.tensor(ctxs, dtype=torch.int64, device=DEV)
+    _full_select_check(B, q, k, s, ctx, oracle_rows=[(b, 0) for b in range(len(ctxs))])
+
+
+def test_full_select_largest_row(B):
+    """131,072 positions: 16,384 blocks, the most one CTA holds."""
+    cap = 131072
+    q, k, s = _index_inputs(1, cap, 4, 32, seed=5)
+    ctx = torch.tensor([cap], dtype=torch.int64, device=DEV)
+    _full_select_check(B, q, k, s, ctx, oracle_rows=[(0, 0)])
+
+
+def test_full_select_causal_queries(B):
+    Bn, Nq, ctx0, H, D = 2, 64, 3000, 16, 128
+    cap = ctx0 + Nq
+    g = torch.Generator(device=DEV).manual_seed(9)
+    k = torch.randint(-127, 128, (Bn, cap, H, D), generator=g, device=DEV, dtype=torch.int8)
+    q = torch.randint(-127, 128, (Bn, Nq, H, D), generator=g, device=DEV, dtype=torch.int8)
+    s = 0.5 + torch.rand((Bn, cap), generator=g, device=DEV)
+    ctx = torch.tensor([cap, cap - 5], dtype=torch.int64, device=DEV)
+    qpos = (ctx0 + torch.arange(Nq, device=DEV)).repeat(Bn, 1).contiguous()
+    _full_select_check(B, q, k, s, ctx, q_pos=qpos, oracle_rows=[(0, 0), (1, 63), (1, 31)])
+
+
+@pytest.mark.parametrize("levels", [1, 2, 5])
+def test_full_select_tie_heavy(B, levels):
+    """Coarse keys and unit scales: long runs of equal block and token scores
+    (levels = 1: every score is zero), decided by position."""
+    ctxs = [30000, 9001]
+    cap = max(ctxs)
+    g = torch.Generator(device=DEV).manual_seed(levels)
+    k = torch.randint(0, levels, (2, cap, 4, 32), generator=g, device=DEV, dtype=torch.int8)
+    q = torch.randint(-3, 4, (2, 1, 4, 32), generator=g, device=DEV, dtype=torch.int8)
+    s = torch.ones((2, cap), device=DEV)
+    ctx = torch.tensor(ctxs, dtype=torch.int64, device=DEV)
+    _full_select_check(B, q, k, s, ctx, oracle_rows=[(0, 0), (1, 0)])
+
+
+def test_full_select_other_sizes(B):
+    """A smaller pool and a ragged k (the shapes the call accepts besides 2048 / 512)."""
+    ctxs = [5000, 300]
+    q, k, s = _index_inputs(2, 5000, 8, 64, seed=77)
+    ctx = torch.tensor(ctxs, dtype=torch.int64, device=DEV)
+    _full_select_check(B, q, k, s, ctx, P=64, K=100)
+    _full_select_check(B, q, k, s, ctx, P=2048, K=4000)
+
+
 def test_reindex_bitexact(B):
     ctxs = [30000, 20001, 9000]
     H, D = 16, 128

@@ -169,6 +169,9 @@ int csa2_pool_gather(const float *tok_score, const int32_t *pool, const int64_t 
  * The result equals csa2_topk (k = P, n_valid = n_blk), csa2_pool_gather and
  * csa2_topk (k = K) in sequence, bit for bit; no intermediate buffer is
  * needed. One CTA per query holds a row in shared memory, hence the limits.
+ * Precondition (as csa2_index_full writes them): blk_score[j] is the maximum
+ * of tok_score over the visible positions of block j. The best K tokens then
+ * lie in the best min(K, P) blocks, and only those blocks' tokens are read.
  *  blk_score [B][Nq][ceil(cap/8)] fp32, n_blk [B][Nq] int32
  *  tok_score [B][Nq][cap] fp32 (no NaN)
  *  ctx_len   [B] int64 (device); q_pos [B][Nq] int64 (device) or NULL

@@ -11,12 +11,15 @@
 // nothing written to global memory between them: for rows that fit in shared
 // memory (at most 16,384 blocks and 16,384 pooled tokens), one CTA per query
 //   1. loads the block scores as 32-bit order keys and selects the best P by
-//      (score desc, block asc) with three radix digits (12, 10, 10 bits) and a
-//      tie rank in index order; writes the pool (ascending block ids);
-//   2. gathers the pooled blocks' token scores (positions below the query's
-//      visible length) into the same key array, in position order;
-//   3. selects the best K tokens the same way and writes their positions
-//      ascending.
+//      (score desc, block asc): radix digits below the bits that every key of
+//      the row shares (so the first histogram spreads), then a tie rank in
+//      index order; writes the pool (ascending block ids);
+//   2. selects the best K blocks the same way (K <= P): every one of the best
+//      K tokens lies in one of them, since each block ranked ahead of a token's
+//      block holds its own maximum, a token ranked ahead of it;
+//   3. gathers those blocks' token scores (positions below the query's visible
+//      length) into the key array, in position order, and selects the best K
+//      tokens, written as ascending positions.
 // Key 0 marks a slot that holds no candidate (no finite score maps to 0).
 // Emission walks each warp's contiguous range with ballots, so the output is
 // in index order without a sort.
@@ -28,12 +31,17 @@ constexpr int FS_THREADS = 512;
 constexpr int FS_WARPS = FS_THREADS / 32;
 constexpr int FS_MAXN = 16384;  // keys held in shared memory
 constexpr int FS_HIST = 4096;
+// Histogram bin b lives at b + b / 32: a thread scanning its run of
+// consecutive bins then hits a different bank from every other lane.
+__device__ __forceinline__ int hpad(int b) { return b + (b >> 5); }
+constexpr int FS_HIST_WORDS = FS_HIST + FS_HIST / 32;
 
 struct FsState {
     uint32_t wsum[32];
     int digit;
     uint32_t above, match, total;
     uint32_t wcnt[FS_WARPS];  // packed (greater << 16 | equal) counts per warp
+    uint32_t wor[FS_WARPS], wand[FS_WARPS], wn[FS_WARPS];
 };
 
 // Bin d where the count of keys in bins >= d first reaches kk (scanning from
@@ -45,7 +53,7 @@ __device__ void fs_find_digit(const uint32_t *hist, int NB, int kk, FsState &st)
     const int b0 = tid * BPT;
     uint32_t local = 0;
     for (int j = 0; j < BPT; j++)
-        if (b0 + j < NB) local += hist[b0 + j];
+        if (b0 + j < NB) local += hist[hpad(b0 + j)];
     uint32_t x = local;  // inclusive suffix sum within the warp
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -63,7 +71,7 @@ __device__ void fs_find_digit(const uint32_t *hist, int NB, int kk, FsState &st)
     for (int j = BPT - 1; j >= 0; j--) {
         const int bin = b0 + j;
         if (bin >= NB) continue;
-        const uint32_t h = hist[bin];
+        const uint32_t h = hist[hpad(bin)];
         if (above < (uint32_t)kk && above + h >= (uint32_t)kk) {
             st.digit = bin;
             st.above = above;
@@ -78,51 +86,87 @@ __device__ void fs_find_digit(const uint32_t *hist, int NB, int kk, FsState &st)
 // The k best of keys[0..n) by (key desc, index asc), as a threshold: every
 // key > T is selected, and of the keys == T the first `take` in index order.
 // T = 0 (take = 0) when all candidates are selected. Returns the number
-// selected.
+// selected. The digits start below the leading bits that all candidate keys
+// share (an OR / AND reduction), 12 bits first, then 10 at a time.
 __device__ int fs_select(const uint32_t *keys, int n, int k, uint32_t *hist, FsState &st,
                          uint32_t &T, int &take) {
-    const int tid = threadIdx.x;
-    for (int b = tid; b < FS_HIST; b += FS_THREADS) hist[b] = 0;
-    __syncthreads();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t kor = 0, kand = 0xFFFFFFFFu, cnt = 0;
     for (int i = tid; i < n; i += FS_THREADS) {
         const uint32_t key = keys[i];
-        if (key) atomicAdd(&hist[key >> 20], 1u);
+        if (key) {
+            kor |= key;
+            kand &= key;
+            cnt++;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        kor |= __shfl_xor_sync(0xffffffffu, kor, o);
+        kand &= __shfl_xor_sync(0xffffffffu, kand, o);
+        cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    }
+    if (lane == 0) {
+        st.wor[warp] = kor;
+        st.wand[warp] = kand;
+        st.wn[warp] = cnt;
     }
     __syncthreads();
-    fs_find_digit(hist, FS_HIST, k, st);
-    const uint32_t total = st.total;
-    if (total <= (uint32_t)k) {
+    kor = 0;
+    kand = 0xFFFFFFFFu;
+    cnt = 0;
+    for (int w = 0; w < FS_WARPS; w++) {
+        kor |= st.wor[w];
+        kand &= st.wand[w];
+        cnt += st.wn[w];
+    }
+    if (cnt <= (uint32_t)k) {
         T = 0;
         take = 0;
-        return (int)total;
+        return (int)cnt;
     }
-    uint32_t prefix = (uint32_t)st.digit;  // digits found so far
-    int kk = k - (int)st.above;
-    // two more digits of 10 bits among the keys that share the prefix
+    // the candidates share their top L bits; all of them equal when L = 32
+    const int L = __clz(kor ^ kand);
+    if (L == 32) {
+        T = kand;
+        take = k;
+        return k;
+    }
+    int shift = 32 - L > 12 ? 32 - L - 12 : 0;
+    int nbits = 32 - L - shift;
+    uint32_t prefix = L == 0 ? 0u : (kand >> (32 - L));  // the matched high bits
+    int pshift = 32 - L;
+    int kk = k;
 #pragma unroll 1
-    for (int shift = 10; shift >= 0; shift -= 10) {
+    while (true) {
+        const uint32_t mask = (1u << nbits) - 1u;
+        for (int b = tid; b <= (int)mask; b += FS_THREADS) hist[hpad(b)] = 0;
         __syncthreads();
-        for (int b = tid; b < 1024; b += FS_THREADS) hist[b] = 0;
-        __syncthreads();
-        const int pshift = shift + 10;
         for (int i = tid; i < n; i += FS_THREADS) {
             const uint32_t key = keys[i];
-            if (key && (key >> pshift) == prefix) atomicAdd(&hist[(key >> shift) & 1023u], 1u);
+            if (key && (pshift >= 32 || (key >> pshift) == prefix))
+                atomicAdd(&hist[hpad((int)((key >> shift) & mask))], 1u);
         }
         __syncthreads();
-        fs_find_digit(hist, 1024, kk, st);
-        prefix = (prefix << 10) | (uint32_t)st.digit;
+        fs_find_digit(hist, (int)mask + 1, kk, st);
+        prefix = (prefix << nbits) | (uint32_t)st.digit;
         kk -= (int)st.above;
+        if (shift == 0) break;
+        pshift = shift;
+        nbits = shift > 10 ? 10 : shift;
+        shift -= nbits;
+        __syncthreads();
     }
     T = prefix;
     take = kk;
     return k;
 }
 
-// Calls f(out_slot, index) for the selected keys in ascending index order.
-// Warp w walks the contiguous range [w R, w R + R), 32 keys per step.
-template <typename F>
-__device__ void fs_emit(const uint32_t *keys, int n, uint32_t T, int take, FsState &st, F f) {
+// Calls f(out_slot, index) for the selected keys (key(i), i < n) in
+// ascending index order. Warp w walks the contiguous range [w R, w R + R),
+// 32 keys per step.
+template <typename KeyF, typename F>
+__device__ void fs_emit(KeyF key_of, int n, uint32_t T, int take, FsState &st, F f) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int R = ((n + FS_WARPS * 32 - 1) / (FS_WARPS * 32)) * 32;
     const int i0 = warp * R;
@@ -130,7 +174,7 @@ __device__ void fs_emit(const uint32_t *keys, int n, uint32_t T, int take, FsSta
     uint32_t gt = 0, eq = 0;
     for (int j = i0; j < i0 + R && j < n; j += 32) {
         const int i = j + lane;
-        const uint32_t key = i < n ? keys[i] : 0u;
+        const uint32_t key = i < n ? key_of(i) : 0u;
         gt += __popc(__ballot_sync(0xffffffffu, key > T));
         eq += __popc(__ballot_sync(0xffffffffu, key != 0 && key == T));
     }
@@ -143,7 +187,7 @@ __device__ void fs_emit(const uint32_t *keys, int n, uint32_t T, int take, FsSta
     }
     for (int j = i0; j < i0 + R && j < n; j += 32) {
         const int i = j + lane;
-        const uint32_t key = i < n ? keys[i] : 0u;
+        const uint32_t key = i < n ? key_of(i) : 0u;
         const bool g = key > T;
         const bool e = key != 0 && key == T;
         const uint32_t bg = __ballot_sync(0xffffffffu, g);
@@ -167,9 +211,12 @@ __global__ void __launch_bounds__(FS_THREADS) full_select_kernel(
     grid_dep_wait();
     grid_dep_launch();
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw);  // [FS_MAXN]
-    uint32_t *hist = keys + FS_MAXN;                           // [FS_HIST]
-    int32_t *pool_s = reinterpret_cast<int32_t *>(hist + FS_HIST);  // [P]
+    const int64_t nkeys = (cap + 7) / 8 > 8 * (int64_t)(K < P ? K : P) ? (cap + 7) / 8
+                                                                       : 8 * (int64_t)(K < P ? K : P);
+    uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw);  // [nkeys]
+    uint32_t *hist = keys + nkeys;                             // [FS_HIST_WORDS]
+    int32_t *pool_s = reinterpret_cast<int32_t *>(hist + FS_HIST_WORDS);  // [P]
+    int32_t *kblk_s = pool_s + P;                                    // [P]
     __shared__ FsState st;
     const int tid = threadIdx.x;
     const int64_t row = blockIdx.x;
@@ -199,7 +246,7 @@ __global__ void __launch_bounds__(FS_THREADS) full_select_kernel(
     uint32_t T;
     int take;
     const int npool = fs_select(keys, nb, P, hist, st, T, take);
-    fs_emit(keys, nb, T, take, st, [&](int slot, int i) { pool_s[slot] = i; });
+    fs_emit([&](int i) { return keys[i]; }, nb, T, take, st, [&](int slot, int i) { pool_s[slot] = i; });
     int32_t *prow = pool + row * P;
     for (int s = tid; s < P; s += FS_THREADS) {
         if (s >= npool) pool_s[s] = -1;
@@ -207,16 +254,27 @@ __global__ void __launch_bounds__(FS_THREADS) full_select_kernel(
     }
     __syncthreads();
 
-    // ---- 2. token scores of the pooled blocks, in position order
+    // ---- 2. the best min(K, P) blocks, found inside the pool (ascending)
+    const int32_t *kblk = pool_s;
+    int nkb = npool;
+    if (K < npool) {
+        fs_select(keys, nb, K, hist, st, T, take);
+        fs_emit([&](int s) { return keys[pool_s[s]]; }, npool, T, take, st,
+                [&](int slot, int s) { kblk_s[slot] = pool_s[s]; });
+        kblk = kblk_s;
+        nkb = K;
+    }
+
+    // ---- 3. their token scores in position order, then the best K tokens
     const float *trow = tok + row * cap;
-    const int n2 = 8 * P;
+    const int n2 = 8 * nkb;
     for (int i0 = 0; i0 < n2; i0 += FS_THREADS * 8) {
         float v[8];
         bool ok[8];
 #pragma unroll
         for (int u = 0; u < 8; u++) {
             const int i = i0 + u * FS_THREADS + tid;
-            const int32_t j = i < n2 ? pool_s[i >> 3] : -1;
+            const int32_t j = i < n2 ? kblk[i >> 3] : -1;
             const int64_t p = 8 * (int64_t)j + (i & 7);
             ok[u] = j >= 0 && p < V;
             v[u] = ok[u] ? __ldg(trow + p) : 0.0f;
@@ -228,16 +286,21 @@ __global__ void __launch_bounds__(FS_THREADS) full_select_kernel(
         }
     }
     __syncthreads();
-
-    // ---- 3. the best K tokens, positions ascending
     const int ntop = fs_select(keys, n2, K, hist, st, T, take);
     int32_t *trow_out = top + row * K;
-    fs_emit(keys, n2, T, take, st,
-            [&](int slot, int i) { trow_out[slot] = 8 * pool_s[i >> 3] + (i & 7); });
+    fs_emit([&](int i) { return keys[i]; }, n2, T, take, st,
+            [&](int slot, int i) { trow_out[slot] = 8 * kblk[i >> 3] + (i & 7); });
     for (int s = ntop + tid; s < K; s += FS_THREADS) trow_out[s] = -1;
 }
 
-size_t full_select_smem(int P) { return (size_t)(FS_MAXN + FS_HIST) * 4 + (size_t)P * 4; }
+// key array (the larger of the block row and the gathered tokens), the
+// histogram, the pool and the best blocks
+size_t full_select_smem(int64_t cap, int P, int K) {
+    const int64_t nb = (cap + 7) / 8;
+    const int64_t n2 = 8 * (int64_t)(K < P ? K : P);
+    const int64_t nkeys = nb > n2 ? nb : n2;
+    return (size_t)(nkeys + FS_HIST_WORDS) * 4 + (size_t)P * 8;
+}
 
 bool full_select_supported(int64_t cap, int P, int K) {
     return (cap + 7) / 8 <= FS_MAXN && P >= 1 && 8 * (int64_t)P <= FS_MAXN && K >= 1 && K <= 8 * P;
@@ -249,11 +312,17 @@ int launch_full_select(const float *blk, const int32_t *n_blk, const float *tok,
     const int64_t rows = (int64_t)B * Nq;
     if (rows == 0) return CSA2_OK;
     if (rows > INT32_MAX) return CSA2_ERR_SHAPE;
-    const size_t smem = full_select_smem(P);
+    const size_t smem = full_select_smem(cap, P, K);
     static bool attr = false;
     if (!attr) {
+        // two CTAs per SM: dynamic shared memory up to the largest row, and the
+        // largest shared-memory carveout
         if (cudaFuncSetAttribute(full_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)full_select_smem(kPoolBlocks)) != cudaSuccess)
+                                 (int)full_select_smem(8 * (int64_t)FS_MAXN, kPoolBlocks,
+                                                       kPoolBlocks)) != cudaSuccess ||
+            cudaFuncSetAttribute(full_select_kernel,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
             return CSA2_ERR_CUDA;
         attr = true;
     }

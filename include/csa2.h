@@ -23,7 +23,9 @@
  *  - Return value: CSA2_OK or a negative csa2_status. On error nothing has
  *    been launched, except CSA2_ERR_CUDA, which reports a failed launch.
  *  - Kernels never trap: an out-of-range position found on the device is
- *    skipped, not written.
+ *    skipped, not written; a wait inside a kernel that runs out its time or
+ *    iteration bound records it in a device flag and the kernel returns
+ *    (csa2_device_status reads the flags).
  *  - bf16 tensors are IEEE bfloat16 bit patterns; fp32 is IEEE binary32.
  *  - Layouts are row-major with the listed dimensions, densely packed.
  *  - Selection order everywhere: score descending, then position ascending.
@@ -55,7 +57,8 @@ typedef enum csa2_status {
     CSA2_ERR_ALIGN = -3,     /* a pointer or row size breaks the alignment rule */
     CSA2_ERR_RANGE = -4,     /* a host-side value is out of range             */
     CSA2_ERR_WORKSPACE = -5, /* ws is NULL or smaller than required           */
-    CSA2_ERR_CUDA = -6       /* a kernel launch failed                        */
+    CSA2_ERR_CUDA = -6,      /* a kernel launch failed                        */
+    CSA2_ERR_DEVICE_TIMEOUT = -7 /* a kernel gave up a bounded wait (device flag) */
 } csa2_status;
 
 /* CSA2 layer modes ([N] CSA2 section). */
@@ -70,6 +73,19 @@ const char *csa2_status_string(int status);
 
 /* CSA2_ABI_VERSION of the loaded library. */
 int csa2_abi_version(void);
+
+/* Device-side error status of the current device: CSA2_ERR_DEVICE_TIMEOUT if
+ * any kernel of the library gave up a bounded wait since the flags were last
+ * cleared, else CSA2_OK (CSA2_ERR_CUDA if the flags cannot be read). With
+ * clear != 0 the flags are reset after reading. Synchronizes the device. The
+ * outputs of a call whose kernel gave up are unspecified; the CUDA context
+ * stays usable. */
+int csa2_device_status(int clear);
+
+/* Self-test of that path: launches one CTA whose wait on an mbarrier that
+ * nothing completes gives up after limit_us microseconds (1..1,000,000) and
+ * records the timeout, as a kernel of the library would. */
+int csa2_selftest_wait_timeout(int limit_us, void *stream);
 
 /* ------------------------------------------------------------------------
  * FP4 append: quantize-and-pack new main-KV rows into the cache.

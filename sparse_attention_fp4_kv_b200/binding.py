@@ -55,6 +55,8 @@ class csa2_layer(ctypes.Structure):
 _SIGS = {
     "csa2_status_string": (ctypes.c_char_p, [_I]),
     "csa2_abi_version": (_I, []),
+    "csa2_device_status": (_I, [_I]),
+    "csa2_selftest_wait_timeout": (_I, [_I, _P]),
     "csa2_kv_append_fp4": (_I, [_P, _I, _I, _I, _P, _I64, _P, _P, _P]),
     "csa2_index_full": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _P, _P, _P, _P]),
     "csa2_topk_workspace_size": (_SZ, [_I, _I64, _I]),
@@ -171,6 +173,17 @@ def csa2_pool_gather(tok_score, pool, ctx_len, pool_score, pool_pos, q_pos=None,
     _check("csa2_pool_gather", lib.csa2_pool_gather(
         _ptr(tok_score), _ptr(pool), _ptr(ctx_len), _ptr(q_pos), B, Nq, P, cap,
         _ptr(pool_score), _ptr(pool_pos), _stream(stream)))
+
+
+def device_status(clear: bool = False) -> int:
+    """CSA2_OK, or CSA2_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait
+    (synchronizes the device; clear resets the flags)."""
+    return lib.csa2_device_status(1 if clear else 0)
+
+
+def selftest_wait_timeout(limit_us: int = 1000, stream=None) -> None:
+    """Launch one CTA whose wait nothing completes; it records a timeout."""
+    _check("csa2_selftest_wait_timeout", lib.csa2_selftest_wait_timeout(limit_us, _stream(stream)))
 
 
 def csa2_full_select(blk_score, n_blk, tok_score, ctx_len, pool, top, q_pos=None,

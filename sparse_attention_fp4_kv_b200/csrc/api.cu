@@ -19,6 +19,7 @@ extern "C" const char *csa2_status_string(int status) {
         case CSA2_ERR_RANGE: return "a host-side value is out of range";
         case CSA2_ERR_WORKSPACE: return "workspace missing or too small";
         case CSA2_ERR_CUDA: return "a CUDA launch failed";
+        case CSA2_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait on the device";
         default: return "unknown status";
     }
 }

@@ -492,6 +492,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace tr
 
+int attn_rows_wait_flag(bool clear) { return read_device_flag(tr::g_attn_rows_error, clear); }
+
 bool attn_rows_supported(const AttnArgs &a) {
     const int nwin = a.n_win < a.swa_rows ? a.n_win : a.swa_rows;
     const bool has_win = nwin > 0 && a.swa != nullptr;

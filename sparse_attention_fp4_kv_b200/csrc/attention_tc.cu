@@ -22,17 +22,21 @@
 //     head), does a chunk-local softmax in fp32 and writes P to shared memory
 //     as bf16 hi + lo parts (P = hi + lo to ~16 bits, so the P V product keeps
 //     fp32-level accuracy with bf16 operands).
-//  4. O = P_hi V + P_lo V: M = 64, N = 256 (two halves of 512 channels), K = 80,
-//     the same shared-memory KV tile read as an MN-major operand.
-//  5. Each CTA writes its unnormalized O (from TMEM), row maxima and sums into
-//     its cluster's exchange slot in the workspace (L2 resident); after a
-//     cluster barrier each CTA combines its 64 channels of all 64 heads over the
-//     8 partial results and writes the output. (Moving the 1 MB of partials of a
-//     cluster through L2 measured about 4x faster than through distributed
-//     shared memory.) Clusters are persistent over query rows (at most 18, one
-//     wave on 148 SMs), so the workspace is 18 slots at most.
-// TMEM: O uses columns 0..511 of lanes 0-15 of each 32-lane subpartition
-// (the M = 64 accumulator layout); S uses lanes 16-31 of columns 0..79.
+//  4. O^T = V^T P_hi^T + V^T P_lo^T: M = 128 channels (4 blocks), N = 64 heads,
+//     K = 80 keys; the shared-memory KV tile is read as an MN-major A operand.
+//     Accumulating O transposed keeps the MMAs at M = 128 (an M = 64 MMA runs at
+//     half rate, and every tcgen05.mma has a fixed cost of about 50 cycles).
+//  5. Each CTA writes its unnormalized O straight from TMEM (lane = channel, so
+//     each warp store covers 128 contiguous bytes of one head), its row maxima
+//     and sums into its cluster's exchange slot in the workspace (L2
+//     resident); after a cluster barrier each CTA combines its 64 channels of
+//     all 64 heads over the 8 partial results and writes the output. (Moving
+//     the 1 MB of partials of a cluster through L2 measured about 4x faster
+//     than through distributed shared memory.) Clusters are persistent over
+//     query rows (at most 18, one wave on 148 SMs), so the workspace is 18
+//     slots at most.
+// TMEM: O^T uses columns 0..255 (all lanes); S uses lanes 16-31 of each 32-lane
+// subpartition (the M = 64 accumulator layout) in columns 256..335.
 // One launch per layer; scratch: one exchange slot (1.05 MB) per cluster.
 #include "attention.cuh"
 #include "tcgen05.cuh"
@@ -73,9 +77,9 @@ constexpr int SMEM_USED = TADDR_OFF + 16;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 // Exchange slot of one cluster in the workspace: partial O [8 sources][8
 // slices][64 heads][64 channels] fp32, row maxima [8][64] and row sums [8][64].
-constexpr int SLICE_BYTES = HQ * 64 * 4;  // 16 KB
-constexpr int STG_OFF = Q_OFF;            // staging of the partial O (128 KB)
-static_assert(CL * SLICE_BYTES <= Q_BYTES + K_BYTES, "staging must fit in the Q + KV tiles");
+// TMEM: O^T channel block c (128 lanes x 64 heads) at columns 64 c; S (M = 64
+// layout, lanes 16-31 of each quadrant) at columns S_COL..S_COL + 79.
+constexpr uint32_t S_COL = 256;
 constexpr int64_t XSLOT_FLOATS = (int64_t)CL * HQ * CH + 2 * CL * HQ;
 // Clusters resident at once (148 SMs / 8); each walks query rows with this stride.
 constexpr int MAX_CLUSTERS = 18;
@@ -281,7 +285,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncthreads();
 
         // ---- S = Q K^T  (M = 64, N = 80, K = 512) into TMEM lanes 16..31
-        const uint32_t s_tmem = tmem + (16u << 16);
+        const uint32_t s_tmem = tmem + (16u << 16) + S_COL;
         if (tid == 0 && ok) {
             tc_fence_after();
             constexpr uint32_t id_s = idesc_bf16(HQ, T, false);
@@ -358,20 +362,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_before();
         __syncthreads();
 
-        // ---- O = P_hi V + P_lo V  (M = 64, N = 256 per half, K = 80)
+        // ---- O^T = V^T P_hi^T + V^T P_lo^T  (M = 128 channels x 4 blocks, N = 64
+        // heads, K = 80 keys): V^T is the KV tile read MN-major, P^T the P tiles
+        // read K-major; block c of 128 channels accumulates in columns 64 c
         if (tid == 0 && ok) {
             tc_fence_after();
-            constexpr uint32_t id_o = idesc_bf16(HQ, 256, true);
+            constexpr uint32_t id_o = idesc_bf16(128, HQ, false, true);
 #pragma unroll 1
-            for (int hf = 0; hf < 2; hf++) {
-#pragma unroll 1
-                for (int kk = 0; kk < T / 16; kk++) {
-                    const uint32_t poff = (kk >> 2) * P_ATOM + (kk & 3) * 32;
-                    const uint64_t vd =
-                        sdesc(base + K_OFF + hf * 4 * K_CHUNK + kk * 2048, K_CHUNK, 1024);
-                    mma_bf16(tmem + hf * 256, sdesc(base + PHI_OFF + poff, 16, 1024), vd, id_o,
-                             kk > 0);
-                    mma_bf16(tmem + hf * 256, sdesc(base + PLO_OFF + poff, 16, 1024), vd, id_o, 1);
+            for (int kk = 0; kk < T / 16; kk++) {
+                const uint32_t poff = (kk >> 2) * P_ATOM + (kk & 3) * 32;
+                const uint64_t phi = sdesc(base + PHI_OFF + poff, 16, 1024);
+                const uint64_t plo = sdesc(base + PLO_OFF + poff, 16, 1024);
+#pragma unroll
+                for (int c = 0; c < 4; c++) {
+                    const uint64_t vd = sdesc(base + K_OFF + 2 * c * K_CHUNK + kk * 2048, K_CHUNK, 1024);
+                    mma_bf16(tmem + 64 * c, vd, phi, id_o, kk > 0);
+                    mma_bf16(tmem + 64 * c, vd, plo, id_o, 1);
                 }
             }
             mma_commit(bar);
@@ -380,45 +386,29 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
 
         // ---- publish this CTA's unnormalized O, row maxima and sums in the
-        // cluster's exchange slot (L2). O is first staged in shared memory
-        // slice-major ([8 slices of 64 channels][64 heads][64 channels]) over the
-        // now idle Q and KV tiles, then copied out as 8 contiguous 16 KB bulk
-        // stores; warps w and w + 4 split the TMEM columns.
+        // cluster's exchange slot (L2), laid out [source][64-channel slice][64
+        // heads][64 channels]. TMEM lane = channel, so every warp store of one
+        // head writes 32 consecutive channels (128 bytes); warps w and w + 4
+        // take channel blocks 0-1 and 2-3.
         {
-            const uint32_t row_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-            const int cbeg = (warp >> 2) * 256;
+            const int q4 = warp & 3;
+            const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
 #pragma unroll 1
-            for (int c0 = cbeg; c0 < cbeg + 256; c0 += 64) {
-                float v[32];
-                tmem_ld_16x32x2_32(row_addr + c0, v);
-                tmem_ld_wait();
-                // 16-byte chunk j of a head's 256-byte row sits at position j ^ (h & 7):
-                // lanes 0-7 of a warp hold 8 consecutive heads, so each store of
-                // the warp covers all 8 bank groups
-                const uint32_t row = base + STG_OFF + (uint32_t)(((c0 >> 6) * HQ + h) * 256);
+            for (int c = 2 * (warp >> 2); c < 2 * (warp >> 2) + 2; c++) {
+                const int ch = 128 * c + 32 * q4 + lane;  // this thread's channel
+                float *dst = xo + ((int64_t)rank * CL + (ch >> 6)) * (HQ * 64) + (ch & 63);
+#pragma unroll 1
+                for (int hc = 0; hc < 2; hc++) {
+                    float v[32];
+                    tmem_ld_32x32b_32(lane_addr + 64 * c + 32 * hc, v);
 #pragma unroll
-                for (int u = 0; u < 8; u++) {
-                    const int j = (half * 8 + u) ^ (h & 7);
-                    const uint4 w = ok ? make_uint4(__float_as_uint(v[4 * u]), __float_as_uint(v[4 * u + 1]),
-                                                    __float_as_uint(v[4 * u + 2]), __float_as_uint(v[4 * u + 3]))
-                                       : make_uint4(0u, 0u, 0u, 0u);
-                    st_shared_v4(row + 16 * j, w);
+                    for (int i = 0; i < 32; i++) dst[(32 * hc + i) * 64] = ok ? v[i] : 0.0f;
                 }
             }
             if (warp < 4 && half == 0) {
                 xm[rank * HQ + h] = ok ? m_s[h] : -INFINITY;
                 xl[rank * HQ + h] = ok ? l_s[h] : 0.0f;
             }
-        }
-        fence_proxy_async();
-        __syncthreads();
-        if (tid == 0) {
-#pragma unroll
-            for (int c = 0; c < CL; c++)
-                bulk_store(xo + ((int64_t)rank * CL + c) * (HQ * 64), base + STG_OFF + c * SLICE_BYTES,
-                           SLICE_BYTES);
-            bulk_store_wait();
-            asm volatile("fence.proxy.async.global;" ::: "memory");
         }
         __syncthreads();
         __threadfence();
@@ -428,7 +418,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ---- combine: this CTA owns channels [64 rank, 64 rank + 64); the slice
         // of source r is contiguous at xo[r][rank]. Thread t takes the 16-byte
         // chunks e = 4 (t + 256 u), u = 0..3, of the [64 heads][64 channels]
-        // slice; chunk position p of head hh holds channels 4 (p ^ (hh & 7)).
+        // slice.
         {
             float *wts = reinterpret_cast<float *>(sm + PHI_OFF);  // [64 heads][8] weight / den
             if (tid < HQ) {
@@ -463,7 +453,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int u = 0; u < 4; u++) {
                 const int e = 4 * (tid + 256 * u);
-                const int hh = e >> 6, ch = 4 * (((e & 63) >> 2) ^ (hh & 7));
+                const int hh = e >> 6, ch = e & 63;
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int r = 0; r < CL; r++) {
@@ -542,6 +532,8 @@ int launch_attn_tc(const AttnArgs &a, cudaStream_t s) {
 }  // namespace csa2
 
 namespace csa2 {
+
+int attn_tc_wait_flag(bool clear) { return read_device_flag(tc::g_attn_error, clear); }
 
 size_t attn_tc_workspace_bytes(int B, int Nq) {
     const int64_t rows = (int64_t)B * Nq;

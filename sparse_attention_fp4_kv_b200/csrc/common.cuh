@@ -57,6 +57,23 @@ inline int launch_kernel(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 blo
     return launch_status();
 }
 
+// Reads a device flag of the library (an int __device__ variable of the
+// calling translation unit), resetting it when clear; -1 if it cannot be read.
+template <typename T>
+inline int read_device_flag(T &symbol, bool clear) {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, symbol, sizeof(int)) != cudaSuccess) return -1;
+    if (clear && v) {
+        const int z = 0;
+        if (cudaMemcpyToSymbol(symbol, &z, sizeof(int)) != cudaSuccess) return -1;
+    }
+    return v;
+}
+// The bounded-wait flags of the kernels that wait on the device.
+int attn_tc_wait_flag(bool clear);
+int attn_rows_wait_flag(bool clear);
+int index_mma_wait_flag(bool clear);
+
 inline int num_sms() {
     static int n = 0;
     if (n == 0) {

@@ -378,6 +378,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace imma
 
+int index_mma_wait_flag(bool clear) { return read_device_flag(imma::g_imma_error, clear); }
+
 // Use the tensor-core scan for multi-query calls whose rows split into whole
 // 128-byte stages.
 bool index_mma_supported(int Nq, int HD, int64_t cap, int B) {

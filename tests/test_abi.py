@@ -46,7 +46,7 @@ def test_binding_covers_the_header():
 
 def test_status_strings():
     from sparse_attention_fp4_kv_b200 import binding as B
-    for st in (0, -1, -2, -3, -4, -5, -6):
+    for st in (0, -1, -2, -3, -4, -5, -6, -7):
         assert B.status_string(st) and B.status_string(st) != "unknown status"
     assert B.status_string(-99) == "unknown status"
 
@@ -80,6 +80,9 @@ def test_host_validation_codes():
     assert L.csa2_index_full(good, good, good, good, None, 0, 1, 16, 128, 10, None, good, None,
                              None) == 0
     assert L.csa2_topk(good, None, None, 0, 10, 5, good, None, 0, None) == 0
+    # the wait-timeout self-test checks its bound on the host
+    assert L.csa2_selftest_wait_timeout(0, None) == -4
+    assert L.csa2_selftest_wait_timeout(2000000, None) == -4
     # fused Full-layer selection: NULL, the shared-memory row limits, empty work
     fs = L.csa2_full_select
     assert fs(None, good, good, good, None, 1, 1, 4096, 2048, 512, good, good, None) == -1

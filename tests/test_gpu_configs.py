@@ -165,7 +165,10 @@ def test_reindex_group_b32_ctx256k_sampled():
 
 
 def test_decoder_stack20_b4_ctx1m_sampled():
+    from sparse_attention_fp4_kv_b200 import binding
+    binding.device_status(clear=True)
     wl = _workload("decoder_stack20_b4_ctx1m")
     _check(wl, [0, 3])
+    assert binding.device_status() == 0  # no kernel gave up a bounded wait
     del wl
     _free()

@@ -481,3 +481,19 @@ def test_index_full_multi_query_tensor_core_path(B, Nq, ctx0, H, D):
             ref = oracle.index_scores(qn[b, i], kn[b, :V], sn[b, :V])
             assert np.array_equal(f32_bits(tok[b, i, :V]), f32_bits(ref))
             assert np.array_equal(f32_bits(blk[b, i, :(V + 7) // 8]), f32_bits(oracle.block_scores(ref, V)))
+
+
+# ----------------------------------------------------------------------------- device-side status
+def test_device_status_reports_a_bounded_wait_timeout(B):
+    """A kernel whose wait nothing completes gives up at its bound, records it,
+    and returns; the host reads the flag and the context stays usable."""
+    B.device_status(clear=True)
+    assert B.device_status() == 0
+    B.selftest_wait_timeout(2000)
+    assert B.device_status() == -7
+    assert B.device_status(clear=True) == -7
+    assert B.device_status() == 0
+    score = torch.arange(100, device=DEV, dtype=torch.float32).view(1, 100)
+    out = torch.empty((1, 10), dtype=torch.int32, device=DEV)
+    B.csa2_topk(score, 10, out)
+    assert out.cpu().tolist() == [list(range(90, 100))]

@@ -61,9 +61,12 @@ def test_prefill_small_all_queries(ctx0, n):
 
 def test_prefill_4096_at_64k_sampled():
     from sparse_attention_fp4_kv_b200.workload import PrefillWorkload
+    from sparse_attention_fp4_kv_b200 import binding
+    binding.device_status(clear=True)
     pw = PrefillWorkload(synth.WORKLOADS["prefill_4096_at_64k"], "cuda", keep_kv_bf16=True)
     pw.step()
     torch.cuda.synchronize()
+    assert binding.device_status() == 0  # no kernel gave up a bounded wait
     _fp4_matches_oracle(pw)
     _check_queries(pw, [0, 1, 127, 128, 2049, 4095])
     del pw

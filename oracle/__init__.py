@@ -45,6 +45,7 @@ BLOCK_TOKENS = 8        # ... of 8 tokens (16,384 positions)
 TOPK = 512              # each query keeps its best 512
 N_WIN = 128             # sliding window: the last 128 tokens
 FP4_GROUP = 16          # one E4M3 scale per 16 channels
+MX_GROUP = 32           # MXFP4 variant: one E8M0 scale per 32 channels
 
 FULL, REINDEX, REUSE = "full", "reindex", "reuse"
 
@@ -86,6 +87,14 @@ def _L():
         lib.orc_fp4_quantize.argtypes = [P, c_i64, c_int, P, P]
         lib.orc_fp4_dequantize.restype = None
         lib.orc_fp4_dequantize.argtypes = [P, P, c_i64, c_int, P]
+        lib.orc_e8m0_value.restype = c_dbl
+        lib.orc_e8m0_value.argtypes = [ctypes.c_uint8]
+        lib.orc_mx_shared_exp.restype = c_int
+        lib.orc_mx_shared_exp.argtypes = [c_dbl]
+        lib.orc_mxfp4_quantize.restype = None
+        lib.orc_mxfp4_quantize.argtypes = [P, c_i64, c_int, P, P]
+        lib.orc_mxfp4_dequantize.restype = None
+        lib.orc_mxfp4_dequantize.argtypes = [P, P, c_i64, c_int, P]
         lib.orc_index_dots.restype = None
         lib.orc_index_dots.argtypes = [P, P, c_i64, c_int, P]
         lib.orc_index_scores.restype = c_int
@@ -163,6 +172,37 @@ def fp4_dequantize(packed: np.ndarray, sf: np.ndarray) -> np.ndarray:
     rows = packed.size // (C // 2)
     out = np.empty(packed.shape[:-1] + (C,), dtype=np.float64)
     _L().orc_fp4_dequantize(_p(packed), _p(sf), rows, C, _p(out))
+    return out
+
+
+def e8m0_value(code: int) -> float:
+    return _L().orc_e8m0_value(int(code))
+
+
+def mx_shared_exp(amax: float) -> int:
+    return int(_L().orc_mx_shared_exp(float(amax)))
+
+
+def mxfp4_quantize(x_bf16: np.ndarray):
+    """MXFP4 variant. x_bf16: uint16 bf16 bit patterns [..., C], C % 32 == 0.
+    Returns (packed uint8 [..., C/2], scales uint8 E8M0 [..., C/32])."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    C = x.shape[-1]
+    assert C % MX_GROUP == 0
+    rows = x.size // C
+    packed = np.empty(x.shape[:-1] + (C // 2,), dtype=np.uint8)
+    sf = np.empty(x.shape[:-1] + (C // MX_GROUP,), dtype=np.uint8)
+    _L().orc_mxfp4_quantize(_p(x), rows, C, _p(packed), _p(sf))
+    return packed, sf
+
+
+def mxfp4_dequantize(packed: np.ndarray, sf: np.ndarray) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    C = packed.shape[-1] * 2
+    rows = packed.size // (C // 2)
+    out = np.empty(packed.shape[:-1] + (C,), dtype=np.float64)
+    _L().orc_mxfp4_dequantize(_p(packed), _p(sf), rows, C, _p(out))
     return out
 
 
@@ -282,16 +322,21 @@ def window_rows(q_pos: int, swa_pos0: int, swa_rows: int, n_win: int = N_WIN):
 
 
 def sparse_attention(q_bf16, kv_bf16_rows_of, top, swa_bf16, q_pos, swa_pos0, scale,
-                     n_win=N_WIN):
+                     n_win=N_WIN, kv_format="nvfp4"):
     """One query (all heads) attends the selected main-KV tokens (quantized to
     FP4 by this oracle, then dequantized) followed by its sliding-window rows.
 
     kv_bf16_rows_of(positions) -> uint16 bf16 rows [len, C] of the main KV
-    before quantization; swa_bf16: [swa_rows, C] uint16 of this layer."""
+    before quantization; swa_bf16: [swa_rows, C] uint16 of this layer;
+    kv_format: "nvfp4" (E4M3 per 16 channels) or "mxfp4" (E8M0 per 32)."""
     sel = np.asarray(top, dtype=np.int64)
     sel = sel[sel >= 0]
-    packed, sf = fp4_quantize(kv_bf16_rows_of(sel))
-    main = fp4_dequantize(packed, sf)
+    if kv_format == "mxfp4":
+        packed, sf = mxfp4_quantize(kv_bf16_rows_of(sel))
+        main = mxfp4_dequantize(packed, sf)
+    else:
+        packed, sf = fp4_quantize(kv_bf16_rows_of(sel))
+        main = fp4_dequantize(packed, sf)
     rows = window_rows(int(q_pos), int(swa_pos0), swa_bf16.shape[0], n_win)
     swa = bf16_to_f64(np.asarray(swa_bf16)[rows])
     return attention(q_bf16, np.concatenate([main, swa], axis=0), scale)

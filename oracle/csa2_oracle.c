@@ -26,6 +26,9 @@
  *  - FP4 element: x / scale in fp32 IEEE division, then nearest E2M1 value,
  *    ties to the even code, saturating at 6, sign taken from x. A zero scale
  *    encodes every element as +0.
+ *  - MXFP4 variant: E8M0 scale per 32 channels = 2^(floor(log2(amax)) - 2),
+ *    clamped to 2^-127..2^127 (2^-127 for an all-zero block); element = nearest
+ *    E2M1 value of x / scale, ties to even, saturating at 6, sign from x.
  *  - Indexer score: (sum over heads and dims of int8*int8, exact) converted to
  *    fp32 with round-to-nearest-even, then one fp32 multiply by the key's scale.
  *  - Block score: max of the visible token scores in the 8-token block.
@@ -189,6 +192,84 @@ void orc_fp4_dequantize(const uint8_t *packed, const uint8_t *sf, int64_t rows, 
             uint8_t byte = packed[r * (C / 2) + c / 2];
             uint8_t code = (c & 1) ? (byte >> 4) : (byte & 0xF);
             double s = orc_e4m3_value(sf[r * (C / 16) + c / 16]);
+            out[r * C + c] = orc_e2m1_value(code) * s;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* MXFP4 variant. [T] mechanism 3 names the cache format MXFP4 and     */
+/* gives no detail; read as the OCP Microscaling format: E2M1 elements  */
+/* sharing one E8M0 scale per block of 32 channels.                     */
+/* E8M0: 8 exponent bits, bias 127, no sign, no mantissa; code e is     */
+/* 2^(e - 127) for e = 0..254, and code 255 is NaN.                     */
+/* ------------------------------------------------------------------ */
+double orc_e8m0_value(uint8_t code)
+{
+    if (code == 255)
+        return NAN;
+    return ldexp(1.0, (int)code - 127);
+}
+
+/* Shared exponent of a block whose largest magnitude is amax: the
+ * exponent of amax (floor(log2(amax))) minus 2, the largest E2M1
+ * exponent, clamped to the E8M0 range [-127, 127]; an all-zero block
+ * takes -127. frexp gives amax = m * 2^ex with m in [0.5, 1), so
+ * floor(log2(amax)) = ex - 1 exactly.                                    */
+int orc_mx_shared_exp(double amax)
+{
+    if (amax == 0.0)
+        return -127;
+    int ex;
+    frexp(amax, &ex);
+    int e = (ex - 1) - 2;
+    if (e < -127)
+        e = -127;
+    if (e > 127)
+        e = 127;
+    return e;
+}
+
+/* MXFP4 quantize-and-pack: per block of 32 channels, the shared scale
+ * 2^e (e from orc_mx_shared_exp of the block's amax); each element is the
+ * nearest E2M1 value of x / 2^e (an exact division by a power of two),
+ * ties to the even code, saturating at 6, sign taken from x.
+ *   packed : rows x C/2 bytes; byte i = code[2i] | code[2i+1] << 4
+ *   sf     : rows x C/32 E8M0 codes (e + 127)                           */
+void orc_mxfp4_quantize(const uint16_t *x, int64_t rows, int C, uint8_t *packed, uint8_t *sf)
+{
+    for (int64_t r = 0; r < rows; r++) {
+        const uint16_t *xr = x + r * C;
+        for (int g = 0; g < C / 32; g++) {
+            double amax = 0.0;
+            for (int c = 0; c < 32; c++) {
+                double v = fabs((double)bf16_to_float(xr[g * 32 + c]));
+                if (v > amax)
+                    amax = v;
+            }
+            int e = orc_mx_shared_exp(amax);
+            sf[r * (C / 32) + g] = (uint8_t)(e + 127);
+            for (int c = 0; c < 32; c += 2) {
+                uint8_t code[2];
+                for (int u = 0; u < 2; u++) {
+                    double v = ldexp((double)bf16_to_float(xr[g * 32 + c + u]), -e);
+                    code[u] = orc_e2m1_encode((float)v);
+                }
+                packed[r * (C / 2) + (g * 32 + c) / 2] = (uint8_t)(code[0] | (code[1] << 4));
+            }
+        }
+    }
+}
+
+/* Dequantize: value = e2m1(code) * e8m0(scale of the 32-channel block). */
+void orc_mxfp4_dequantize(const uint8_t *packed, const uint8_t *sf, int64_t rows, int C,
+                          double *out)
+{
+    for (int64_t r = 0; r < rows; r++) {
+        for (int c = 0; c < C; c++) {
+            uint8_t byte = packed[r * (C / 2) + c / 2];
+            uint8_t code = (c & 1) ? (byte >> 4) : (byte & 0xF);
+            double s = orc_e8m0_value(sf[r * (C / 32) + c / 32]);
             out[r * C + c] = orc_e2m1_value(code) * s;
         }
     }

@@ -101,6 +101,31 @@ class DecodeWorkload:
         """One decode step: append the new token, then every layer of the stack."""
         self.stack(stream)
 
+    def io_set(self):
+        """A second set of the per-step inputs (new KV row, main and indexer Q)
+        and outputs (attention outputs, top-k indices) with its own decode
+        stack over the same caches, pool and window rows, so that one step's
+        host copies can overlap another step's compute. Returns (stack,
+        inputs, outputs)."""
+        kv_new = self.kv_new.clone()
+        q = [t.clone() for t in self.q]
+        q_idx = [t.clone() if t is not None else None for t in self.q_idx]
+        out = [torch.empty_like(t) for t in self.out]
+        topk = [torch.empty_like(t) if t is not None else None for t in self.topk]
+        stack = csa2.DecodeStack(self.modes, q_idx, q, self.swa, out, topk, self.k_idx,
+                                 self.k_scale, self.kv_fp4, self.kv_sf, self.ctx_len, self.swa_pos0,
+                                 self.pool, self.scale, kv_new=kv_new, pool_ready=self.pool_ready)
+        inputs = [kv_new] + q + [t for t in q_idx if t is not None]
+        outputs = out + [t for t in topk if t is not None]
+        return stack, inputs, outputs
+
+    def io_tensors(self):
+        """The per-step inputs and outputs of the workload's own stack (same
+        order as io_set)."""
+        inputs = [self.kv_new] + list(self.q) + [t for t in self.q_idx if t is not None]
+        outputs = list(self.out) + [t for t in self.topk if t is not None]
+        return inputs, outputs
+
     def launches_per_step(self) -> int:
         """libcsa2 kernels one step launches: the append, then per Full layer
         the scan, the pool selection, the gather and the token selection; per

@@ -201,3 +201,117 @@ def test_fp4_row_bytes_match_pages():
     assert oracle.fp4_row_bytes(512) == int(vals["fp4_row_bytes_512"]) == 288
     packed, sf = oracle.fp4_quantize(np.zeros((3, 512), np.uint16))
     assert packed.shape[1] + sf.shape[1] == 288
+
+
+# ----------------------------------------------------------------------------- MXFP4 variant
+# [T] mechanism 3 names the cache format MXFP4; read as the OCP Microscaling
+# format: E2M1 elements, one E8M0 scale per 32 channels, shared exponent
+# floor(log2(amax)) - 2.
+def _bf16(x):
+    return np.asarray(x, dtype=np.float32).view(np.uint32) >> 16
+
+
+def _floor_log2(x: float) -> int:
+    """floor(log2(x)) of a positive float by exact integer arithmetic."""
+    n, d = Fraction(x).as_integer_ratio()
+    k = n.bit_length() - d.bit_length()
+    return k if (Fraction(n, d) >= Fraction(2) ** k) else k - 1
+
+
+def test_e8m0_decode_all_codes_closed_form_and_library():
+    lib = np.arange(256, dtype=np.uint8).view(ml_dtypes.float8_e8m0fnu).astype(np.float64)
+    for c in range(255):
+        v = oracle.e8m0_value(c)
+        assert v == lib[c] and Fraction(v) == Fraction(2) ** (c - 127), c
+    assert np.isnan(oracle.e8m0_value(255)) and np.isnan(lib[255])
+
+
+def test_mx_shared_exponent_closed_form():
+    rng = np.random.default_rng(21)
+    vals = list(2.0 ** rng.uniform(-140, 127, 3000)) + [1.0, 6.0, 7.99, 8.0, 0.25, 2.0 ** -126,
+                                                       2.0 ** -149, 3.0e38]
+    for amax in vals:
+        amax = float(np.float32(amax))
+        if amax == 0.0:
+            continue
+        ref = min(127, max(-127, _floor_log2(amax) - 2))
+        assert oracle.mx_shared_exp(amax) == ref, amax
+    assert oracle.mx_shared_exp(0.0) == -127
+    assert oracle.mx_shared_exp(6.0) == 0 and oracle.mx_shared_exp(1.0) == -2
+    assert oracle.mx_shared_exp(7.99) == 0 and oracle.mx_shared_exp(8.0) == 1
+
+
+def test_mxfp4_quantize_is_e2m1_of_the_scaled_block():
+    """Scale codes from the exact exponent of each block's amax; element codes
+    from the (library-pinned) E2M1 encoder of x / 2^e; packing low nibble first."""
+    rng = np.random.default_rng(22)
+    x = (rng.standard_normal((40, 128)) * np.exp(rng.uniform(-20, 20, (40, 1)))).astype(np.float32)
+    x[3, :32] = 0.0
+    x[5, 40:48] *= 1e4
+    xb = _bf16(x).astype(np.uint16)
+    xf = (xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    packed, sf = oracle.mxfp4_quantize(xb)
+    for r in range(x.shape[0]):
+        for g in range(4):
+            blk = xf[r, 32 * g:32 * g + 32]
+            amax = float(np.abs(blk).max())
+            e = -127 if amax == 0 else min(127, max(-127, _floor_log2(amax) - 2))
+            assert sf[r, g] == e + 127
+            codes = oracle.e2m1_encode_array((blk / 2.0 ** e).astype(np.float32))
+            got = np.stack([packed[r, 16 * g:16 * g + 16] & 15, packed[r, 16 * g:16 * g + 16] >> 4], 1)
+            assert np.array_equal(got.ravel(), codes), (r, g)
+
+
+def test_mxfp4_exact_round_trip_and_invariants():
+    rng = np.random.default_rng(23)
+    e2m1 = np.array([oracle.e2m1_value(c) for c in range(16)])
+    for _ in range(50):
+        s = int(rng.integers(-120, 120))
+        codes = rng.integers(0, 16, 32)
+        codes[rng.integers(0, 32)] = 6 + int(rng.integers(0, 2))   # amax in [4, 6]
+        x = e2m1[codes] * 2.0 ** s
+        xb = _bf16(x).astype(np.uint16)
+        packed, sf = oracle.mxfp4_quantize(xb[None])
+        assert sf[0, 0] == s + 127
+        assert np.array_equal(oracle.mxfp4_dequantize(packed, sf)[0], x)
+        # scaling by 2^t shifts only the scale code; negation flips only the signs
+        t = int(rng.integers(-5, 5))
+        p2, sf2 = oracle.mxfp4_quantize(_bf16(x * 2.0 ** t).astype(np.uint16)[None])
+        assert int(sf2[0, 0]) == int(sf[0, 0]) + t and np.array_equal(p2, packed)
+        p3, sf3 = oracle.mxfp4_quantize(_bf16(-x).astype(np.uint16)[None])
+        assert np.array_equal(sf3, sf)
+        assert np.all((p3 ^ packed) == 0x88)  # every sign bit flips (zeros too)
+
+
+def test_mxfp4_error_bound_saturation_and_zero_block():
+    rng = np.random.default_rng(24)
+    x = rng.standard_normal((64, 64)).astype(np.float32) * 3.0
+    xb = _bf16(x).astype(np.uint16)
+    xf = (xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    packed, sf = oracle.mxfp4_quantize(xb)
+    xh = oracle.mxfp4_dequantize(packed, sf)
+    scale = np.repeat(2.0 ** (sf.astype(np.float64) - 127), 32, axis=1)
+    v = np.abs(xf) / scale
+    err = np.abs(xf - xh) / scale
+    # spacing of E2M1 is 0.5 below 2, 1 below 4, 2 below 6; |v| < 8 saturates at 6
+    assert np.all(v < 8)
+    assert np.all(err[v <= 2] <= 0.25) and np.all(err[(v > 2) & (v <= 4)] <= 0.5)
+    assert np.all(err[(v > 4) & (v <= 6)] <= 1.0) and np.all(err[v > 6] <= 2.0)
+    z, zs = oracle.mxfp4_quantize(np.zeros((1, 32), np.uint16))
+    assert zs[0, 0] == 0 and np.all(z == 0) and np.all(oracle.mxfp4_dequantize(z, zs) == 0)
+
+
+def test_mxfp4_dequantize_every_code_and_scale_is_exact_product():
+    codes = np.arange(16, dtype=np.uint8)
+    packed = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)
+    packed = np.tile(packed, 4)[None]                      # 32 channels
+    for e in range(255):
+        out = oracle.mxfp4_dequantize(packed, np.array([[e]], np.uint8))[0]
+        for c in range(32):
+            assert Fraction(out[c]) == Fraction(oracle.e2m1_value(c % 16)) * Fraction(2) ** (e - 127)
+
+
+def test_mxfp4_row_bytes():
+    # 512 channels: 256 bytes of E2M1 codes + 16 E8M0 scales
+    packed, sf = oracle.mxfp4_quantize(np.zeros((1, 512), np.uint16))
+    assert packed.shape[-1] + sf.shape[-1] == 272

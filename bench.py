@@ -374,11 +374,12 @@ def _e2e(wl, args, stream, world, local_rank):
     """Same metric through the public API with pinned host buffers: every step
     copies that step's inputs host->device (the new KV row, every layer's main Q
     and indexer Q), runs the decode stack, and reads every layer's output and
-    top-k indices back to the host. As in a serving loop, the copies run on a
-    second stream and overlap the neighbouring steps' compute: two sets of
-    per-step device buffers alternate, events order each step's copy-in,
-    compute and copy-out, and compute stays strictly in step order on one
-    stream. The timed region spans the first copy-in to the last copy-out."""
+    top-k indices back to the host. As in a serving loop, the copies overlap the
+    neighbouring steps' compute: inputs go up on one stream and results come
+    back on another, two sets of per-step device buffers alternate, events
+    order each step's copy-in, compute and copy-out, and compute stays strictly
+    in step order on one stream. The timed region spans the first copy-in to
+    the last copy-out."""
     import torch.distributed as dist
     dev = wl.device
     sets = []
@@ -396,7 +397,8 @@ def _e2e(wl, args, stream, world, local_rank):
     h2d = sum(h.numel() * h.element_size() for _, h in sets[0][1])
     d2h = sum(h.numel() * h.element_size() for _, h in sets[0][2])
     E = max(1, min(args.steps, 200))
-    copy = torch.cuda.Stream(device=dev)
+    up = torch.cuda.Stream(device=dev)
+    down = torch.cuda.Stream(device=dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_done = [torch.cuda.Event() for _ in range(2)]
     ev_out = [torch.cuda.Event() for _ in range(2)]
@@ -405,22 +407,22 @@ def _e2e(wl, args, stream, world, local_rank):
     def enqueue(k):
         i = k % 2
         stack, ins, outs = sets[i]
-        with torch.cuda.stream(copy):
+        with torch.cuda.stream(up):
             if started[i]:
-                copy.wait_event(ev_done[i])  # the set's previous step has read its inputs
+                up.wait_event(ev_done[i])  # the set's previous step has read its inputs
             for d, h in ins:
                 d.copy_(h, non_blocking=True)
-            ev_in[i].record(copy)
+            ev_in[i].record(up)
         stream.wait_event(ev_in[i])
         if started[i]:
             stream.wait_event(ev_out[i])  # ... and its outputs have been read back
         stack(stream)
         ev_done[i].record(stream)
-        with torch.cuda.stream(copy):
-            copy.wait_event(ev_done[i])
+        with torch.cuda.stream(down):
+            down.wait_event(ev_done[i])
             for d, h in outs:
                 h.copy_(d, non_blocking=True)
-            ev_out[i].record(copy)
+            ev_out[i].record(down)
         started[i] = True
 
     for k in range(4):
@@ -430,7 +432,7 @@ def _e2e(wl, args, stream, world, local_rank):
         dist.barrier(device_ids=[local_rank])
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    copy.wait_event(a)
+    up.wait_event(a)
     for k in range(E):
         enqueue(k)
     stream.wait_event(ev_out[(E - 1) % 2])
@@ -441,7 +443,7 @@ def _e2e(wl, args, stream, world, local_rank):
     ms = replicas.slowest([ms], dev)[0]
     return {"value": replicas.aggregate_rate(wl.w.n_layers, world, ms), "unit": UNIT, "ms_per_step": ms,
             "steps": E, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "overlap": "copies on a second stream, two alternating buffer sets"}
+            "overlap": "inputs and results copied on two more streams, two alternating buffer sets"}
 
 
 def main():

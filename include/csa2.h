@@ -108,6 +108,20 @@ int csa2_kv_append_fp4(const void *kv_bf16, int B, int n_new, int C, const int64
                        int64_t cap, uint8_t *kv_fp4, uint8_t *kv_sf, void *stream);
 
 /* ------------------------------------------------------------------------
+ * MXFP4 variant of the append ([T] mechanism 3 calls the cache format MXFP4
+ * and gives no detail; read as the OCP Microscaling format): E2M1 elements,
+ * one E8M0 scale per 32 channels.
+ * For token row (b, i) at p = start_pos[b] + i, per 32-channel block g:
+ *   e = clamp(floor(log2(amax_g)) - 2, -127, 127)   (-127 when amax_g = 0)
+ *   element c: code = E2M1_rn_satfinite(x_c * 2^-e)   (an exact scaling)
+ *   kv_fp4[b][p][c/2]: as csa2_kv_append_fp4;  kv_sf[b][p][g] = e + 127
+ *  kv_sf [B][cap][C/32] uint8 (E8M0); C % 32 == 0, 32 <= C <= 8192; other
+ *  arguments and errors as csa2_kv_append_fp4.
+ * ------------------------------------------------------------------------ */
+int csa2_kv_append_mxfp4(const void *kv_bf16, int B, int n_new, int C, const int64_t *start_pos,
+                         int64_t cap, uint8_t *kv_fp4, uint8_t *kv_sf, void *stream);
+
+/* ------------------------------------------------------------------------
  * Full-mode indexer scan ([N] CSA2 section: a Full layer projects indexer K
  * and scores the context; [G] indexer section: 8-token blocks).
  *
@@ -243,6 +257,15 @@ int csa2_sparse_attn_decode(const void *q_bf16, const uint8_t *kv_fp4, const uin
                             const int64_t *swa_pos0, int swa_rows, const int64_t *q_pos,
                             int n_win, int B, int Nq, int Hq, int C, float softmax_scale,
                             float *out, void *ws, size_t ws_bytes, void *stream);
+
+/* The same attention over an MXFP4 cache (csa2_kv_append_mxfp4): kv_sf is
+ * [B][cap][C/32] E8M0, a row's value is e2m1(code) * 2^(e - 127); C % 32 == 0.
+ * Everything else, including the workspace size, as csa2_sparse_attn_decode. */
+int csa2_sparse_attn_decode_mxfp4(const void *q_bf16, const uint8_t *kv_fp4, const uint8_t *kv_sf,
+                                  int64_t cap, const int32_t *topk, int K, const void *swa_bf16,
+                                  const int64_t *swa_pos0, int swa_rows, const int64_t *q_pos,
+                                  int n_win, int B, int Nq, int Hq, int C, float softmax_scale,
+                                  float *out, void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
  * One decode step of a CSA2 layer stack ([N] CSA2 section: static per-layer

@@ -58,6 +58,7 @@ _SIGS = {
     "csa2_device_status": (_I, [_I]),
     "csa2_selftest_wait_timeout": (_I, [_I, _P]),
     "csa2_kv_append_fp4": (_I, [_P, _I, _I, _I, _P, _I64, _P, _P, _P]),
+    "csa2_kv_append_mxfp4": (_I, [_P, _I, _I, _I, _P, _I64, _P, _P, _P]),
     "csa2_index_full": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _P, _P, _P, _P]),
     "csa2_topk_workspace_size": (_SZ, [_I, _I64, _I]),
     "csa2_topk": (_I, [_P, _P, _P, _I, _I64, _I, _P, _P, _SZ, _P]),
@@ -67,6 +68,8 @@ _SIGS = {
     "csa2_sparse_attn_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "csa2_sparse_attn_decode": (_I, [_P, _P, _P, _I64, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I,
                                      _I, _F, _P, _P, _SZ, _P]),
+    "csa2_sparse_attn_decode_mxfp4": (_I, [_P, _P, _P, _I64, _P, _I, _P, _P, _I, _P, _I, _I, _I,
+                                           _I, _I, _F, _P, _P, _SZ, _P]),
     "csa2_decode_stack_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I64]),
     "csa2_decode_stack": (_I, [ctypes.POINTER(csa2_layer), _I, _P, _P, _P, _P, _P, _I64, _P, _P,
                                _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _P, _SZ, _P]),
@@ -115,17 +118,19 @@ def _want(t: torch.Tensor, dtype, name: str):
 
 # ----------------------------------------------------------------------------- calls
 def csa2_kv_append_fp4(kv_bf16: torch.Tensor, start_pos: torch.Tensor, kv_fp4: torch.Tensor,
-                       kv_sf: torch.Tensor, stream=None) -> None:
+                       kv_sf: torch.Tensor, stream=None, mx: bool = False) -> None:
     """kv_bf16 [B][n_new][C] bf16; start_pos [B] int64; kv_fp4 [B][cap][C/2] uint8;
-    kv_sf [B][cap][C/16] uint8."""
+    kv_sf [B][cap][C/16] uint8 (E4M3), or with mx the MXFP4 variant's
+    [B][cap][C/32] E8M0 (csa2_kv_append_mxfp4)."""
     _want(kv_bf16, torch.bfloat16, "kv_bf16")
     _want(start_pos, torch.int64, "start_pos")
     _want(kv_fp4, torch.uint8, "kv_fp4")
     _want(kv_sf, torch.uint8, "kv_sf")
     B, n, C = kv_bf16.shape
     cap = kv_fp4.shape[1]
-    assert kv_fp4.shape == (B, cap, C // 2) and kv_sf.shape == (B, cap, C // 16)
-    _check("csa2_kv_append_fp4", lib.csa2_kv_append_fp4(
+    assert kv_fp4.shape == (B, cap, C // 2) and kv_sf.shape == (B, cap, C // (32 if mx else 16))
+    name = "csa2_kv_append_mxfp4" if mx else "csa2_kv_append_fp4"
+    _check(name, getattr(lib, name)(
         _ptr(kv_bf16), B, n, C, _ptr(start_pos), cap, _ptr(kv_fp4), _ptr(kv_sf), _stream(stream)))
 
 
@@ -220,9 +225,10 @@ def sparse_attn_workspace_size(B, Nq, Hq, C, K, n_win=N_WIN) -> int:
 
 
 def csa2_sparse_attn_decode(q_bf16, kv_fp4, kv_sf, topk, swa_bf16, swa_pos0, out, softmax_scale,
-                            q_pos=None, n_win=N_WIN, ws=None, stream=None) -> None:
+                            q_pos=None, n_win=N_WIN, ws=None, stream=None, mx: bool = False) -> None:
     """q_bf16 [B][Nq][Hq][C]; topk [B][Nq][K] int32; swa_bf16 [B][rows][C] bf16;
-    swa_pos0 [B] int64; out [B][Nq][Hq][C] fp32."""
+    swa_pos0 [B] int64; out [B][Nq][Hq][C] fp32; with mx the cache is the MXFP4
+    variant (csa2_sparse_attn_decode_mxfp4)."""
     _want(q_bf16, torch.bfloat16, "q_bf16")
     _want(out, torch.float32, "out")
     B, Nq, Hq, C = q_bf16.shape
@@ -233,7 +239,8 @@ def csa2_sparse_attn_decode(q_bf16, kv_fp4, kv_sf, topk, swa_bf16, swa_pos0, out
     if need and ws is None:
         ws = torch.empty(need, dtype=torch.uint8, device=q_bf16.device)
     wsb = ws.numel() * ws.element_size() if ws is not None else 0
-    _check("csa2_sparse_attn_decode", lib.csa2_sparse_attn_decode(
+    name = "csa2_sparse_attn_decode_mxfp4" if mx else "csa2_sparse_attn_decode"
+    _check(name, getattr(lib, name)(
         _ptr(q_bf16), _ptr(kv_fp4), _ptr(kv_sf), cap, _ptr(topk), K, _ptr(swa_bf16),
         _ptr(swa_pos0), rows, _ptr(q_pos), n_win, B, Nq, Hq, C, float(softmax_scale), _ptr(out),
         _ptr(ws), wsb, _stream(stream)))

@@ -49,11 +49,11 @@ __global__ void __launch_bounds__(256) attn_general_kernel(AttnArgs a) {
             if (valid) {
                 const int64_t cell = (int64_t)b * a.cap + pos;
                 const uint8_t *row = a.kv_fp4 + cell * (C / 2);
-                const uint8_t *sfr = a.kv_sf + cell * (C / 16);
+                const uint8_t *sfr = a.kv_sf + cell * (C / (a.mx ? 32 : 16));
                 for (int u = 0; u < CPL; u += 2) {
                     const int c = lane * CPL + u;
                     const uint32_t byte = row[c / 2];
-                    const float s = e4m3_to_f32(sfr[c / 16]);
+                    const float s = kv_group_scale(sfr, c / 16, a.mx);
                     dot += qs[c] * (e2m1_to_f32(byte & 0xF) * s);
                     dot += qs[c + 1] * (e2m1_to_f32(byte >> 4) * s);
                 }
@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(256) attn_general_kernel(AttnArgs a) {
             const int64_t cell = (int64_t)b * a.cap + a.topk[bq * a.K + j];
             const uint32_t byte = a.kv_fp4[cell * (C / 2) + c / 2];
             const float v = e2m1_to_f32((c & 1) ? (byte >> 4) : (byte & 0xF)) *
-                            e4m3_to_f32(a.kv_sf[cell * (C / 16) + c / 16]);
+                            kv_group_scale(a.kv_sf + cell * (C / (a.mx ? 32 : 16)), c / 16, a.mx);
             acc += p * v;
         }
         const uint16_t *swa = reinterpret_cast<const uint16_t *>(a.swa) +
@@ -146,6 +146,18 @@ extern "C" int csa2_sparse_attn_decode(const void *q_bf16, const uint8_t *kv_fp4
                                        void *ws, size_t ws_bytes, void *stream) {
     AttnArgs a{q_bf16, kv_fp4, kv_sf, cap, topk, K, swa_bf16, swa_pos0, swa_rows, q_pos,
                n_win, B, Nq, Hq, C, softmax_scale, out, ws, false, false};
+    return attn_checked_launch(a, ws_bytes, (cudaStream_t)stream);
+}
+
+extern "C" int csa2_sparse_attn_decode_mxfp4(const void *q_bf16, const uint8_t *kv_fp4,
+                                             const uint8_t *kv_sf, int64_t cap, const int32_t *topk,
+                                             int K, const void *swa_bf16, const int64_t *swa_pos0,
+                                             int swa_rows, const int64_t *q_pos, int n_win, int B,
+                                             int Nq, int Hq, int C, float softmax_scale, float *out,
+                                             void *ws, size_t ws_bytes, void *stream) {
+    if (C % 32) return CSA2_ERR_SHAPE;
+    AttnArgs a{q_bf16, kv_fp4, kv_sf, cap, topk, K, swa_bf16, swa_pos0, swa_rows, q_pos,
+               n_win, B, Nq, Hq, C, softmax_scale, out, ws, false, false, true};
     return attn_checked_launch(a, ws_bytes, (cudaStream_t)stream);
 }
 

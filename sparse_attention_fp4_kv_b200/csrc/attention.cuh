@@ -29,6 +29,9 @@ struct AttnArgs {
     // kernels earlier, so the selected rows may be gathered and dequantized
     // before the wait.
     bool prefetch;
+    // Scales of the FP4 rows: E4M3 per 16 channels (kv_sf [B][cap][C/16]), or
+    // with mx the MXFP4 variant's E8M0 per 32 channels (kv_sf [B][cap][C/32]).
+    bool mx;
 };
 
 // Sliding-window rows of query bq: rows [row0, row0 + n) of the SWA tensor,

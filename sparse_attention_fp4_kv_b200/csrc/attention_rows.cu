@@ -340,7 +340,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                         const int64_t src = (int64_t)b * a.cap + pos;
                         codes[u] = vrow[u] ? __ldg(reinterpret_cast<const uint2 *>(a.kv_fp4 + src * 256) + lane)
                                            : make_uint2(0, 0);
-                        const uint32_t sb = vrow[u] ? (uint32_t)__ldg(a.kv_sf + src * 32 + lane) : 0u;
+                        // E4M3 of this lane's 16-channel group, or the E8M0 of its 32-channel block
+                        const uint32_t sb =
+                            vrow[u] ? (uint32_t)__ldg(a.mx ? a.kv_sf + src * 16 + (lane >> 1)
+                                                           : a.kv_sf + src * 32 + lane)
+                                    : 0u;
                         scl[u >> 2] |= sb << (8 * (u & 3));
                     }
                     // indices of the next selected tile, while these loads are in flight
@@ -363,7 +367,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int u = 0; u < LROWS; u++) {
                         const int j = wl + (NLOAD / 32) * u;
-                        const float s = e4m3_to_f32((scl[u >> 2] >> (8 * (u & 3))) & 0xFF);
+                        const uint32_t sc = (scl[u >> 2] >> (8 * (u & 3))) & 0xFF;
+                        const float s = a.mx ? e8m0_to_f32(sc) : e4m3_to_f32(sc);
                         uint32_t wds[8];
 #pragma unroll
                         for (int e = 0; e < 8; e++) {

@@ -243,10 +243,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (waited && tid == 0) issue_q_swa();
         for (int i = tid; i < T * 18; i += THREADS) {  // (slot, 16-byte piece of its 288 B)
             const int j = i / 18, pc = i - j * 18;
-            if (slot_kind[j] != 1) continue;
+            if (slot_kind[j] != 1 || (a.mx && pc == 17)) continue;  // MXFP4: 16 scale bytes
             const int64_t cell = slot_src[j];
-            const uint8_t *src =
-                pc < 16 ? a.kv_fp4 + cell * 256 + pc * 16 : a.kv_sf + cell * 32 + (pc - 16) * 16;
+            const uint8_t *src = pc < 16 ? a.kv_fp4 + cell * 256 + pc * 16
+                                         : a.kv_sf + cell * (a.mx ? 16 : 32) + (pc - 16) * 16;
             cp_async16(base + FP4_STAGE_OFF + j * 288 + pc * 16, src);
         }
         cp_async_wait_all();
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int j = i >> 5, g = i & 31;
             if (slot_kind[j] != 1) continue;
             const uint2 codes = *reinterpret_cast<const uint2 *>(stage + j * 288 + g * 8);
-            const float s = e4m3_to_f32(stage[j * 288 + 256 + g]);
+            const float s = kv_group_scale(stage + j * 288 + 256, g, a.mx);
             uint32_t wds[8];
 #pragma unroll
             for (int u = 0; u < 8; u++) {

@@ -109,6 +109,18 @@ __device__ __forceinline__ float e2m1_to_f32(uint32_t c4) {
 }
 
 // fp32 -> E4M3 with round-to-nearest-even and saturation to +-448 (PTX cvt).
+// E8M0 scale (MXFP4 variant): code e is 2^(e - 127), 255 is NaN; code 0 is the
+// fp32 subnormal 2^-127.
+__device__ __forceinline__ float e8m0_to_f32(uint32_t code) {
+    if (code == 255u) return __uint_as_float(0x7FC00000u);
+    return code == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(code << 23);
+}
+// Scale of 16-channel group g of a row whose scale bytes start at sf: E4M3
+// per 16 channels, or (mx) E8M0 per 32 channels.
+__device__ __forceinline__ float kv_group_scale(const uint8_t *sf, int g, bool mx) {
+    return mx ? e8m0_to_f32(sf[g >> 1]) : e4m3_to_f32(sf[g]);
+}
+
 __device__ __forceinline__ uint32_t f32_to_e4m3_satfinite(float x) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));

@@ -60,6 +60,57 @@ __global__ void __launch_bounds__(256) kv_append_fp4_kernel(
     sf[cell * G + g] = (uint8_t)scode;
 }
 
+// MXFP4 variant: one thread per 32-channel block. The shared exponent is the
+// exponent of the block's amax minus 2 (the largest E2M1 exponent), clamped to
+// the E8M0 range: read straight from the fp32 exponent field, so an all-zero or
+// subnormal amax gives 2^-127. Elements are x * 2^-e, an exact scaling since
+// the result stays below 8, then the same E2M1 pair conversion.
+__global__ void __launch_bounds__(256) kv_append_mxfp4_kernel(
+    const uint16_t *__restrict__ kv, int B, int n_new, int C, const int64_t *__restrict__ start_pos,
+    int64_t pos_offset, int64_t cap, uint8_t *__restrict__ fp4, uint8_t *__restrict__ sf) {
+    grid_dep_wait();
+    grid_dep_launch();
+    const int G = C / 32;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t total = (int64_t)B * n_new * G;
+    if (gid >= total) return;
+    const int g = (int)(gid % G);
+    const int64_t row = gid / G;
+    const int i = (int)(row % n_new);
+    const int b = (int)(row / n_new);
+    const int64_t pos = start_pos[b] + pos_offset + i;
+    if (pos < 0 || pos >= cap) return;
+
+    const uint4 *src = reinterpret_cast<const uint4 *>(kv + row * C + (int64_t)g * 32);
+    float x[32];
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+        const uint4 a = src[q];
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            x[8 * q + 2 * j] = bf16_lo(w[j]);
+            x[8 * q + 2 * j + 1] = bf16_hi(w[j]);
+        }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; j++) amax = fmaxf(amax, fabsf(x[j]));
+    const int E = (int)((__float_as_uint(amax) >> 23) & 0xFF);  // 0 for zero / subnormal
+    int e = E == 0 ? -127 : E - 129;
+    e = e < -127 ? -127 : e;
+    // 2^-e as an fp32 (2^-127 .. 2^127; -e = -127 is the subnormal 2^-127)
+    const float inv = -e >= -126 ? __uint_as_float((uint32_t)(127 - e) << 23) : __uint_as_float(0x00400000u);
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; j++) v[j] = x[j] * inv;
+    const int64_t cell = (int64_t)b * cap + pos;
+    uint2 *dst = reinterpret_cast<uint2 *>(fp4 + cell * (C / 2) + (int64_t)g * 16);
+    dst[0] = make_uint2(f32x8_to_e2m1x8(v), f32x8_to_e2m1x8(v + 8));
+    dst[1] = make_uint2(f32x8_to_e2m1x8(v + 16), f32x8_to_e2m1x8(v + 24));
+    sf[cell * G + g] = (uint8_t)(e + 127);
+}
+
 int launch_kv_append(const uint16_t *kv, int B, int n_new, int C, const int64_t *pos_base,
                      int64_t pos_offset, int64_t cap, uint8_t *fp4, uint8_t *sf, cudaStream_t s,
                      bool pdl) {
@@ -83,4 +134,21 @@ extern "C" int csa2_kv_append_fp4(const void *kv_bf16, int B, int n_new, int C,
     if (!aligned(kv_bf16, 16) || !aligned(kv_fp4, 8)) return CSA2_ERR_ALIGN;
     return launch_kv_append((const uint16_t *)kv_bf16, B, n_new, C, start_pos, 0, cap, kv_fp4,
                             kv_sf, (cudaStream_t)stream);
+}
+
+extern "C" int csa2_kv_append_mxfp4(const void *kv_bf16, int B, int n_new, int C,
+                                    const int64_t *start_pos, int64_t cap, uint8_t *kv_fp4,
+                                    uint8_t *kv_sf, void *stream) {
+    using namespace csa2;
+    if (!kv_bf16 || !start_pos || !kv_fp4 || !kv_sf) return CSA2_ERR_NULL;
+    if (B < 0 || n_new < 0 || cap < 0 || C < 32 || C > 8192 || C % 32) return CSA2_ERR_SHAPE;
+    if (!aligned(kv_bf16, 16) || !aligned(kv_fp4, 8)) return CSA2_ERR_ALIGN;
+    const int64_t total = (int64_t)B * n_new * (C / 32);
+    if (total == 0) return CSA2_OK;
+    const int threads = 256;
+    const int64_t blocks = (total + threads - 1) / threads;
+    if (blocks > INT32_MAX) return CSA2_ERR_SHAPE;
+    return launch_kernel(false, kv_append_mxfp4_kernel, dim3((unsigned)blocks), dim3(threads), 0,
+                         (cudaStream_t)stream, (const uint16_t *)kv_bf16, B, n_new, C, start_pos,
+                         (int64_t)0, cap, kv_fp4, kv_sf);
 }

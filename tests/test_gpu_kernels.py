@@ -101,6 +101,63 @@ def test_append_out_of_range_positions_are_skipped(B):
     assert np.all(sfn[1, :1] != 0) and np.all(sfn[1, 1:] == 0)
 
 
+# ----------------------------------------------------------------------------- MXFP4 variant
+def _append_mx_and_compare(B, x_bf16: torch.Tensor, cap_extra=3):
+    """MXFP4 append (E8M0 per 32 channels) against the oracle, bit for bit."""
+    Bn, n, C = x_bf16.shape
+    cap = n + cap_extra
+    start = (torch.arange(Bn, dtype=torch.int64) % (cap_extra + 1)).to(DEV)
+    fp4 = torch.full((Bn, cap, C // 2), 0xAB, dtype=torch.uint8, device=DEV)
+    sf = torch.full((Bn, cap, C // 32), 0xCD, dtype=torch.uint8, device=DEV)
+    B.csa2_kv_append_fp4(x_bf16, start, fp4, sf, mx=True)
+    torch.cuda.synchronize()
+    xp, xs = oracle.mxfp4_quantize(bf16_np(x_bf16))
+    g4, gs = fp4.cpu().numpy(), sf.cpu().numpy()
+    for b in range(Bn):
+        s0 = int(start[b])
+        assert np.array_equal(g4[b, s0:s0 + n], xp[b]), f"packed bytes differ (b={b})"
+        assert np.array_equal(gs[b, s0:s0 + n], xs[b]), f"E8M0 scales differ (b={b})"
+        assert np.all(g4[b, :s0] == 0xAB) and np.all(gs[b, s0 + n:] == 0xCD)
+
+
+def test_append_mxfp4_synthetic_rows_and_random_bits(B):
+    w = synth.scaled(synth.WORKLOADS["decoder_group1_b8_ctx128k"], ctx=300)
+    _append_mx_and_compare(B, torch.stack([synth.main_kv_bf16(w, b, 0, 300, DEV) for b in range(3)]))
+    g = torch.Generator(device=DEV).manual_seed(15)
+    bits = torch.randint(0, 1 << 16, (3, 129, 512), generator=g, device=DEV, dtype=torch.int32)
+    x = bits.to(torch.int16).view(torch.bfloat16)
+    x = torch.where(torch.isfinite(x.float()), x, torch.zeros_like(x))
+    _append_mx_and_compare(B, x.contiguous())
+
+
+def test_append_mxfp4_special_blocks(B):
+    """Zero and negative-zero blocks, subnormal and near-maximum amax, amax at
+    and just below powers of two, E2M1 ties and the saturation band (6, 8)."""
+    rows = [np.zeros(32), -np.zeros(32), np.full(32, 2.0 ** -130), np.full(32, -(2.0 ** -133)),
+            np.array([3.0e38] + [1.0] * 31), np.array([2.0 ** 10] + [3.0] * 31),
+            np.array([2.0 ** 10 - 4.0] + [-3.0] * 31)]
+    for k in range(-6, 7, 3):
+        s = 2.0 ** k
+        ties = np.array([.25, .75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.5, 7.0, 7.75, -0.25, -2.5, -5.0,
+                         4.0, 0.0, -0.0] * 2) * s
+        rows.append(ties)
+    x = torch.from_numpy(np.stack(rows).astype(np.float32)).to(torch.bfloat16).to(DEV)
+    _append_mx_and_compare(B, x.view(1, -1, 32).contiguous(), cap_extra=0)
+
+
+@pytest.mark.parametrize("C", [32, 96, 512])
+def test_append_mxfp4_channel_counts(B, C):
+    g = torch.Generator(device=DEV).manual_seed(C + 1)
+    _append_mx_and_compare(B, (torch.randn(2, 17, C, generator=g, device=DEV) * 5).to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("Bn,ctx,C,Hq,K,Nq", [(3, 4000, 512, 64, 512, 1),     # split-key clusters
+                                              (70, 900, 512, 64, 512, 1),      # one CTA per row
+                                              (2, 2000, 128, 8, 512, 1)])      # general kernel
+def test_sparse_attention_mxfp4(B, Bn, ctx, C, Hq, K, Nq):
+    _attention_case(B, Bn, ctx, C, Hq, K, 128, seed=Bn + ctx + 3, Nq=Nq, drop=7, mx=True)
+
+
 # ----------------------------------------------------------------------------- a2/a3 scan
 def _index_inputs(Bn, cap, H, D, seed):
     g = torch.Generator(device=DEV).manual_seed(seed)
@@ -365,13 +422,13 @@ def test_reindex_bitexact(B):
 
 
 # ----------------------------------------------------------------------------- a8 attention
-def _attention_case(B, Bn, ctx, C, Hq, K, n_win, seed, q_pos=None, Nq=1, drop=0):
+def _attention_case(B, Bn, ctx, C, Hq, K, n_win, seed, q_pos=None, Nq=1, drop=0, mx=False):
     w = synth.scaled(synth.WORKLOADS["decoder_group1_b8_ctx128k"], B=Bn, ctx=ctx, C=C, Hq=Hq,
                      seed=seed)
     kv = torch.stack([synth.main_kv_bf16(w, b, 0, ctx, DEV) for b in range(Bn)])
     fp4 = torch.empty((Bn, ctx, C // 2), dtype=torch.uint8, device=DEV)
-    sf = torch.empty((Bn, ctx, C // 16), dtype=torch.uint8, device=DEV)
-    B.csa2_kv_append_fp4(kv, torch.zeros(Bn, dtype=torch.int64, device=DEV), fp4, sf)
+    sf = torch.empty((Bn, ctx, C // (32 if mx else 16)), dtype=torch.uint8, device=DEV)
+    B.csa2_kv_append_fp4(kv, torch.zeros(Bn, dtype=torch.int64, device=DEV), fp4, sf, mx=mx)
     q = synth.main_q(w, 0, Nq, DEV)
     g = torch.Generator(device=DEV).manual_seed(seed)
     kk = min(K, ctx)
@@ -387,14 +444,15 @@ def _attention_case(B, Bn, ctx, C, Hq, K, n_win, seed, q_pos=None, Nq=1, drop=0)
     out = torch.empty((Bn, Nq, Hq, C), device=DEV)
     scale = 1.0 / math.sqrt(C)
     B.csa2_sparse_attn_decode(q, fp4, sf, top.contiguous(), swa, pos0, out, scale, q_pos=q_pos,
-                              n_win=n_win)
+                              n_win=n_win, mx=mx)
     torch.cuda.synchronize()
     kvn, qn, topn, swan = bf16_np(kv), bf16_np(q), top.cpu().numpy(), bf16_np(swa)
     for b in range(Bn):
         for i in range(Nq):
             p = (ctx - 1) if q_pos is None else int(q_pos[b, i])
             ref = oracle.sparse_attention(qn[b, i], lambda P: kvn[b][P], topn[b, i], swan[b], p,
-                                          ctx - rows, scale, n_win)
+                                          ctx - rows, scale, n_win,
+                                          kv_format="mxfp4" if mx else "nvfp4")
             assert_attn_close(out[b, i].cpu().numpy(), ref, f"b={b} i={i}")
 
 

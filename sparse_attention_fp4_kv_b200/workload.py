@@ -101,6 +101,18 @@ class DecodeWorkload:
         """One decode step: append the new token, then every layer of the stack."""
         self.stack(stream)
 
+    def capture_step_graph(self):
+        """One decode step (the csa2_decode_stack call) captured as a CUDA graph
+        on a side stream; replay() runs the step again on the same buffers.
+        Call a step first, outside the capture (one-time kernel set-up)."""
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device=self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.graph(graph, stream=side):
+            self.stack(side)
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        return graph
+
     def io_set(self):
         """A second set of the per-step inputs (new KV row, main and indexer Q)
         and outputs (attention outputs, top-k indices) with its own decode

@@ -122,6 +122,28 @@ def test_launches_per_step_matches_profiler(ctx):
     _free()
 
 
+def test_decode_step_replays_as_a_cuda_graph():
+    """The step captured as a CUDA graph (dependent launches become graph
+    edges) gives the same pools, indices and outputs, bit for bit, as the
+    directly launched step."""
+    wl = _workload("decoder_stack20_b4_ctx1m", B=2, ctx=30011)
+    wl.step()
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in wl.topk if t is not None] + [o.clone() for o in wl.out] + [wl.pool.clone()]
+    for t in [t for t in wl.topk if t is not None] + list(wl.out):
+        t.zero_()
+    g = wl.capture_step_graph()
+    g.replay()
+    torch.cuda.synchronize()
+    got = [t for t in wl.topk if t is not None] + list(wl.out) + [wl.pool]
+    for x, y in zip(ref, got):
+        assert torch.equal(x, y)
+    from sparse_attention_fp4_kv_b200 import binding
+    assert binding.device_status() == 0
+    del g, wl
+    _free()
+
+
 def test_decode_step_is_deterministic():
     wl = _workload("decoder_stack20_b4_ctx1m", B=2, ctx=30000)
     wl.step()

@@ -235,6 +235,13 @@ def run_reference(args, name):
     print(json.dumps(line), flush=True)
 
 
+def synth_n_new(name: str) -> int:
+    """New tokens (queries) per sequence of a workload: more than one means the
+    multi-query Full-layer path (chunked prefill, multi-token decode)."""
+    from sparse_attention_fp4_kv_b200 import synth
+    return int(getattr(synth.WORKLOADS[name], "n_new", 1) or 1)
+
+
 def run_prefill(args, name, rank, world, local_rank):
     """Chunked-prefill workload (one Full layer, n_new causal queries): tokens
     (queries) per second, and the tensor-core indexer against the int8 roofline."""
@@ -279,6 +286,23 @@ def run_prefill(args, name, rank, world, local_rank):
     ops = pw.index_ops()
     tops = ops / (scan_ms / 1e3) / 1e12
     tokens = world * w.B * w.n_new
+    # A few queries per sequence (multi-token decode): the scan streams every
+    # key once and is bound by HBM, not by the tensor cores.
+    key_bytes = w.B * w.ctx * (w.H_idx * w.D_idx + 4)
+    hbm_bound = ops / key_bytes < 2.0 * bf16 * 1e12 / (float(peaks.get("hbm_gbs", 6650.0)) * 1e9)
+    if hbm_bound:
+        hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
+        gbs = key_bytes / (scan_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": "index_mma_kernel (tcgen05 kind::i8, few queries)",
+                "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                "peak_kind": "measured" if "hbm_gbs" in peaks else "fallback",
+                "traffic": None, "algorithmic_bytes": key_bytes, "launch_ms": scan_ms}
+    else:
+        roof = {"bound": "tensor", "kernel": "index_mma_kernel (tcgen05 kind::i8)",
+                "achieved": tops, "peak": int8_peak, "unit": "TOPS", "frac": tops / int8_peak,
+                "peak_kind": "measured bf16 burst x 2 (nominal int8/bf16 ratio)"
+                if peaks else "fallback bf16 x 2",
+                "traffic": None, "algorithmic_ops": ops, "launch_ms": scan_ms}
     line = {"metric": "CSA2 chunked-prefill tokens/s (Full layer: append, causal indexer, "
                       "pool, top-512, attention)", "value": tokens / (ms / 1e3),
             "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms,
@@ -286,13 +310,7 @@ def run_prefill(args, name, rank, world, local_rank):
             "dtype": "int8/fp32", "data": "synthetic",
             "config": {"workload": name, "batch_per_gpu": w.B, "ctx": w.ctx, "new_tokens": w.n_new,
                        "indexer": f"int8 {w.H_idx}x{w.D_idx}", "q_heads": w.Hq, "C": w.C},
-            "roofline": {"bound": "tensor", "kernel": "index_mma_kernel (tcgen05 kind::i8)",
-                         "achieved": tops, "peak": int8_peak, "unit": "TOPS",
-                         "frac": tops / int8_peak,
-                         "peak_kind": "measured bf16 burst x 2 (nominal int8/bf16 ratio)"
-                         if peaks else "fallback bf16 x 2",
-                         "traffic": None, "algorithmic_ops": ops, "launch_ms": scan_ms},
-            "clocks": clk, "gpu_launches": pw.launches_per_step() * K}
+            "roofline": roof, "clocks": clk, "gpu_launches": pw.launches_per_step() * K}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -496,7 +514,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
-        if args.workload.startswith("prefill"):
+        if synth_n_new(args.workload) > 1:
             run_prefill(args, args.workload, rank, world, local_rank)
         else:
             run_csa2(args, args.workload, rank, world, local_rank)

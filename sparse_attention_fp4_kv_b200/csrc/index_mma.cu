@@ -380,10 +380,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 int index_mma_wait_flag(bool clear) { return read_device_flag(imma::g_imma_error, clear); }
 
-// Use the tensor-core scan for multi-query calls whose rows split into whole
-// 128-byte stages.
+// Use the tensor-core scan for every multi-query call whose rows split into
+// whole 128-byte stages. It reads each key tile once for all the queries of a
+// sequence (the per-query scan would stream the keys once per query); with a
+// few queries (speculative decode tokens) most of the 128-row query tile is
+// padding, but the MMA work per key tile (about 6 us per SM) stays below the
+// time to stream that tile from HBM (about 12 us), so the scan stays HBM-bound.
 bool index_mma_supported(int Nq, int HD, int64_t cap, int B) {
-    return Nq >= 16 && HD % imma::BK == 0 && HD <= 65536 && (int64_t)B * Nq < INT32_MAX &&
+    return Nq >= 2 && HD % imma::BK == 0 && HD <= 65536 && (int64_t)B * Nq < INT32_MAX &&
            (int64_t)B * cap < INT32_MAX;
 }
 

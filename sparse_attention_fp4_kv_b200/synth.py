@@ -79,6 +79,11 @@ WORKLOADS = {
     "encoder_stack18_b4_ctx1m": Workload("encoder_stack18_b4_ctx1m", B=4, ctx=1048576, C=512,
                                          Hq=64, H_idx=16, D_idx=128, modes=list(ENCODER_MODES),
                                          outlier_frac=0.01, outlier_mult=16.0, seed=5),
+    # Multi-token decode (speculative / MTP tokens): 4 new tokens per sequence
+    # appended to a 1M context, each a causal query of one Full layer.
+    "decode_mtp4_b4_ctx1m": Workload("decode_mtp4_b4_ctx1m", B=4, ctx=1048576 + 4, C=512, Hq=64,
+                                     H_idx=16, D_idx=128, modes=[FULL], outlier_frac=0.01,
+                                     outlier_mult=16.0, seed=6, n_new=4, prefill_queries=4),
     # Chunked prefill: 4096 new tokens appended to a 65536-token context.
     "prefill_4096_at_64k": Workload("prefill_4096_at_64k", B=1, ctx=65536 + 4096, C=512, Hq=64,
                                     H_idx=16, D_idx=128, modes=[FULL], outlier_frac=0.01,

@@ -493,10 +493,12 @@ def test_sparse_attention_one_cta_per_row_causal_positions(B):
 
 # ----------------------------------------------------------------------------- a9 prefill scan
 @pytest.mark.parametrize("Nq,ctx0,H,D", [(300, 5000, 16, 128), (129, 2048, 8, 128), (40, 777, 4, 64),
-                                         (256, 7936, 16, 128)])
+                                         (256, 7936, 16, 128), (2, 3000, 16, 128), (4, 5001, 16, 128),
+                                         (7, 1234, 8, 128)])
 def test_index_full_multi_query_tensor_core_path(B, Nq, ctx0, H, D):
-    """Nq >= 16 runs the tcgen05 kind::i8 kernel: causal scores and block maxima
-    must equal the oracle bit for bit, and equal the per-query dp4a scan."""
+    """Nq >= 2 runs the tcgen05 kind::i8 kernel (a few queries: speculative
+    decode tokens): causal scores and block maxima must equal the oracle bit
+    for bit, and equal the per-query dp4a scan."""
     Bn = 2
     cap = ctx0 + Nq
     g = torch.Generator(device=DEV).manual_seed(Nq + ctx0)

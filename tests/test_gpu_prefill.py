@@ -71,3 +71,22 @@ def test_prefill_4096_at_64k_sampled():
     _check_queries(pw, [0, 1, 127, 128, 2049, 4095])
     del pw
     torch.cuda.empty_cache()
+
+
+def test_multi_token_decode_sampled():
+    """Four speculative tokens per sequence at 1M context: the tensor-core scan
+    with a mostly padded query tile, the three-call selection (the rows are too
+    long for the fused kernel) and split-key attention; sampled queries."""
+    from sparse_attention_fp4_kv_b200.workload import PrefillWorkload
+    from sparse_attention_fp4_kv_b200 import binding
+    w = synth.scaled(synth.WORKLOADS["decode_mtp4_b4_ctx1m"], B=2, ctx=200003 + 4)
+    pw = PrefillWorkload(w, "cuda", keep_kv_bf16=True)
+    assert not pw.fused_select
+    binding.device_status(clear=True)
+    pw.step()
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    _fp4_matches_oracle(pw)
+    _check_queries(pw, [0, 3])
+    del pw
+    torch.cuda.empty_cache()

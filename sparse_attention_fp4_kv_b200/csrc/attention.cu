@@ -183,7 +183,7 @@ int attn_checked_launch(const AttnArgs &a, size_t ws_bytes, cudaStream_t s) {
 // workspace; the general kernel needs none. The size covers the tensor-core
 // path whenever its shape constraints could hold.
 size_t attn_workspace_bytes(int B, int Nq, int Hq, int C, int K, int n_win) {
-    if (C == 512 && Hq == 64 && K % 16 == 0 && K + (n_win > 0 ? n_win : 0) <= 640)
+    if (C == 512 && Hq == 64 && K > 0 && K <= 640)
         return attn_tc_workspace_bytes(B, Nq);
     return 0;
 }

@@ -7,37 +7,41 @@
 // layer has its own main Q and SWA KV; the window is the last 128 tokens.
 // FP4 section of both pages: E2M1 elements with one E4M3 scale per 16 channels.
 //
-// One thread-block cluster of 8 CTAs (256 threads each) per query; CTA r takes
-// keys [80 r, 80 r + 80) of the query's key list (selected rows, then window
-// rows).
-//  1. One thread issues TMA copies of the query's 64 x 512 bf16 Q and of the
-//     CTA's window rows straight into 128-byte-swizzled K-major tiles (they
-//     complete on an mbarrier); all threads gather the selected FP4 rows (256 B
-//     of codes, 32 B of scales each) with 16-byte cp.async into a staging area.
-//     The FP4 rows are then dequantized from shared memory by all 8 warps
-//     (hardware E2M1 -> f16 conversion, times the E4M3 scale; exact in bf16).
+// One thread-block cluster of 8 CTAs (256 threads each) per (query row, head
+// group); CTA r takes keys [80 r, 80 r + 80) of the row's key list (selected
+// rows, then window rows) for the group's HPC heads. With few rows the 64
+// heads are split into groups of 16 or 32 (HPC), so that more SMs share the
+// row and each CTA's partial result is smaller; with many rows a cluster takes
+// all 64 heads and loops over rows.
+//  1. All threads gather the CTA's selected FP4 rows (256 B of codes, 32 B of
+//     scales each) straight into registers, 16-byte loads all issued before
+//     the first use, and dequantize them into the 128-byte-swizzled K-major KV
+//     tile (hardware E2M1 -> f16 conversion, times the E4M3 scale; exact in
+//     bf16). One thread issues TMA copies of the group's HPC x 512 bf16 Q rows
+//     and of the CTA's window rows, which complete on an mbarrier.
 //  2. One thread issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32):
-//     S = Q K^T with M = 64 heads, N = 80 keys, K = 512, accumulated in TMEM.
-//  3. Each of the 4 warps reads its 16 heads' logits from TMEM (two threads per
-//     head), does a chunk-local softmax in fp32 and writes P to shared memory
-//     as bf16 hi + lo parts (P = hi + lo to ~16 bits, so the P V product keeps
-//     fp32-level accuracy with bf16 operands).
-//  4. O^T = V^T P_hi^T + V^T P_lo^T: M = 128 channels (4 blocks), N = 64 heads,
-//     K = 80 keys; the shared-memory KV tile is read as an MN-major A operand.
-//     Accumulating O transposed keeps the MMAs at M = 128 (an M = 64 MMA runs at
-//     half rate, and every tcgen05.mma has a fixed cost of about 50 cycles).
+//     S = Q K^T with M = 64 (HPC real heads), N = 80 keys, K = 512 in TMEM.
+//  3. HPC / 16 warps read the heads' logits from TMEM (two threads per head),
+//     do a chunk-local softmax in fp32 and write P to shared memory as bf16 hi
+//     + lo parts (P = hi + lo to ~16 bits, so the P V product keeps fp32-level
+//     accuracy with bf16 operands).
+//  4. O^T = V^T P_hi^T + V^T P_lo^T: M = 128 channels (4 blocks), N = HPC
+//     heads, K = 80 keys; the shared-memory KV tile is read as an MN-major A
+//     operand. Accumulating O transposed keeps the MMAs at M = 128 (an M = 64
+//     MMA runs at half rate, and every tcgen05.mma has a fixed cost of about
+//     50 cycles).
 //  5. Each CTA writes its unnormalized O straight from TMEM (lane = channel, so
 //     each warp store covers 128 contiguous bytes of one head), its row maxima
 //     and sums into its cluster's exchange slot in the workspace (L2
 //     resident); after a cluster barrier each CTA combines its 64 channels of
-//     all 64 heads over the 8 partial results and writes the output. (Moving
-//     the 1 MB of partials of a cluster through L2 measured about 4x faster
-//     than through distributed shared memory.) Clusters are persistent over
-//     query rows (at most 18, one wave on 148 SMs), so the workspace is 18
-//     slots at most.
-// TMEM: O^T uses columns 0..255 (all lanes); S uses lanes 16-31 of each 32-lane
-// subpartition (the M = 64 accumulator layout) in columns 256..335.
-// One launch per layer; scratch: one exchange slot (1.05 MB) per cluster.
+//     the group's heads over the 8 partial results and writes the output.
+//     (Moving the partials through L2 measured about 4x faster than through
+//     distributed shared memory.) Clusters are persistent over (row, group)
+//     items, at most as many as can be resident at once (and at most 18), so
+//     the workspace is 18 slots at most.
+// TMEM: O^T block c at columns HPC c (all lanes); S uses lanes 16-31 of each
+// 32-lane subpartition (the M = 64 accumulator layout) from column S_COL.
+// One launch per layer.
 #include "attention.cuh"
 #include "tcgen05.cuh"
 #include "tma.cuh"
@@ -48,64 +52,55 @@ namespace tc {
 constexpr int HQ = 64;
 constexpr int CH = 512;
 constexpr int T = 80;        // keys per CTA
-constexpr int CL = 8;        // CTAs per query (cluster size)
+constexpr int CL = 8;        // CTAs per (row, head group) (cluster size)
 constexpr int THREADS = 256;
-constexpr int SWA_BOX = 16;  // window rows per TMA box
+constexpr int SWA_BOX = 8;   // window rows per TMA box
 constexpr int KEYS_MAX = T * CL;
-
-constexpr int Q_CHUNK = HQ * 128;  // one 64-channel column of Q: 64 rows x 128 B
-constexpr int Q_BYTES = HQ * CH * 2;
 constexpr int K_CHUNK = T * 128;   // one 64-channel column of the KV tile
 constexpr int K_BYTES = T * CH * 2;
-constexpr int P_ATOM = HQ * 128;   // 64 tokens of P for 64 heads
-constexpr int P_BYTES = 2 * P_ATOM;
-
-constexpr int Q_OFF = 0;
-constexpr int K_OFF = Q_OFF + Q_BYTES;
-constexpr int PHI_OFF = K_OFF + K_BYTES;
-constexpr int PLO_OFF = PHI_OFF + P_BYTES;
-constexpr int M_OFF = PLO_OFF + P_BYTES;  // fp32 row max (log2 domain) [64]
-constexpr int L_OFF = M_OFF + HQ * 4;     // fp32 row sum [64]
-constexpr int SLOT_OFF = L_OFF + HQ * 4;  // int64 source offset per key slot [T]
-constexpr int KIND_OFF = SLOT_OFF + T * 8;
-constexpr int FP4_STAGE_OFF = PHI_OFF;    // raw FP4 rows [T][288], before P is written
-static_assert(T * 288 <= 2 * P_BYTES, "FP4 staging must fit in the P buffers");
-constexpr int BAR_OFF = (KIND_OFF + T + 15) / 16 * 16;  // [0] loads, [1] MMAs
-constexpr int TADDR_OFF = BAR_OFF + 16;
-
-constexpr int SMEM_USED = TADDR_OFF + 16;
-constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
-// Exchange slot of one cluster in the workspace: partial O [8 sources][8
-// slices][64 heads][64 channels] fp32, row maxima [8][64] and row sums [8][64].
-// TMEM: O^T channel block c (128 lanes x 64 heads) at columns 64 c; S (M = 64
-// layout, lanes 16-31 of each quadrant) at columns S_COL..S_COL + 79.
-constexpr uint32_t S_COL = 256;
-constexpr int64_t XSLOT_FLOATS = (int64_t)CL * HQ * CH + 2 * CL * HQ;
-// Clusters resident at once (148 SMs / 8); each walks query rows with this stride.
+constexpr int GATHER_PER_THREAD = T * 16 / THREADS;  // (slot, 32-channel group) items
+static_assert(GATHER_PER_THREAD * THREADS == T * 16, "gather split");
 constexpr int MAX_CLUSTERS = 18;
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-
 constexpr float LOG2E = 1.4426950408889634f;
-constexpr long WAIT_LIMIT = 1L << 24;
+constexpr uint64_t WAIT_NS = 200ull * 1000 * 1000;
+
+// Shared-memory layout and TMEM columns of a CTA that takes HPC heads.
+template <int HPC>
+struct Cfg {
+    static constexpr int HG = HQ / HPC;            // head groups per row
+    static constexpr int Q_CHUNK = HPC * 128;      // one 64-channel column of Q
+    static constexpr int Q_BYTES = HPC * CH * 2;
+    static constexpr int P_ATOM = HPC * 128;       // 64 tokens of P for HPC heads
+    static constexpr int P_BYTES = 2 * P_ATOM;
+    static constexpr int Q_OFF = 0;
+    // S is an M = 64 MMA: its A operand spans 64 rows of each Q column, of
+    // which rows HPC..63 run on into the next columns and (for the last column)
+    // the KV tile. Those rows only produce accumulator rows that are never
+    // read, and they stay inside this CTA's shared memory.
+    static constexpr int K_OFF = Q_OFF + Q_BYTES;
+    static constexpr int PHI_OFF = K_OFF + K_BYTES;
+    static constexpr int PLO_OFF = PHI_OFF + P_BYTES;
+    static constexpr int M_OFF = PLO_OFF + P_BYTES;  // fp32 row max (log2 domain) [HPC]
+    static constexpr int L_OFF = M_OFF + HPC * 4;    // fp32 row sum [HPC]
+    static constexpr int SLOT_OFF = L_OFF + HPC * 4; // int64 source row per key slot [T]
+    static constexpr int KIND_OFF = SLOT_OFF + T * 8;
+    static constexpr int BAR_OFF = (KIND_OFF + T + 15) / 16 * 16;  // [0] loads, [1] MMAs
+    static constexpr int TADDR_OFF = BAR_OFF + 16;
+    static constexpr int SMEM_USED = TADDR_OFF + 16;
+    static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
+    static constexpr int MIN_BLOCKS = SMEM_BYTES <= 112 * 1024 ? 2 : 1;
+    static constexpr uint32_t S_COL = HPC == 64 ? 256 : 128;
+    static constexpr uint32_t TMEM_COLS = HPC == 64 ? 512 : 256;
+    static constexpr int64_t XSLOT_FLOATS = (int64_t)CL * HPC * CH + 2 * CL * HPC;
+    static_assert(64 * 128 <= Q_BYTES - 7 * Q_CHUNK + K_BYTES, "S A-operand rows inside the CTA");
+    static_assert(4 * HPC <= (int)S_COL && S_COL + T <= TMEM_COLS, "TMEM columns");
+    static_assert(HPC * CL * 4 <= P_BYTES, "combine weights fit in the P tiles");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
 
 __device__ int g_attn_error = 0;
 
 // ---------------------------------------------------------------- PTX wrappers
-// Bounded wait on an mbarrier phase; returns false if the limit ran out.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase) {
-    for (long it = 0; it < WAIT_LIMIT; it++) {
-        uint32_t done;
-        asm volatile(
-            "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-            "selp.u32 %0, 1, 0, p;\n}"
-            : "=r"(done)
-            : "r"(bar), "r"(phase)
-            : "memory");
-        if (done) return true;
-    }
-    return false;
-}
-
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -115,36 +110,31 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::
                      : "memory");
 }
-__device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void st_dsmem_v4(uint32_t addr, float4 v) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x),
-                 "f"(v.y), "f"(v.z), "f"(v.w)
-                 : "memory");
-}
-__device__ __forceinline__ void st_dsmem_f32(uint32_t addr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
+
+// O^T columns [col, col + HPC) of the 32 lanes of this warp's subpartition
+// into v[0..HPC) (HPC = 16, 32 or 64).
+template <int HPC>
+__device__ __forceinline__ void load_ot(uint32_t taddr, float (&v)[HPC]) {
+    if constexpr (HPC == 16) {
+        tmem_ld_32x32b_16(taddr, v);
+    } else {
+#pragma unroll
+        for (int hc = 0; hc < HPC / 32; hc++) {
+            float w[32];
+            tmem_ld_32x32b_32(taddr + 32 * hc, w);
+#pragma unroll
+            for (int i = 0; i < 32; i++) v[32 * hc + i] = w[i];
+        }
+    }
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+// Slots of a CTA: [0, ks) for its ks selected keys, [ks, ks + wsz) for its wsz
+// window rows (ks and wsz multiples of 8, ks + wsz <= T).
+template <int HPC>
+__global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tswa,
-                   AttnArgs a) {
+                   AttnArgs a, int ks, int wsz) {
+    using L = Cfg<HPC>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -152,16 +142,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t rank = cluster_rank();
 
-    float *m_s = reinterpret_cast<float *>(sm + M_OFF);
-    float *l_s = reinterpret_cast<float *>(sm + L_OFF);
-    int64_t *slot_src = reinterpret_cast<int64_t *>(sm + SLOT_OFF);
-    uint8_t *slot_kind = sm + KIND_OFF;
-    const uint32_t bar_ld = base + BAR_OFF, bar = base + BAR_OFF + 8;
-    uint32_t *taddr_s = reinterpret_cast<uint32_t *>(sm + TADDR_OFF);
+    float *m_s = reinterpret_cast<float *>(sm + L::M_OFF);
+    float *l_s = reinterpret_cast<float *>(sm + L::L_OFF);
+    int64_t *slot_src = reinterpret_cast<int64_t *>(sm + L::SLOT_OFF);
+    uint8_t *slot_kind = sm + L::KIND_OFF;
+    const uint32_t bar_ld = base + L::BAR_OFF, bar = base + L::BAR_OFF + 8;
+    uint32_t *taddr_s = reinterpret_cast<uint32_t *>(sm + L::TADDR_OFF);
     // this cluster's exchange slot in the workspace
-    float *xo = reinterpret_cast<float *>(a.ws) + (int64_t)blockIdx.y * XSLOT_FLOATS;
-    float *xm = xo + CL * HQ * CH;
-    float *xl = xm + CL * HQ;
+    float *xo = reinterpret_cast<float *>(a.ws) + (int64_t)blockIdx.y * L::XSLOT_FLOATS;
+    float *xm = xo + CL * HPC * CH;
+    float *xl = xm + CL * HPC;
 
     // ---- once per CTA: mbarriers and TMEM
     if (tid == 0) {
@@ -169,109 +159,135 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) tmem_alloc(base + TADDR_OFF, 512);
+    if (warp == 0) tmem_alloc(base + L::TADDR_OFF, L::TMEM_COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *taddr_s;
-    const int64_t rows = (int64_t)a.B * a.Nq;
+    const int64_t items = (int64_t)a.B * a.Nq * L::HG;
     uint32_t ld_phase = 0;
     bool ok = true;
     // dependency on the previous kernel of the stream: at once, or (prefetch)
-    // after the first row's selected FP4 rows are gathered and dequantized
+    // after the first item's selected FP4 rows are gathered and dequantized
     bool waited = !a.prefetch;
     if (waited) {
         grid_dep_wait();
         grid_dep_launch();
     }
 
-    // The cluster walks query rows blockIdx.y, blockIdx.y + gridDim.y, ...
-    for (int64_t bq = blockIdx.y; bq < rows; bq += gridDim.y) {
+    // The cluster walks (row, head group) items blockIdx.y, blockIdx.y + gridDim.y, ...
+    for (int64_t it = blockIdx.y; it < items; it += gridDim.y) {
+        const int64_t bq = it / L::HG;
+        const int hg = (int)(it - bq * L::HG);
         const int b = (int)(bq / a.Nq);
         const AttnWindow w = attn_window(a, b, bq);
-        // Window slots of this CTA: [js, je) are window keys; TMA copies them in
-        // boxes of SWA_BOX rows starting at js (a multiple of 16).
-        const int k0 = (int)rank * T;
-        int js = a.K - k0;
-        js = js < 0 ? 0 : (js > T ? T : js);
-        int je = a.K + w.n - k0;
-        je = je < js ? js : (je > T ? T : je);
-        const int nbox = (je - js + SWA_BOX - 1) / SWA_BOX;
-        const int cover_end = js + nbox * SWA_BOX;  // slots written by the window boxes
+        // CTA r takes selected keys [r ks, r ks + ks) and window rows
+        // [r wsz, r wsz + wsz), so that every CTA gathers about as many FP4 rows
+        // and copies about as many window rows. The window rows arrive by TMA
+        // in boxes of SWA_BOX rows from slot ks; slots [ks, cover_end) are
+        // written by the boxes.
+        const int w0 = (int)rank * wsz;
+        int wn = w.n - w0;
+        wn = wn < 0 ? 0 : (wn > wsz ? wsz : wn);
+        const int js = ks;
+        const int nbox = (wn + SWA_BOX - 1) / SWA_BOX;
+        const int cover_end = js + nbox * SWA_BOX;
 
         if (tid < T) {
-            const int kidx = k0 + tid;
             uint8_t kind = 0;
             int64_t src = 0;
-            if (kidx < a.K) {
-                const int32_t pos = a.topk[bq * a.K + kidx];
-                if (pos >= 0 && pos < a.cap) {
-                    kind = 1;
-                    src = (int64_t)b * a.cap + pos;
+            if (tid < ks) {
+                const int kidx = (int)rank * ks + tid;
+                if (kidx < a.K) {
+                    const int32_t pos = a.topk[bq * a.K + kidx];
+                    if (pos >= 0 && pos < a.cap) {
+                        kind = 1;
+                        src = (int64_t)b * a.cap + pos;
+                    }
                 }
-            } else if (kidx - a.K < w.n) {
+            } else if (tid - ks < wn) {
                 kind = 2;
             }
             slot_kind[tid] = kind;
             slot_src[tid] = src;
         }
         if (tid == 0)
-            mbar_expect_tx(bar_ld, (uint32_t)Q_BYTES + (uint32_t)nbox * 8u * SWA_BOX * 128u);
+            mbar_expect_tx(bar_ld, (uint32_t)L::Q_BYTES + (uint32_t)nbox * 8u * SWA_BOX * 128u);
         __syncthreads();
 
-        // ---- load phase: Q and window rows by TMA, FP4 rows by cp.async
-        // slots that no copy writes (invalid keys outside the window boxes) are zeroed
-        for (int i = tid; i < T * 64; i += THREADS) {
-            const int j = i >> 6, pg = i & 63;
-            if (slot_kind[j] == 0 && (j < js || j >= cover_end))
-                st_shared_v4(base + K_OFF + (pg >> 3) * K_CHUNK + sw128(j, pg & 7),
-                             make_uint4(0, 0, 0, 0));
-        }
-        // Q and this CTA's window rows by TMA (one thread)
+        // Q rows of the group and this CTA's window rows by TMA (one thread)
         auto issue_q_swa = [&]() {
-            const int qrow = (int)(bq * HQ);
+            const int qrow = (int)(bq * HQ + hg * HPC);
 #pragma unroll
             for (int cc = 0; cc < 8; cc++)
-                tma_load_2d(base + Q_OFF + cc * Q_CHUNK, &tq, cc * 64, qrow, bar_ld);
-            const int wrow0 = (int)((int64_t)b * a.swa_rows + w.row0 + (k0 + js - a.K));
+                tma_load_2d(base + L::Q_OFF + cc * L::Q_CHUNK, &tq, cc * 64, qrow, bar_ld);
+            const int wrow0 = (int)((int64_t)b * a.swa_rows + w.row0 + w0);
             for (int bx = 0; bx < nbox; bx++)
 #pragma unroll
                 for (int cc = 0; cc < 8; cc++)
-                    tma_load_2d(base + K_OFF + cc * K_CHUNK + (js + bx * SWA_BOX) * 128, &tswa,
-                                cc * 64, wrow0 + bx * SWA_BOX, bar_ld);
+                    tma_load_2d(base + L::K_OFF + cc * K_CHUNK + (js + bx * SWA_BOX) * 128,
+                                &tswa, cc * 64, wrow0 + bx * SWA_BOX, bar_ld);
         };
         if (waited && tid == 0) issue_q_swa();
-        for (int i = tid; i < T * 18; i += THREADS) {  // (slot, 16-byte piece of its 288 B)
-            const int j = i / 18, pc = i - j * 18;
-            if (slot_kind[j] != 1 || (a.mx && pc == 17)) continue;  // MXFP4: 16 scale bytes
-            const int64_t cell = slot_src[j];
-            const uint8_t *src = pc < 16 ? a.kv_fp4 + cell * 256 + pc * 16
-                                         : a.kv_sf + cell * (a.mx ? 16 : 32) + (pc - 16) * 16;
-            cp_async16(base + FP4_STAGE_OFF + j * 288 + pc * 16, src);
+        // Before the wait: warm L2 with the rows that the copies after the wait
+        // read (a prefetch only; the data is read after the wait)
+        if (!waited && tid == 32) {
+            bulk_prefetch_l2(static_cast<const uint8_t *>(a.q) + (bq * HQ + hg * HPC) * (int64_t)CH * 2,
+                             (uint32_t)(HPC * CH * 2));
+            if (wn > 0)
+                bulk_prefetch_l2(static_cast<const uint8_t *>(a.swa) +
+                                     ((int64_t)b * a.swa_rows + w.row0 + w0) * CH * 2,
+                                 (uint32_t)(wn * CH * 2));
         }
-        cp_async_wait_all();
-        __syncthreads();
 
-        // ---- dequantize the FP4 rows into the KV tile (slots of kind 1; the
-        // TMA copies write only window slots, so this need not wait for them)
-        const uint8_t *stage = sm + FP4_STAGE_OFF;
-        for (int i = tid; i < T * 32; i += THREADS) {  // (slot, 16-channel group)
-            const int j = i >> 5, g = i & 31;
-            if (slot_kind[j] != 1) continue;
-            const uint2 codes = *reinterpret_cast<const uint2 *>(stage + j * 288 + g * 8);
-            const float s = kv_group_scale(stage + j * 288 + 256, g, a.mx);
-            uint32_t wds[8];
+        // ---- selected FP4 rows: codes and scales into registers (all loads
+        // first, unconditionally: a slot without a selected row reads row 0),
+        // then dequantized into the KV tile. Item i = (slot i / 16, 32-channel
+        // group i % 16): 16 bytes of codes and the group's two E4M3 scales (one
+        // E8M0 with MXFP4); a warp reads two rows' 256 code bytes. Slots that no
+        // copy writes (invalid keys outside the window boxes) are zeroed; the TMA
+        // copies write only window slots, so this need not wait for them.
+        {
+            uint4 codes[GATHER_PER_THREAD];
+            uint32_t sfb[GATHER_PER_THREAD];
 #pragma unroll
-            for (int u = 0; u < 8; u++) {
-                const uint32_t byte = ((u < 4 ? codes.x : codes.y) >> (8 * (u & 3))) & 0xFF;
-                const float2 f = e2m1x2_to_f32x2(byte);
-                wds[u] = pack_bf16x2(f.x * s, f.y * s);
+            for (int u = 0; u < GATHER_PER_THREAD; u++) {
+                const int i = tid + THREADS * u, j = i >> 4, gp = i & 15;
+                const int64_t cell = slot_src[j];
+                codes[u] = __ldcg(reinterpret_cast<const uint4 *>(a.kv_fp4 + cell * 256) + gp);
+                sfb[u] = a.mx ? (uint32_t)__ldcg(a.kv_sf + cell * 16 + gp)
+                              : (uint32_t)__ldcg(
+                                    reinterpret_cast<const unsigned short *>(a.kv_sf + cell * 32) + gp);
             }
-            const int pg = g * 2;  // two 16-byte pieces
-            const uint32_t d0 = base + K_OFF + (pg >> 3) * K_CHUNK + sw128(j, pg & 7);
-            const uint32_t d1 = base + K_OFF + ((pg + 1) >> 3) * K_CHUNK + sw128(j, (pg + 1) & 7);
-            st_shared_v4(d0, make_uint4(wds[0], wds[1], wds[2], wds[3]));
-            st_shared_v4(d1, make_uint4(wds[4], wds[5], wds[6], wds[7]));
+#pragma unroll
+            for (int u = 0; u < GATHER_PER_THREAD; u++) {
+                const int i = tid + THREADS * u, j = i >> 4, gp = i & 15;
+                const int kind = slot_kind[j];
+                if (kind == 2 || (kind == 0 && j >= js && j < cover_end)) continue;
+                uint32_t wds[16];
+                if (kind == 1) {
+                    // channels 32 gp .. 32 gp + 15 take the first scale, the rest the second
+                    const float s0 = a.mx ? e8m0_to_f32(sfb[u]) : e4m3_to_f32(sfb[u] & 0xFF);
+                    const float s1 = a.mx ? s0 : e4m3_to_f32(sfb[u] >> 8);
+                    const uint32_t cw[4] = {codes[u].x, codes[u].y, codes[u].z, codes[u].w};
+#pragma unroll
+                    for (int e = 0; e < 16; e++) {
+                        const uint32_t byte = (cw[e >> 2] >> (8 * (e & 3))) & 0xFF;
+                        const float2 f = e2m1x2_to_f32x2(byte);
+                        const float sc = e < 8 ? s0 : s1;
+                        wds[e] = pack_bf16x2(f.x * sc, f.y * sc);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; e++) wds[e] = 0u;
+                }
+#pragma unroll
+                for (int q = 0; q < 4; q++) {
+                    const int pg = gp * 4 + q;  // 16-byte piece (8 channels) of the row
+                    st_shared_v4(base + L::K_OFF + (pg >> 3) * K_CHUNK + sw128(j, pg & 7),
+                                 make_uint4(wds[4 * q], wds[4 * q + 1], wds[4 * q + 2], wds[4 * q + 3]));
+                }
+            }
         }
         fence_proxy_async();
         if (!waited) {
@@ -280,31 +296,31 @@ __global__ void __launch_bounds__(THREADS, 1)
             waited = true;
             if (tid == 0) issue_q_swa();
         }
-        if (ok) ok = mbar_wait(bar_ld, ld_phase);
+        if (tid == 0 && ok) ok = mbar_wait_bounded(bar_ld, ld_phase, WAIT_NS);
         ld_phase ^= 1;
-        __syncthreads();
+        ok = __syncthreads_and(ok) != 0;
 
         // ---- S = Q K^T  (M = 64, N = 80, K = 512) into TMEM lanes 16..31
-        const uint32_t s_tmem = tmem + (16u << 16) + S_COL;
+        const uint32_t s_tmem = tmem + (16u << 16) + L::S_COL;
         if (tid == 0 && ok) {
             tc_fence_after();
-            constexpr uint32_t id_s = idesc_bf16(HQ, T, false);
+            constexpr uint32_t id_s = idesc_bf16(64, T, false);
 #pragma unroll 1
             for (int kk = 0; kk < CH / 16; kk++) {
                 const uint32_t off = (kk & 3) * 32;
-                const uint64_t ad = sdesc(base + Q_OFF + (kk >> 2) * Q_CHUNK + off, 16, 1024);
-                const uint64_t bd = sdesc(base + K_OFF + (kk >> 2) * K_CHUNK + off, 16, 1024);
+                const uint64_t ad = sdesc(base + L::Q_OFF + (kk >> 2) * L::Q_CHUNK + off, 16, 1024);
+                const uint64_t bd = sdesc(base + L::K_OFF + (kk >> 2) * K_CHUNK + off, 16, 1024);
                 mma_bf16(s_tmem, ad, bd, id_s, kk > 0);
             }
             mma_commit(bar);
         }
-        if (ok) ok = mbar_wait(bar, 0);
-        tc_fence_after();
 
-        // ---- softmax over this CTA's keys (warps 0-3; two threads per head)
-        const int h = (warp & 3) * 16 + (lane & 15);
+        // ---- softmax over this CTA's keys (warps 0 .. HPC/16 - 1; two threads per head)
+        const int h = warp * 16 + (lane & 15);
         const int half = lane >> 4;
-        if (warp < 4) {
+        if (warp < HPC / 16) {
+            if (ok) ok = mbar_wait_bounded(bar, 0, WAIT_NS);
+            tc_fence_after();
             const float sl2 = a.scale * LOG2E;
             float p[40];
             {
@@ -353,40 +369,41 @@ __global__ void __launch_bounds__(THREADS, 1)
                     hi[u] = *reinterpret_cast<const uint32_t *>(&hb);
                     lo[u] = pack_bf16x2(pp[2 * u] - hf.x, pp[2 * u + 1] - hf.y);
                 }
-                const uint32_t off = (tok0 >> 6) * P_ATOM + sw128(h, (tok0 & 63) >> 3);
-                st_shared_v4(base + PHI_OFF + off, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-                st_shared_v4(base + PLO_OFF + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+                const uint32_t off = (tok0 >> 6) * L::P_ATOM + sw128(h, (tok0 & 63) >> 3);
+                st_shared_v4(base + L::PHI_OFF + off, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+                st_shared_v4(base + L::PLO_OFF + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
             }
+            fence_proxy_async();
+            tc_fence_before();
         }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
+        ok = __syncthreads_and(ok) != 0;
 
-        // ---- O^T = V^T P_hi^T + V^T P_lo^T  (M = 128 channels x 4 blocks, N = 64
+        // ---- O^T = V^T P_hi^T + V^T P_lo^T  (M = 128 channels x 4 blocks, N = HPC
         // heads, K = 80 keys): V^T is the KV tile read MN-major, P^T the P tiles
-        // read K-major; block c of 128 channels accumulates in columns 64 c
+        // read K-major; block c of 128 channels accumulates in columns HPC c
         if (tid == 0 && ok) {
             tc_fence_after();
-            constexpr uint32_t id_o = idesc_bf16(128, HQ, false, true);
+            constexpr uint32_t id_o = idesc_bf16(128, HPC, false, true);
 #pragma unroll 1
             for (int kk = 0; kk < T / 16; kk++) {
-                const uint32_t poff = (kk >> 2) * P_ATOM + (kk & 3) * 32;
-                const uint64_t phi = sdesc(base + PHI_OFF + poff, 16, 1024);
-                const uint64_t plo = sdesc(base + PLO_OFF + poff, 16, 1024);
+                const uint32_t poff = (kk >> 2) * L::P_ATOM + (kk & 3) * 32;
+                const uint64_t phi = sdesc(base + L::PHI_OFF + poff, 16, 1024);
+                const uint64_t plo = sdesc(base + L::PLO_OFF + poff, 16, 1024);
 #pragma unroll
                 for (int c = 0; c < 4; c++) {
-                    const uint64_t vd = sdesc(base + K_OFF + 2 * c * K_CHUNK + kk * 2048, K_CHUNK, 1024);
-                    mma_bf16(tmem + 64 * c, vd, phi, id_o, kk > 0);
-                    mma_bf16(tmem + 64 * c, vd, plo, id_o, 1);
+                    const uint64_t vd =
+                        sdesc(base + L::K_OFF + 2 * c * K_CHUNK + kk * 2048, K_CHUNK, 1024);
+                    mma_bf16(tmem + HPC * c, vd, phi, id_o, kk > 0);
+                    mma_bf16(tmem + HPC * c, vd, plo, id_o, 1);
                 }
             }
             mma_commit(bar);
         }
-        if (ok) ok = mbar_wait(bar, 1);
+        if (ok) ok = mbar_wait_bounded(bar, 1, WAIT_NS);
         tc_fence_after();
 
         // ---- publish this CTA's unnormalized O, row maxima and sums in the
-        // cluster's exchange slot (L2), laid out [source][64-channel slice][64
+        // cluster's exchange slot (L2), laid out [source][64-channel slice][HPC
         // heads][64 channels]. TMEM lane = channel, so every warp store of one
         // head writes 32 consecutive channels (128 bytes); warps w and w + 4
         // take channel blocks 0-1 and 2-3.
@@ -396,37 +413,35 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
             for (int c = 2 * (warp >> 2); c < 2 * (warp >> 2) + 2; c++) {
                 const int ch = 128 * c + 32 * q4 + lane;  // this thread's channel
-                float *dst = xo + ((int64_t)rank * CL + (ch >> 6)) * (HQ * 64) + (ch & 63);
-#pragma unroll 1
-                for (int hc = 0; hc < 2; hc++) {
-                    float v[32];
-                    tmem_ld_32x32b_32(lane_addr + 64 * c + 32 * hc, v);
+                float *dst = xo + ((int64_t)rank * CL + (ch >> 6)) * (HPC * 64) + (ch & 63);
+                float v[HPC];
+                load_ot<HPC>(lane_addr + HPC * c, v);
 #pragma unroll
-                    for (int i = 0; i < 32; i++) dst[(32 * hc + i) * 64] = ok ? v[i] : 0.0f;
-                }
+                for (int i = 0; i < HPC; i++) dst[i * 64] = ok ? v[i] : 0.0f;
             }
-            if (warp < 4 && half == 0) {
-                xm[rank * HQ + h] = ok ? m_s[h] : -INFINITY;
-                xl[rank * HQ + h] = ok ? l_s[h] : 0.0f;
+            if (warp < HPC / 16 && half == 0) {
+                xm[rank * HPC + h] = ok ? m_s[h] : -INFINITY;
+                xl[rank * HPC + h] = ok ? l_s[h] : 0.0f;
             }
         }
         __syncthreads();
         __threadfence();
         tc_fence_before();
-        cluster_sync();  // all partial results of this row are in the slot
+        cluster_sync();  // all partial results of this item are in the slot
 
         // ---- combine: this CTA owns channels [64 rank, 64 rank + 64); the slice
         // of source r is contiguous at xo[r][rank]. Thread t takes the 16-byte
-        // chunks e = 4 (t + 256 u), u = 0..3, of the [64 heads][64 channels]
+        // chunks e = 4 (t + 256 u), u < HPC / 16, of the [HPC heads][64 channels]
         // slice.
         {
-            float *wts = reinterpret_cast<float *>(sm + PHI_OFF);  // [64 heads][8] weight / den
-            if (tid < HQ) {
+            constexpr int U = HPC / 16;
+            float *wts = reinterpret_cast<float *>(sm + L::PHI_OFF);  // [HPC heads][8] weight / den
+            if (tid < HPC) {
                 float mr[CL], lr[CL];
 #pragma unroll
                 for (int r = 0; r < CL; r++) {
-                    mr[r] = __ldcg(xm + r * HQ + tid);
-                    lr[r] = __ldcg(xl + r * HQ + tid);
+                    mr[r] = __ldcg(xm + r * HPC + tid);
+                    lr[r] = __ldcg(xl + r * HPC + tid);
                 }
                 float M = -INFINITY;
 #pragma unroll
@@ -441,17 +456,17 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                 for (int r = 0; r < CL; r++) wts[tid * CL + r] = wg[r] * inv;
             }
-            float4 f[4][CL];
+            float4 f[U][CL];
 #pragma unroll
-            for (int u = 0; u < 4; u++)
+            for (int u = 0; u < U; u++)
 #pragma unroll
                 for (int r = 0; r < CL; r++)
                     f[u][r] = __ldcg(reinterpret_cast<const float4 *>(
-                                         xo + ((int64_t)r * CL + rank) * (HQ * 64)) +
+                                         xo + ((int64_t)r * CL + rank) * (HPC * 64)) +
                                      tid + 256 * u);
             __syncthreads();  // weights ready
 #pragma unroll
-            for (int u = 0; u < 4; u++) {
+            for (int u = 0; u < U; u++) {
                 const int e = 4 * (tid + 256 * u);
                 const int hh = e >> 6, ch = e & 63;
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -463,45 +478,106 @@ __global__ void __launch_bounds__(THREADS, 1)
                     acc.z += wr * f[u][r].z;
                     acc.w += wr * f[u][r].w;
                 }
-                *reinterpret_cast<float4 *>(a.out + (bq * HQ + hh) * (int64_t)CH + (int)rank * 64 + ch) =
-                    acc;
+                *reinterpret_cast<float4 *>(a.out + (bq * HQ + hg * HPC + hh) * (int64_t)CH +
+                                            (int)rank * 64 + ch) = acc;
             }
         }
-        // the slot, the tiles and TMEM are free for the next row (after the last
-        // row nothing is shared any more: the exchange went through global memory)
-        if (bq + (int64_t)gridDim.y < rows) cluster_sync();
+        // the slot, the tiles and TMEM are free for the next item (after the last
+        // item nothing is shared any more: the exchange went through global memory)
+        if (it + (int64_t)gridDim.y < items) cluster_sync();
     }
-    if (!ok && tid == 0) atomicExch(&g_attn_error, 1);
+    if (!ok) atomicExch(&g_attn_error, 1);
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, L::TMEM_COLS);
     }
 }
 
 }  // namespace tc
 
+// Heads per CTA for a call of `rows` query rows: split the 64 heads while the
+// (row, head group) items still run in one wave of 8-CTA clusters (15 fit on a
+// B200 at one CTA per SM). Per-phase timestamps at 200K context put a 1-row call
+// at 10.7 / 11.1 / 12.4 us from first CTA start to last CTA end with 16 / 32 /
+// 64 heads per CTA, a 6-row call at 12.0 us with 32 and 13.3 us with 64. With
+// dependent launches two consecutive layers share the 15 cluster slots: a
+// layer that gathers before its wait (Reuse) keeps to 7 clusters and one that
+// waits first to 8, so that the next layer's clusters all start (and gather)
+// while this one runs.
+static int tc_heads_per_cta(int64_t rows, bool pdl, bool prefetch) {
+    if (!pdl) return rows <= 2 ? 16 : rows <= 7 ? 32 : 64;
+    const int64_t lim = prefetch ? 7 : 8;
+    return 4 * rows <= lim ? 16 : 2 * rows <= lim ? 32 : 64;
+}
+
+// Slots per CTA: ks for selected keys, wsz for window rows, each rounded up to
+// a multiple of 8 (window boxes then land on 1024-byte boundaries of the tile).
+struct TcSplit {
+    int ks, wsz;
+};
+static TcSplit tc_split(const AttnArgs &a) {
+    int nwin = a.n_win < a.swa_rows ? a.n_win : a.swa_rows;
+    if (a.swa == nullptr || nwin < 0) nwin = 0;
+    const int ks = ((a.K + tc::CL - 1) / tc::CL + 7) / 8 * 8;
+    const int wsz = ((nwin + tc::CL - 1) / tc::CL + 7) / 8 * 8;
+    return {ks, wsz};
+}
+
 bool attn_tc_supported(const AttnArgs &a) {
     const int nwin = a.n_win < a.swa_rows ? a.n_win : a.swa_rows;
     const bool has_win = nwin > 0 && a.swa != nullptr;
-    return a.C == tc::CH && a.Hq == tc::HQ && a.K + (nwin > 0 ? nwin : 0) <= tc::KEYS_MAX &&
-           a.K % 16 == 0 && aligned(a.q, 16) && aligned(a.kv_fp4, 16) && aligned(a.kv_sf, 16) &&
+    const TcSplit sp = tc_split(a);
+    return a.C == tc::CH && a.Hq == tc::HQ && a.K > 0 && a.K <= tc::KEYS_MAX &&
+           sp.ks + sp.wsz <= tc::T && aligned(a.q, 16) && aligned(a.kv_fp4, 16) &&
+           aligned(a.kv_sf, 16) &&
            (!has_win || (aligned(a.swa, 16) && (int64_t)a.B * a.swa_rows >= tc::SWA_BOX)) &&
            (int64_t)a.B * a.Nq * tc::HQ < INT32_MAX && (int64_t)a.B * a.swa_rows < INT32_MAX;
 }
 
-int launch_attn_tc(const AttnArgs &a, cudaStream_t s) {
+// Clusters of the HPC-head kernel that can be resident at once (the
+// persistent loop then runs in one wave); MAX_CLUSTERS if the query fails.
+template <int HPC>
+int tc_max_active_clusters() {
+    static int n = 0;
+    if (n == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(tc::CL, tc::MAX_CLUSTERS, 1);
+        cfg.blockDim = dim3(tc::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = tc::Cfg<HPC>::SMEM_BYTES;
+        cudaLaunchAttribute at;
+        at.id = cudaLaunchAttributeClusterDimension;
+        at.val.clusterDim.x = tc::CL;
+        at.val.clusterDim.y = 1;
+        at.val.clusterDim.z = 1;
+        cfg.attrs = &at;
+        cfg.numAttrs = 1;
+        int m = 0;
+        if (cudaFuncSetAttribute(tc::attn_tc_kernel<HPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::Cfg<HPC>::SMEM_BYTES) == cudaSuccess &&
+            cudaOccupancyMaxActiveClusters(&m, tc::attn_tc_kernel<HPC>, &cfg) == cudaSuccess && m > 0)
+            n = m;
+        else
+            n = tc::MAX_CLUSTERS;
+        (void)cudaGetLastError();
+    }
+    return n;
+}
+
+template <int HPC>
+static int launch_tc(const AttnArgs &a, cudaStream_t s) {
+    using L = tc::Cfg<HPC>;
     static bool attr = false;
     if (!attr) {
-        if (cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tc::SMEM_BYTES) != cudaSuccess)
+        if (cudaFuncSetAttribute(tc::attn_tc_kernel<HPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 L::SMEM_BYTES) != cudaSuccess)
             return CSA2_ERR_CUDA;
         attr = true;
     }
     const int64_t rows = (int64_t)a.B * a.Nq;
-    if (a.ws == nullptr) return CSA2_ERR_WORKSPACE;
+    const int64_t items = rows * L::HG;
     CUtensorMap tq, tswa;
     if (!make_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.q, tc::CH, (uint64_t)rows * tc::HQ,
-                      tc::CH * 2, 64, 64))
+                      tc::CH * 2, 64, HPC))
         return CSA2_ERR_CUDA;
     const bool has_win = a.swa != nullptr && a.swa_rows > 0 && a.n_win > 0;
     // without a window the map is never used; describe the Q tensor instead
@@ -510,10 +586,11 @@ int launch_attn_tc(const AttnArgs &a, cudaStream_t s) {
                       tc::SWA_BOX))
         return CSA2_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
-    const int64_t clusters = rows < tc::MAX_CLUSTERS ? rows : tc::MAX_CLUSTERS;
+    int64_t clusters = items < tc::MAX_CLUSTERS ? items : tc::MAX_CLUSTERS;
+    if (clusters > tc_max_active_clusters<HPC>()) clusters = tc_max_active_clusters<HPC>();
     cfg.gridDim = dim3(tc::CL, (unsigned)clusters, 1);
     cfg.blockDim = dim3(tc::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = tc::SMEM_BYTES;
+    cfg.dynamicSmemBytes = L::SMEM_BYTES;
     cfg.stream = s;
     cudaLaunchAttribute attr_cl[2];
     attr_cl[0].id = cudaLaunchAttributeClusterDimension;
@@ -524,21 +601,36 @@ int launch_attn_tc(const AttnArgs &a, cudaStream_t s) {
     attr_cl[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr_cl;
     cfg.numAttrs = a.pdl ? 2 : 1;
-    if (cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel, tq, tswa, a) != cudaSuccess)
+    const TcSplit sp = tc_split(a);
+    if (cudaLaunchKernelEx(&cfg, tc::attn_tc_kernel<HPC>, tq, tswa, a, sp.ks, sp.wsz) != cudaSuccess)
         return CSA2_ERR_CUDA;
     return launch_status();
 }
 
-}  // namespace csa2
-
-namespace csa2 {
+int launch_attn_tc(const AttnArgs &a, cudaStream_t s) {
+    if (a.ws == nullptr) return CSA2_ERR_WORKSPACE;
+    switch (tc_heads_per_cta((int64_t)a.B * a.Nq, a.pdl, a.prefetch)) {
+    case 16: return launch_tc<16>(a, s);
+    case 32: return launch_tc<32>(a, s);
+    default: return launch_tc<64>(a, s);
+    }
+}
 
 int attn_tc_wait_flag(bool clear) { return read_device_flag(tc::g_attn_error, clear); }
 
 size_t attn_tc_workspace_bytes(int B, int Nq) {
+    // the largest of the head splits a call of this size can take
     const int64_t rows = (int64_t)B * Nq;
-    const int64_t clusters = rows < tc::MAX_CLUSTERS ? rows : tc::MAX_CLUSTERS;
-    return (size_t)clusters * tc::XSLOT_FLOATS * sizeof(float);
+    size_t most = 0;
+    for (int v = 0; v < 3; v++) {
+        const int hpc = tc_heads_per_cta(rows, v > 0, v > 1);
+        const int64_t items = rows * (tc::HQ / hpc);
+        const int64_t clusters = items < tc::MAX_CLUSTERS ? items : tc::MAX_CLUSTERS;
+        const int64_t slot = (int64_t)tc::CL * hpc * tc::CH + 2 * tc::CL * hpc;
+        const size_t bytes = (size_t)clusters * slot * sizeof(float);
+        if (bytes > most) most = bytes;
+    }
+    return most;
 }
 
 }  // namespace csa2

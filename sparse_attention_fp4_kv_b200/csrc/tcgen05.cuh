@@ -165,6 +165,26 @@ __device__ __forceinline__ void tmem_ld_32x32b_32(uint32_t taddr, float (&v)[32]
 #pragma unroll
     for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
 }
+// The 16-column form of the load above (columns [col, col + 16)).
+__device__ __forceinline__ void tmem_ld_32x32b_16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; i++) v[i] = __uint_as_float(r[i]);
+}
 // The matching store; completed by tmem_st_wait().
 __device__ __forceinline__ void tmem_st_32x32b_32(uint32_t taddr, const float (&v)[32]) {
     asm volatile(
@@ -208,6 +228,33 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
+}
+
+// mbarrier.try_wait with a suspend-time hint (ns): the thread sleeps until the
+// phase of the given parity completes or about `ns` pass.
+__device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        "selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity), "r"(ns)
+        : "memory");
+    return done != 0;
+}
+// Wait for the phase of the given parity, sleeping in try_wait between checks;
+// false when `limit_ns` of global time pass first.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; it++) {
+        if (mbar_try_wait_ns(bar, parity, 100000u)) return true;
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) {
+            t0 = now;
+        } else if (now - t0 > limit_ns) {
+            return false;
+        }
+    }
 }
 
 }  // namespace csa2

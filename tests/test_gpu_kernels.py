@@ -152,6 +152,7 @@ def test_append_mxfp4_channel_counts(B, C):
 
 
 @pytest.mark.parametrize("Bn,ctx,C,Hq,K,Nq", [(3, 4000, 512, 64, 512, 1),     # split-key clusters
+                                              (7, 3000, 512, 64, 512, 1),      # 32-head groups
                                               (70, 900, 512, 64, 512, 1),      # one CTA per row
                                               (2, 2000, 128, 8, 512, 1)])      # general kernel
 def test_sparse_attention_mxfp4(B, Bn, ctx, C, Hq, K, Nq):
@@ -456,7 +457,8 @@ def _attention_case(B, Bn, ctx, C, Hq, K, n_win, seed, q_pos=None, Nq=1, drop=0,
             assert_attn_close(out[b, i].cpu().numpy(), ref, f"b={b} i={i}")
 
 
-@pytest.mark.parametrize("Bn,ctx,C,Hq,K", [(3, 5000, 512, 64, 512), (2, 3000, 128, 8, 512),
+@pytest.mark.parametrize("Bn,ctx,C,Hq,K", [(3, 5000, 512, 64, 512), (2, 3000, 512, 64, 488),
+                                           (2, 3000, 128, 8, 512),
                                            (1, 300, 512, 64, 512), (2, 100, 256, 16, 512),
                                            (1, 2000, 64, 3, 100)])
 def test_sparse_attention_matches_oracle(B, Bn, ctx, C, Hq, K):
@@ -474,9 +476,19 @@ def test_sparse_attention_prefill_positions(B):
     _attention_case(B, 1, ctx, 512, 64, 512, 128, seed=3, q_pos=q_pos, Nq=4)
 
 
-# One CTA per query row: calls with 19 or more rows (and any call with more than
+# The split-key cluster kernel divides the 64 heads of a row into groups with few
+# rows: 16 heads per cluster up to 4 rows, 32 up to 9, all 64 beyond (clusters
+# then loop over rows). Each grouping, with masked slots and short windows.
+@pytest.mark.parametrize("Bn,Nq,drop,n_win", [(1, 1, 0, 128), (2, 2, 4, 128), (5, 1, 0, 128),
+                                              (3, 3, 6, 100), (10, 1, 0, 128), (19, 1, 9, 64)])
+def test_sparse_attention_head_groups(B, Bn, Nq, drop, n_win):
+    _attention_case(B, Bn, 2600, 512, 64, 512, n_win, seed=31 * Bn + Nq, Nq=Nq, drop=drop)
+
+
+# One CTA per query row: calls with 64 or more rows (and any call with more than
 # 640 keys per row) take the per-row kernel; its window tiles, masked slots and
-# online-softmax rescaling are covered here.
+# online-softmax rescaling are covered here (the 20- to 40-row cases run the
+# split-key kernel with all 64 heads per cluster).
 @pytest.mark.parametrize("Bn,Nq,K,n_win,drop", [(20, 1, 512, 128, 0), (24, 1, 512, 128, 5),
                                                 (2, 1, 1024, 128, 0), (20, 1, 512, 0, 0),
                                                 (3, 8, 576, 64, 7)])

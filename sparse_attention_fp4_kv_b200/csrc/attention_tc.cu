@@ -171,6 +171,23 @@ __global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
     // after the first item's selected FP4 rows are gathered and dequantized
     bool waited = !a.prefetch;
     if (waited) {
+        // warm L2 with the first item's Q and window rows (inputs of this
+        // layer, read after the wait; the prefetch only moves them into L2)
+        if (tid == 32 && (int64_t)blockIdx.y < items) {
+            const int64_t bq0 = (int64_t)blockIdx.y / L::HG;
+            const int hg0 = (int)((int64_t)blockIdx.y - bq0 * L::HG);
+            const int b0 = (int)(bq0 / a.Nq);
+            const AttnWindow w = attn_window(a, b0, bq0);
+            const int w0 = (int)rank * wsz;
+            int wn = w.n - w0;
+            wn = wn < 0 ? 0 : (wn > wsz ? wsz : wn);
+            bulk_prefetch_l2(static_cast<const uint8_t *>(a.q) + (bq0 * HQ + hg0 * HPC) * (int64_t)CH * 2,
+                             (uint32_t)(HPC * CH * 2));
+            if (wn > 0)
+                bulk_prefetch_l2(static_cast<const uint8_t *>(a.swa) +
+                                     ((int64_t)b0 * a.swa_rows + w.row0 + w0) * CH * 2,
+                                 (uint32_t)(wn * CH * 2));
+        }
         grid_dep_wait();
         grid_dep_launch();
     }

@@ -91,6 +91,12 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 
 // E4M3 code -> fp32 from the format definition (1 sign, 4 exponent bits with
 // bias 7, 3 mantissa bits; exponent field 0 is subnormal m * 2^-9). Exact.
+// Prefetch of a contiguous global range into L2 (16-byte aligned, size a
+// multiple of 16); no data reaches the issuing CTA.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
     uint32_t e = (code >> 3) & 0xF, m = code & 7;
     float mag = (e == 0) ? (float)m * 0.001953125f                     // m * 2^-9

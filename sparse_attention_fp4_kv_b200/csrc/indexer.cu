@@ -264,24 +264,37 @@ __device__ __forceinline__ int64_t reindex_block(const ReindexArgs &a, int64_t b
 
 // One warp per pooled block (no persistence: the kernel is short, so a grid
 // of one warp per item hides the ramp-up and tail better), 16 loads per lane
-// in flight.
+// in flight. Before its grid-dependency wait a warp finds its block from the
+// pool and the context lengths and pulls the block's keys into L2, so that
+// with dependent launches the key stream overlaps the previous kernel (a
+// latency-bound attention layer that leaves HBM idle). The pool comes from the
+// Full layer's selection, which is always two or more kernels earlier (its
+// token selection and attention follow it), and the keys and context lengths
+// are not written during a step; the layer's own indexer query, the only input
+// the previous kernel may produce, is read after the wait.
 template <int HD>
 __global__ void __launch_bounds__(256) index_reindex_kernel(ReindexArgs a) {
-    grid_dep_wait();
-    grid_dep_launch();
     using RS = RowShape<HD>;
     const int lane = threadIdx.x & 31;
     const int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t items = (int64_t)a.B * a.Nq * a.P;
+    int64_t bq = 0, t0 = -1;
+    int s = 0, b = 0, ntok = 0;
+    if (it < items) {
+        bq = it / a.P;
+        s = (int)(it - bq * a.P);
+        b = (int)(bq / a.Nq);
+        const int i = (int)(bq % a.Nq);
+        int64_t V = visible_len(a.ctx_len, a.q_pos, b, i, a.Nq);
+        if (V > a.cap) V = a.cap;
+        t0 = reindex_block(a, bq, s, V, ntok);
+        if (t0 >= 0 && lane == 0)
+            bulk_prefetch_l2(a.k + ((int64_t)b * a.cap + t0) * HD, (uint32_t)(ntok * HD));
+    }
+    grid_dep_wait();
+    grid_dep_launch();
     if (it >= items) return;
     const int my_tok = reduce_token_of_lane(lane);
-    const int64_t bq = it / a.P;
-    const int s = (int)(it - bq * a.P);
-    const int b = (int)(bq / a.Nq), i = (int)(bq % a.Nq);
-    int64_t V = visible_len(a.ctx_len, a.q_pos, b, i, a.Nq);
-    if (V > a.cap) V = a.cap;
-    int ntok;
-    const int64_t t0 = reindex_block(a, bq, s, V, ntok);
     const int64_t slot = bq * 8 * (int64_t)a.P + 8 * (int64_t)s;
     if (t0 < 0) {
         if (lane < 8) {

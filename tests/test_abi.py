@@ -117,3 +117,36 @@ def test_decode_stack_schedule_checks():
     # unknown mode
     layers[1] = B.csa2_layer(7, good, good, good, good, good)
     assert B.lib.csa2_decode_stack(layers, 2, None, *args) == -4
+
+
+def _attn_slot_bytes(hpc):
+    # one cluster's exchange slot: 8 CTAs' partial O [hpc][512] fp32, row maxima and sums
+    return (8 * hpc * 512 + 2 * 8 * hpc) * 4
+
+
+def _attn_heads_per_cta(rows, pdl, prefetch):
+    # the launcher's head split: 16 or 32 of the 64 heads per cluster while the
+    # (row, head group) items fit the resident clusters (a dependent launch
+    # leaves room for the next layer's clusters), else all 64
+    if not pdl:
+        return 16 if rows <= 2 else 32 if rows <= 7 else 64
+    lim = 7 if prefetch else 8
+    return 16 if 4 * rows <= lim else 32 if 2 * rows <= lim else 64
+
+
+def test_attention_workspace_covers_every_head_split(lib):
+    ws = lib.csa2_sparse_attn_workspace_size
+    ws.restype = ctypes.c_size_t
+    ws.argtypes = [ctypes.c_int] * 6
+    for B, Nq in [(1, 1), (2, 1), (3, 1), (4, 1), (5, 1), (7, 1), (8, 1), (9, 1), (16, 1), (4, 4),
+                  (63, 1), (64, 1)]:
+        rows = B * Nq
+        need = []
+        for pdl, prefetch in [(False, False), (True, False), (True, True)]:
+            hpc = _attn_heads_per_cta(rows, pdl, prefetch)
+            need.append(min(rows * (64 // hpc), 18) * _attn_slot_bytes(hpc))
+        got = ws(B, Nq, 64, 512, 512, 128)
+        assert got == max(need), (B, Nq, got, need)
+    # the tensor-core kernels need no workspace outside their shape, nor does the general kernel
+    assert ws(2, 1, 8, 128, 512, 128) == 0
+    assert ws(2, 1, 64, 512, 1024, 128) == 0

@@ -23,9 +23,12 @@ together in the order the pages give them:
 * "890 bytes per token: how DeepSeek V4.1-Flash's KV cache works", mechanism 4:
   attention runs only over the selected candidates.
 
-Parity pins: every function here is checked by ``tests/test_oracle_pins.py``
+Parity pins: every function here is checked by ``tests/test_oracle_formats.py``,
+``tests/test_oracle_selection.py`` and ``tests/test_oracle_attention.py``
 against closed forms, the ml_dtypes format library, numpy/torch library
-routines, brute force on tiny inputs and the invariants the pages fix.
+routines, brute force on tiny inputs and the invariants the pages fix;
+``tests/test_oracle_mutants.py`` plants single mistakes in copies of the oracle
+and checks that those pins catch each one.
 """
 from __future__ import annotations
 
@@ -52,7 +55,12 @@ FULL, REINDEX, REUSE = "full", "reindex", "reuse"
 
 def build(force: bool = False) -> str:
     """Compile the oracle with gcc (plain -O2, no fast-math: IEEE fp32 division
-    and conversion must be exact). Returns the path of the shared library."""
+    and conversion must be exact). Returns the path of the shared library.
+    CSA2_ORACLE_LIB names a library to load instead (the mutation tests build
+    copies of this source with one planted mistake each)."""
+    override = os.environ.get("CSA2_ORACLE_LIB")
+    if override:
+        return override
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         os.makedirs(os.path.dirname(_LIB_PATH), exist_ok=True)
         tmp = _LIB_PATH + f".tmp{os.getpid()}"

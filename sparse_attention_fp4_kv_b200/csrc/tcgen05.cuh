@@ -1,6 +1,6 @@
 // Device-side wrappers shared by the tensor-core attention kernels: shared
 // memory and proxy fences, mbarriers, TMEM allocation and loads/stores,
-// tcgen05.mma (kind::f16) descriptors, cp.async, and the FP4 -> bf16 helpers.
+// tcgen05.mma (kind::f16) descriptors, and the FP4 -> bf16 helpers.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -109,12 +109,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
-}
 // Byte offset of 16-byte piece p (0..7) of row r inside a 128B-swizzled,
 // 8-row-atom column (rows at 128 B, atoms at 1024 B).
 __device__ __forceinline__ uint32_t sw128(int r, int p) {

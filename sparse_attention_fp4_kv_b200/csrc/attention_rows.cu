@@ -333,19 +333,25 @@ __global__ void __launch_bounds__(THREADS, 1)
                     uint2 codes[LROWS];
                     uint32_t scl[LROWS / 4] = {};
                     bool vrow[LROWS];
+                    // every load is issued, all before the first use (a row that is
+                    // not selected reads row 0 and is zeroed after the loads)
 #pragma unroll
                     for (int u = 0; u < LROWS; u++) {
                         const int32_t pos = pos_next[u];
                         vrow[u] = pos >= 0 && pos < a.cap;
-                        const int64_t src = (int64_t)b * a.cap + pos;
-                        codes[u] = vrow[u] ? __ldg(reinterpret_cast<const uint2 *>(a.kv_fp4 + src * 256) + lane)
-                                           : make_uint2(0, 0);
+                        const int64_t src = vrow[u] ? (int64_t)b * a.cap + pos : 0;
+                        codes[u] = __ldg(reinterpret_cast<const uint2 *>(a.kv_fp4 + src * 256) + lane);
                         // E4M3 of this lane's 16-channel group, or the E8M0 of its 32-channel block
-                        const uint32_t sb =
-                            vrow[u] ? (uint32_t)__ldg(a.mx ? a.kv_sf + src * 16 + (lane >> 1)
-                                                           : a.kv_sf + src * 32 + lane)
-                                    : 0u;
+                        const uint32_t sb = (uint32_t)__ldg(a.mx ? a.kv_sf + src * 16 + (lane >> 1)
+                                                                 : a.kv_sf + src * 32 + lane);
                         scl[u >> 2] |= sb << (8 * (u & 3));
+                    }
+#pragma unroll
+                    for (int u = 0; u < LROWS; u++) {
+                        if (!vrow[u]) {
+                            codes[u] = make_uint2(0, 0);
+                            scl[u >> 2] &= ~(0xFFu << (8 * (u & 3)));
+                        }
                     }
                     // indices of the next selected tile, while these loads are in flight
                     if (t + 1 < n_sel_tiles) {

@@ -177,6 +177,10 @@ def test_quantize_error_bound_and_zero_group():
     z = np.zeros((1, 32), np.uint16)
     p, s = oracle.fp4_quantize(z)
     assert np.all(p == 0) and np.all(s == 0)
+    # a group of negative zeros: its scale is 0, so every code is +0 (no sign kept)
+    nz = np.full((1, 16), 0x8000, np.uint16)
+    p, s = oracle.fp4_quantize(nz)
+    assert np.all(p == 0) and np.all(s == 0)
     # a group whose amax/6 rounds below the smallest E4M3 subnormal: scale 0, codes +0
     tiny = _bf16(np.full(16, 2.0 ** -13, np.float32))[None, :]
     p, s = oracle.fp4_quantize(tiny)

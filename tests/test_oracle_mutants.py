@@ -86,6 +86,28 @@ C_MUTANTS = [
      "dot += (double)bf16_to_float(q[h * C + c]) * kv[c * n + j];", 1, ["attention"]),
     ("attention values shifted by a channel", "acc += logit[j] * kv[j * C + c];",
      "acc += logit[j] * kv[j * C + (c + 1) % C];", 1, ["attention"]),
+    ("mx zero block takes exponent 0", "    if (amax == 0.0)\n        return -127;",
+     "    if (amax == 0.0)\n        return 0;", 1, ["formats"]),
+    ("mx exponent clamped at -126", "    if (e < -127)\n        e = -127;",
+     "    if (e < -126)\n        e = -126;", 1, ["formats"]),
+    ("e4m3 code 0x7F read as 480", "    if (e == 0xF && m == 0x7)\n        return NAN;\n", "", 1,
+     ["formats"]),
+    ("e4m3 saturates at 240", "    if (ax > 448.0)\n        ax = 448.0;", "    if (ax > 240.0)\n        ax = 240.0;",
+     1, ["formats"]),
+    ("zero-scale group keeps the sign of zeros",
+     "                    if (s == 0.0f) {\n                        code[u] = 0;",
+     "                    if (s == 0.0f) {\n                        code[u] = signbit(xv) ? 0x8 : 0;", 1,
+     ["formats"]),
+    ("mx elements scaled one exponent low",
+     "double v = ldexp((double)bf16_to_float(xr[g * 32 + c + u]), -e);",
+     "double v = ldexp((double)bf16_to_float(xr[g * 32 + c + u]), -e - 1);", 1, ["formats"]),
+    ("mx dequantize takes the wrong block's scale", "double s = orc_e8m0_value(sf[r * (C / 32) + c / 32]);",
+     "double s = orc_e8m0_value(sf[r * (C / 32) + c / 64]);", 1, ["formats"]),
+    ("index score overflow not rejected",
+     "        if (acc > INT32_MAX || acc < INT32_MIN)\n            return -1;\n", "", 1, ["selection"]),
+    ("block max ignores the first token", "        float m = score[8 * j];",
+     "        float m = score[8 * j + 1 < n_visible ? 8 * j + 1 : 8 * j];", 1, ["selection"]),
+    ("selection padded with 0", "        out[i] = -1;", "        out[i] = 0;", 1, ["selection"]),
 ]
 
 # (name, text in oracle/__init__.py, replacement, pin files)
@@ -104,6 +126,15 @@ PY_MUTANTS = [
      "top, _, _ = reindex_layer(q_idx_of(0), k_idx, k_scale, pool, n_visible)", ["selection"]),
     ("bf16 read one bit low", "u = np.ascontiguousarray(x_bf16, dtype=np.uint16).astype(np.uint32) << 16",
      "u = np.ascontiguousarray(x_bf16, dtype=np.uint16).astype(np.uint32) << 15", ["attention"]),
+    ("window ends one position early", "hi = min(q_pos, swa_pos0 + swa_rows - 1)",
+     "hi = min(q_pos - 1, swa_pos0 + swa_rows - 1)", ["attention"]),
+    ("Full top-k one short", "top = topk(tok[ppos], ppos, k_top)", "top = topk(tok[ppos], ppos, k_top - 1)",
+     ["selection"]),
+    ("Reindex key scales doubled", "sc = index_scores(q_idx, k_idx[ppos], k_scale[ppos])",
+     "sc = index_scores(q_idx, k_idx[ppos], k_scale[ppos] * 2)", ["selection"]),
+    ("attention drops selected position 0", "sel = sel[sel >= 0]", "sel = sel[sel > 0]", ["attention"]),
+    ("stack returns the pool reversed", "            pools[l] = pool", "            pools[l] = pool[::-1].copy()",
+     ["selection"]),
 ]
 
 

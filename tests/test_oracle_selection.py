@@ -216,6 +216,10 @@ def test_stack_reuse_layers_take_producer_indices():
     modes = oracle.decoder_schedule()
     tops, pools = oracle.stack_indices(modes, lambda l: qs[l], k, s, ctx)
     assert list(pools) == [0]
+    # the Full layer's pool and indices, as the layer alone computes them (ascending, -1 padded)
+    full = oracle.full_layer(qs[0], k, s, ctx)
+    assert np.array_equal(pools[0], full["pool"]) and np.array_equal(tops[0], full["top"])
+    assert np.all(np.diff(pools[0][pools[0] >= 0]) > 0)
     for l, m in enumerate(modes):
         producer = max(i for i in range(l + 1) if modes[i] != oracle.REUSE)
         assert np.array_equal(tops[l], tops[producer])

@@ -72,6 +72,7 @@ def test_append_ties_zeros_and_tiny_groups(B):
     for s in e4:
         rows.append(mult * s)
     rows.append(np.zeros(16))
+    rows.append(-np.zeros(16))                      # negative zeros: scale 0, codes +0
     rows.append(np.full(16, 2.0 ** -13))            # amax/6 below the smallest E4M3 subnormal
     rows.append(np.full(16, -(2.0 ** -12)))
     rows.append(np.array([3e38] + [1.0] * 15))       # scale saturates at 448

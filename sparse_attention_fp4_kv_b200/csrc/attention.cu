@@ -189,9 +189,11 @@ size_t attn_workspace_bytes(int B, int Nq, int Hq, int C, int K, int n_win) {
 }
 
 // Tensor-core kernels where their shape constraints hold (64 heads, 512
-// channels): one CTA per row when there are more rows than the split-key
-// kernel's clusters cover in one wave (and for more than 640 keys per row),
-// the split-key cluster kernel otherwise; the general kernel for other shapes.
+// channels): one CTA per row from kAttnRowsMin (64) rows, where the per-row
+// kernel's 148 persistent CTAs outrun the split-key clusters looping over rows
+// (and whenever the split-key kernel cannot take the call, e.g. more than 640
+// keys per row); the split-key cluster kernel below that; the general kernel
+// for other shapes.
 int launch_attn(const AttnArgs &a, cudaStream_t s) {
     const int64_t rows = (int64_t)a.B * a.Nq;
     const bool rows_ok = attn_rows_supported(a);

@@ -67,8 +67,9 @@ int launch_attn_general(const AttnArgs &a, cudaStream_t s);
 bool attn_tc_supported(const AttnArgs &a);
 size_t attn_tc_workspace_bytes(int B, int Nq);
 int launch_attn_tc(const AttnArgs &a, cudaStream_t s);
-// One CTA per query row (attention_rows.cu): no workspace; for calls with
-// more rows than the split-key kernel runs at once.
+// One CTA per query row (attention_rows.cu): no workspace; for calls of
+// kAttnRowsMin rows or more (below that the split-key clusters measured
+// faster: at 32 rows and fewer, the decode batches).
 bool attn_rows_supported(const AttnArgs &a);
 int launch_attn_rows(const AttnArgs &a, cudaStream_t s);
 constexpr int64_t kAttnRowsMin = 64;

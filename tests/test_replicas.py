@@ -1,5 +1,6 @@
 """Multi-process (gloo, world size 2, CPU) tests of the host logic that
-bench.py uses on N GPUs: per-rank workloads and max-over-ranks timing."""
+bench.py uses on N GPUs: per-rank workloads and max-over-ranks timing; and the
+bench's clock record."""
 import os
 import socket
 
@@ -55,3 +56,41 @@ def test_single_process_is_a_no_op():
     assert replicas.rank_workload(w, 0, 1) is w
     assert replicas.slowest([1.5, 2.5]) == [1.5, 2.5]
     assert replicas.aggregate_rate(20, 1, 2.0) == pytest.approx(10000.0)
+
+
+def test_clock_summary_of_sampled_lines():
+    """The bench's clock record: median SM clock under load, the max clock and
+    every throttle reason reported active (from nvidia-smi CSV lines)."""
+    import importlib.util
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(root, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    lines = "\n".join([
+        "0, 1965, 1965, 812.4, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1920, 1965, 998.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1965, 1965, 905.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+        "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ])
+    c = bench.summarize_clocks(lines)
+    assert c == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    hot = "0, 1400, 1965, 1000, 0x48, Active, Active, Not Active, Not Active"
+    assert bench.summarize_clocks(hot)["reasons"] == ["hw_slowdown", "hw_thermal_slowdown"]
+    assert bench.summarize_clocks("")["samples"] == 0
+    # the sampler's stop(): ends the sampling process, reads and removes its file
+    import tempfile
+
+    class _Proc:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    cs = bench.ClockSampler.__new__(bench.ClockSampler)
+    cs.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+    cs.file.write(lines + "\n")
+    cs.proc = _Proc()
+    name = cs.file.name
+    assert cs.stop() == c and not os.path.exists(name)

@@ -459,6 +459,7 @@ def _attention_case(B, Bn, ctx, C, Hq, K, n_win, seed, q_pos=None, Nq=1, drop=0,
 
 
 @pytest.mark.parametrize("Bn,ctx,C,Hq,K", [(3, 5000, 512, 64, 512), (2, 3000, 512, 64, 488),
+                                           (2, 3000, 512, 64, 100),
                                            (2, 3000, 128, 8, 512),
                                            (1, 300, 512, 64, 512), (2, 100, 256, 16, 512),
                                            (1, 2000, 64, 3, 100)])

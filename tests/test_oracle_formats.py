@@ -187,6 +187,123 @@ def test_quantize_error_bound_and_zero_group():
     assert s[0, 0] == 0 and np.all(p == 0)
 
 
+def _nvfp4_pack_restated(x_bf16):
+    """The FP4 pack of [N] "FP4 KV Quantization and Cache Lifetime Management"
+    (E2M1 elements, one E4M3 scale per 16 channels, NVFP4 without its global
+    scale) restated with numpy float32 arithmetic and the ml_dtypes format
+    casts, sharing nothing with the oracle's C code: per group amax, then
+    s_f = float32(amax) / float32(6) (IEEE division), scale = E4M3 RNE of s_f
+    saturating at 448, each element float32(x) / float32(scale) (IEEE
+    division) cast to E2M1 (RNE, saturating, sign kept), a zero scale giving
+    +0 codes, two codes per byte with the even channel in the low nibble."""
+    x = np.ascontiguousarray(x_bf16, np.uint16)
+    rows, C = x.shape
+    xf = (x.astype(np.uint32) << 16).view(np.float32).reshape(rows, C // 16, 16)
+    amax = np.abs(xf).max(axis=2)
+    s_f = amax / np.float32(6)
+    assert s_f.dtype == np.float32
+    s_code = np.minimum(s_f, np.float32(448)).astype(ml_dtypes.float8_e4m3fn)
+    s = s_code.astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = xf / s[:, :, None]
+    assert v.dtype == np.float32
+    codes = v.astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF
+    codes = np.where(s[:, :, None] == 0, np.uint8(0), codes).reshape(rows, C)
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    return packed, s_code.view(np.uint8)
+
+
+def _tie_multiple_groups():
+    """One group per (E4M3 scale s, E2M1 tie point k): an element 6 s (so amax/6
+    is exactly s) and the others k s for the seven ties k = 0.25 ... 5 with both
+    signs, all exactly representable in bf16. x / s is then exactly the tie; a
+    division that is off by one ulp breaks it the other way."""
+    e4 = np.arange(1, 0x7F, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    groups = []
+    for s in e4:
+        for lead in (1.0, -1.0):
+            g = np.concatenate([[6.0 * lead], ties, -ties, [0.0]]) * s
+            groups.append(g)
+    x = np.array(groups, np.float32)
+    return _bf16(x)
+
+
+def _scale_midpoint_groups():
+    """Groups whose amax / 6 is exactly the midpoint of two neighbouring E4M3
+    values (a tie of the scale rounding), with tie-multiple elements of the
+    scale that the midpoint rounds to."""
+    e4 = np.arange(0, 0x7F, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    mids = (e4[1:] + e4[:-1]) / 2
+    out = []
+    for m in mids:
+        amax = 6.0 * m
+        if amax > 3.0e38:
+            continue
+        body = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1.5, 3.0, 4.0, 6.0, 2.0, 1.0, 0.0]) * m
+        for sign in (1.0, -1.0):
+            out.append(np.concatenate([[sign * amax], body * sign]))
+    x = np.array(out, np.float32)
+    u = x.view(np.uint32)
+    keep = np.all((u & 0xFFFF) == 0, axis=1)       # every value exact in bf16
+    return (u[keep] >> 16).astype(np.uint16)
+
+
+def _random_finite_bf16_groups(n_groups, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.integers(0, 1 << 16, size=(n_groups, 16), dtype=np.uint32).astype(np.uint16)
+    finite = (x & 0x7F80) != 0x7F80
+    return np.where(finite, x, np.uint16(0)).astype(np.uint16)
+
+
+@pytest.mark.parametrize("inputs", ["tie_multiples", "scale_midpoints", "random_bits"])
+def test_quantize_matches_independent_nvfp4_restatement(inputs):
+    if inputs == "tie_multiples":
+        x = _tie_multiple_groups()
+        assert x.shape[0] == 2 * 126
+    elif inputs == "scale_midpoints":
+        x = _scale_midpoint_groups()
+        assert x.shape[0] >= 200
+    else:
+        x = _random_finite_bf16_groups(262_144, seed=29)
+    # rows of 16 groups (256 channels) keep the layout of a real cache row
+    pad = (-x.shape[0]) % 16
+    x = np.concatenate([x, np.zeros((pad, 16), np.uint16)]).reshape(-1, 256)
+    packed, sf = oracle.fp4_quantize(x)
+    rp, rs = _nvfp4_pack_restated(x)
+    bad_s = np.argwhere(sf != rs)
+    assert bad_s.size == 0, bad_s[:5]
+    bad_p = np.argwhere(packed != rp)
+    assert bad_p.size == 0, [(tuple(i), int(packed[tuple(i)]), int(rp[tuple(i)])) for i in bad_p[:5]]
+
+
+def every_bf16_amax_groups():
+    """One 16-channel group per finite bf16 magnitude a (both signs): a in
+    channel 0, a/2 rounded down to bf16 in channel 1, zeros elsewhere. The
+    group's amax runs over every finite bf16 value."""
+    b = np.arange(1, 0x7F80, dtype=np.uint16)
+    g = np.zeros((2 * b.size, 16), np.uint16)
+    g[:b.size, 0] = b
+    g[b.size:, 0] = b | 0x8000
+    half = _trunc_bf16(((b.astype(np.uint32) << 16).view(np.float32) / np.float32(2)))
+    g[:b.size, 1] = half
+    g[b.size:, 1] = half | 0x8000
+    return g
+
+
+def test_quantize_scale_for_every_bf16_amax():
+    """The scale step alone, exhaustively: for every finite bf16 amax the
+    oracle's scale byte is E4M3_RNE_satfinite(float32(amax) / 6)."""
+    g = every_bf16_amax_groups()
+    _, sf = oracle.fp4_quantize(g)
+    a = np.abs((g[:, 0].astype(np.uint32) << 16).view(np.float32))
+    ref = np.minimum(a / np.float32(6), np.float32(448)).astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    bad = np.nonzero(sf[:, 0] != ref)[0]
+    assert bad.size == 0, [(float(a[i]), int(sf[i, 0]), int(ref[i])) for i in bad[:5]]
+    rp, rs = _nvfp4_pack_restated(g)
+    assert np.array_equal(rs[:, 0], sf[:, 0])
+
+
 def test_dequantize_every_code_and_scale_is_exact_product():
     codes = np.arange(16, dtype=np.uint8)
     packed = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)
@@ -211,7 +328,8 @@ def test_fp4_row_bytes_match_pages():
 # [T] mechanism 3 names the cache format MXFP4; read as the OCP Microscaling
 # format: E2M1 elements, one E8M0 scale per 32 channels, shared exponent
 # floor(log2(amax)) - 2.
-def _bf16(x):
+def _trunc_bits(x):
+    """float32 values -> bf16 bit patterns (as uint32) by dropping the low 16 bits."""
     return np.asarray(x, dtype=np.float32).view(np.uint32) >> 16
 
 
@@ -252,7 +370,7 @@ def test_mxfp4_quantize_is_e2m1_of_the_scaled_block():
     x = (rng.standard_normal((40, 128)) * np.exp(rng.uniform(-20, 20, (40, 1)))).astype(np.float32)
     x[3, :32] = 0.0
     x[5, 40:48] *= 1e4
-    xb = _bf16(x).astype(np.uint16)
+    xb = _trunc_bits(x).astype(np.uint16)
     xf = (xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     packed, sf = oracle.mxfp4_quantize(xb)
     for r in range(x.shape[0]):
@@ -274,15 +392,15 @@ def test_mxfp4_exact_round_trip_and_invariants():
         codes = rng.integers(0, 16, 32)
         codes[rng.integers(0, 32)] = 6 + int(rng.integers(0, 2))   # amax in [4, 6]
         x = e2m1[codes] * 2.0 ** s
-        xb = _bf16(x).astype(np.uint16)
+        xb = _trunc_bits(x).astype(np.uint16)
         packed, sf = oracle.mxfp4_quantize(xb[None])
         assert sf[0, 0] == s + 127
         assert np.array_equal(oracle.mxfp4_dequantize(packed, sf)[0], x)
         # scaling by 2^t shifts only the scale code; negation flips only the signs
         t = int(rng.integers(-5, 5))
-        p2, sf2 = oracle.mxfp4_quantize(_bf16(x * 2.0 ** t).astype(np.uint16)[None])
+        p2, sf2 = oracle.mxfp4_quantize(_trunc_bits(x * 2.0 ** t).astype(np.uint16)[None])
         assert int(sf2[0, 0]) == int(sf[0, 0]) + t and np.array_equal(p2, packed)
-        p3, sf3 = oracle.mxfp4_quantize(_bf16(-x).astype(np.uint16)[None])
+        p3, sf3 = oracle.mxfp4_quantize(_trunc_bits(-x).astype(np.uint16)[None])
         assert np.array_equal(sf3, sf)
         assert np.all((p3 ^ packed) == 0x88)  # every sign bit flips (zeros too)
 
@@ -290,7 +408,7 @@ def test_mxfp4_exact_round_trip_and_invariants():
 def test_mxfp4_error_bound_saturation_and_zero_block():
     rng = np.random.default_rng(24)
     x = rng.standard_normal((64, 64)).astype(np.float32) * 3.0
-    xb = _bf16(x).astype(np.uint16)
+    xb = _trunc_bits(x).astype(np.uint16)
     xf = (xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     packed, sf = oracle.mxfp4_quantize(xb)
     xh = oracle.mxfp4_dequantize(packed, sf)

@@ -108,6 +108,22 @@ C_MUTANTS = [
     ("block max ignores the first token", "        float m = score[8 * j];",
      "        float m = score[8 * j + 1 < n_visible ? 8 * j + 1 : 8 * j];", 1, ["selection"]),
     ("selection padded with 0", "        out[i] = -1;", "        out[i] = 0;", 1, ["selection"]),
+    ("fp4 element by reciprocal multiply", "float v = xv / s; /* fp32 IEEE division */",
+     "float v = xv * (1.0f / s);", 1, ["formats"]),
+]
+
+# Mutants that change the arithmetic but not a single output over the oracle's
+# input domain (bf16 values), so no pin can catch them. Each is built and
+# checked to give the unmutated oracle's bytes on every input of the step it
+# changes; if that ever stopped holding, it would belong in C_MUTANTS.
+#   fp4 scale by reciprocal multiply: fp32(amax * fp32(1/6)) differs from
+#   fp32(amax / 6) for some bf16 amax (about 10,600 of 32,640), but never by
+#   enough to change the E4M3 code it rounds to: an E4M3 midpoint m has at most
+#   5 significant bits, so amax / 6 lands on it only when amax = 6 m exactly,
+#   where both forms give m.
+EQUIVALENT_C_MUTANTS = [
+    ("fp4 scale by reciprocal multiply", "float s_f = amax / 6.0f; /* fp32 IEEE division */",
+     "float s_f = amax * (1.0f / 6.0f);", 1),
 ]
 
 # (name, text in oracle/__init__.py, replacement, pin files)
@@ -211,6 +227,30 @@ def test_every_python_mutant_fails_a_pin(tmp_path):
         results = list(ex.map(one, range(len(PY_MUTANTS))))
     survivors = [name for name, rc in results if rc == 0]
     assert not survivors, f"mutants no pin catches: {survivors}"
+
+
+@pytest.mark.parametrize("name,old,new,nth", EQUIVALENT_C_MUTANTS, ids=[m[0] for m in EQUIVALENT_C_MUTANTS])
+def test_equivalent_mutant_changes_no_output(tmp_path, name, old, new, nth):
+    """The mutant's FP4 bytes and scales equal the oracle's for a group of
+    every finite bf16 amax (both signs)."""
+    src = open(C_SRC).read()
+    lib = _compile(_replace_nth(src, old, new, nth), str(tmp_path / "eq"))
+    code = (f"import sys; sys.path.insert(0, {ROOT!r}); sys.path.insert(0, {os.path.join(ROOT, 'tests')!r}); "
+            "import numpy as np, oracle, test_oracle_formats as F; "
+            "g = F.every_bf16_amax_groups(); p, s = oracle.fp4_quantize(g); "
+            "np.save(sys.argv[1], np.concatenate([p, s], axis=1))")
+    outs = []
+    for i, l in enumerate([lib, oracle_lib()]):
+        f = str(tmp_path / f"out{i}.npy")
+        subprocess.check_call([sys.executable, "-c", code, f], cwd=ROOT, env=dict(os.environ, CSA2_ORACLE_LIB=l),
+                              timeout=600)
+        outs.append(__import__("numpy").load(f))
+    assert (outs[0] == outs[1]).all(), name
+
+
+def oracle_lib():
+    from oracle import build
+    return build()
 
 
 @pytest.mark.parametrize("name,old,new,nth,files", C_MUTANTS, ids=[m[0] for m in C_MUTANTS])

@@ -129,8 +129,7 @@ def summarize_clocks(text: str) -> dict:
             "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def _config(wl, name):
-    w = wl.w
+def _config(w, name):
     return {"workload": name, "batch_per_gpu": w.B, "ctx": w.ctx, "layers": w.n_layers,
             "schedule": "".join("FRU"[m] for m in w.modes), "main_kv": f"fp4 e2m1+e4m3/16, {w.C} ch",
             "q_heads": w.Hq, "indexer": f"int8 {w.H_idx}x{w.D_idx}", "pool_blocks": 2048,
@@ -141,12 +140,20 @@ def _config(wl, name):
 
 
 # ----------------------------------------------------------------------------- oracle timing
+def _host_cores() -> dict:
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except AttributeError:
+        usable = os.cpu_count()
+    return {"cpu_count": os.cpu_count(), "usable": usable}
+
+
 def _oracle_sequence_step(inp):
     """The oracle's decode step for one sequence of the stack (all layers)."""
     import oracle
     modes = inp["modes"]
     ctx = inp["ctx"]
-    kn, sn, kvb = inp["k_idx"], inp["k_scale"], inp["kv_bf16_rows"]
+    kn, sn, kv = inp["k_idx"], inp["k_scale"], inp["kv_bf16"]
     pool = inp.get("pool0")
     top = None
     outs = []
@@ -156,86 +163,116 @@ def _oracle_sequence_step(inp):
             pool, top = r["pool"], r["top"]
         elif m == 1:
             top, _, _ = oracle.reindex_layer(inp["q_idx"][l], kn, sn, pool, ctx)
-        outs.append(oracle.sparse_attention(inp["q"][l], lambda P: kvb(P), top, inp["swa"][l],
+        outs.append(oracle.sparse_attention(inp["q"][l], lambda P: kv[P], top, inp["swa"][l],
                                             ctx - 1, ctx - inp["swa_rows"], inp["scale"]))
     return outs
 
 
+def _bits(t):
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
 def _oracle_inputs_from_device(wl, b):
-    """Host copies of sequence b's inputs (the same buffers the GPU arm uses)."""
-    def bits(t):
-        return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    """Host copies of sequence b's inputs: the buffers the GPU arm uses, with
+    the bf16 main-KV rows (before quantization) re-drawn on the device."""
     from sparse_attention_fp4_kv_b200 import synth
+    import oracle
     w = wl.w
-    kv_rows = {}
-
-    def kvb(P):
-        P = np.asarray(P, dtype=np.int64)
-        # re-draw the bf16 rows of the requested positions (seeded, chunked)
-        out = np.empty((P.size, w.C), dtype=np.uint16)
-        for j, p in enumerate(P.tolist()):
-            c = p // 8192
-            if c not in kv_rows:
-                kv_rows[c] = bits(synth.main_kv_bf16(w, b, c * 8192, min(w.ctx, c * 8192 + 8192),
-                                                     wl.device))
-            out[j] = kv_rows[c][p - c * 8192]
-        return out
-
     inp = dict(modes=list(wl.modes), ctx=w.ctx, k_idx=wl.k_idx[b].cpu().numpy(),
-               k_scale=wl.k_scale[b].cpu().numpy(), kv_bf16_rows=kvb,
+               k_scale=wl.k_scale[b].cpu().numpy(),
+               kv_bf16=_bits(synth.main_kv_bf16(w, b, 0, w.ctx, wl.device)),
                q_idx={l: q[b, 0].cpu().numpy() for l, q in enumerate(wl.q_idx) if q is not None},
-               q=[bits(q[b, 0]) for q in wl.q], swa=[bits(s[b]) for s in wl.swa],
+               q=[_bits(q[b, 0]) for q in wl.q], swa=[_bits(s[b]) for s in wl.swa],
                swa_rows=wl.swa_rows, scale=wl.scale)
     if wl.pool_ready:
-        import oracle
         inp["pool0"] = oracle.full_layer(wl.pool_q_idx[b, 0].cpu().numpy(), inp["k_idx"],
                                          inp["k_scale"], w.ctx)["pool"]
     return inp
 
 
-def _time_oracle(inp, B, n_layers, reps=1):
+def _oracle_inputs_on_host(w, b):
+    """Sequence b's inputs drawn on the host by the seeded generators alone (no
+    GPU, no libcsa2): the same shapes and distributions as the GPU arm's
+    (values drawn on the CPU differ from values drawn on a GPU)."""
+    from sparse_attention_fp4_kv_b200 import synth
+    import oracle
+    rows = min(w.n_win, w.ctx)
+    k_idx = synth.indexer_keys(w, b, w.ctx, "cpu")
+    q_idx = {l: synth.indexer_q(w, l, 1, "cpu") for l, m in enumerate(w.modes) if m != synth.REUSE}
+    inp = dict(modes=list(w.modes), ctx=w.ctx, k_scale=synth.indexer_key_scale(w, b, w.ctx, "cpu").numpy(),
+               kv_bf16=_bits(synth.main_kv_bf16(w, b, 0, w.ctx, "cpu")),
+               q=[_bits(synth.main_q(w, l, 1, "cpu")[b, 0]) for l in range(w.n_layers)],
+               swa=[_bits(synth.swa_kv(w, l, rows, "cpu")[b]) for l in range(w.n_layers)],
+               swa_rows=rows, scale=1.0 / np.sqrt(w.C))
+    if w.modes[0] == synth.REINDEX:
+        # set-up: plant the correlated blocks, then the pool of a preceding Full layer
+        q_r = q_idx[0]
+        if w.planted_blocks:
+            synth.plant(w, b, k_idx, q_r[b, 0])
+        inp["pool0"] = oracle.full_layer(synth.pool_builder_q(w, q_r)[b, 0].numpy(), k_idx.numpy(),
+                                         inp["k_scale"], w.ctx)["pool"]
+    inp["k_idx"] = k_idx.numpy()
+    inp["q_idx"] = {l: q[b, 0].numpy() for l, q in q_idx.items()}
+    return inp
+
+
+def _time_oracle(inp, reps=3):
+    """Seconds per oracle step of one sequence: one untimed warm-up, then the
+    median of `reps` timed runs on the same pre-drawn inputs."""
+    _oracle_sequence_step(inp)
     ts = []
     for _ in range(reps):
         t0 = time.perf_counter()
         _oracle_sequence_step(inp)
         ts.append(time.perf_counter() - t0)
-    t_seq = statistics.median(ts)
-    # the oracle is single-threaded; a decode step of the batch is B sequences
-    return n_layers / (B * t_seq), t_seq
+    return statistics.median(ts)
 
 
 # ----------------------------------------------------------------------------- arms
+REFERENCE_BUDGET_S = 150.0
+
+
 def run_reference(args, name):
-    """CPU oracle arm: each step is the oracle's full decode step of one
-    sequence (all layers), a bounded sample of the batch; the rate is scaled to
-    the batch by the number of sequences."""
+    """CPU oracle arm (the OpenMP build, every usable host core). A step is the
+    oracle's decode step (every layer) of S sequences of the batch: the whole
+    batch (S = B) when K + W such steps fit in REFERENCE_BUDGET_S, else as many
+    sequences as fit (at least one). ms_per_step is the measured time of those
+    S sequences; value is the batch rate at that time per sequence."""
     from sparse_attention_fp4_kv_b200 import synth
     import oracle
-    oracle.build()
+    threads = oracle.use_openmp(True)
     w = synth.WORKLOADS[name]
-    dev = "cuda" if torch.cuda.is_available() else "cpu"
-    from sparse_attention_fp4_kv_b200.workload import DecodeWorkload
-    wl = DecodeWorkload(w, dev)
-    inp = _oracle_inputs_from_device(wl, 0)
-    cfg = _config(wl, name)
-    del wl
-    if dev == "cuda":
-        torch.cuda.empty_cache()
+    t_setup = time.perf_counter()
+    inputs = [_oracle_inputs_on_host(w, 0)]
+    t_seq = _time_oracle(inputs[0], reps=1)
+    n_steps = args.steps + args.warmup
+    S = int(max(1, min(w.B, REFERENCE_BUDGET_S // max(n_steps * t_seq, 1e-9))))
+    for b in range(1, S):
+        inputs.append(_oracle_inputs_on_host(w, b))
+    t_setup = time.perf_counter() - t_setup
+
+    def step():
+        for inp in inputs:
+            _oracle_sequence_step(inp)
+
     for _ in range(args.warmup):
-        _oracle_sequence_step(inp)
+        step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        _oracle_sequence_step(inp)
-    t_seq = (time.perf_counter() - t0) / args.steps
-    ms = t_seq * w.B * 1e3
-    value = w.n_layers / (ms / 1e3)
-    sample = (f"sequence 0 of {w.B}: Full-layer scan over all {w.ctx} tokens, pool, every "
-              f"layer's top-512 and attention ({w.n_layers} layers); rate scaled x1/{w.B}")
+        step()
+    ms = (time.perf_counter() - t0) / args.steps * 1e3
+    value = w.n_layers * S / w.B / (ms / 1e3)
+    sample = (f"{S} of {w.B} sequences per step (all {w.n_layers} layers each: Full-layer scan over "
+              f"all {w.ctx} tokens, pool, every layer's top-512 and attention); value = rate of the "
+              f"{w.B}-sequence batch at the measured time per sequence; inputs drawn on the host by "
+              f"the seeded generators ({t_setup:.0f} s set-up, untimed); OpenMP oracle build, "
+              f"{threads} threads")
+    cfg = _config(w, name)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "int64/fp64", "data": "synthetic", "config": cfg,
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "dtype": "int64/fp64", "data": "synthetic", "config": cfg, "host_cores": _host_cores(),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -391,6 +428,9 @@ def run_csa2(args, name, rank, world, local_rank):
 
     # ---- end to end through the public API with host buffers
     e2e = _e2e(wl, args, stream, world, local_rank)
+    from sparse_attention_fp4_kv_b200 import binding
+    # every bounded wait of the timed steps completed (0); otherwise the outputs are invalid
+    status = binding.device_status()
 
     nbytes = wl.step_bytes()
     peak, peak_kind = _peaks()
@@ -399,7 +439,7 @@ def run_csa2(args, name, rank, world, local_rank):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8/fp32", "data": "synthetic",
-            "config": _config(wl, name),
+            "config": _config(w, name),
             "roofline": {"bound": "hbm", "kernel": "index_full_kernel (Full-layer indexer scan)",
                          "achieved": scan_gbs, "peak": peak, "unit": "GB/s",
                          "frac": scan_gbs / peak, "peak_kind": peak_kind,
@@ -412,14 +452,25 @@ def run_csa2(args, name, rank, world, local_rank):
             "timing": {"value_from": "CUDA graph replays" if graph_ms is not None else "direct launches",
                        "graph_ms_per_step": graph_ms / K if graph_ms is not None else None,
                        "direct_ms_per_step": ms_direct / K, "note": graph_note}}
+    line["device_status"] = status
+    line["host_cores"] = _host_cores()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        threads = oracle.use_openmp(True)
         inp = _oracle_inputs_from_device(wl, 0)
-        v, t_seq = _time_oracle(inp, w.B, w.n_layers)
-        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
-                                "sample": f"sequence 0 of {w.B}, all {w.n_layers} layers "
-                                          f"({t_seq:.1f} s), rate scaled x1/{w.B}"}
+        t_seq = _time_oracle(inp, reps=3)
+        line["cpu_baseline"] = {"value": w.n_layers / (w.B * t_seq), "unit": UNIT, "cores": threads,
+                                "kind": "oracle",
+                                "sample": f"sequence 0 of {w.B}, all {w.n_layers} layers, the GPU arm's "
+                                          f"inputs copied to the host; median of 3 runs after one "
+                                          f"warm-up ({t_seq:.2f} s per sequence); rate of the "
+                                          f"{w.B}-sequence batch at that time per sequence; OpenMP "
+                                          f"oracle build, {threads} threads"}
     if rank == 0:
         print(json.dumps(line), flush=True)
+    if status != 0:
+        raise SystemExit(f"a kernel gave up a bounded wait (csa2_device_status = {status}): "
+                         "the step's outputs are invalid")
 
 
 def _e2e(wl, args, stream, world, local_rank):

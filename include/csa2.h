@@ -339,6 +339,10 @@ int csa2_decode_stack(const csa2_layer *layers, int n_layers, const void *kv_new
  * Set-up: the first call on each device, with that device current, looks up
  * the array's device address (cudaGetSymbolAddress) and keeps it. Make that
  * first call before any stream capture. A failed look-up returns CSA2_ERR_CUDA.
+ * The kept address belongs to the device's current CUDA context: after
+ * cudaDeviceReset (or anything else that destroys that context) it no longer
+ * names the array, so a process that resets a device must not call this entry
+ * point on that device again.
  * Sharing: every call uses the same array, which keeps the last call's
  * contents. Calls that overlap on the GPU (other streams, other host threads)
  * race and must be serialised by the caller. No part of the array has to

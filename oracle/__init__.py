@@ -41,6 +41,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "csa2_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "_build", "libcsa2_oracle.so")
+_LIB_OMP_PATH = os.path.join(_HERE, "_build", "libcsa2_oracle_omp.so")
 
 # Constants the pages fix.
 POOL_BLOCKS = 2048      # candidate pool: 2,048 blocks ...
@@ -53,30 +54,53 @@ MX_GROUP = 32           # MXFP4 variant: one E8M0 scale per 32 channels
 FULL, REINDEX, REUSE = "full", "reindex", "reuse"
 
 
-def build(force: bool = False) -> str:
+def build(force: bool = False, openmp: bool = False) -> str:
     """Compile the oracle with gcc (plain -O2, no fast-math: IEEE fp32 division
     and conversion must be exact). Returns the path of the shared library.
-    CSA2_ORACLE_LIB names a library to load instead (the mutation tests build
-    copies of this source with one planted mistake each)."""
+    CSA2_ORACLE_LIB names a library to load instead of the plain build (the
+    mutation tests build copies of this source with one planted mistake each).
+    openmp=True builds the timing variant (-fopenmp): the same source, its
+    independent outer loops shared among threads, results identical."""
     override = os.environ.get("CSA2_ORACLE_LIB")
-    if override:
+    if override and not openmp:
         return override
-    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
-        os.makedirs(os.path.dirname(_LIB_PATH), exist_ok=True)
-        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    path = _LIB_OMP_PATH if openmp else _LIB_PATH
+    if force or not os.path.exists(path) or os.path.getmtime(path) < os.path.getmtime(_SRC):
+        os.makedirs(os.path.dirname(path), exist_ok=True)
+        tmp = path + f".tmp{os.getpid()}"
+        flags = ["-fopenmp"] if openmp else []
         subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off",
-                               "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB_PATH)
-    return _LIB_PATH
+                               *flags, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, path)
+    return path
 
 
 _lib = None
+_use_openmp = False
+
+
+def use_openmp(on: bool = True) -> int:
+    """Route every oracle call through the OpenMP timing build (on=True) or the
+    plain build. Returns the number of threads the loaded build uses."""
+    global _lib, _use_openmp
+    if on != _use_openmp:
+        _use_openmp = on
+        _lib = None
+    return num_threads()
+
+
+def num_threads() -> int:
+    """Threads the loaded oracle build shares its outer loops among (1 for the
+    plain build)."""
+    return int(_L().orc_num_threads())
 
 
 def _L():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
+        lib = ctypes.CDLL(build(openmp=_use_openmp))
+        lib.orc_num_threads.restype = ctypes.c_int
+        lib.orc_num_threads.argtypes = []
         c_i64, c_int, c_dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_double
         P = ctypes.c_void_p
         lib.orc_e4m3_value.restype = c_dbl

@@ -41,6 +41,23 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* The library is built twice: plain (what every test loads) and with
+ * -fopenmp, a timing build for the CPU baseline in which the independent
+ * outer loops (rows, tokens, heads) are shared among threads. The pragmas
+ * change no arithmetic: every output element is computed by one thread in
+ * the same order as in the plain build. */
+int orc_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
 
 /* ------------------------------------------------------------------ */
 /* bf16: the upper 16 bits of an IEEE binary32.                        */
@@ -154,6 +171,7 @@ void orc_e2m1_encode_n(const float *v, int64_t n, uint8_t *out)
 /* ------------------------------------------------------------------ */
 void orc_fp4_quantize(const uint16_t *x, int64_t rows, int C, uint8_t *packed, uint8_t *sf)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; r++) {
         const uint16_t *xr = x + r * C;
         for (int g = 0; g < C / 16; g++) {
@@ -286,6 +304,7 @@ void orc_mxfp4_dequantize(const uint8_t *packed, const uint8_t *sf, int64_t rows
 /* ------------------------------------------------------------------ */
 void orc_index_dots(const int8_t *q, const int8_t *k, int64_t n, int HD, int64_t *S)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < n; t++) {
         int64_t acc = 0;
         for (int i = 0; i < HD; i++)
@@ -298,16 +317,20 @@ void orc_index_dots(const int8_t *q, const int8_t *k, int64_t n, int HD, int64_t
 int orc_index_scores(const int8_t *q, const int8_t *k, const float *kscale, int64_t n, int HD,
                      float *score)
 {
+    int out_of_range = 0;
+#pragma omp parallel for schedule(static) reduction(|| : out_of_range)
     for (int64_t t = 0; t < n; t++) {
         int64_t acc = 0;
         for (int i = 0; i < HD; i++)
             acc += (int64_t)q[i] * (int64_t)k[t * HD + i];
-        if (acc > INT32_MAX || acc < INT32_MIN)
-            return -1;
+        if (acc > INT32_MAX || acc < INT32_MIN) {
+            out_of_range = 1;
+            continue;
+        }
         float s = (float)acc; /* round to nearest even */
         score[t] = s * kscale[t];
     }
-    return 0;
+    return out_of_range ? -1 : 0;
 }
 
 /* Block score: max over the visible tokens of each 8-token block.
@@ -382,8 +405,9 @@ int64_t orc_topk(const float *score, const int64_t *pos, int64_t n, int64_t k, i
 void orc_attention(const uint16_t *q, int Hq, int C, const double *kv, int64_t n, double scale,
                    double *out)
 {
-    double *logit = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+#pragma omp parallel for schedule(dynamic, 1)
     for (int h = 0; h < Hq; h++) {
+        double *logit = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
         double mx = -INFINITY;
         for (int64_t j = 0; j < n; j++) {
             double dot = 0.0;
@@ -404,6 +428,6 @@ void orc_attention(const uint16_t *q, int Hq, int C, const double *kv, int64_t n
                 acc += logit[j] * kv[j * C + c];
             out[h * C + c] = acc / z;
         }
+        free(logit);
     }
-    free(logit);
 }

@@ -515,13 +515,8 @@ bool attn_rows_supported(const AttnArgs &a) {
 }
 
 int launch_attn_rows(const AttnArgs &a, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(tr::attn_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tr::SMEM_BYTES) != cudaSuccess)
-            return CSA2_ERR_CUDA;
-        attr = true;
-    }
+    static PerDevice smem_set;
+    if (!set_smem_limit_once(smem_set, tr::attn_rows_kernel, tr::SMEM_BYTES)) return CSA2_ERR_CUDA;
     const int64_t rows = (int64_t)a.B * a.Nq;
     const int nwin = a.n_win < a.swa_rows ? a.n_win : a.swa_rows;
     const bool has_win = nwin > 0 && a.swa != nullptr;

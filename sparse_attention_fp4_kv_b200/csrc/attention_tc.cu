@@ -555,8 +555,9 @@ bool attn_tc_supported(const AttnArgs &a) {
 // persistent loop then runs in one wave); MAX_CLUSTERS if the query fails.
 template <int HPC>
 int tc_max_active_clusters() {
-    static int n = 0;
-    if (n == 0) {
+    static PerDevice cache;
+    return cache.get([] {
+        int n = 0;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(tc::CL, tc::MAX_CLUSTERS, 1);
         cfg.blockDim = dim3(tc::THREADS, 1, 1);
@@ -576,20 +577,15 @@ int tc_max_active_clusters() {
         else
             n = tc::MAX_CLUSTERS;
         (void)cudaGetLastError();
-    }
-    return n;
+        return n;
+    });
 }
 
 template <int HPC>
 static int launch_tc(const AttnArgs &a, cudaStream_t s) {
     using L = tc::Cfg<HPC>;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(tc::attn_tc_kernel<HPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 L::SMEM_BYTES) != cudaSuccess)
-            return CSA2_ERR_CUDA;
-        attr = true;
-    }
+    static PerDevice smem_set;
+    if (!set_smem_limit_once(smem_set, tc::attn_tc_kernel<HPC>, L::SMEM_BYTES)) return CSA2_ERR_CUDA;
     const int64_t rows = (int64_t)a.B * a.Nq;
     const int64_t items = rows * L::HG;
     CUtensorMap tq, tswa;

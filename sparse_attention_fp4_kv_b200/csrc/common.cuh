@@ -4,6 +4,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "csa2.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
@@ -21,6 +24,49 @@ inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_
 
 inline int launch_status() {
     return cudaGetLastError() == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- per-device set-up
+// Function attributes (the dynamic shared-memory limit, the carveout) and
+// occupancy figures belong to one device. Launchers keep their one-time set-up
+// in a PerDevice table indexed by the current device ordinal, so a process that
+// drives several GPUs sets each one up once, and host threads may race to the
+// first call safely.
+constexpr int kMaxDevices = 64;
+
+class PerDevice {
+  public:
+    // The value for the current device; fn() computes it the first time and
+    // returns a value >= 0, or < 0 on failure (then nothing is cached and the
+    // next call tries again). Devices past kMaxDevices are never cached.
+    template <class F>
+    int get(F &&fn) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return fn();
+        int v = value_[dev].load(std::memory_order_acquire);
+        if (v > 0) return v - 1;
+        std::lock_guard<std::mutex> lock(mutex_);
+        v = value_[dev].load(std::memory_order_relaxed);
+        if (v > 0) return v - 1;
+        const int r = fn();
+        if (r >= 0) value_[dev].store(r + 1, std::memory_order_release);
+        return r;
+    }
+
+  private:
+    std::mutex mutex_;
+    std::atomic<int> value_[kMaxDevices] = {};  // value + 1; 0 = not yet computed
+};
+
+// Sets the dynamic shared-memory limit of `kernel` on the current device once.
+template <typename K>
+inline bool set_smem_limit_once(PerDevice &done, K kernel, size_t bytes) {
+    return done.get([&] {
+        return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) ==
+                       cudaSuccess
+                   ? 1
+                   : -1;
+    }) >= 0;
 }
 
 // ---------------------------------------------------------------- dependent launches
@@ -74,29 +120,30 @@ int attn_tc_wait_flag(bool clear);
 int attn_rows_wait_flag(bool clear);
 int index_mma_wait_flag(bool clear);
 
+// Streaming multiprocessors of the current device (148 on B200 if the query fails).
 inline int num_sms() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
+    static PerDevice cache;
+    return cache.get([] {
+        int dev = 0, n = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        return n;
+    });
 }
 
 // ---------------------------------------------------------------- bf16 / fp8 / fp4
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// E4M3 code -> fp32 from the format definition (1 sign, 4 exponent bits with
-// bias 7, 3 mantissa bits; exponent field 0 is subnormal m * 2^-9). Exact.
 // Prefetch of a contiguous global range into L2 (16-byte aligned, size a
 // multiple of 16); no data reaches the issuing CTA.
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// E4M3 code -> fp32 from the format definition (1 sign, 4 exponent bits with
+// bias 7, 3 mantissa bits; exponent field 0 is subnormal m * 2^-9). Exact.
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
     uint32_t e = (code >> 3) & 0xF, m = code & 7;
     float mag = (e == 0) ? (float)m * 0.001953125f                     // m * 2^-9
@@ -114,7 +161,6 @@ __device__ __forceinline__ float e2m1_to_f32(uint32_t c4) {
     return (c4 & 8) ? -v : v;
 }
 
-// fp32 -> E4M3 with round-to-nearest-even and saturation to +-448 (PTX cvt).
 // E8M0 scale (MXFP4 variant): code e is 2^(e - 127), 255 is NaN; code 0 is the
 // fp32 subnormal 2^-127.
 __device__ __forceinline__ float e8m0_to_f32(uint32_t code) {

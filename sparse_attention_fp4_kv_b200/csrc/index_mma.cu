@@ -399,13 +399,8 @@ int launch_index_mma(const int8_t *q, const int8_t *k, const float *kscale, cons
     if (!make_tmap_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, HD, (uint64_t)B * Nq, HD, BK, BM) ||
         !make_tmap_2d(&mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, k, HD, (uint64_t)B * cap, HD, BK, BN))
         return CSA2_ERR_CUDA;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(index_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 SMEM_BYTES) != cudaSuccess)
-            return CSA2_ERR_CUDA;
-        attr = true;
-    }
+    static PerDevice smem_set;
+    if (!set_smem_limit_once(smem_set, index_mma_kernel, SMEM_BYTES)) return CSA2_ERR_CUDA;
     Args a;
     a.kscale = kscale;
     a.ctx_len = ctx_len;

@@ -99,8 +99,9 @@ __global__ void __launch_bounds__(256) kv_append_mxfp4_kernel(
     const int E = (int)((__float_as_uint(amax) >> 23) & 0xFF);  // 0 for zero / subnormal
     int e = E == 0 ? -127 : E - 129;
     e = e < -127 ? -127 : e;
-    // 2^-e as an fp32 (2^-127 .. 2^127; -e = -127 is the subnormal 2^-127)
-    const float inv = -e >= -126 ? __uint_as_float((uint32_t)(127 - e) << 23) : __uint_as_float(0x00400000u);
+    // 2^-e as an fp32: e lies in [-127, 126], so 2^-e is a normal number
+    // (2^-126 .. 2^127)
+    const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
     float v[32];
 #pragma unroll
     for (int j = 0; j < 32; j++) v[j] = x[j] * inv;

@@ -13,7 +13,9 @@
 //
 // The host needs the array's device address. The first call on each device,
 // with that device current, looks it up once with cudaGetSymbolAddress and
-// caches it. Make that first call before any stream capture. Every call shares
+// caches it for the life of the process (a cudaDeviceReset destroys the context
+// the cached address belongs to; the entry point must not be called on that
+// device afterwards). Make that first call before any stream capture. Every call shares
 // the one array: calls that overlap on the GPU (different streams, or
 // concurrent host threads on the same device) race on it. Nothing in it has to
 // start at zero: each call writes every scratch byte it reads before reading it.

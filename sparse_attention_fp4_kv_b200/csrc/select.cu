@@ -313,19 +313,20 @@ int launch_full_select(const float *blk, const int32_t *n_blk, const float *tok,
     if (rows == 0) return CSA2_OK;
     if (rows > INT32_MAX) return CSA2_ERR_SHAPE;
     const size_t smem = full_select_smem(cap, P, K);
-    static bool attr = false;
-    if (!attr) {
-        // two CTAs per SM: dynamic shared memory up to the largest row, and the
-        // largest shared-memory carveout
-        if (cudaFuncSetAttribute(full_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)full_select_smem(8 * (int64_t)FS_MAXN, kPoolBlocks,
-                                                       kPoolBlocks)) != cudaSuccess ||
-            cudaFuncSetAttribute(full_select_kernel,
-                                 cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
-            return CSA2_ERR_CUDA;
-        attr = true;
-    }
+    static PerDevice attrs_set;
+    // two CTAs per SM: dynamic shared memory up to the largest row, and the
+    // largest shared-memory carveout
+    if (attrs_set.get([] {
+            return cudaFuncSetAttribute(full_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)full_select_smem(8 * (int64_t)FS_MAXN, kPoolBlocks,
+                                                              kPoolBlocks)) == cudaSuccess &&
+                           cudaFuncSetAttribute(full_select_kernel,
+                                                cudaFuncAttributePreferredSharedMemoryCarveout,
+                                                (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess
+                       ? 1
+                       : -1;
+        }) < 0)
+        return CSA2_ERR_CUDA;
     return launch_kernel(pdl, full_select_kernel, dim3((unsigned)rows), dim3(FS_THREADS), smem, s,
                          blk, n_blk, tok, ctx_len, q_pos, B, Nq, cap, P, K, pool, top);
 }

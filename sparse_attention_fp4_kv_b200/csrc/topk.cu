@@ -682,17 +682,11 @@ int launch_topk_from_hist(const float *score, const int32_t *cand_pos, const int
                           int R, int64_t n, int k, int32_t *out, void *ws, cudaStream_t s) {
     if (R == 0) return CSA2_OK;
     if (R > 65535) return CSA2_ERR_SHAPE;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)TK_SMEM) != cudaSuccess ||
-            cudaFuncSetAttribute(topk_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)TK_SMEM) != cudaSuccess ||
-            cudaFuncSetAttribute(topk_row_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)TK_SMEM) != cudaSuccess)
-            return CSA2_ERR_CUDA;
-        attr = true;
-    }
+    static PerDevice smem_set[3];
+    if (!set_smem_limit_once(smem_set[0], topk_kernel, TK_SMEM) ||
+        !set_smem_limit_once(smem_set[1], topk_finish_kernel, TK_SMEM) ||
+        !set_smem_limit_once(smem_set[2], topk_row_hist_kernel, TK_SMEM))
+        return CSA2_ERR_CUDA;
     TopkArgs a{score, cand_pos, n_valid, R, n, k, out};
     TopkHistWs w = topk_hist_ws(ws, R, k);
     if (n <= TS_MAX_N)
@@ -721,13 +715,8 @@ extern "C" int csa2_topk(const float *score, const int32_t *cand_pos, const int3
     if (!score || !out) return CSA2_ERR_NULL;
     if (R < 0 || n < 1 || n >= ((int64_t)1 << 31) || k < 1 || k > TK_MAXK) return CSA2_ERR_SHAPE;
     if (R == 0) return CSA2_OK;
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)TK_SMEM) != cudaSuccess)
-            return CSA2_ERR_CUDA;
-        attr_set = true;
-    }
+    static PerDevice smem_set;
+    if (!set_smem_limit_once(smem_set, topk_kernel, TK_SMEM)) return CSA2_ERR_CUDA;
     TopkArgs a{score, cand_pos, n_valid, R, n, k, out};
     topk_kernel<<<R, TK_THREADS, TK_SMEM, (cudaStream_t)stream>>>(a);
     return launch_status();

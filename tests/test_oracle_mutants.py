@@ -104,7 +104,8 @@ C_MUTANTS = [
     ("mx dequantize takes the wrong block's scale", "double s = orc_e8m0_value(sf[r * (C / 32) + c / 32]);",
      "double s = orc_e8m0_value(sf[r * (C / 32) + c / 64]);", 1, ["formats"]),
     ("index score overflow not rejected",
-     "        if (acc > INT32_MAX || acc < INT32_MIN)\n            return -1;\n", "", 1, ["selection"]),
+     "        if (acc > INT32_MAX || acc < INT32_MIN) {\n            out_of_range = 1;\n            continue;\n        }\n",
+     "", 1, ["selection"]),
     ("block max ignores the first token", "        float m = score[8 * j];",
      "        float m = score[8 * j + 1 < n_visible ? 8 * j + 1 : 8 * j];", 1, ["selection"]),
     ("selection padded with 0", "        out[i] = -1;", "        out[i] = 0;", 1, ["selection"]),

@@ -94,3 +94,28 @@ def test_clock_summary_of_sampled_lines():
     cs.proc = _Proc()
     name = cs.file.name
     assert cs.stop() == c and not os.path.exists(name)
+
+
+def test_reference_arm_runs_on_host_inputs_without_the_cuda_library():
+    """bench.py --impl reference draws its inputs with the seeded generators on
+    the host and runs only the oracle: libcsa2 is never imported or loaded."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import sys, json; sys.argv = ['bench.py', '--impl', 'reference', '--workload', "
+            "'full_b1_ctx4k', '--steps', '3', '--warmup', '3']; sys.path.insert(0, %r); import bench; "
+            "bench.main(); maps = open('/proc/self/maps').read(); "
+            "print(json.dumps({'binding': 'sparse_attention_fp4_kv_b200.binding' in sys.modules, "
+            "'libcsa2': 'libcsa2.so' in maps, 'omp': 'libcsa2_oracle_omp.so' in maps}))" % root)
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    line, loaded = lines[0], lines[-1]
+    assert loaded == {"binding": False, "libcsa2": False, "omp": True}
+    assert line["impl"] == "reference" and line["steps"] == 3 and line["warmup"] == 3
+    assert line["config"]["workload"] == "full_b1_ctx4k" and line["unit"] == "layer-steps/s"
+    assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] > 0
+    # a 4K-context step is short enough that every step covers the whole batch
+    assert "1 of 1 sequences per step" in line["cpu_baseline"]["sample"]

@@ -66,13 +66,14 @@ def test_noalloc_matches_regular_entry_point(name, kw):
 
 def test_noalloc_rejects_problems_beyond_the_scratch_limit():
     from sparse_attention_fp4_kv_b200 import binding as B
-    P = ctypes.c_void_p
-    good = P(4096)
-    layers = (B.csa2_layer * 1)(B.csa2_layer(B.MODE_FULL, good, good, good, good, good))
+    # every device pointer is NULL: the size check comes first and returns
+    # CSA2_ERR_WORKSPACE; were it ever to run later, the NULL checks would stop
+    # the call on the host (CSA2_ERR_NULL) before any kernel could launch
+    layers = (B.csa2_layer * 1)(B.csa2_layer(B.MODE_FULL, None, None, None, None, None))
     B_, cap = 8, 1 << 20                       # needs ~38 MB of scratch
     need = B.lib.csa2_decode_stack_workspace_size(B_, 64, 512, 16, 128, cap)
     assert need > (24 << 20)
-    st = B.lib.csa2_decode_stack_noalloc(layers, 1, None, good, good, good, good, cap, good, good,
-                                         128, B_, 64, 512, 16, 128, ctypes.c_float(0.04), good, 0,
+    st = B.lib.csa2_decode_stack_noalloc(layers, 1, None, None, None, None, None, cap, None, None,
+                                         128, B_, 64, 512, 16, 128, ctypes.c_float(0.04), None, 0,
                                          None)
     assert st == -5 and B.status_string(st) == "workspace missing or too small"

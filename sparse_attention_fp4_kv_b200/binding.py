@@ -26,6 +26,12 @@ TOPK_SHORT_ROW = 65536
 # csa2_full_select holds a row of block scores (and of pooled token scores) in
 # shared memory: at most this many of each.
 FULL_SELECT_MAX = 16384
+# The decode stack launches the attention of a layer group (a Full or Reindex
+# layer and the Reuse layers after it, up to ATTN_GROUP_MAX layers) as one
+# kernel when the tensor-core cluster kernel takes the shape (512 channels, 64
+# heads, fewer than ATTN_ROWS_MIN query rows); otherwise one kernel per layer.
+ATTN_GROUP_MAX = 8
+ATTN_ROWS_MIN = 64
 MODE_FULL, MODE_REINDEX, MODE_REUSE = 0, 1, 2
 
 

@@ -39,9 +39,11 @@ struct StackWs {
     int32_t *n_blk;
     float *pscore;
     int32_t *ppos;
+    int *row_done;     // per-row layer counters of the grouped attention launches
     void *sel_blk;     // histogram-fed top-k workspace of the pool selection
     void *sel_tok;     // ... and of the token top-512
     size_t hist_bytes; // leading bytes of each that must be zero before a step
+    size_t zero_bytes; // bytes from row_done that must be zero (counters + sel_blk's histogram)
     void *attn;
     size_t attn_bytes;
     size_t total;
@@ -63,11 +65,14 @@ StackWs stack_layout(void *base, int B, int Hq, int C, int64_t cap) {
     off += up(sizeof(float) * (size_t)B * P8);
     w.ppos = reinterpret_cast<int32_t *>(p + off);
     off += up(sizeof(int32_t) * (size_t)B * P8);
+    w.row_done = reinterpret_cast<int *>(p + off);
+    off += up(sizeof(int) * (size_t)B);
     w.sel_blk = p + off;
     off += up(topk_hist_ws_bytes(B, kPoolBlocks));
     w.sel_tok = p + off;
     off += up(topk_hist_ws_bytes(B, kTopK));
     w.hist_bytes = up((size_t)B * kHistBins * 4) + up((size_t)B * 2 * 4);
+    w.zero_bytes = up(sizeof(int) * (size_t)B) + w.hist_bytes;
     w.attn = p + off;
     w.attn_bytes = up(attn_workspace_bytes(B, 1, Hq, C, kTopK, CSA2_N_WIN));
     off += w.attn_bytes;
@@ -128,14 +133,16 @@ extern "C" int csa2_decode_stack(const csa2_layer *layers, int n_layers,
                               kv_sf, s, true);
         if (st) return st;
     }
-    // the selection histograms and counters start the step at zero (every
-    // finishing top-k kernel leaves its rows clear for the next producer)
-    if (cudaMemsetAsync(w.sel_blk, 0, w.hist_bytes, s) != cudaSuccess ||
+    // the selection histograms and counters and the attention layer counters
+    // start the step at zero (every finishing top-k kernel leaves its rows
+    // clear for the next producer)
+    if (cudaMemsetAsync(w.row_done, 0, w.zero_bytes, s) != cudaSuccess ||
         cudaMemsetAsync(w.sel_tok, 0, w.hist_bytes, s) != cudaSuccess)
         return CSA2_ERR_CUDA;
     uint32_t *hist_blk = topk_hist_ptr_of(w.sel_blk);
     uint32_t *hist_tok = topk_hist_ptr_of(w.sel_tok);
-    for (int l = 0; l < n_layers; l++) {
+    int row_base = 0;  // value of every per-row layer counter before the next group
+    for (int l = 0; l < n_layers;) {
         const csa2_layer &L = layers[l];
         if (L.mode == CSA2_MODE_FULL) {
             const bool timed = scan_events && !scan_timed;
@@ -166,16 +173,49 @@ extern "C" int csa2_decode_stack(const csa2_layer *layers, int n_layers,
             if (st) return st;
             cur = L.topk;
         }
-        // Every kernel of the step is launched with programmatic stream
-        // serialization. A Reuse layer's attention follows the previous layer's
-        // attention, and its indices come from an earlier selection kernel, so
-        // it gathers and dequantizes its rows before waiting for that kernel;
-        // Q and the window rows (the layer's own inputs) are read after the wait.
+        // The attention group: this layer and the Reuse layers after it, which
+        // attend the same selected rows. Every kernel of the step is launched
+        // with programmatic stream serialization.
+        int g = 1;
+        while (l + g < n_layers && g < attn_group_max_layers() &&
+               layers[l + g].mode == CSA2_MODE_REUSE)
+            g++;
+        // A launch led by a Reuse layer (a run of Reuse layers longer than one
+        // launch takes, or layers launched one by one) follows an attention
+        // launch, and its indices come from an earlier selection kernel, so it
+        // gathers and dequantizes its rows before waiting; Q and the window rows
+        // (the layers' own inputs) are read after the wait.
         AttnArgs aa{L.q, kv_fp4, kv_sf, cap, cur, kTopK, L.swa, swa_pos0, swa_rows, nullptr,
                     CSA2_N_WIN, B, 1, Hq, C, softmax_scale, L.out, w.attn, true,
                     L.mode == CSA2_MODE_REUSE};
-        st = attn_checked_launch(aa, w.attn_bytes, s);
+        st = attn_checked_launch(aa, w.attn_bytes, s, /*validate_only=*/true);
         if (st) return st;
+        if (attn_tc_supported(aa) && (int64_t)B < kAttnRowsMin) {
+            // one launch for the group; layer i + 1 of a sequence follows layer i
+            // of that sequence through the per-row counters
+            const void *gq[kMaxGroupLayers], *gswa[kMaxGroupLayers];
+            float *gout[kMaxGroupLayers];
+            for (int i = 0; i < g; i++) {
+                gq[i] = layers[l + i].q;
+                gswa[i] = layers[l + i].swa;
+                gout[i] = layers[l + i].out;
+            }
+            int adds = 0;
+            st = launch_attn_tc_group(aa, gq, gswa, gout, g, w.row_done, row_base, &adds, s);
+            if (st) return st;
+            row_base += adds;
+        } else {
+            for (int i = 0; i < g; i++) {
+                const csa2_layer &Li = layers[l + i];
+                aa.q = Li.q;
+                aa.swa = Li.swa;
+                aa.out = Li.out;
+                aa.prefetch = i > 0 || L.mode == CSA2_MODE_REUSE;
+                st = attn_checked_launch(aa, w.attn_bytes, s);
+                if (st) return st;
+            }
+        }
+        l += g;
     }
     return CSA2_OK;
 }

@@ -163,7 +163,7 @@ extern "C" int csa2_sparse_attn_decode_mxfp4(const void *q_bf16, const uint8_t *
 
 namespace csa2 {
 
-int attn_checked_launch(const AttnArgs &a, size_t ws_bytes, cudaStream_t s) {
+int attn_checked_launch(const AttnArgs &a, size_t ws_bytes, cudaStream_t s, bool validate_only) {
     if (!a.q || !a.kv_fp4 || !a.kv_sf || !a.out) return CSA2_ERR_NULL;
     if (a.K > 0 && !a.topk) return CSA2_ERR_NULL;
     if (a.n_win > 0 && a.swa_rows > 0 && (!a.swa || !a.swa_pos0)) return CSA2_ERR_NULL;
@@ -175,7 +175,7 @@ int attn_checked_launch(const AttnArgs &a, size_t ws_bytes, cudaStream_t s) {
         return CSA2_ERR_ALIGN;
     if (ws_bytes < attn_workspace_bytes(a.B, a.Nq, a.Hq, a.C, a.K, a.n_win))
         return CSA2_ERR_WORKSPACE;
-    if ((int64_t)a.B * a.Nq == 0) return CSA2_OK;
+    if ((int64_t)a.B * a.Nq == 0 || validate_only) return CSA2_OK;
     return launch_attn(a, s);
 }
 

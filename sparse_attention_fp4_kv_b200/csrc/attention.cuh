@@ -61,12 +61,26 @@ __device__ __forceinline__ AttnWindow attn_window(const AttnArgs &a, int b, int6
 size_t attn_workspace_bytes(int B, int Nq, int Hq, int C, int K, int n_win);
 // Validates the arguments of a sparse-attention call (status codes of
 // csa2_sparse_attn_decode) and launches it.
-int attn_checked_launch(const AttnArgs &a, size_t ws_bytes, cudaStream_t s);
+// With validate_only, only the checks run (CSA2_OK when the call would launch).
+int attn_checked_launch(const AttnArgs &a, size_t ws_bytes, cudaStream_t s,
+                        bool validate_only = false);
 int launch_attn(const AttnArgs &a, cudaStream_t s);
 int launch_attn_general(const AttnArgs &a, cudaStream_t s);
 bool attn_tc_supported(const AttnArgs &a);
 size_t attn_tc_workspace_bytes(int B, int Nq);
 int launch_attn_tc(const AttnArgs &a, cudaStream_t s);
+// The tensor-core kernel over a group of n layers that share a's selected rows
+// (layer i: Q q[i], window rows swa[i], output out[i]; a.q / a.swa / a.out are
+// ignored). Layer i + 1 of a query row runs once layer i of that row is
+// written: row_done holds one counter per query row (B Nq ints, each equal to
+// row_base at launch; used when n > 1) and *adds receives how much the launch
+// adds to each.
+int launch_attn_tc_group(const AttnArgs &a, const void *const *q, const void *const *swa,
+                         float *const *out, int n, int *row_done, int row_base, int *adds,
+                         cudaStream_t s);
+// Most layers one group launch takes (kMaxGroupLayers).
+int attn_group_max_layers();
+constexpr int kMaxGroupLayers = 8;
 // One CTA per query row (attention_rows.cu): no workspace; for calls of
 // kAttnRowsMin rows or more (below that the split-key clusters measured
 // faster: at 32 rows and fewer, the decode batches).

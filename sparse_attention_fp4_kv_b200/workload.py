@@ -141,18 +141,29 @@ class DecodeWorkload:
     def launches_per_step(self) -> int:
         """libcsa2 kernels one step launches: the append, then per Full layer
         the scan, the pool selection, the gather and the token selection; per
-        Reindex layer the rescoring and the token selection; one attention
-        kernel per layer. A selection is one kernel for rows of at most
-        TOPK_SHORT_ROW candidates, else two (compaction + finish). (The
-        per-step histogram clear is a memset, not counted.)"""
+        Reindex layer the rescoring and the token selection. Attention: one
+        kernel per layer group (a Full or Reindex layer and the Reuse layers
+        after it, at most ATTN_GROUP_MAX layers per kernel) where the
+        tensor-core cluster kernel takes the shape, else one per layer. A
+        selection is one kernel for rows of at most TOPK_SHORT_ROW candidates,
+        else two (compaction + finish). (The per-step clear of the histograms
+        and counters is a memset, not counted.)"""
         def sel(n):
             return 1 if n <= csa2.TOPK_SHORT_ROW else 2
+        w = self.w
         nblk = (self.kv_fp4.shape[1] + 7) // 8
         pooled = csa2.POOL_BLOCKS * csa2.BLOCK_TOKENS
+        grouped = w.C == 512 and w.Hq == 64 and w.B < csa2.ATTN_ROWS_MIN
         n = 1
+        run = 0  # layers in the current attention launch
         for m in self.modes:
             n += {synth.FULL: 2 + sel(nblk) + sel(pooled), synth.REINDEX: 1 + sel(pooled),
-                  synth.REUSE: 0}[m] + 1
+                  synth.REUSE: 0}[m]
+            if grouped and m == synth.REUSE and 0 < run < csa2.ATTN_GROUP_MAX:
+                run += 1
+            else:
+                n += 1
+                run = 1
         return n
 
     # ---- algorithmic bytes of one step (what the method must move)

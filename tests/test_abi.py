@@ -124,27 +124,17 @@ def _attn_slot_bytes(hpc):
     return (8 * hpc * 512 + 2 * 8 * hpc) * 4
 
 
-def _attn_heads_per_cta(rows, pdl, prefetch):
-    # the launcher's head split: 16 or 32 of the 64 heads per cluster while the
-    # (row, head group) items fit the resident clusters (a dependent launch
-    # leaves room for the next layer's clusters), else all 64
-    if not pdl:
-        return 16 if rows <= 2 else 32 if rows <= 7 else 64
-    lim = 7 if prefetch else 8
-    return 16 if 4 * rows <= lim else 32 if 2 * rows <= lim else 64
-
-
 def test_attention_workspace_covers_every_head_split(lib):
+    """The launcher splits the 64 heads into clusters of 16, 32 or 64 (one
+    layer at a time, or a whole layer group per launch, at most 18 clusters);
+    the workspace holds the exchange slots of the largest of those splits."""
     ws = lib.csa2_sparse_attn_workspace_size
     ws.restype = ctypes.c_size_t
     ws.argtypes = [ctypes.c_int] * 6
     for B, Nq in [(1, 1), (2, 1), (3, 1), (4, 1), (5, 1), (7, 1), (8, 1), (9, 1), (16, 1), (4, 4),
                   (63, 1), (64, 1)]:
         rows = B * Nq
-        need = []
-        for pdl, prefetch in [(False, False), (True, False), (True, True)]:
-            hpc = _attn_heads_per_cta(rows, pdl, prefetch)
-            need.append(min(rows * (64 // hpc), 18) * _attn_slot_bytes(hpc))
+        need = [min(rows * (64 // hpc), 18) * _attn_slot_bytes(hpc) for hpc in (16, 32, 64)]
         got = ws(B, Nq, 64, 512, 512, 128)
         assert got == max(need), (B, Nq, got, need)
     # the tensor-core kernels need no workspace outside their shape, nor does the general kernel

@@ -88,6 +88,16 @@ def test_scaled_stack(name, kw):
     _free()
 
 
+def test_stack_reuse_run_longer_than_one_attention_launch():
+    """A Full layer followed by 10 Reuse layers: the attention of the first 8
+    layers runs as one launch and the last 3 as a second launch led by a Reuse
+    layer (it gathers its rows before its dependency wait)."""
+    wl = _workload("decoder_stack20_b4_ctx1m", B=3, ctx=9001, modes=[synth.FULL] + [synth.REUSE] * 10)
+    _check(wl, range(wl.w.B))
+    del wl
+    _free()
+
+
 @pytest.mark.parametrize("levels", [1, 3])
 def test_stack_tie_heavy_keys(levels):
     """Coarse indexer keys give many equal scores: with levels=1 every score is

@@ -8,126 +8,200 @@
 // as E2M1 codes with one E4M3 scale per 16 channels; dequantization
 // e2m1 * e4m3 is exact in fp32.
 //
-// General kernel: one CTA per (query, head). Warps compute one logit per key
-// (lane = C/32 channels, dequantized in registers, fp32 dot, shuffle reduce),
-// the CTA does the softmax in shared memory, and each thread then accumulates
-// its channels over all keys. Used for shapes outside the tensor-core
-// kernel's constraints (attention_tc.cu).
-#include <cfloat>
-
+// General kernel: one CTA per (query, head), 8 warps. Lane l of a warp holds
+// channel pairs l, l + 32, ... (pair i = channels 2i, 2i + 1 = one FP4 byte).
+//  1. The query's selected positions go to shared memory.
+//  2. Logits: warp w takes keys w, w + 8, ..., GEN_U keys per round with all
+//     their loads issued before the first use; fp32 dot, shuffle reduce.
+//  3. Softmax statistics over the logits in shared memory.
+//  4. P V: warp w accumulates p_j row_j over the same keys in registers (the
+//     lane's channels), GEN_U keys per round; the 8 warps' sums are added in
+//     shared memory.
+// Used for shapes outside the tensor-core kernels' constraints (other channel
+// and head counts, e.g. 8 heads of 128 channels).
 #include "attention.cuh"
 
 namespace csa2 {
 
-__global__ void __launch_bounds__(256) attn_general_kernel(AttnArgs a) {
+constexpr int GEN_THREADS = 256;
+constexpr int GEN_WARPS = GEN_THREADS / 32;
+constexpr int GEN_U = 4;  // keys per warp per round
+
+// Key j of query bq (j < K: selected row, else window row j - K) as NP channel
+// pairs per lane, dequantized; valid = false for an empty selected slot.
+template <int NP>
+__device__ __forceinline__ void gen_load_key(const AttnArgs &a, int b, const int32_t *sel,
+                                             const AttnWindow &w, int j, int lane, float2 (&v)[NP],
+                                             bool &valid) {
+    const int C = a.C, npairs = C / 2;
+    if (j < a.K) {
+        const int32_t pos = sel[j];
+        valid = pos >= 0 && pos < a.cap;
+        const int64_t cell = (int64_t)b * a.cap + (valid ? pos : 0);
+        const uint8_t *row = a.kv_fp4 + cell * (C / 2);
+        const uint8_t *sfr = a.kv_sf + cell * (C / (a.mx ? 32 : 16));
+        uint32_t byte[NP];
+        float sc[NP];
+#pragma unroll
+        for (int i = 0; i < NP; i++) {
+            const int p = lane + 32 * i;
+            byte[i] = p < npairs ? __ldg(row + p) : 0u;
+            sc[i] = p < npairs ? kv_group_scale(sfr, p >> 3, a.mx) : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < NP; i++)
+            v[i] = valid ? make_float2(e2m1_to_f32(byte[i] & 0xF) * sc[i], e2m1_to_f32(byte[i] >> 4) * sc[i])
+                         : make_float2(0.0f, 0.0f);
+    } else {
+        valid = true;
+        const uint32_t *row = reinterpret_cast<const uint32_t *>(a.swa) +
+                              ((int64_t)b * a.swa_rows + w.row0 + (j - a.K)) * (C / 2);
+#pragma unroll
+        for (int i = 0; i < NP; i++) {
+            const int p = lane + 32 * i;
+            const uint32_t u = p < npairs ? __ldg(row + p) : 0u;
+            v[i] = make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+        }
+    }
+}
+
+template <int NP>
+__global__ void __launch_bounds__(GEN_THREADS) attn_general_kernel(AttnArgs a) {
     grid_dep_wait();
     grid_dep_launch();
     extern __shared__ float sm[];
-    const int C = a.C;
-    float *qs = sm;            // [C]
-    float *lg = sm + C;        // [K + n_win]
-    __shared__ float red[32];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarp = blockDim.x >> 5;
+    const int C = a.C, npairs = C / 2;
+    float *lg = sm;                                    // [K + n_win] logits, then p
+    float *red = sm + a.K + a.n_win;                   // [GEN_WARPS][C] partial sums
+    int32_t *sel = reinterpret_cast<int32_t *>(red + GEN_WARPS * C);  // [K]
+    __shared__ float wred[GEN_WARPS];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t bq = blockIdx.x / a.Hq;
     const int h = (int)(blockIdx.x % a.Hq);
     const int b = (int)(bq / a.Nq);
-
-    AttnWindow w = attn_window(a, b, bq);
+    const AttnWindow w = attn_window(a, b, bq);
     const int nkeys = a.K + w.n;
+    for (int j = tid; j < a.K; j += GEN_THREADS) sel[j] = a.topk[bq * a.K + j];
 
-    const uint16_t *q = reinterpret_cast<const uint16_t *>(a.q) + (bq * a.Hq + h) * (int64_t)C;
-    for (int c = tid; c < C; c += blockDim.x) qs[c] = __uint_as_float((uint32_t)q[c] << 16);
-    __syncthreads();
-
-    const int CPL = C / 32;  // channels per lane
-    for (int j = warp; j < nkeys; j += nwarp) {
-        float dot = 0.0f;
-        bool valid = true;
-        if (j < a.K) {
-            const int32_t pos = a.topk[bq * a.K + j];
-            valid = pos >= 0 && pos < a.cap;
-            if (valid) {
-                const int64_t cell = (int64_t)b * a.cap + pos;
-                const uint8_t *row = a.kv_fp4 + cell * (C / 2);
-                const uint8_t *sfr = a.kv_sf + cell * (C / (a.mx ? 32 : 16));
-                for (int u = 0; u < CPL; u += 2) {
-                    const int c = lane * CPL + u;
-                    const uint32_t byte = row[c / 2];
-                    const float s = kv_group_scale(sfr, c / 16, a.mx);
-                    dot += qs[c] * (e2m1_to_f32(byte & 0xF) * s);
-                    dot += qs[c + 1] * (e2m1_to_f32(byte >> 4) * s);
-                }
-            }
-        } else {
-            const uint16_t *row = reinterpret_cast<const uint16_t *>(a.swa) +
-                                  ((int64_t)b * a.swa_rows + w.row0 + (j - a.K)) * C;
-            for (int u = 0; u < CPL; u++) {
-                const int c = lane * CPL + u;
-                dot += qs[c] * __uint_as_float((uint32_t)row[c] << 16);
-            }
-        }
+    // this lane's query channels
+    const uint32_t *q = reinterpret_cast<const uint32_t *>(a.q) + (bq * a.Hq + h) * (int64_t)(C / 2);
+    float2 qv[NP];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        if (lane == 0) lg[j] = valid ? dot * a.scale : -INFINITY;
+    for (int i = 0; i < NP; i++) {
+        const int p = lane + 32 * i;
+        const uint32_t u = p < npairs ? __ldg(q + p) : 0u;
+        qv[i] = make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
     }
     __syncthreads();
 
-    // softmax statistics
+    // ---- logits
+    for (int j0 = warp * GEN_U; j0 < nkeys; j0 += GEN_WARPS * GEN_U) {
+        float2 v[GEN_U][NP];
+        bool valid[GEN_U];
+#pragma unroll
+        for (int u = 0; u < GEN_U; u++) {
+            valid[u] = false;
+            if (j0 + u < nkeys) gen_load_key<NP>(a, b, sel, w, j0 + u, lane, v[u], valid[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < GEN_U; u++) {
+            float dot = 0.0f;
+#pragma unroll
+            for (int i = 0; i < NP; i++) dot += qv[i].x * v[u][i].x + qv[i].y * v[u][i].y;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+            if (lane == 0 && j0 + u < nkeys) lg[j0 + u] = valid[u] ? dot * a.scale : -INFINITY;
+        }
+    }
+    __syncthreads();
+
+    // ---- softmax statistics
     float m = -INFINITY;
-    for (int j = tid; j < nkeys; j += blockDim.x) m = fmaxf(m, lg[j]);
+    for (int j = tid; j < nkeys; j += GEN_THREADS) m = fmaxf(m, lg[j]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) red[warp] = m;
+    if (lane == 0) wred[warp] = m;
     __syncthreads();
     m = -INFINITY;
-    for (int w2 = 0; w2 < nwarp; w2++) m = fmaxf(m, red[w2]);
+    for (int w2 = 0; w2 < GEN_WARPS; w2++) m = fmaxf(m, wred[w2]);
     __syncthreads();
     float z = 0.0f;
-    for (int j = tid; j < nkeys; j += blockDim.x) {
+    for (int j = tid; j < nkeys; j += GEN_THREADS) {
         const float p = (lg[j] == -INFINITY) ? 0.0f : expf(lg[j] - m);
         lg[j] = p;
         z += p;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    if (lane == 0) red[warp] = z;
+    if (lane == 0) wred[warp] = z;
     __syncthreads();
     z = 0.0f;
-    for (int w2 = 0; w2 < nwarp; w2++) z += red[w2];
+    for (int w2 = 0; w2 < GEN_WARPS; w2++) z += wred[w2];
     const float inv = z > 0.0f ? 1.0f / z : 0.0f;
 
+    // ---- P V over the same keys
+    float2 acc[NP];
+#pragma unroll
+    for (int i = 0; i < NP; i++) acc[i] = make_float2(0.0f, 0.0f);
+    for (int j0 = warp * GEN_U; j0 < nkeys; j0 += GEN_WARPS * GEN_U) {
+        float2 v[GEN_U][NP];
+        bool valid[GEN_U];
+#pragma unroll
+        for (int u = 0; u < GEN_U; u++) {
+            valid[u] = false;
+            if (j0 + u < nkeys && lg[j0 + u] != 0.0f) gen_load_key<NP>(a, b, sel, w, j0 + u, lane, v[u], valid[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < GEN_U; u++) {
+            if (!valid[u]) continue;
+            const float p = lg[j0 + u];
+#pragma unroll
+            for (int i = 0; i < NP; i++) {
+                acc[i].x += p * v[u][i].x;
+                acc[i].y += p * v[u][i].y;
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NP; i++) {
+        const int p = lane + 32 * i;
+        if (p < npairs) {
+            red[warp * C + 2 * p] = acc[i].x;
+            red[warp * C + 2 * p + 1] = acc[i].y;
+        }
+    }
+    __syncthreads();
     float *out = a.out + (bq * a.Hq + h) * (int64_t)C;
-    for (int c = tid; c < C; c += blockDim.x) {
-        float acc = 0.0f;
-        for (int j = 0; j < a.K; j++) {
-            const float p = lg[j];
-            if (p == 0.0f) continue;
-            const int64_t cell = (int64_t)b * a.cap + a.topk[bq * a.K + j];
-            const uint32_t byte = a.kv_fp4[cell * (C / 2) + c / 2];
-            const float v = e2m1_to_f32((c & 1) ? (byte >> 4) : (byte & 0xF)) *
-                            kv_group_scale(a.kv_sf + cell * (C / (a.mx ? 32 : 16)), c / 16, a.mx);
-            acc += p * v;
-        }
-        const uint16_t *swa = reinterpret_cast<const uint16_t *>(a.swa) +
-                              ((int64_t)b * a.swa_rows + w.row0) * C;
-        for (int j = 0; j < w.n; j++) {
-            const float p = lg[a.K + j];
-            acc += p * __uint_as_float((uint32_t)swa[(int64_t)j * C + c] << 16);
-        }
-        out[c] = acc * inv;
+    for (int c = tid; c < C; c += GEN_THREADS) {
+        float sum = 0.0f;
+#pragma unroll
+        for (int w2 = 0; w2 < GEN_WARPS; w2++) sum += red[w2 * C + c];
+        out[c] = sum * inv;
     }
 }
 
+template <int NP>
+static int launch_general(const AttnArgs &a, size_t smem, int64_t grid, cudaStream_t s) {
+    static PerDevice smem_set;
+    if (smem > 48 * 1024 && !set_smem_limit_once(smem_set, attn_general_kernel<NP>, 227 * 1024))
+        return CSA2_ERR_CUDA;
+    return launch_kernel(a.pdl, attn_general_kernel<NP>, dim3((unsigned)grid), dim3(GEN_THREADS), smem,
+                         s, a);
+}
+
 int launch_attn_general(const AttnArgs &a, cudaStream_t s) {
-    const size_t smem = sizeof(float) * ((size_t)a.C + a.K + a.n_win);
-    if (smem > 48 * 1024) {
-        if (cudaFuncSetAttribute(attn_general_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess)
-            return CSA2_ERR_CUDA;
-    }
+    // logits [K + n_win], partial sums [8][C], selected positions [K]
+    const size_t smem = sizeof(float) * ((size_t)a.K + a.n_win + (size_t)GEN_WARPS * a.C) +
+                        sizeof(int32_t) * (size_t)a.K;
+    if (smem > 227 * 1024) return CSA2_ERR_SHAPE;
     const int64_t grid = (int64_t)a.B * a.Nq * a.Hq;
     if (grid > INT32_MAX) return CSA2_ERR_SHAPE;
-    return launch_kernel(a.pdl, attn_general_kernel, dim3((unsigned)grid), dim3(256), smem, s, a);
+    const int pairs_per_lane = (a.C / 2 + 31) / 32;  // 1 .. 16 (C <= 1024)
+    if (pairs_per_lane <= 1) return launch_general<1>(a, smem, grid, s);
+    if (pairs_per_lane <= 2) return launch_general<2>(a, smem, grid, s);
+    if (pairs_per_lane <= 4) return launch_general<4>(a, smem, grid, s);
+    if (pairs_per_lane <= 8) return launch_general<8>(a, smem, grid, s);
+    return launch_general<16>(a, smem, grid, s);
 }
 
 }  // namespace csa2

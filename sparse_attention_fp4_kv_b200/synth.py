@@ -75,6 +75,13 @@ WORKLOADS = {
     "decoder_stack20_b4_ctx1m": Workload("decoder_stack20_b4_ctx1m", B=4, ctx=1048576, C=512,
                                          Hq=64, H_idx=16, D_idx=128, modes=list(DECODER_MODES),
                                          outlier_frac=0.01, outlier_mult=16.0, seed=3),
+    # The same stack at 256K context: its Reindex, selection and attention
+    # launches are those of the 1M stack (the pool is 2,048 blocks either way)
+    # with a quarter of the scan; small enough on the device for multi-pass
+    # profiler captures.
+    "decoder_stack20_b4_ctx256k": Workload("decoder_stack20_b4_ctx256k", B=4, ctx=262144, C=512,
+                                           Hq=64, H_idx=16, D_idx=128, modes=list(DECODER_MODES),
+                                           outlier_frac=0.01, outlier_mult=16.0, seed=7),
     # The 18 CSA2 encoder layers of a decode step, batch 4, 1M context.
     "encoder_stack18_b4_ctx1m": Workload("encoder_stack18_b4_ctx1m", B=4, ctx=1048576, C=512,
                                          Hq=64, H_idx=16, D_idx=128, modes=list(ENCODER_MODES),

@@ -356,6 +356,18 @@ int csa2_decode_stack_noalloc(const csa2_layer *layers, int n_layers, const void
                               int D, float softmax_scale, int32_t *pool, int pool_ready,
                               void *stream);
 
+/* ------------------------------------------------------------------------
+ * csa2_attn_resident_clusters: how many 8-CTA clusters of the tensor-core
+ * attention kernel can be resident at once on the current device when each
+ * cluster takes heads_per_cluster (16, 32 or 64) of the 64 query heads. The
+ * decode stack splits the heads as finely as the (query row, head group)
+ * items still fit in that many clusters. An introspection aid for callers
+ * sizing batches; the pages have no counterpart. Returns the count (at least
+ * 1; the library's upper bound of 18 when the occupancy query fails), or
+ * CSA2_ERR_RANGE for another heads_per_cluster. Needs a current device.
+ * ------------------------------------------------------------------------ */
+int csa2_attn_resident_clusters(int heads_per_cluster);
+
 #ifdef __cplusplus
 }
 #endif

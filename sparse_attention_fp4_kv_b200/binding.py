@@ -81,6 +81,7 @@ _SIGS = {
                                _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _P, _SZ, _P]),
     "csa2_decode_stack_noalloc": (_I, [ctypes.POINTER(csa2_layer), _I, _P, _P, _P, _P, _P, _I64,
                                        _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P]),
+    "csa2_attn_resident_clusters": (_I, [_I]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -184,6 +185,12 @@ def csa2_pool_gather(tok_score, pool, ctx_len, pool_score, pool_pos, q_pos=None,
     _check("csa2_pool_gather", lib.csa2_pool_gather(
         _ptr(tok_score), _ptr(pool), _ptr(ctx_len), _ptr(q_pos), B, Nq, P, cap,
         _ptr(pool_score), _ptr(pool_pos), _stream(stream)))
+
+
+def attn_resident_clusters(heads_per_cluster: int) -> int:
+    """8-CTA attention clusters that fit on the current device at once with
+    heads_per_cluster (16, 32 or 64) query heads each."""
+    return lib.csa2_attn_resident_clusters(heads_per_cluster)
 
 
 def device_status(clear: bool = False) -> int:

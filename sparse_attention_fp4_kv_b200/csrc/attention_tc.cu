@@ -791,3 +791,13 @@ size_t attn_tc_workspace_bytes(int B, int Nq) {
 int attn_group_max_layers() { return tc::MAXL; }
 
 }  // namespace csa2
+
+extern "C" int csa2_attn_resident_clusters(int heads_per_cluster) {
+    using namespace csa2;
+    switch (heads_per_cluster) {
+    case 16: return tc_max_active_clusters<16>();
+    case 32: return tc_max_active_clusters<32>();
+    case 64: return tc_max_active_clusters<64>();
+    default: return CSA2_ERR_RANGE;
+    }
+}

@@ -87,6 +87,23 @@ int csa2_device_status(int clear);
  * records the timeout, as a kernel of the library would. */
 int csa2_selftest_wait_timeout(int limit_us, void *stream);
 
+/* Per-call error word. The workspaces of csa2_sparse_attn_decode(_mxfp4) and
+ * csa2_decode_stack start with the call's error word: the call clears it on
+ * `stream` before its kernels run, and a kernel of that call that gives up a
+ * bounded wait sets it (besides the library flags above), so a timeout can be
+ * told apart from other calls on other streams. csa2_workspace_status reads
+ * the word at the start of ws on `stream` and synchronizes that stream:
+ * CSA2_ERR_DEVICE_TIMEOUT if it is set, else CSA2_OK; with clear != 0 a set
+ * word is reset (on the stream). CSA2_ERR_NULL for a NULL ws, CSA2_ERR_CUDA if
+ * the word cannot be read. csa2_decode_stack_noalloc keeps its word inside
+ * the library: use csa2_device_status for it. */
+int csa2_workspace_status(const void *ws, int clear, void *stream);
+
+/* Self-test of the per-call word: as csa2_selftest_wait_timeout, and the
+ * timeout also sets the error word at the start of ws (device memory of at
+ * least 4 bytes; the call does not clear it first). */
+int csa2_selftest_workspace_timeout(int limit_us, void *ws, void *stream);
+
 /* ------------------------------------------------------------------------
  * FP4 append: quantize-and-pack new main-KV rows into the cache.
  * [G] FP4 section and [N] FP4 section: E2M1 elements, one E4M3 scale per 16
@@ -249,7 +266,10 @@ int csa2_index_reindex(const int8_t *q_idx, const int8_t *k_idx, const float *k_
  *  swa_bf16 [B][swa_rows][C] bf16, 16-byte aligned; swa_pos0 [B] int64 (device)
  *  out      [B][Nq][Hq][C] fp32
  *  C % 32 == 0, 32 <= C <= 1024; 1 <= Hq <= 256; 0 <= K <= 4096; 0 <= n_win <= 4096.
- *  ws/ws_bytes: at least csa2_sparse_attn_workspace_size(...) bytes.
+ *  ws/ws_bytes: at least csa2_sparse_attn_workspace_size(...) bytes (0 for
+ *           shapes whose kernel has no bounded wait and no scratch: then ws
+ *           may be NULL). It starts with the call's error word (read with
+ *           csa2_workspace_status); the rest is the kernels' exchange space.
  * ------------------------------------------------------------------------ */
 size_t csa2_sparse_attn_workspace_size(int B, int Nq, int Hq, int C, int K, int n_win);
 int csa2_sparse_attn_decode(const void *q_bf16, const uint8_t *kv_fp4, const uint8_t *kv_sf,
@@ -277,6 +297,11 @@ int csa2_sparse_attn_decode_mxfp4(const void *q_bf16, const uint8_t *kv_fp4, con
  * Reuse -> nothing; then, for every layer, csa2_sparse_attn_decode with the
  * indices of the most recent Full/Reindex layer. One query per sequence
  * (Nq = 1) at position ctx_len[b] - 1, seeing the whole context.
+ * With 512 channels, 64 heads and fewer than 64 sequences, the attention of a
+ * Full or Reindex layer and the Reuse layers after it (up to 8 layers) runs as
+ * one kernel launch: layer l + 1 of a sequence starts once layer l of that
+ * sequence is written (per-sequence counters in the workspace; sequences are
+ * independent and never wait for each other).
  * When kv_new_bf16 ([B][C] bf16, 16-byte aligned) is not NULL, the step first
  * appends that row to the FP4 cache at position ctx_len[b] - 1 (as
  * csa2_kv_append_fp4 does); the new token's indexer key is expected to be in
@@ -298,6 +323,9 @@ int csa2_sparse_attn_decode_mxfp4(const void *q_bf16, const uint8_t *kv_fp4, con
  *  scan_events: NULL, or two cudaEvent_t that are recorded on `stream` right
  *         before and right after the first Full layer's indexer scan (to time
  *         that kernel inside the step).
+ *  ws/ws_bytes: at least csa2_decode_stack_workspace_size(...) bytes; it
+ *         starts with the call's error word (csa2_workspace_status), cleared
+ *         by the call.
  *  Errors: CSA2_ERR_RANGE if a Reuse layer has no preceding Full/Reindex
  *  layer or a Reindex layer has no pool; nothing is launched then.
  * ------------------------------------------------------------------------ */

@@ -82,6 +82,8 @@ _SIGS = {
     "csa2_decode_stack_noalloc": (_I, [ctypes.POINTER(csa2_layer), _I, _P, _P, _P, _P, _P, _I64,
                                        _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P]),
     "csa2_attn_resident_clusters": (_I, [_I]),
+    "csa2_workspace_status": (_I, [_P, _I, _P]),
+    "csa2_selftest_workspace_timeout": (_I, [_I, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -185,6 +187,12 @@ def csa2_pool_gather(tok_score, pool, ctx_len, pool_score, pool_pos, q_pos=None,
     _check("csa2_pool_gather", lib.csa2_pool_gather(
         _ptr(tok_score), _ptr(pool), _ptr(ctx_len), _ptr(q_pos), B, Nq, P, cap,
         _ptr(pool_score), _ptr(pool_pos), _stream(stream)))
+
+
+def workspace_status(ws: torch.Tensor, clear: bool = False, stream=None) -> int:
+    """Status of the call whose workspace is ws (its error word): 0, or
+    CSA2_ERR_DEVICE_TIMEOUT (-7) if a kernel of that call gave up a wait."""
+    return lib.csa2_workspace_status(_ptr(ws), int(clear), _stream(stream))
 
 
 def attn_resident_clusters(heads_per_cluster: int) -> int:

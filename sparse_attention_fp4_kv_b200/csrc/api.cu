@@ -26,6 +26,18 @@ extern "C" const char *csa2_status_string(int status) {
 
 extern "C" int csa2_abi_version(void) { return CSA2_ABI_VERSION; }
 
+extern "C" int csa2_workspace_status(const void *ws, int clear, void *stream) {
+    if (!ws) return CSA2_ERR_NULL;
+    cudaStream_t s = (cudaStream_t)stream;
+    int v = 0;
+    if (cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return CSA2_ERR_CUDA;
+    if (clear && v && cudaMemsetAsync(const_cast<void *>(ws), 0, sizeof(int), s) != cudaSuccess)
+        return CSA2_ERR_CUDA;
+    return v ? CSA2_ERR_DEVICE_TIMEOUT : CSA2_OK;
+}
+
 namespace {
 
 uint32_t *topk_hist_ptr_of(void *ws) { return static_cast<uint32_t *>(ws); }
@@ -34,6 +46,7 @@ constexpr size_t kAlign = 256;
 inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct StackWs {
+    int *err;          // the call's error word (set when a kernel gives up a bounded wait)
     float *tok;
     float *blk;
     int32_t *n_blk;
@@ -43,18 +56,32 @@ struct StackWs {
     void *sel_blk;     // histogram-fed top-k workspace of the pool selection
     void *sel_tok;     // ... and of the token top-512
     size_t hist_bytes; // leading bytes of each that must be zero before a step
-    size_t zero_bytes; // bytes from row_done that must be zero (counters + sel_blk's histogram)
+    size_t zero_bytes; // bytes from err that must be zero (error word, counters, sel_blk's histogram)
     void *attn;
     size_t attn_bytes;
     size_t total;
 };
 
+// Layout: the error word first (where csa2_workspace_status reads it), then
+// the regions that start every step at zero (the attention layer counters and
+// the pool selection's histogram follow it contiguously, so one memset clears
+// all three), then the scores and the attention scratch.
 StackWs stack_layout(void *base, int B, int Hq, int C, int64_t cap) {
     StackWs w{};
     size_t off = 0;
     char *p = static_cast<char *>(base);
     const int64_t nblk = (cap + 7) / 8;
     const int64_t P8 = (int64_t)kPoolBlocks * kBlockTokens;
+    w.err = reinterpret_cast<int *>(p + off);
+    off += kErrWordBytes;
+    w.row_done = reinterpret_cast<int *>(p + off);
+    off += up(sizeof(int) * (size_t)B);
+    w.sel_blk = p + off;
+    off += up(topk_hist_ws_bytes(B, kPoolBlocks));
+    w.sel_tok = p + off;
+    off += up(topk_hist_ws_bytes(B, kTopK));
+    w.hist_bytes = up((size_t)B * kHistBins * 4) + up((size_t)B * 2 * 4);
+    w.zero_bytes = kErrWordBytes + up(sizeof(int) * (size_t)B) + w.hist_bytes;
     w.tok = reinterpret_cast<float *>(p + off);
     off += up(sizeof(float) * (size_t)B * cap);
     w.blk = reinterpret_cast<float *>(p + off);
@@ -65,16 +92,8 @@ StackWs stack_layout(void *base, int B, int Hq, int C, int64_t cap) {
     off += up(sizeof(float) * (size_t)B * P8);
     w.ppos = reinterpret_cast<int32_t *>(p + off);
     off += up(sizeof(int32_t) * (size_t)B * P8);
-    w.row_done = reinterpret_cast<int *>(p + off);
-    off += up(sizeof(int) * (size_t)B);
-    w.sel_blk = p + off;
-    off += up(topk_hist_ws_bytes(B, kPoolBlocks));
-    w.sel_tok = p + off;
-    off += up(topk_hist_ws_bytes(B, kTopK));
-    w.hist_bytes = up((size_t)B * kHistBins * 4) + up((size_t)B * 2 * 4);
-    w.zero_bytes = up(sizeof(int) * (size_t)B) + w.hist_bytes;
     w.attn = p + off;
-    w.attn_bytes = up(attn_workspace_bytes(B, 1, Hq, C, kTopK, CSA2_N_WIN));
+    w.attn_bytes = up(attn_scratch_bytes(B, 1, Hq, C, kTopK));
     off += w.attn_bytes;
     w.total = off;
     return w;
@@ -136,7 +155,7 @@ extern "C" int csa2_decode_stack(const csa2_layer *layers, int n_layers,
     // the selection histograms and counters and the attention layer counters
     // start the step at zero (every finishing top-k kernel leaves its rows
     // clear for the next producer)
-    if (cudaMemsetAsync(w.row_done, 0, w.zero_bytes, s) != cudaSuccess ||
+    if (cudaMemsetAsync(w.err, 0, w.zero_bytes, s) != cudaSuccess ||
         cudaMemsetAsync(w.sel_tok, 0, w.hist_bytes, s) != cudaSuccess)
         return CSA2_ERR_CUDA;
     uint32_t *hist_blk = topk_hist_ptr_of(w.sel_blk);
@@ -187,7 +206,7 @@ extern "C" int csa2_decode_stack(const csa2_layer *layers, int n_layers,
         // (the layers' own inputs) are read after the wait.
         AttnArgs aa{L.q, kv_fp4, kv_sf, cap, cur, kTopK, L.swa, swa_pos0, swa_rows, nullptr,
                     CSA2_N_WIN, B, 1, Hq, C, softmax_scale, L.out, w.attn, true,
-                    L.mode == CSA2_MODE_REUSE};
+                    L.mode == CSA2_MODE_REUSE, false, w.err};
         st = attn_checked_launch(aa, w.attn_bytes, s, /*validate_only=*/true);
         if (st) return st;
         if (attn_tc_supported(aa) && (int64_t)B < kAttnRowsMin) {

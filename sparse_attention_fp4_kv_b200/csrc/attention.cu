@@ -220,7 +220,7 @@ extern "C" int csa2_sparse_attn_decode(const void *q_bf16, const uint8_t *kv_fp4
                                        void *ws, size_t ws_bytes, void *stream) {
     AttnArgs a{q_bf16, kv_fp4, kv_sf, cap, topk, K, swa_bf16, swa_pos0, swa_rows, q_pos,
                n_win, B, Nq, Hq, C, softmax_scale, out, ws, false, false};
-    return attn_checked_launch(a, ws_bytes, (cudaStream_t)stream);
+    return attn_call(a, ws_bytes, (cudaStream_t)stream);
 }
 
 extern "C" int csa2_sparse_attn_decode_mxfp4(const void *q_bf16, const uint8_t *kv_fp4,
@@ -232,7 +232,7 @@ extern "C" int csa2_sparse_attn_decode_mxfp4(const void *q_bf16, const uint8_t *
     if (C % 32) return CSA2_ERR_SHAPE;
     AttnArgs a{q_bf16, kv_fp4, kv_sf, cap, topk, K, swa_bf16, swa_pos0, swa_rows, q_pos,
                n_win, B, Nq, Hq, C, softmax_scale, out, ws, false, false, true};
-    return attn_checked_launch(a, ws_bytes, (cudaStream_t)stream);
+    return attn_call(a, ws_bytes, (cudaStream_t)stream);
 }
 
 namespace csa2 {
@@ -247,19 +247,40 @@ int attn_checked_launch(const AttnArgs &a, size_t ws_bytes, cudaStream_t s, bool
         return CSA2_ERR_SHAPE;
     if (!aligned(a.q, 16) || (a.swa && !aligned(a.swa, 16)) || !aligned(a.kv_fp4, 8))
         return CSA2_ERR_ALIGN;
-    if (ws_bytes < attn_workspace_bytes(a.B, a.Nq, a.Hq, a.C, a.K, a.n_win))
+    if ((a.ws == nullptr ? 0 : ws_bytes) < attn_scratch_bytes(a.B, a.Nq, a.Hq, a.C, a.K))
         return CSA2_ERR_WORKSPACE;
     if ((int64_t)a.B * a.Nq == 0 || validate_only) return CSA2_OK;
     return launch_attn(a, s);
 }
 
-// The tensor-core kernel exchanges per-CTA partial results through the
-// workspace; the general kernel needs none. The size covers the tensor-core
-// path whenever its shape constraints could hold.
-size_t attn_workspace_bytes(int B, int Nq, int Hq, int C, int K, int n_win) {
-    if (C == 512 && Hq == 64 && K > 0 && K <= 640)
-        return attn_tc_workspace_bytes(B, Nq);
+// A standalone call: its workspace starts with the call's error word, cleared
+// at the call's start; the kernels' scratch follows it.
+int attn_call(AttnArgs a, size_t ws_bytes, cudaStream_t s) {
+    const size_t need = attn_workspace_bytes(a.B, a.Nq, a.Hq, a.C, a.K, a.n_win);
+    if (need == 0) return attn_checked_launch(a, ws_bytes, s);
+    if (a.ws == nullptr || ws_bytes < need) return CSA2_ERR_WORKSPACE;
+    a.err = static_cast<int *>(a.ws);
+    if (cudaMemsetAsync(a.err, 0, sizeof(int), s) != cudaSuccess) return CSA2_ERR_CUDA;
+    a.ws = static_cast<char *>(a.ws) + kErrWordBytes;
+    return attn_checked_launch(a, ws_bytes - kErrWordBytes, s);
+}
+
+// Scratch of the kernels (a.ws): the cluster kernel's exchange slots for its
+// per-CTA partial results when its shape constraints could hold; the other
+// kernels need none.
+size_t attn_scratch_bytes(int B, int Nq, int Hq, int C, int K) {
+    if (C == 512 && Hq == 64 && K > 0 && K <= 640) return attn_tc_workspace_bytes(B, Nq);
     return 0;
+}
+
+// Workspace of a standalone call: the call's error word (kErrWordBytes)
+// whenever a tensor-core kernel, whose waits are bounded, may take the call
+// (512 channels, 64 heads), followed by the kernels' scratch. The general
+// kernel waits on nothing and needs none.
+size_t attn_workspace_bytes(int B, int Nq, int Hq, int C, int K, int n_win) {
+    (void)n_win;
+    if (C != 512 || Hq != 64) return 0;
+    return kErrWordBytes + attn_scratch_bytes(B, Nq, Hq, C, K);
 }
 
 // Tensor-core kernels where their shape constraints hold (64 heads, 512

@@ -32,7 +32,14 @@ struct AttnArgs {
     // Scales of the FP4 rows: E4M3 per 16 channels (kv_sf [B][cap][C/16]), or
     // with mx the MXFP4 variant's E8M0 per 32 channels (kv_sf [B][cap][C/32]).
     bool mx;
+    // The call's error word (the first word of the caller's workspace), or
+    // NULL: a kernel that gives up a bounded wait sets it to 1 besides the
+    // library's device flag.
+    int *err = nullptr;
 };
+
+// Bytes at the start of a workspace that hold the call's error word.
+constexpr size_t kErrWordBytes = 256;
 
 // Sliding-window rows of query bq: rows [row0, row0 + n) of the SWA tensor,
 // i.e. positions max(0, p - n_win + 1) .. p that the tensor holds.
@@ -59,6 +66,11 @@ __device__ __forceinline__ AttnWindow attn_window(const AttnArgs &a, int b, int6
 }
 
 size_t attn_workspace_bytes(int B, int Nq, int Hq, int C, int K, int n_win);
+// The kernels' scratch (AttnArgs::ws) without the error word.
+size_t attn_scratch_bytes(int B, int Nq, int Hq, int C, int K);
+// A standalone call (csa2_sparse_attn_decode): the error word at the start of
+// ws is cleared, then the call is checked and launched with the rest as scratch.
+int attn_call(AttnArgs a, size_t ws_bytes, cudaStream_t s);
 // Validates the arguments of a sparse-attention call (status codes of
 // csa2_sparse_attn_decode) and launches it.
 // With validate_only, only the checks run (CSA2_OK when the call would launch).

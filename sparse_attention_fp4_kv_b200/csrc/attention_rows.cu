@@ -490,6 +490,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     __syncthreads();
     if (*abort) {
+        if (tid == 0 && a.err) atomicExch(a.err, 1);
         // let copies and MMAs still in flight land before the CTA's memory is released
         const uint64_t t0 = globaltimer_ns();
         while (globaltimer_ns() - t0 < 2000000ull) {

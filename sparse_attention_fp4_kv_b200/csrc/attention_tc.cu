@@ -594,7 +594,10 @@ __global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
             if (!keep && !last) cluster_sync();
         }
     }
-    if (!ok) atomicExch(&g_attn_error, 1);
+    if (!ok) {
+        atomicExch(&g_attn_error, 1);
+        if (a.err) atomicExch(a.err, 1);
+    }
     // copies still in flight into this CTA's shared memory land before it exits
     if (tid == 0 && ld_pending) (void)mbar_wait_bounded(bar_ld, ld_phase, WAIT_NS);
     __syncthreads();

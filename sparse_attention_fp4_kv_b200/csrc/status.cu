@@ -9,7 +9,7 @@ namespace csa2 {
 
 __device__ int g_selftest_error = 0;
 
-__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+__global__ void selftest_wait_kernel(uint64_t limit_ns, int *err) {
     __shared__ __align__(8) uint64_t bar;
     const uint32_t b = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
     if (threadIdx.x == 0) {
@@ -32,7 +32,10 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns) {
         done = d != 0;
         asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     } while (!done && t - t0 < limit_ns);
-    if (!done && threadIdx.x == 0) atomicExch(&g_selftest_error, 1);
+    if (!done && threadIdx.x == 0) {
+        atomicExch(&g_selftest_error, 1);
+        if (err) atomicExch(err, 1);
+    }
 }
 
 }  // namespace csa2
@@ -54,6 +57,14 @@ extern "C" int csa2_device_status(int clear) {
 
 extern "C" int csa2_selftest_wait_timeout(int limit_us, void *stream) {
     if (limit_us < 1 || limit_us > 1000000) return CSA2_ERR_RANGE;
-    selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)limit_us * 1000ull);
+    selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)limit_us * 1000ull, nullptr);
+    return launch_status();
+}
+
+extern "C" int csa2_selftest_workspace_timeout(int limit_us, void *ws, void *stream) {
+    if (!ws) return CSA2_ERR_NULL;
+    if (limit_us < 1 || limit_us > 1000000) return CSA2_ERR_RANGE;
+    selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)limit_us * 1000ull,
+                                                               static_cast<int *>(ws));
     return launch_status();
 }

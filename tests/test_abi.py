@@ -136,7 +136,15 @@ def test_attention_workspace_covers_every_head_split(lib):
         rows = B * Nq
         need = [min(rows * (64 // hpc), 18) * _attn_slot_bytes(hpc) for hpc in (16, 32, 64)]
         got = ws(B, Nq, 64, 512, 512, 128)
-        assert got == max(need), (B, Nq, got, need)
+        assert got == 256 + max(need), (B, Nq, got, need)   # error word + exchange slots
+    # more than 640 keys: the per-row kernel, which has bounded waits but no slots
+    assert ws(2, 1, 64, 512, 1024, 128) == 256
     # the tensor-core kernels need no workspace outside their shape, nor does the general kernel
     assert ws(2, 1, 8, 128, 512, 128) == 0
-    assert ws(2, 1, 64, 512, 1024, 128) == 0
+
+
+def test_workspace_status_rejects_a_null_workspace(lib):
+    """The per-call error word is read from the workspace; a NULL workspace is
+    rejected on the host before any CUDA call."""
+    assert lib.csa2_workspace_status(None, 0, None) == -1
+    assert lib.csa2_selftest_workspace_timeout(1000, None, None) == -1

@@ -571,3 +571,27 @@ def test_device_status_reports_a_bounded_wait_timeout(B):
     out = torch.empty((1, 10), dtype=torch.int32, device=DEV)
     B.csa2_topk(score, 10, out)
     assert out.cpu().tolist() == [list(range(90, 100))]
+
+
+def test_workspace_error_word_attributes_a_timeout_to_its_call(B):
+    """The error word at the start of a call's workspace: a kernel that gives up
+    a bounded wait sets it (besides the library flag), another call's word on
+    another stream stays clear, and a decode step clears its own word."""
+    B.device_status(clear=True)
+    ws_a = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    ws_b = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    assert B.lib.csa2_selftest_workspace_timeout(2000, B._ptr(ws_a), B._stream(s1)) == 0
+    assert B.workspace_status(ws_a, stream=s1) == -7
+    assert B.workspace_status(ws_b, stream=s2) == 0
+    assert B.workspace_status(ws_a, clear=True, stream=s1) == -7
+    assert B.workspace_status(ws_a, stream=s1) == 0
+    assert B.device_status(clear=True) == -7          # the library flag saw it too
+    # a decode step clears its word and leaves it clear when every wait completes
+    from sparse_attention_fp4_kv_b200 import synth
+    from sparse_attention_fp4_kv_b200.workload import DecodeWorkload
+    wl = DecodeWorkload(synth.scaled(synth.WORKLOADS["decoder_stack20_b4_ctx1m"], B=2, ctx=9001), DEV)
+    wl.stack.ws[:4].fill_(1)
+    wl.step()
+    assert B.workspace_status(wl.stack.ws) == 0
+    assert B.device_status() == 0

@@ -173,14 +173,10 @@ extern "C" int csa2_decode_stack(const csa2_layer *layers, int n_layers,
                 cudaEventRecord((cudaEvent_t)scan_events[1], (cudaStream_t)stream);
                 scan_timed = true;
             }
-            st = launch_topk_from_hist(w.blk, nullptr, w.n_blk, B, nblk, kPoolBlocks, pool,
-                                       w.sel_blk, s);
-            if (st) return st;
-            st = launch_pool_gather_hist(w.tok, pool, ctx_len, B, kPoolBlocks, cap, w.pscore, w.ppos,
-                                         hist_tok, s);
-            if (st) return st;
-            st = launch_topk_from_hist(w.pscore, w.ppos, nullptr, B, P8, kTopK, L.topk, w.sel_tok,
-                                       s);
+            // the pool and the top-512 among the pooled tokens in one selection
+            // (a compaction kernel first for rows of more than 65,536 blocks)
+            st = launch_pool_and_tokens(w.blk, w.n_blk, B, nblk, kPoolBlocks, pool, w.sel_blk, w.tok,
+                                        ctx_len, cap, kTopK, L.topk, s);
             if (st) return st;
             cur = L.topk;
         } else if (L.mode == CSA2_MODE_REINDEX) {

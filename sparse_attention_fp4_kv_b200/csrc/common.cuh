@@ -119,6 +119,7 @@ inline int read_device_flag(T &symbol, bool clear) {
 int attn_tc_wait_flag(bool clear);
 int attn_rows_wait_flag(bool clear);
 int index_mma_wait_flag(bool clear);
+int index_scan_wait_flag(bool clear);
 
 // Streaming multiprocessors of the current device (148 on B200 if the query fails).
 inline int num_sms() {
@@ -246,6 +247,10 @@ __device__ __forceinline__ uint32_t hist_bin(float score) { return f32_order_key
 // the three score producers below serve the decode step only and launch with
 // programmatic stream serialization.
 size_t topk_hist_ws_bytes(int R, int k);
+// Pool and top tokens of the decode Full layer in one selection (topk.cu).
+int launch_pool_and_tokens(const float *blk, const int32_t *n_blk, int R, int64_t nblk, int P,
+                           int32_t *pool, void *ws, const float *tok, const int64_t *ctx_len,
+                           int64_t cap, int ktop, int32_t *top, cudaStream_t s);
 int launch_topk_from_hist(const float *score, const int32_t *cand_pos, const int32_t *n_valid,
                           int R, int64_t n, int k, int32_t *out, void *ws, cudaStream_t s);
 

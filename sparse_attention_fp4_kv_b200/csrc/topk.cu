@@ -570,13 +570,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_finish_kernel(TopkArgs a, 
 constexpr int64_t TS_MAX_N = 65536;
 constexpr int TS_PER = 16;
 
-__global__ void __launch_bounds__(TK_THREADS, 1) topk_row_hist_kernel(TopkArgs a, uint32_t *ghist) {
-    grid_dep_wait();
-    grid_dep_launch();
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    __shared__ TopkState st;
-    TopkShared sh = topk_shared(smem_raw);
-    const int64_t r = blockIdx.x;
+__device__ void topk_row_hist_body(const TopkArgs &a, int64_t r, uint32_t *ghist, TopkShared sh,
+                                   TopkState &st) {
     const int lane = threadIdx.x & 31;
     int64_t nv = a.n;
     if (a.n_valid) {
@@ -648,6 +643,183 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_row_hist_kernel(TopkArgs a
     for (int b = threadIdx.x; b < TK_HIST; b += TK_THREADS) ghist[r * TK_HIST + b] = 0;
 }
 
+__global__ void __launch_bounds__(TK_THREADS, 1) topk_row_hist_kernel(TopkArgs a, uint32_t *ghist) {
+    grid_dep_wait();
+    grid_dep_launch();
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __shared__ TopkState st;
+    topk_row_hist_body(a, blockIdx.x, ghist, topk_shared(smem_raw), st);
+}
+
+// ------------------------------------------------------------------ pool + tokens
+// The decode Full layer's selection after its scan, in one CTA per row: the
+// pool (best P blocks, from the producer's histogram, as the two selection
+// kernels above do) and then the row's top-K tokens among the pooled blocks'
+// tokens. The pooled tokens' rank keys are gathered into shared memory in pool
+// order, which is position order (the pool is written ascending), and selected
+// there: a 12-bit first digit, then the remaining digits of the threshold
+// bin's keys, then emission in index order (= ascending positions) through a
+// bitmap. An empty slot holds key 0, which no finite score produces.
+constexpr int PT_MAX = kPoolBlocks * kBlockTokens;                  // 16,384 pooled tokens
+constexpr size_t PT_SMEM = TK_HIST * 4 + TK_MAXK * 4 + (size_t)PT_MAX * 8;  // 160 KB
+static_assert((size_t)PT_MAX * 8 >= (size_t)TK_BUF * 8, "the key array holds the tie buffer");
+
+__device__ __forceinline__ TopkShared pool_tokens_shared(uint8_t *smem_raw) {
+    return TopkShared{reinterpret_cast<uint32_t *>(smem_raw),
+                      reinterpret_cast<uint64_t *>(smem_raw + TK_HIST * 4 + TK_MAXK * 4),
+                      reinterpret_cast<int32_t *>(smem_raw + TK_HIST * 4)};
+}
+
+struct PoolTokArgs {
+    const float *tok;        // [R][cap] token scores of the scan
+    const int64_t *ctx_len;  // [R] visible length of each row
+    int64_t cap;
+    int k;                   // tokens to keep (<= TK_MAXK)
+    int32_t *top;            // [R][k] ascending positions, -1 padded
+};
+
+// Top-pa.k tokens of row r among the tokens of the a.k pool blocks this CTA
+// just wrote to a.out (row r, ascending block ids, -1 padded). All threads of
+// the CTA, after a barrier that follows the pool's writes.
+__device__ void pool_tokens_select(const TopkArgs &a, const PoolTokArgs &pa, int64_t r,
+                                   TopkShared sh, TopkState &st) {
+    const int P = a.k, n = P * kBlockTokens;
+    uint64_t *keys = sh.buf;
+    int64_t V = pa.ctx_len[r];
+    if (V > pa.cap) V = pa.cap;
+    const int32_t *pool = a.out + r * (int64_t)P;
+    const float *tok = pa.tok + r * pa.cap;
+    for (int i = threadIdx.x; i < n; i += TK_THREADS) {
+        const int32_t blk = pool[i >> 3];
+        const int64_t pos = 8 * (int64_t)blk + (i & 7);
+        keys[i] = (blk >= 0 && pos < V) ? rank_key(tok[pos], (int32_t)pos) : 0ull;
+    }
+    for (int b = threadIdx.x; b < TK_HIST; b += TK_THREADS) sh.hist[b] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += TK_THREADS) {
+        const uint64_t key = keys[i];
+        if (key) atomicAdd(&sh.hist[key >> 52], 1u);
+    }
+    __syncthreads();
+    find_digit(sh.hist, TK_HIST, pa.k, st);
+    const bool all = st.total <= (uint32_t)pa.k;
+    const uint64_t d = (uint64_t)st.digit;
+    if (threadIdx.x == 0) {
+        st.kk = pa.k - (int)st.above;
+        st.prefix = d << 52;
+        st.mask = (uint64_t)(TK_HIST - 1) << 52;
+    }
+    __syncthreads();
+    if (!all && st.match != (uint32_t)st.kk) {
+        // only part of the threshold bin is taken: further digits over its keys
+        const int widths[6] = {10, 10, 8, 8, 8, 8};
+        int shift = 52;
+        for (int wi = 0; wi < 6; wi++) {
+            shift -= widths[wi];
+            const int NB = 1 << widths[wi];
+            smem_hist_pass(keys, n, sh.hist, NB, shift, st.prefix, st.mask);
+            find_digit(sh.hist, NB, st.kk, st);
+            if (threadIdx.x == 0) {
+                st.kk -= (int)st.above;
+                st.prefix |= (uint64_t)st.digit << shift;
+                st.mask |= (uint64_t)(NB - 1) << shift;
+            }
+            __syncthreads();
+            if (st.match == (uint32_t)st.kk) break;
+        }
+    }
+    const uint64_t p = st.prefix, m = st.mask;
+    // bitmap of the selected indices over [0, n), in the histogram's space
+    uint32_t *bm = sh.hist;
+    const int nwords = n / 32;
+    for (int i = threadIdx.x; i < nwords; i += TK_THREADS) bm[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += TK_THREADS) {
+        const uint64_t key = keys[i];
+        const bool take = key && (all || (key >> 52) > d || ((key & m) >= p && (key >> 52) == d));
+        if (take) atomicOr(&bm[i >> 5], 1u << (i & 31));
+    }
+    __syncthreads();
+    const int per = (nwords + TK_THREADS - 1) / TK_THREADS;
+    const int w0 = threadIdx.x * per;
+    int c = 0;
+    for (int i = 0; i < per; i++)
+        if (w0 + i < nwords) c += __popc(bm[w0 + i]);
+    int rank = block_excl_scan(c, st);
+    int32_t *out = pa.top + r * (int64_t)pa.k;
+    for (int i = 0; i < per; i++) {
+        if (w0 + i >= nwords) break;
+        uint32_t bits = bm[w0 + i];
+        while (bits) {
+            const int b = __ffs(bits) - 1;
+            bits &= bits - 1;
+            if (rank < pa.k) out[rank] = rank_key_pos(keys[(w0 + i) * 32 + b]);
+            rank++;
+        }
+    }
+    // the last thread's rank is the number selected: -1 after them
+    if (threadIdx.x == TK_THREADS - 1) st.nsel = rank;
+    __syncthreads();
+    for (int i = st.nsel + threadIdx.x; i < pa.k; i += TK_THREADS) out[i] = -1;
+}
+
+// Pool from the compacted global lists (as topk_finish_kernel), then the row's
+// top tokens among the pooled tokens.
+__global__ void __launch_bounds__(TK_THREADS, 1)
+    topk_finish_pool_tokens_kernel(TopkArgs a, TopkHistWs ws, PoolTokArgs pa) {
+    grid_dep_wait();
+    grid_dep_launch();
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __shared__ TopkState st;
+    TopkShared sh = pool_tokens_shared(smem_raw);
+    const int64_t r = blockIdx.x;
+    load_hist<TK_THREADS>(sh.hist, ws.hist + r * TK_HIST);
+    const int nsel0 = min(ws.cnt[2 * r], a.k);
+    const int ntie = ws.cnt[2 * r + 1];
+    if (threadIdx.x == 0) {
+        st.prefix = 0;
+        st.mask = 0;
+        st.nsel = 0;
+        st.nbuf = 0;
+    }
+    __syncthreads();
+    find_digit(sh.hist, TK_HIST, a.k, st);
+    const bool all = st.total <= (uint32_t)a.k;
+    if ((!all && ntie > TK_BUF) || a.n > TF_MAX_N) {
+        __syncthreads();
+        topk_row_full(a, r, sh, st);  // rare: the tie list or the bitmap does not fit
+    } else {
+        load_batched(sh.sel, ws.sel + r * a.k, nsel0);
+        if (threadIdx.x == 0) st.nsel = nsel0;
+        if (!all) {
+            load_batched(sh.buf, ws.tie + r * TK_BUF, ntie);
+            resolve_ties(sh, st, ntie, a.k);
+        }
+        __syncthreads();
+        emit_in_index_order(a, r, sh, st, min(st.nsel, a.k));
+    }
+    // leave the histogram and counters of this row clear for the next producer
+    __syncthreads();
+    for (int b = threadIdx.x; b < TK_HIST; b += TK_THREADS) ws.hist[r * TK_HIST + b] = 0;
+    if (threadIdx.x < 2) ws.cnt[2 * r + threadIdx.x] = 0;
+    __syncthreads();
+    pool_tokens_select(a, pa, r, sh, st);
+}
+
+// Pool from one pass over the row (as topk_row_hist_kernel), then the row's top
+// tokens among the pooled tokens.
+__global__ void __launch_bounds__(TK_THREADS, 1)
+    topk_row_pool_tokens_kernel(TopkArgs a, uint32_t *ghist, PoolTokArgs pa) {
+    grid_dep_wait();
+    grid_dep_launch();
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __shared__ TopkState st;
+    TopkShared sh = pool_tokens_shared(smem_raw);
+    topk_row_hist_body(a, blockIdx.x, ghist, sh, st);
+    __syncthreads();
+    pool_tokens_select(a, pa, blockIdx.x, sh, st);
+}
+
 }  // namespace csa2
 
 using namespace csa2;
@@ -697,6 +869,33 @@ int launch_topk_from_hist(const float *score, const int32_t *cand_pos, const int
                                  dim3(TC_THREADS), 0, s, a, w);
     if (st) return st;
     return launch_kernel(true, topk_finish_kernel, dim3(R), dim3(TK_THREADS), TK_SMEM, s, a, w);
+}
+
+// The decode Full layer's pool (k = P blocks of the block scores blk, whose
+// histogram the scan filled) and the top ktop tokens among the pooled tokens
+// (token scores tok [R][cap]): written to pool and top. One kernel per row, or
+// compaction + one kernel per row for rows longer than TS_MAX_N blocks.
+int launch_pool_and_tokens(const float *blk, const int32_t *n_blk, int R, int64_t nblk, int P,
+                           int32_t *pool, void *ws, const float *tok, const int64_t *ctx_len,
+                           int64_t cap, int ktop, int32_t *top, cudaStream_t s) {
+    if (R == 0) return CSA2_OK;
+    if (R > 65535 || P * kBlockTokens > PT_MAX || ktop > TK_MAXK) return CSA2_ERR_SHAPE;
+    static PerDevice smem_set[2];
+    if (!set_smem_limit_once(smem_set[0], topk_finish_pool_tokens_kernel, PT_SMEM) ||
+        !set_smem_limit_once(smem_set[1], topk_row_pool_tokens_kernel, PT_SMEM))
+        return CSA2_ERR_CUDA;
+    TopkArgs a{blk, nullptr, n_blk, R, nblk, P, pool};
+    PoolTokArgs pa{tok, ctx_len, cap, ktop, top};
+    TopkHistWs w = topk_hist_ws(ws, R, P);
+    if (nblk <= TS_MAX_N)
+        return launch_kernel(true, topk_row_pool_tokens_kernel, dim3(R), dim3(TK_THREADS), PT_SMEM, s,
+                             a, w.hist, pa);
+    const int64_t slices = (nblk + TC_SLICE - 1) / TC_SLICE;
+    const int st = launch_kernel(true, topk_compact_kernel, dim3((unsigned)slices, (unsigned)R),
+                                 dim3(TC_THREADS), 0, s, a, w);
+    if (st) return st;
+    return launch_kernel(true, topk_finish_pool_tokens_kernel, dim3(R), dim3(TK_THREADS), PT_SMEM, s, a,
+                         w, pa);
 }
 
 }  // namespace csa2

@@ -140,8 +140,8 @@ class DecodeWorkload:
 
     def launches_per_step(self) -> int:
         """libcsa2 kernels one step launches: the append, then per Full layer
-        the scan, the pool selection, the gather and the token selection; per
-        Reindex layer the rescoring and the token selection. Attention: one
+        the scan and one selection of the pool and its top tokens; per Reindex
+        layer the rescoring and the token selection. Attention: one
         kernel per layer group (a Full or Reindex layer and the Reuse layers
         after it, at most ATTN_GROUP_MAX layers per kernel) where the
         tensor-core cluster kernel takes the shape, else one per layer. A
@@ -157,8 +157,7 @@ class DecodeWorkload:
         n = 1
         run = 0  # layers in the current attention launch
         for m in self.modes:
-            n += {synth.FULL: 2 + sel(nblk) + sel(pooled), synth.REINDEX: 1 + sel(pooled),
-                  synth.REUSE: 0}[m]
+            n += {synth.FULL: 1 + sel(nblk), synth.REINDEX: 1 + sel(pooled), synth.REUSE: 0}[m]
             if grouped and m == synth.REUSE and 0 < run < csa2.ATTN_GROUP_MAX:
                 run += 1
             else:

@@ -119,7 +119,6 @@ inline int read_device_flag(T &symbol, bool clear) {
 int attn_tc_wait_flag(bool clear);
 int attn_rows_wait_flag(bool clear);
 int index_mma_wait_flag(bool clear);
-int index_scan_wait_flag(bool clear);
 
 // Streaming multiprocessors of the current device (148 on B200 if the query fails).
 inline int num_sms() {

@@ -207,198 +207,6 @@ __global__ void __launch_bounds__(256) index_full_kernel(ScanArgs a) {
     }
 }
 
-// TMA-fed variant of the scan for 16 x 128 keys (16 KB blocks): one
-// persistent CTA per SM, one producer thread that streams the CTA's blocks
-// (items blockIdx.x, blockIdx.x + gridDim.x, ...) with cp.async.bulk into a
-// ring of SCAN_STAGES shared-memory stages (128 KB in flight per SM), and
-// SCAN_CONS consumer warps, warp w taking the items whose stage is w. The
-// arithmetic per block is the register kernel's: dp4a dots of 16-byte
-// vectors (lane l takes vectors 32 i + l), the 9-shuffle transpose-reduce,
-// fp32 score, block max and histogram count. Every wait is bounded; a wait
-// that runs out sets the scan's device flag and the CTA stops, letting the
-// copies it issued land before it exits.
-constexpr int SCAN_CONS = 8;
-constexpr int SCAN_STAGES = 8;
-constexpr int SCAN_THREADS = 32 * (SCAN_CONS + 1);
-constexpr int SCAN_HD = 2048;
-constexpr int SCAN_STAGE_BYTES = 8 * SCAN_HD;
-constexpr size_t SCAN_SMEM = (size_t)SCAN_STAGES * SCAN_STAGE_BYTES;
-constexpr uint64_t SCAN_WAIT_NS = 200ull * 1000 * 1000;
-static_assert(SCAN_STAGES == SCAN_CONS, "consumer warp w owns stage w");
-
-__device__ int g_scan_error = 0;
-
-__device__ __forceinline__ uint32_t scan_smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ bool scan_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
-        "selp.u32 %0, 1, 0, p;\n}"
-        : "=r"(done)
-        : "r"(bar), "r"(parity), "r"(20000u)
-        : "memory");
-    return done != 0;
-}
-// Bounded wait for the phase of the given parity (or until *stop is set).
-__device__ __forceinline__ bool scan_wait(uint32_t bar, uint32_t parity, volatile int *stop) {
-    uint64_t t0 = 0;
-    for (;;) {
-        if (scan_try_wait(bar, parity)) return true;
-        if (*stop) return false;
-        uint64_t now;
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
-        if (t0 == 0) {
-            t0 = now;
-        } else if (now - t0 > SCAN_WAIT_NS) {
-            *stop = 1;
-            atomicExch(&g_scan_error, 1);
-            return false;
-        }
-    }
-}
-
-__global__ void __launch_bounds__(SCAN_THREADS, 1) index_full_tma_kernel(ScanArgs a) {
-    using RS = RowShape<SCAN_HD>;
-    extern __shared__ __align__(128) uint8_t stage_mem[];
-    __shared__ __align__(8) uint64_t full_bar[SCAN_STAGES], empty_bar[SCAN_STAGES];
-    __shared__ int64_t issued[SCAN_STAGES];  // uses of each stage the producer issued
-    __shared__ int stop;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) {
-        for (int st = 0; st < SCAN_STAGES; st++) {
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(scan_smem_u32(&full_bar[st]))
-                         : "memory");
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(scan_smem_u32(&empty_bar[st]))
-                         : "memory");
-            issued[st] = 0;
-        }
-        stop = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncthreads();
-    grid_dep_wait();
-    grid_dep_launch();
-    const int64_t items = (int64_t)a.B * a.Nq * a.nblk_cap;
-    const int64_t nmine =
-        (int64_t)blockIdx.x < items ? (items - 1 - (int64_t)blockIdx.x) / gridDim.x + 1 : 0;
-
-    if (warp == SCAN_CONS) {
-        // ---- producer: one thread issues the CTA's block copies in order
-        if (lane == 0) {
-            volatile int *vstop = &stop;
-            for (int64_t k = 0; k < nmine && !*vstop; k++) {
-                const int st = (int)(k % SCAN_STAGES);
-                const uint32_t use = (uint32_t)(k / SCAN_STAGES);
-                if (k >= SCAN_STAGES &&
-                    !scan_wait(scan_smem_u32(&empty_bar[st]), (use - 1) & 1, &stop))
-                    break;
-                const int64_t it = (int64_t)blockIdx.x + k * gridDim.x;
-                const int64_t bq = it / a.nblk_cap;
-                const int64_t j = it - bq * a.nblk_cap;
-                const int b = (int)(bq / a.Nq), i = (int)(bq % a.Nq);
-                int64_t V = visible_len(a.ctx_len, a.q_pos, b, i, a.Nq);
-                if (V > a.cap) V = a.cap;
-                const int64_t ntok = 8 * j < V ? (V - 8 * j < 8 ? V - 8 * j : 8) : 0;
-                const uint32_t fb = scan_smem_u32(&full_bar[st]);
-                if (ntok > 0) {
-                    const uint32_t bytes = (uint32_t)(ntok * SCAN_HD);
-                    const int8_t *src = a.k + ((int64_t)b * a.cap + 8 * j) * SCAN_HD;
-                    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb),
-                                 "r"(bytes)
-                                 : "memory");
-                    asm volatile(
-                        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], "
-                        "%2, [%3];" ::"r"(scan_smem_u32(stage_mem + (size_t)st * SCAN_STAGE_BYTES)),
-                        "l"(src), "r"(bytes), "r"(fb)
-                        : "memory");
-                } else {
-                    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(fb) : "memory");
-                }
-                issued[st] = (int64_t)use + 1;
-            }
-        }
-    } else {
-        // ---- consumers: warp w scores the blocks of stage w
-        const int my_tok = reduce_token_of_lane(lane);
-        int64_t cur_bq = -1, V = 0;
-        uint4 qf[RS::QV];
-        const uint4 *sv = reinterpret_cast<const uint4 *>(stage_mem + (size_t)warp * SCAN_STAGE_BYTES);
-        for (int64_t k = warp; k < nmine; k += SCAN_STAGES) {
-            const uint32_t use = (uint32_t)(k / SCAN_STAGES);
-            bool ok = true;
-            if (lane == 0) ok = scan_wait(scan_smem_u32(&full_bar[warp]), use & 1, &stop);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) break;
-            const int64_t it = (int64_t)blockIdx.x + k * gridDim.x;
-            const int64_t bq = it / a.nblk_cap;
-            const int64_t j = it - bq * a.nblk_cap;
-            const int b = (int)(bq / a.Nq), i = (int)(bq % a.Nq);
-            if (bq != cur_bq) {
-                cur_bq = bq;
-                V = visible_len(a.ctx_len, a.q_pos, b, i, a.Nq);
-                if (V > a.cap) V = a.cap;
-                load_qfrag<SCAN_HD>(a.q + bq * SCAN_HD, qf, lane);
-            }
-            if (j == 0 && lane == 0 && a.n_blk) a.n_blk[bq] = (int32_t)((V + 7) / 8);
-            if (8 * j < V) {
-                const int ntok = (int)(V - 8 * j < 8 ? V - 8 * j : 8);
-                int part[8];
-#pragma unroll
-                for (int t = 0; t < 8; t++) part[t] = 0;
-#pragma unroll
-                for (int i0 = 0; i0 < RS::VPL; i0 += 8) {
-                    uint4 kv[8];
-#pragma unroll
-                    for (int u = 0; u < 8; u++) {
-                        const int v = 32 * (i0 + u) + lane;
-                        kv[u] = (v / RS::VPT < ntok) ? sv[v] : make_uint4(0, 0, 0, 0);
-                    }
-#pragma unroll
-                    for (int u = 0; u < 8; u++) {
-                        const int v = 32 * (i0 + u) + lane;
-                        const int tok = v / RS::VPT;
-                        const int sdot = dot16(kv[u], qf[(i0 + u) % RS::QV], 0);
-#pragma unroll
-                        for (int t = 0; t < 8; t++) part[t] += (tok == t) ? sdot : 0;
-                    }
-                }
-                const int S = transpose_reduce8(part, lane);
-                const int64_t t0 = (int64_t)b * a.cap + 8 * j;
-                const float sc = lane_score(S, a.kscale + t0, my_tok, ntok);
-                const float m = warp_block_max(sc);
-                if (a.tok && (lane & 3) == 0 && my_tok < ntok) a.tok[bq * a.cap + 8 * j + my_tok] = sc;
-                if (lane == 0) {
-                    a.blk[bq * a.nblk_cap + j] = m;
-                    if (a.hist) atomicAdd(&a.hist[bq * kHistBins + hist_bin(m)], 1u);
-                }
-            }
-            __syncwarp();
-            if (lane == 0)
-                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(
-                                 scan_smem_u32(&empty_bar[warp]))
-                             : "memory");
-        }
-    }
-    __syncthreads();
-    if (*(volatile int *)&stop && threadIdx.x == 0) {
-        // the copies issued last on each stage land before the CTA's memory is released
-        for (int st = 0; st < SCAN_STAGES; st++) {
-            if (issued[st] == 0) continue;
-            const uint32_t fb = scan_smem_u32(&full_bar[st]);
-            uint64_t t0, now;
-            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-            do {
-                if (scan_try_wait(fb, (uint32_t)(issued[st] - 1) & 1)) break;
-                asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
-            } while (now - t0 < SCAN_WAIT_NS);
-        }
-    }
-}
-
-int index_scan_wait_flag(bool clear) { return read_device_flag(g_scan_error, clear); }
-
 __global__ void __launch_bounds__(256) index_full_generic_kernel(ScanArgs a) {
     grid_dep_wait();
     grid_dep_launch();
@@ -590,13 +398,6 @@ using namespace csa2;
 static int dispatch_scan(const ScanArgs &a, cudaStream_t s, bool pdl) {
     const int64_t items = (int64_t)a.B * a.Nq * a.nblk_cap;
     const int T = 256;
-    if (a.HD == SCAN_HD && aligned(a.k, 16) && aligned(a.q, 16)) {
-        static PerDevice smem_set;
-        if (!set_smem_limit_once(smem_set, index_full_tma_kernel, SCAN_SMEM)) return CSA2_ERR_CUDA;
-        const int64_t g = items < num_sms() ? items : num_sms();
-        return launch_kernel(pdl, index_full_tma_kernel, dim3((unsigned)(g < 1 ? 1 : g)),
-                             dim3(SCAN_THREADS), SCAN_SMEM, s, a);
-    }
     switch (a.HD) {
 #define CSA2_SCAN_CASE(HDV)                                                             \
     case HDV: {                                                                         \

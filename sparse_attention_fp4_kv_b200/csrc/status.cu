@@ -44,8 +44,8 @@ using namespace csa2;
 
 extern "C" int csa2_device_status(int clear) {
     if (cudaDeviceSynchronize() != cudaSuccess) return CSA2_ERR_CUDA;
-    const int flags[5] = {attn_tc_wait_flag(clear != 0), attn_rows_wait_flag(clear != 0),
-                          index_mma_wait_flag(clear != 0), index_scan_wait_flag(clear != 0),
+    const int flags[4] = {attn_tc_wait_flag(clear != 0), attn_rows_wait_flag(clear != 0),
+                          index_mma_wait_flag(clear != 0),
                           read_device_flag(g_selftest_error, clear != 0)};
     int any = 0;
     for (int f : flags) {

@@ -651,6 +651,159 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_row_hist_kernel(TopkArgs a
     topk_row_hist_body(a, blockIdx.x, ghist, topk_shared(smem_raw), st);
 }
 
+// ------------------------------------------------------------------ short rows, fast path
+// Rows of at most FT_N candidates (the 16,384 pooled tokens of a Reindex layer)
+// with k <= FT_K and the producer's first-digit histogram: one CTA of FT_THREADS
+// threads per row holds every candidate's 64-bit rank key (score order bits,
+// inverted index) and its position in shared memory.
+//  1. The histogram row (8 bins per thread, in registers) gives the threshold
+//     bin d by one block-wide suffix scan.
+//  2. One pass over the candidates (32 per thread, 16-byte loads): keys and
+//     positions to shared memory; the candidates above d go straight to a
+//     bitmap over the indices.
+//  3. When only part of bin d is taken, the remaining digits (10, 10, then the
+//     index bytes) are resolved over the keys in shared memory; every key is
+//     distinct, so the last digit decides.
+//  4. Emission in index order (= position order inside the step) through a
+//     block prefix count of the bitmap words; -1 padding; the histogram row is
+//     cleared for the next producer.
+constexpr int FT_THREADS = 512;
+constexpr int FT_N = 16384;
+constexpr int FT_K = 512;
+constexpr int FT_PER = FT_N / FT_THREADS;                       // 32 candidates per thread
+constexpr int FT_BPT = TK_HIST / FT_THREADS;                    // 8 histogram bins per thread
+constexpr size_t FT_SMEM = (size_t)FT_N * 8 + (size_t)FT_N * 4 + (size_t)(FT_N / 32) * 4 + 1024 * 4;
+
+__global__ void __launch_bounds__(FT_THREADS, 1) topk_fast_kernel(TopkArgs a, uint32_t *ghist) {
+    grid_dep_wait();
+    grid_dep_launch();
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __shared__ TopkState st;
+    uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);
+    int32_t *pos = reinterpret_cast<int32_t *>(smem_raw + (size_t)FT_N * 8);
+    uint32_t *bm = reinterpret_cast<uint32_t *>(smem_raw + (size_t)FT_N * 12);
+    uint32_t *hist = bm + FT_N / 32;  // 1024 bins for the refinement digits
+    const int64_t r = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int nv = (int)a.n;
+    if (a.n_valid) {
+        const int64_t v = a.n_valid[r];
+        nv = v < 0 ? 0 : (v < a.n ? (int)v : (int)a.n);
+    }
+    const int k = a.k;
+    // ---- 1. threshold bin from the histogram row (bins [8 tid, 8 tid + 8))
+    uint32_t hb[FT_BPT];
+    {
+        const uint4 *hp = reinterpret_cast<const uint4 *>(ghist + r * TK_HIST) + 2 * tid;
+        const uint4 h0 = hp[0], h1 = hp[1];
+        hb[0] = h0.x; hb[1] = h0.y; hb[2] = h0.z; hb[3] = h0.w;
+        hb[4] = h1.x; hb[5] = h1.y; hb[6] = h1.z; hb[7] = h1.w;
+    }
+    for (int i = tid; i < FT_N / 32; i += FT_THREADS) bm[i] = 0;
+    uint32_t local = 0;
+#pragma unroll
+    for (int j = 0; j < FT_BPT; j++) local += hb[j];
+    uint32_t x = local;  // inclusive suffix sum over the lanes of the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
+        if (lane + o < 32) x += y;
+    }
+    if (lane == 0) st.wsum[warp] = x;
+    if (tid == 0) st.digit = -1;
+    __syncthreads();
+    uint32_t above = x - local, total = 0;
+    for (int w = 0; w < FT_THREADS / 32; w++) {
+        total += st.wsum[w];
+        if (w > warp) above += st.wsum[w];
+    }
+    const bool all = total <= (uint32_t)k;
+#pragma unroll
+    for (int j = FT_BPT - 1; j >= 0; j--) {
+        if (!all && above < (uint32_t)k && above + hb[j] >= (uint32_t)k) {
+            st.digit = FT_BPT * tid + j;
+            st.above = above;
+            st.match = hb[j];
+        }
+        above += hb[j];
+    }
+    __syncthreads();
+    const int d = all ? -1 : st.digit;
+    // ---- 2. candidates: keys and positions to shared memory, those above d to the bitmap
+    const bool vec = ((r * a.n) % 4 == 0) && aligned16(a.score) &&
+                     (a.cand_pos == nullptr || aligned16(a.cand_pos));
+#pragma unroll
+    for (int u = 0; u < FT_PER / 4; u++) {
+        const int i0 = 4 * (u * FT_THREADS + tid);
+        uint64_t kq[4];
+        bool ok[4];
+        load_cand4(a, r, i0, nv, vec, kq, ok);
+#pragma unroll
+        for (int v = 0; v < 4; v++) {
+            const int i = i0 + v;
+            // rank key with the index (not the position) in the low bits: ties go to the
+            // lower index, which inside the step is the lower position
+            const uint64_t key = ok[v] ? ((kq[v] & 0xFFFFFFFF00000000ull) | (uint32_t)~(uint32_t)i) : 0ull;
+            keys[i] = key;
+            pos[i] = ok[v] ? rank_key_pos(kq[v]) : -1;
+            if (ok[v] && (all || (int)(key >> 52) > d)) atomicOr(&bm[i >> 5], 1u << (i & 31));
+        }
+    }
+    if (tid == 0) {
+        st.kk = all ? 0 : k - (int)st.above;
+        st.prefix = (uint64_t)(all ? 0 : d) << 52;
+        st.mask = (uint64_t)(TK_HIST - 1) << 52;
+    }
+    __syncthreads();
+    // ---- 3. the threshold bin: all of it, or the best kk of it by the remaining digits
+    if (!all) {
+        if (st.match != (uint32_t)st.kk) {
+            const int widths[6] = {10, 10, 8, 8, 8, 8};
+            int shift = 52;
+            for (int wi = 0; wi < 6; wi++) {
+                shift -= widths[wi];
+                const int NB = 1 << widths[wi];
+                smem_hist_pass<FT_THREADS>(keys, FT_N, hist, NB, shift, st.prefix, st.mask);
+                find_digit<FT_THREADS>(hist, NB, st.kk, st);
+                if (tid == 0) {
+                    st.kk -= (int)st.above;
+                    st.prefix |= (uint64_t)st.digit << shift;
+                    st.mask |= (uint64_t)(NB - 1) << shift;
+                }
+                __syncthreads();
+                if (st.match == (uint32_t)st.kk) break;
+            }
+        }
+        const uint64_t p = st.prefix, m = st.mask;
+        for (int i = tid; i < FT_N; i += FT_THREADS) {
+            const uint64_t key = keys[i];
+            if (key && (int)(key >> 52) == d && (key & m) >= p) atomicOr(&bm[i >> 5], 1u << (i & 31));
+        }
+        __syncthreads();
+    }
+    // ---- 4. emission in index order: thread t owns bitmap word t
+    const uint32_t word = bm[tid];
+    const int c = __popc(word);
+    int rank = block_excl_scan(c, st);
+    int32_t *out = a.out + r * a.k;
+    uint32_t bits = word;
+    while (bits) {
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (rank < k) out[rank] = pos[32 * tid + b];
+        rank++;
+    }
+    if (tid == FT_THREADS - 1) st.nsel = rank;
+    // clear the histogram row for the next producer
+    {
+        uint4 *hp = reinterpret_cast<uint4 *>(ghist + r * TK_HIST) + 2 * tid;
+        hp[0] = make_uint4(0, 0, 0, 0);
+        hp[1] = make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+    for (int i = st.nsel + tid; i < k; i += FT_THREADS) out[i] = -1;
+}
+
 // ------------------------------------------------------------------ pool + tokens
 // The decode Full layer's selection after its scan, in one CTA per row: the
 // pool (best P blocks, from the producer's histogram, as the two selection
@@ -861,6 +1014,11 @@ int launch_topk_from_hist(const float *score, const int32_t *cand_pos, const int
         return CSA2_ERR_CUDA;
     TopkArgs a{score, cand_pos, n_valid, R, n, k, out};
     TopkHistWs w = topk_hist_ws(ws, R, k);
+    if (n <= FT_N && k <= FT_K) {
+        static PerDevice fast_set;
+        if (!set_smem_limit_once(fast_set, topk_fast_kernel, FT_SMEM)) return CSA2_ERR_CUDA;
+        return launch_kernel(true, topk_fast_kernel, dim3(R), dim3(FT_THREADS), FT_SMEM, s, a, w.hist);
+    }
     if (n <= TS_MAX_N)
         return launch_kernel(true, topk_row_hist_kernel, dim3(R), dim3(TK_THREADS), TK_SMEM, s, a,
                              w.hist);

@@ -8,24 +8,30 @@
 // as E2M1 codes with one E4M3 scale per 16 channels; dequantization
 // e2m1 * e4m3 is exact in fp32.
 //
-// General kernel: one CTA per (query, head), 8 warps. Lane l of a warp holds
+// General kernel: one CTA per (query, head), 16 warps when a lane holds at
+// most 2 channel pairs (C <= 128), else 8. Lane l of a warp holds
 // channel pairs l, l + 32, ... (pair i = channels 2i, 2i + 1 = one FP4 byte).
 //  1. The query's selected positions go to shared memory.
-//  2. Logits: warp w takes keys w, w + 8, ..., GEN_U keys per round with all
-//     their loads issued before the first use; fp32 dot, shuffle reduce.
+//  2. Logits: warp w takes keys in runs of U (= 32 / NP, at least 2: as many
+//     as the registers hold) with all their loads issued before the first use;
+//     fp32 dot, shuffle reduce.
 //  3. Softmax statistics over the logits in shared memory.
 //  4. P V: warp w accumulates p_j row_j over the same keys in registers (the
-//     lane's channels), GEN_U keys per round; the 8 warps' sums are added in
-//     shared memory.
+//     lane's channels), U keys per round; the warps' sums are added in shared
+//     memory.
 // Used for shapes outside the tensor-core kernels' constraints (other channel
 // and head counts, e.g. 8 heads of 128 channels).
 #include "attention.cuh"
 
 namespace csa2 {
 
-constexpr int GEN_THREADS = 256;
-constexpr int GEN_WARPS = GEN_THREADS / 32;
-constexpr int GEN_U = 4;  // keys per warp per round
+// threads of the CTA for NP channel pairs per lane
+template <int NP>
+constexpr int gen_threads() { return NP <= 2 ? 512 : 256; }
+constexpr int GEN_MAX_WARPS = 16;
+// keys per warp per round with NP channel pairs per lane
+template <int NP>
+constexpr int gen_keys_per_round() { return NP >= 16 ? 2 : 32 / NP; }
 
 // Key j of query bq (j < K: selected row, else window row j - K) as NP channel
 // pairs per lane, dequantized; valid = false for an empty selected slot.
@@ -66,15 +72,18 @@ __device__ __forceinline__ void gen_load_key(const AttnArgs &a, int b, const int
 }
 
 template <int NP>
-__global__ void __launch_bounds__(GEN_THREADS) attn_general_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(gen_threads<NP>()) attn_general_kernel(AttnArgs a) {
+    constexpr int GEN_U = gen_keys_per_round<NP>();
+    constexpr int GEN_THREADS = gen_threads<NP>();
+    constexpr int GEN_WARPS = GEN_THREADS / 32;
     grid_dep_wait();
     grid_dep_launch();
     extern __shared__ float sm[];
     const int C = a.C, npairs = C / 2;
     float *lg = sm;                                    // [K + n_win] logits, then p
-    float *red = sm + a.K + a.n_win;                   // [GEN_WARPS][C] partial sums
+    float *red = sm + a.K + a.n_win;                   // [warps][C] partial sums
     int32_t *sel = reinterpret_cast<int32_t *>(red + GEN_WARPS * C);  // [K]
-    __shared__ float wred[GEN_WARPS];
+    __shared__ float wred[GEN_MAX_WARPS];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t bq = blockIdx.x / a.Hq;
     const int h = (int)(blockIdx.x % a.Hq);
@@ -185,18 +194,19 @@ static int launch_general(const AttnArgs &a, size_t smem, int64_t grid, cudaStre
     static PerDevice smem_set;
     if (smem > 48 * 1024 && !set_smem_limit_once(smem_set, attn_general_kernel<NP>, 227 * 1024))
         return CSA2_ERR_CUDA;
-    return launch_kernel(a.pdl, attn_general_kernel<NP>, dim3((unsigned)grid), dim3(GEN_THREADS), smem,
-                         s, a);
+    return launch_kernel(a.pdl, attn_general_kernel<NP>, dim3((unsigned)grid), dim3(gen_threads<NP>()),
+                         smem, s, a);
 }
 
 int launch_attn_general(const AttnArgs &a, cudaStream_t s) {
-    // logits [K + n_win], partial sums [8][C], selected positions [K]
-    const size_t smem = sizeof(float) * ((size_t)a.K + a.n_win + (size_t)GEN_WARPS * a.C) +
+    // logits [K + n_win], partial sums [warps][C], selected positions [K]
+    const int pairs_per_lane = (a.C / 2 + 31) / 32;  // 1 .. 16 (C <= 1024)
+    const int warps = pairs_per_lane <= 2 ? 16 : 8;
+    const size_t smem = sizeof(float) * ((size_t)a.K + a.n_win + (size_t)warps * a.C) +
                         sizeof(int32_t) * (size_t)a.K;
     if (smem > 227 * 1024) return CSA2_ERR_SHAPE;
     const int64_t grid = (int64_t)a.B * a.Nq * a.Hq;
     if (grid > INT32_MAX) return CSA2_ERR_SHAPE;
-    const int pairs_per_lane = (a.C / 2 + 31) / 32;  // 1 .. 16 (C <= 1024)
     if (pairs_per_lane <= 1) return launch_general<1>(a, smem, grid, s);
     if (pairs_per_lane <= 2) return launch_general<2>(a, smem, grid, s);
     if (pairs_per_lane <= 4) return launch_general<4>(a, smem, grid, s);

@@ -224,9 +224,16 @@ __global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
     const int64_t rows = (int64_t)a.B * a.Nq;
     const int64_t items = rows * L::HG;
     const int NL = lay.n;
-    // a cluster with at most one item keeps its dequantized selected rows for
-    // every layer; otherwise they are gathered again per item and layer
+    // A cluster with at most one item keeps its dequantized selected rows for
+    // every layer. With 64 heads per cluster a cluster owns whole rows, so it
+    // takes its rows one after another and runs all layers of a row before the
+    // next (row_major): one gather per row and no wait on other clusters.
+    // Otherwise (several head groups per row, more items than clusters) the
+    // cluster walks its items layer by layer and gathers per item and layer.
     const bool keep = (int64_t)gridDim.y >= items;
+    const bool row_major = !keep && L::HG == 1;
+    const int64_t n_mine =
+        (int64_t)blockIdx.y < items ? (items - 1 - (int64_t)blockIdx.y) / gridDim.y + 1 : 0;
     uint32_t ld_phase = 0;
     bool ld_pending = false;  // (thread 0) copies issued on bar_ld and not yet waited for
     bool ok = true;
@@ -261,11 +268,14 @@ __global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
         grid_dep_launch();
     }
 
-    // Layer by layer; within a layer the cluster walks (row, head group) items
-    // blockIdx.y, blockIdx.y + gridDim.y, ... (with keep, just one).
-    for (int l = 0; l < NL; l++) {
-        const bool gather = (l == 0) || !keep;
-        for (int64_t it = blockIdx.y; it < items; it += gridDim.y) {
+    // The cluster's (row, head group) items are blockIdx.y, blockIdx.y +
+    // gridDim.y, ... (with keep, just one). Step s is (layer, item) in layer
+    // order, or with row_major (item, layer) in item order.
+    for (int64_t step = 0; step < n_mine * NL; step++) {
+        const int l = row_major ? (int)(step % NL) : (int)(step / n_mine);
+        const int64_t it = (int64_t)blockIdx.y + (row_major ? step / NL : step % n_mine) * gridDim.y;
+        const bool gather = (l == 0) || (!keep && !row_major);
+        {
             const int64_t bq = it / L::HG;
             const int hg = (int)(it - bq * L::HG);
             const int b = (int)(bq / a.Nq);
@@ -301,8 +311,9 @@ __global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
                 slot_src[tid] = src;
             }
             // layer l of this row follows layer l - 1 of the same row: every
-            // CTA of the row has written its part of that output
-            if (l > 0 && tid == 0 && ok)
+            // CTA of the row has written its part of that output (with
+            // row_major this cluster wrote all of it, before its last barrier)
+            if (l > 0 && !row_major && tid == 0 && ok)
                 ok = wait_counter_bounded(lay.row_done + bq, lay.row_base + l * L::HG * CL, WAIT_NS);
             if (tid == 0)
                 mbar_expect_tx(bar_ld, (uint32_t)L::Q_BYTES + (uint32_t)nbox * 8u * SWA_BOX * 128u);
@@ -590,7 +601,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
             // next layer of the same row, which first waits until every CTA of
             // the row has written this layer's output (after its combine); after
             // the last item of the last layer nothing is shared any more.
-            const bool last = (l == NL - 1) && (it + (int64_t)gridDim.y >= items);
+            const bool last = step == n_mine * NL - 1;
             if (!keep && !last) cluster_sync();
         }
     }

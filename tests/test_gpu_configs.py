@@ -78,6 +78,9 @@ def _free():
     ("decoder_group1_b8_ctx128k", dict(B=5, ctx=3001)),
     ("decoder_group1_b8_ctx128k", dict(B=1, ctx=100)),
     ("reindex_group_b32_ctx256k", dict(B=3, ctx=50001)),
+    # more rows than resident clusters: clusters take whole rows (64 heads) one
+    # after another and run every layer of a row before the next
+    ("reindex_group_b32_ctx256k", dict(B=20, ctx=9001)),
     ("encoder_stack18_b4_ctx1m", dict(B=2, ctx=40007)),
     ("full_b1_ctx4k", dict(B=2, ctx=777)),
 ])

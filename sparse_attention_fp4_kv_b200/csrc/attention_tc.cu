@@ -530,7 +530,8 @@ __global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
                 }
             }
             __syncthreads();
-            __threadfence();
+            // the cluster barrier's release/acquire orders these stores for the
+            // cluster's CTAs, the only readers of the slot
             tc_fence_before();
             cluster_sync();  // all partial results of this item are in the slot
 

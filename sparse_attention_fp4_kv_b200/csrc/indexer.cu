@@ -262,18 +262,20 @@ __device__ __forceinline__ int64_t reindex_block(const ReindexArgs &a, int64_t b
     return t0;
 }
 
-// RI_ITEMS pooled blocks per warp (items w, w + nwarps, w + 2 nwarps, ...; nwarps = the
+// RI_ITEMS pooled blocks per warp (items w, w + nwarps, ...; nwarps = the
 // grid's warp count), 16 loads per lane in flight. Before its grid-dependency
 // wait a warp finds its blocks from the pool and the context lengths and pulls
 // the blocks' keys into L2, so that with dependent launches the key stream
 // overlaps the previous kernel (a latency-bound attention launch that leaves
-// HBM idle); with four blocks per warp the grid (256 CTAs at 4 rows) is small
-// enough to be resident beside that kernel and prefetch early. The pool comes
+// HBM idle). One block per warp measured best: with four per warp (a grid
+// small enough to be resident beside that kernel) the 134 MB of prefetches
+// overran L2 and the smaller grid streamed the rest more slowly (1M step
+// 1.725 against 1.681 ms, same B200). The pool comes
 // from the Full layer's selection, which is always two or more kernels earlier
 // (its attention follows it), and the keys and context lengths are not
 // written during a step; the layer's own indexer query, the only input the
 // previous kernel may produce, is read after the wait.
-constexpr int RI_ITEMS = 4;
+constexpr int RI_ITEMS = 1;
 
 template <int HD>
 __global__ void __launch_bounds__(256) index_reindex_kernel(ReindexArgs a) {

@@ -414,16 +414,32 @@ __global__ void __launch_bounds__(TC_THREADS) topk_compact_kernel(TopkArgs a, To
             else if (ok[v] && bin == d) tiem |= 1u << j;
         }
     }
+    // slots in the row's two lists: warp prefix sums, then one global atomic
+    // per list for the whole CTA (the 32 or more CTAs of a row share the counters)
     const int ns = __popc(selm), nt = __popc(tiem);
     const int is = warp_incl_scan(ns), it = warp_incl_scan(nt);
-    const int lane = threadIdx.x & 31;
-    int bs = 0, bt = 0;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __shared__ int wsel[TC_THREADS / 32], wtie[TC_THREADS / 32], cbase[2];
     if (lane == 31) {
-        if (is) bs = atomicAdd(ws.cnt + 2 * r, is);
-        if (it) bt = atomicAdd(ws.cnt + 2 * r + 1, it);
+        wsel[warp] = is;
+        wtie[warp] = it;
     }
-    bs = __shfl_sync(0xffffffffu, bs, 31) + is - ns;
-    bt = __shfl_sync(0xffffffffu, bt, 31) + it - nt;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int ts = 0, tt = 0;
+        for (int w = 0; w < TC_THREADS / 32; w++) {
+            const int a1 = wsel[w], a2 = wtie[w];
+            wsel[w] = ts;
+            wtie[w] = tt;
+            ts += a1;
+            tt += a2;
+        }
+        cbase[0] = ts ? atomicAdd(ws.cnt + 2 * r, ts) : 0;
+        cbase[1] = tt ? atomicAdd(ws.cnt + 2 * r + 1, tt) : 0;
+    }
+    __syncthreads();
+    int bs = cbase[0] + wsel[warp] + is - ns;
+    int bt = cbase[1] + wtie[warp] + it - nt;
 #pragma unroll
     for (int j = 0; j < TC_PER; j++) {
         if (selm & (1u << j)) {
@@ -654,16 +670,17 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_row_hist_kernel(TopkArgs a
 // ------------------------------------------------------------------ short rows, fast path
 // Rows of at most FT_N candidates (the 16,384 pooled tokens of a Reindex layer)
 // with k <= FT_K and the producer's first-digit histogram: one CTA of FT_THREADS
-// threads per row holds every candidate's 64-bit rank key (score order bits,
-// inverted index) and its position in shared memory.
+// threads per row holds every candidate's position, and the rank keys (score
+// order bits, inverted index) of the threshold bin's candidates, in shared
+// memory.
 //  1. The histogram row (8 bins per thread, in registers) gives the threshold
 //     bin d by one block-wide suffix scan.
-//  2. One pass over the candidates (32 per thread, 16-byte loads): keys and
-//     positions to shared memory; the candidates above d go straight to a
-//     bitmap over the indices.
+//  2. One pass over the candidates (32 per thread, all 16-byte loads issued
+//     first): positions to shared memory; the candidates above d go straight
+//     to a bitmap over the indices, the keys of bin d to a compact tie list.
 //  3. When only part of bin d is taken, the remaining digits (10, 10, then the
-//     index bytes) are resolved over the keys in shared memory; every key is
-//     distinct, so the last digit decides.
+//     index bytes) are resolved over the tie list; every key is distinct, so
+//     the last digit decides.
 //  4. Emission in index order (= position order inside the step) through a
 //     block prefix count of the bitmap words; -1 padding; the histogram row is
 //     cleared for the next producer.
@@ -710,7 +727,10 @@ __global__ void __launch_bounds__(FT_THREADS, 1) topk_fast_kernel(TopkArgs a, ui
         if (lane + o < 32) x += y;
     }
     if (lane == 0) st.wsum[warp] = x;
-    if (tid == 0) st.digit = -1;
+    if (tid == 0) {
+        st.digit = -1;
+        st.nbuf = 0;
+    }
     __syncthreads();
     uint32_t above = x - local, total = 0;
     for (int w = 0; w < FT_THREADS / 32; w++) {
@@ -729,41 +749,58 @@ __global__ void __launch_bounds__(FT_THREADS, 1) topk_fast_kernel(TopkArgs a, ui
     }
     __syncthreads();
     const int d = all ? -1 : st.digit;
-    // ---- 2. candidates: keys and positions to shared memory, those above d to the bitmap
+    // ---- 2. candidates: every load of the thread issued first (32 candidates,
+    // 16-byte loads), then the positions to shared memory, the candidates above
+    // d to the bitmap and the threshold bin's keys to a compact tie list (rank
+    // key with the index, not the position, in the low bits: ties go to the
+    // lower index, which inside the step is the lower position)
     const bool vec = ((r * a.n) % 4 == 0) && aligned16(a.score) &&
                      (a.cand_pos == nullptr || aligned16(a.cand_pos));
+    uint64_t kq[FT_PER / 4][4];
+    bool ok[FT_PER / 4][4];
 #pragma unroll
-    for (int u = 0; u < FT_PER / 4; u++) {
-        const int i0 = 4 * (u * FT_THREADS + tid);
-        uint64_t kq[4];
-        bool ok[4];
-        load_cand4(a, r, i0, nv, vec, kq, ok);
+    for (int u = 0; u < FT_PER / 4; u++) load_cand4(a, r, 4 * (u * FT_THREADS + tid), nv, vec, kq[u], ok[u]);
+    int nt = 0;
+#pragma unroll
+    for (int u = 0; u < FT_PER / 4; u++)
 #pragma unroll
         for (int v = 0; v < 4; v++) {
-            const int i = i0 + v;
-            // rank key with the index (not the position) in the low bits: ties go to the
-            // lower index, which inside the step is the lower position
-            const uint64_t key = ok[v] ? ((kq[v] & 0xFFFFFFFF00000000ull) | (uint32_t)~(uint32_t)i) : 0ull;
-            keys[i] = key;
-            pos[i] = ok[v] ? rank_key_pos(kq[v]) : -1;
-            if (ok[v] && (all || (int)(key >> 52) > d)) atomicOr(&bm[i >> 5], 1u << (i & 31));
+            const int i = 4 * (u * FT_THREADS + tid) + v;
+            pos[i] = ok[u][v] ? rank_key_pos(kq[u][v]) : -1;
+            const int bin = (int)(kq[u][v] >> 52);
+            if (ok[u][v] && (all || bin > d)) atomicOr(&bm[i >> 5], 1u << (i & 31));
+            nt += (ok[u][v] && !all && bin == d) ? 1 : 0;
         }
-    }
+    // one shared atomic per warp for the tie list
+    const int nt_incl = warp_incl_scan(nt);
+    int tbase = 0;
+    if (lane == 31 && nt_incl) tbase = atomicAdd(&st.nbuf, nt_incl);
+    tbase = __shfl_sync(0xffffffffu, tbase, 31) + nt_incl - nt;
+#pragma unroll
+    for (int u = 0; u < FT_PER / 4; u++)
+#pragma unroll
+        for (int v = 0; v < 4; v++) {
+            const int i = 4 * (u * FT_THREADS + tid) + v;
+            if (ok[u][v] && !all && (int)(kq[u][v] >> 52) == d)
+                keys[tbase++] = (kq[u][v] & 0xFFFFFFFF00000000ull) | (uint32_t)~(uint32_t)i;
+        }
     if (tid == 0) {
         st.kk = all ? 0 : k - (int)st.above;
         st.prefix = (uint64_t)(all ? 0 : d) << 52;
         st.mask = (uint64_t)(TK_HIST - 1) << 52;
     }
     __syncthreads();
-    // ---- 3. the threshold bin: all of it, or the best kk of it by the remaining digits
+    // ---- 3. the threshold bin (its keys in the tie list): all of it, or its
+    // best kk by the remaining digits
     if (!all) {
-        if (st.match != (uint32_t)st.kk) {
+        const int ntie = st.nbuf;
+        if (ntie != st.kk) {
             const int widths[6] = {10, 10, 8, 8, 8, 8};
             int shift = 52;
             for (int wi = 0; wi < 6; wi++) {
                 shift -= widths[wi];
                 const int NB = 1 << widths[wi];
-                smem_hist_pass<FT_THREADS>(keys, FT_N, hist, NB, shift, st.prefix, st.mask);
+                smem_hist_pass<FT_THREADS>(keys, ntie, hist, NB, shift, st.prefix, st.mask);
                 find_digit<FT_THREADS>(hist, NB, st.kk, st);
                 if (tid == 0) {
                     st.kk -= (int)st.above;
@@ -775,9 +812,12 @@ __global__ void __launch_bounds__(FT_THREADS, 1) topk_fast_kernel(TopkArgs a, ui
             }
         }
         const uint64_t p = st.prefix, m = st.mask;
-        for (int i = tid; i < FT_N; i += FT_THREADS) {
+        for (int i = tid; i < ntie; i += FT_THREADS) {
             const uint64_t key = keys[i];
-            if (key && (int)(key >> 52) == d && (key & m) >= p) atomicOr(&bm[i >> 5], 1u << (i & 31));
+            if ((key & m) >= p) {
+                const int idx = (int)~(uint32_t)key;
+                atomicOr(&bm[idx >> 5], 1u << (idx & 31));
+            }
         }
         __syncthreads();
     }
@@ -842,10 +882,33 @@ __device__ void pool_tokens_select(const TopkArgs &a, const PoolTokArgs &pa, int
     if (V > pa.cap) V = pa.cap;
     const int32_t *pool = a.out + r * (int64_t)P;
     const float *tok = pa.tok + r * pa.cap;
-    for (int i = threadIdx.x; i < n; i += TK_THREADS) {
-        const int32_t blk = pool[i >> 3];
-        const int64_t pos = 8 * (int64_t)blk + (i & 7);
-        keys[i] = (blk >= 0 && pos < V) ? rank_key(tok[pos], (int32_t)pos) : 0ull;
+    // thread t takes pool slots t, t + TK_THREADS, ...: its pool entries first,
+    // then all its tokens' score loads, then the keys
+    constexpr int SPT = PT_MAX / kBlockTokens / TK_THREADS;  // pool slots per thread
+    static_assert(SPT * kBlockTokens * TK_THREADS == PT_MAX, "gather split");
+    int32_t blk[SPT];
+#pragma unroll
+    for (int u = 0; u < SPT; u++) {
+        const int sl = threadIdx.x + u * TK_THREADS;
+        blk[u] = sl < P ? pool[sl] : -1;
+    }
+    float sc[SPT][kBlockTokens];
+#pragma unroll
+    for (int u = 0; u < SPT; u++)
+#pragma unroll
+        for (int t = 0; t < kBlockTokens; t++) {
+            const int64_t p = 8 * (int64_t)blk[u] + t;
+            sc[u][t] = (blk[u] >= 0 && p < V) ? tok[p] : 0.0f;
+        }
+#pragma unroll
+    for (int u = 0; u < SPT; u++) {
+        const int sl = threadIdx.x + u * TK_THREADS;
+        if (sl >= P) continue;
+#pragma unroll
+        for (int t = 0; t < kBlockTokens; t++) {
+            const int64_t p = 8 * (int64_t)blk[u] + t;
+            keys[sl * kBlockTokens + t] = (blk[u] >= 0 && p < V) ? rank_key(sc[u][t], (int32_t)p) : 0ull;
+        }
     }
     for (int b = threadIdx.x; b < TK_HIST; b += TK_THREADS) sh.hist[b] = 0;
     __syncthreads();
@@ -863,14 +926,32 @@ __device__ void pool_tokens_select(const TopkArgs &a, const PoolTokArgs &pa, int
         st.mask = (uint64_t)(TK_HIST - 1) << 52;
     }
     __syncthreads();
-    if (!all && st.match != (uint32_t)st.kk) {
+    // The threshold bin's keys are resolved over a compact list in the sel
+    // region when they fit there (with the index, which orders like the
+    // position, in their low bits), else over the whole key array.
+    uint64_t *ties = reinterpret_cast<uint64_t *>(sh.sel);
+    const bool partial = !all && st.match != (uint32_t)st.kk;
+    const bool listed = partial && st.match <= (uint32_t)(TK_MAXK / 2);
+    if (listed) {
+        if (threadIdx.x == 0) st.nbuf = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < n; i += TK_THREADS) {
+            const uint64_t key = keys[i];
+            if (key && (key >> 52) == d)
+                ties[atomicAdd(&st.nbuf, 1)] = (key & 0xFFFFFFFF00000000ull) | (uint32_t)~(uint32_t)i;
+        }
+        __syncthreads();
+    }
+    if (partial) {
         // only part of the threshold bin is taken: further digits over its keys
+        const uint64_t *tk = listed ? ties : keys;
+        const int ntk = listed ? st.nbuf : n;
         const int widths[6] = {10, 10, 8, 8, 8, 8};
         int shift = 52;
         for (int wi = 0; wi < 6; wi++) {
             shift -= widths[wi];
             const int NB = 1 << widths[wi];
-            smem_hist_pass(keys, n, sh.hist, NB, shift, st.prefix, st.mask);
+            smem_hist_pass(tk, ntk, sh.hist, NB, shift, st.prefix, st.mask);
             find_digit(sh.hist, NB, st.kk, st);
             if (threadIdx.x == 0) {
                 st.kk -= (int)st.above;
@@ -889,8 +970,18 @@ __device__ void pool_tokens_select(const TopkArgs &a, const PoolTokArgs &pa, int
     __syncthreads();
     for (int i = threadIdx.x; i < n; i += TK_THREADS) {
         const uint64_t key = keys[i];
-        const bool take = key && (all || (key >> 52) > d || ((key & m) >= p && (key >> 52) == d));
+        const bool take =
+            key && (all || (key >> 52) > d || (!listed && (key & m) >= p && (key >> 52) == d));
         if (take) atomicOr(&bm[i >> 5], 1u << (i & 31));
+    }
+    if (listed) {
+        for (int i = threadIdx.x; i < st.nbuf; i += TK_THREADS) {
+            const uint64_t key = ties[i];
+            if ((key & m) >= p) {
+                const int idx = (int)~(uint32_t)key;
+                atomicOr(&bm[idx >> 5], 1u << (idx & 31));
+            }
+        }
     }
     __syncthreads();
     const int per = (nwords + TK_THREADS - 1) / TK_THREADS;

@@ -402,6 +402,7 @@ def run_csa2(args, name, rank, world, local_rank):
     # ---- the same step captured once as a CUDA graph and replayed K times (the
     # kernels keep their programmatic dependencies as graph edges)
     graph_ms, graph_note = None, None
+    graph = None
     try:
         graph = wl.capture_step_graph()
         for _ in range(3):
@@ -466,11 +467,77 @@ def run_csa2(args, name, rank, world, local_rank):
                                           f"warm-up ({t_seq:.2f} s per sequence); rate of the "
                                           f"{w.B}-sequence batch at that time per sequence; OpenMP "
                                           f"oracle build, {threads} threads"}
+    if world == 1 and not args.no_extra_configs and name == DEFAULT_WORKLOAD:
+        del graph, wl
+        torch.cuda.empty_cache()
+        line["configs"] = _extra_configs(dev)
+        status = status or binding.device_status()
+        line["device_status"] = status
     if rank == 0:
         print(json.dumps(line), flush=True)
     if status != 0:
         raise SystemExit(f"a kernel gave up a bounded wait (csa2_device_status = {status}): "
                          "the step's outputs are invalid")
+
+
+# The metric is quoted for 128K-1M contexts: the other decode workloads of that
+# range and the chunked prefill are measured in the same run (one GPU), each
+# after the previous one's buffers are freed.
+EXTRA_CONFIGS = ("decoder_group1_b8_ctx128k", "reindex_group_b32_ctx256k", "prefill_4096_at_64k")
+EXTRA_STEPS, EXTRA_WARMUP = 30, 3
+
+
+def _extra_configs(dev):
+    from sparse_attention_fp4_kv_b200 import synth
+    from sparse_attention_fp4_kv_b200.workload import DecodeWorkload, PrefillWorkload
+    peak, peak_kind = _peaks()
+    out = {}
+    for name in EXTRA_CONFIGS:
+        w = synth.WORKLOADS[name]
+        stream = torch.cuda.current_stream()
+        if synth_n_new(name) > 1:
+            pw = PrefillWorkload(w, dev)
+            for _ in range(EXTRA_WARMUP):
+                pw.step()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(EXTRA_STEPS // 6):
+                pw.step()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / (EXTRA_STEPS // 6)
+            out[name] = {"metric": "chunked-prefill tokens/s", "value": w.B * w.n_new / (ms / 1e3),
+                         "unit": "tokens/s", "ms_per_step": ms, "steps": EXTRA_STEPS // 6,
+                         "gpu_launches_per_step": pw.launches_per_step()}
+            del pw
+        else:
+            wl = DecodeWorkload(w, dev)
+            for _ in range(EXTRA_WARMUP):
+                wl.step()
+            torch.cuda.synchronize()
+            g = wl.capture_step_graph()
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(EXTRA_STEPS):
+                g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / EXTRA_STEPS
+            nbytes = wl.step_bytes()["total"]
+            out[name] = {"metric": METRIC, "value": w.n_layers / (ms / 1e3), "unit": UNIT,
+                         "ms_per_step": ms, "steps": EXTRA_STEPS, "timing": "CUDA graph replays",
+                         "step_hbm": {"algorithmic_bytes": nbytes,
+                                      "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
+                                      "frac": nbytes / (ms / 1e3) / 1e9 / peak, "peak_kind": peak_kind},
+                         "gpu_launches_per_step": wl.launches_per_step()}
+            del g, wl
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
 
 
 def _e2e(wl, args, stream, world, local_rank):
@@ -557,6 +624,8 @@ def main():
     ap.add_argument("--impl", default="csa2", choices=["csa2", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-configs", action="store_true",
+                    help="skip the other decode workloads and the prefill in the line's 'configs'")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -675,9 +675,9 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_row_hist_kernel(TopkArgs a
 // memory.
 //  1. The histogram row (8 bins per thread, in registers) gives the threshold
 //     bin d by one block-wide suffix scan.
-//  2. One pass over the candidates (32 per thread, all 16-byte loads issued
-//     first): positions to shared memory; the candidates above d go straight
-//     to a bitmap over the indices, the keys of bin d to a compact tie list.
+//  2. One pass over the candidates (32 per thread, 16-byte loads): positions
+//     to shared memory; the candidates above d go straight to a bitmap over
+//     the indices, the keys of bin d to a compact tie list.
 //  3. When only part of bin d is taken, the remaining digits (10, 10, then the
 //     index bytes) are resolved over the tie list; every key is distinct, so
 //     the last digit decides.
@@ -749,41 +749,29 @@ __global__ void __launch_bounds__(FT_THREADS, 1) topk_fast_kernel(TopkArgs a, ui
     }
     __syncthreads();
     const int d = all ? -1 : st.digit;
-    // ---- 2. candidates: every load of the thread issued first (32 candidates,
-    // 16-byte loads), then the positions to shared memory, the candidates above
-    // d to the bitmap and the threshold bin's keys to a compact tie list (rank
-    // key with the index, not the position, in the low bits: ties go to the
-    // lower index, which inside the step is the lower position)
+    // ---- 2. candidates (32 per thread, 16-byte loads): the positions to shared
+    // memory, the candidates above d to the bitmap and the threshold bin's keys
+    // to a compact tie list (rank key with the index, not the position, in the
+    // low bits: ties go to the lower index, which inside the step is the lower
+    // position)
     const bool vec = ((r * a.n) % 4 == 0) && aligned16(a.score) &&
                      (a.cand_pos == nullptr || aligned16(a.cand_pos));
-    uint64_t kq[FT_PER / 4][4];
-    bool ok[FT_PER / 4][4];
 #pragma unroll
-    for (int u = 0; u < FT_PER / 4; u++) load_cand4(a, r, 4 * (u * FT_THREADS + tid), nv, vec, kq[u], ok[u]);
-    int nt = 0;
-#pragma unroll
-    for (int u = 0; u < FT_PER / 4; u++)
-#pragma unroll
-        for (int v = 0; v < 4; v++) {
-            const int i = 4 * (u * FT_THREADS + tid) + v;
-            pos[i] = ok[u][v] ? rank_key_pos(kq[u][v]) : -1;
-            const int bin = (int)(kq[u][v] >> 52);
-            if (ok[u][v] && (all || bin > d)) atomicOr(&bm[i >> 5], 1u << (i & 31));
-            nt += (ok[u][v] && !all && bin == d) ? 1 : 0;
-        }
-    // one shared atomic per warp for the tie list
-    const int nt_incl = warp_incl_scan(nt);
-    int tbase = 0;
-    if (lane == 31 && nt_incl) tbase = atomicAdd(&st.nbuf, nt_incl);
-    tbase = __shfl_sync(0xffffffffu, tbase, 31) + nt_incl - nt;
-#pragma unroll
-    for (int u = 0; u < FT_PER / 4; u++)
+    for (int u = 0; u < FT_PER / 4; u++) {
+        const int i0 = 4 * (u * FT_THREADS + tid);
+        uint64_t kq[4];
+        bool ok[4];
+        load_cand4(a, r, i0, nv, vec, kq, ok);
 #pragma unroll
         for (int v = 0; v < 4; v++) {
-            const int i = 4 * (u * FT_THREADS + tid) + v;
-            if (ok[u][v] && !all && (int)(kq[u][v] >> 52) == d)
-                keys[tbase++] = (kq[u][v] & 0xFFFFFFFF00000000ull) | (uint32_t)~(uint32_t)i;
+            const int i = i0 + v;
+            pos[i] = ok[v] ? rank_key_pos(kq[v]) : -1;
+            const int bin = (int)(kq[v] >> 52);
+            if (ok[v] && (all || bin > d)) atomicOr(&bm[i >> 5], 1u << (i & 31));
+            else if (ok[v] && bin == d)
+                keys[atomicAdd(&st.nbuf, 1)] = (kq[v] & 0xFFFFFFFF00000000ull) | (uint32_t)~(uint32_t)i;
         }
+    }
     if (tid == 0) {
         st.kk = all ? 0 : k - (int)st.above;
         st.prefix = (uint64_t)(all ? 0 : d) << 52;
@@ -882,33 +870,10 @@ __device__ void pool_tokens_select(const TopkArgs &a, const PoolTokArgs &pa, int
     if (V > pa.cap) V = pa.cap;
     const int32_t *pool = a.out + r * (int64_t)P;
     const float *tok = pa.tok + r * pa.cap;
-    // thread t takes pool slots t, t + TK_THREADS, ...: its pool entries first,
-    // then all its tokens' score loads, then the keys
-    constexpr int SPT = PT_MAX / kBlockTokens / TK_THREADS;  // pool slots per thread
-    static_assert(SPT * kBlockTokens * TK_THREADS == PT_MAX, "gather split");
-    int32_t blk[SPT];
-#pragma unroll
-    for (int u = 0; u < SPT; u++) {
-        const int sl = threadIdx.x + u * TK_THREADS;
-        blk[u] = sl < P ? pool[sl] : -1;
-    }
-    float sc[SPT][kBlockTokens];
-#pragma unroll
-    for (int u = 0; u < SPT; u++)
-#pragma unroll
-        for (int t = 0; t < kBlockTokens; t++) {
-            const int64_t p = 8 * (int64_t)blk[u] + t;
-            sc[u][t] = (blk[u] >= 0 && p < V) ? tok[p] : 0.0f;
-        }
-#pragma unroll
-    for (int u = 0; u < SPT; u++) {
-        const int sl = threadIdx.x + u * TK_THREADS;
-        if (sl >= P) continue;
-#pragma unroll
-        for (int t = 0; t < kBlockTokens; t++) {
-            const int64_t p = 8 * (int64_t)blk[u] + t;
-            keys[sl * kBlockTokens + t] = (blk[u] >= 0 && p < V) ? rank_key(sc[u][t], (int32_t)p) : 0ull;
-        }
+    for (int i = threadIdx.x; i < n; i += TK_THREADS) {
+        const int32_t blk = pool[i >> 3];
+        const int64_t pos = 8 * (int64_t)blk + (i & 7);
+        keys[i] = (blk >= 0 && pos < V) ? rank_key(tok[pos], (int32_t)pos) : 0ull;
     }
     for (int b = threadIdx.x; b < TK_HIST; b += TK_THREADS) sh.hist[b] = 0;
     __syncthreads();

@@ -262,21 +262,18 @@ __device__ __forceinline__ int64_t reindex_block(const ReindexArgs &a, int64_t b
     return t0;
 }
 
-// RI_ITEMS pooled blocks per warp (items w, w + nwarps, ...; nwarps = the
-// grid's warp count), 16 loads per lane in flight. Before its grid-dependency
-// wait a warp finds its blocks from the pool and the context lengths and pulls
-// the blocks' keys into L2, so that with dependent launches the key stream
-// overlaps the previous kernel (a latency-bound attention launch that leaves
-// HBM idle). One block per warp measured best: with four per warp (a grid
-// small enough to be resident beside that kernel) the 134 MB of prefetches
-// overran L2 and the smaller grid streamed the rest more slowly (1M step
-// 1.725 against 1.681 ms, same B200). The pool comes
-// from the Full layer's selection, which is always two or more kernels earlier
-// (its attention follows it), and the keys and context lengths are not
-// written during a step; the layer's own indexer query, the only input the
-// previous kernel may produce, is read after the wait.
-constexpr int RI_ITEMS = 1;
-
+// A grid of warps walks the pooled blocks (items w, w + nwarps, ...; nwarps =
+// the grid's warp count), 16 loads per lane in flight. Before its
+// grid-dependency wait a warp finds its first block from the pool and the
+// context lengths and pulls the block's keys into L2, so that with dependent
+// launches the key stream overlaps the previous kernel (a latency-bound
+// attention launch that leaves HBM idle). The pool comes from the Full layer's
+// selection, which is always two or more kernels earlier (its attention
+// follows it), and the keys and context lengths are not written during a
+// step; the layer's own indexer query, the only input the previous kernel may
+// produce, is read after the wait. (Four blocks per warp, all prefetched,
+// measured slower: 1M step 1.725 against 1.681 ms, same B200, the prefetches
+// overran L2.)
 template <int HD>
 __global__ void __launch_bounds__(256) index_reindex_kernel(ReindexArgs a) {
     using RS = RowShape<HD>;
@@ -284,49 +281,48 @@ __global__ void __launch_bounds__(256) index_reindex_kernel(ReindexArgs a) {
     const int64_t w0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int64_t items = (int64_t)a.B * a.Nq * a.P;
-    int64_t bq[RI_ITEMS], t0[RI_ITEMS];
-    int s[RI_ITEMS], b[RI_ITEMS], ntok[RI_ITEMS];
-#pragma unroll
-    for (int u = 0; u < RI_ITEMS; u++) {
-        const int64_t it = w0 + u * nwarps;
-        bq[u] = 0;
-        t0[u] = -1;
-        s[u] = b[u] = ntok[u] = 0;
-        if (it < items) {
-            bq[u] = it / a.P;
-            s[u] = (int)(it - bq[u] * a.P);
-            b[u] = (int)(bq[u] / a.Nq);
-            const int i = (int)(bq[u] % a.Nq);
-            int64_t V = visible_len(a.ctx_len, a.q_pos, b[u], i, a.Nq);
-            if (V > a.cap) V = a.cap;
-            t0[u] = reindex_block(a, bq[u], s[u], V, ntok[u]);
-            if (t0[u] >= 0 && lane == 0)
-                bulk_prefetch_l2(a.k + ((int64_t)b[u] * a.cap + t0[u]) * HD, (uint32_t)(ntok[u] * HD));
-        }
+    // item -> (query row, pool slot, sequence, first token (-1: empty), tokens)
+    auto locate = [&](int64_t it, int64_t &bq, int &s, int &b, int64_t &t0, int &ntok) {
+        bq = it / a.P;
+        s = (int)(it - bq * a.P);
+        b = (int)(bq / a.Nq);
+        int64_t V = visible_len(a.ctx_len, a.q_pos, b, (int)(bq % a.Nq), a.Nq);
+        if (V > a.cap) V = a.cap;
+        t0 = reindex_block(a, bq, s, V, ntok);
+    };
+    int64_t bq = 0, t0 = -1;
+    int s = 0, b = 0, ntok = 0;
+    if (w0 < items) {
+        locate(w0, bq, s, b, t0, ntok);
+        if (t0 >= 0 && lane == 0)
+            bulk_prefetch_l2(a.k + ((int64_t)b * a.cap + t0) * HD, (uint32_t)(ntok * HD));
     }
     grid_dep_wait();
     grid_dep_launch();
     const int my_tok = reduce_token_of_lane(lane);
-#pragma unroll
-    for (int u = 0; u < RI_ITEMS; u++) {
-        if (w0 + u * nwarps >= items) break;
-        const int64_t slot = bq[u] * 8 * (int64_t)a.P + 8 * (int64_t)s[u];
-        if (t0[u] < 0) {
+    int64_t cur_bq = -1;
+    uint4 qf[RS::QV];
+    for (int64_t it = w0; it < items; it += nwarps) {
+        if (it != w0) locate(it, bq, s, b, t0, ntok);
+        const int64_t slot = bq * 8 * (int64_t)a.P + 8 * (int64_t)s;
+        if (t0 < 0) {
             if (lane < 8) {
                 a.ppos[slot + lane] = -1;
                 a.pscore[slot + lane] = 0.0f;
             }
             continue;
         }
-        uint4 qf[RS::QV];
-        load_qfrag<HD>(a.q + bq[u] * HD, qf, lane);
-        const int64_t row0 = (int64_t)b[u] * a.cap + t0[u];
-        const int S = block_dots<HD, 16>(a.k + row0 * HD, qf, lane, ntok[u]);
-        const float sc = lane_score(S, a.kscale + row0, my_tok, ntok[u]);
+        if (bq != cur_bq) {
+            cur_bq = bq;
+            load_qfrag<HD>(a.q + bq * HD, qf, lane);
+        }
+        const int64_t row0 = (int64_t)b * a.cap + t0;
+        const int S = block_dots<HD, 16>(a.k + row0 * HD, qf, lane, ntok);
+        const float sc = lane_score(S, a.kscale + row0, my_tok, ntok);
         if ((lane & 3) == 0) {
-            a.ppos[slot + my_tok] = my_tok < ntok[u] ? (int32_t)(t0[u] + my_tok) : -1;
-            a.pscore[slot + my_tok] = my_tok < ntok[u] ? sc : 0.0f;
-            if (a.hist && my_tok < ntok[u]) atomicAdd(&a.hist[bq[u] * kHistBins + hist_bin(sc)], 1u);
+            a.ppos[slot + my_tok] = my_tok < ntok ? (int32_t)(t0 + my_tok) : -1;
+            a.pscore[slot + my_tok] = my_tok < ntok ? sc : 0.0f;
+            if (a.hist && my_tok < ntok) atomicAdd(&a.hist[bq * kHistBins + hist_bin(sc)], 1u);
         }
     }
 }
@@ -440,8 +436,7 @@ static int dispatch_reindex(const ReindexArgs &a, cudaStream_t s, bool pdl) {
     switch (a.HD) {
 #define CSA2_RI_CASE(HDV)                                                               \
     case HDV: {                                                                         \
-        const int64_t g = (items + RI_ITEMS * (T / 32) - 1) / (RI_ITEMS * (T / 32));    \
-        if (g > INT32_MAX) return CSA2_ERR_SHAPE;                                       \
+        const int g = persistent_grid(index_reindex_kernel<HDV>, T, items);             \
         return launch_kernel(pdl, index_reindex_kernel<HDV>, dim3((unsigned)g), dim3(T), 0, s, \
                              a);                                                        \
     }

@@ -271,9 +271,10 @@ __device__ __forceinline__ int64_t reindex_block(const ReindexArgs &a, int64_t b
 // selection, which is always two or more kernels earlier (its attention
 // follows it), and the keys and context lengths are not written during a
 // step; the layer's own indexer query, the only input the previous kernel may
-// produce, is read after the wait. (Four blocks per warp, all prefetched,
-// measured slower: 1M step 1.725 against 1.681 ms, same B200, the prefetches
-// overran L2.)
+// produce, is read after the wait. The launch has one warp per block (the
+// loop runs once): four blocks per warp, all prefetched, measured 1.725
+// against 1.681 ms per 1M step (the prefetches overran L2), and a persistent
+// grid of one resident wave 1.697 against 1.664 ms (same B200 each time).
 template <int HD>
 __global__ void __launch_bounds__(256) index_reindex_kernel(ReindexArgs a) {
     using RS = RowShape<HD>;
@@ -436,7 +437,7 @@ static int dispatch_reindex(const ReindexArgs &a, cudaStream_t s, bool pdl) {
     switch (a.HD) {
 #define CSA2_RI_CASE(HDV)                                                               \
     case HDV: {                                                                         \
-        const int g = persistent_grid(index_reindex_kernel<HDV>, T, items);             \
+        const int g = (int)((items + T / 32 - 1) / (T / 32));                            \
         return launch_kernel(pdl, index_reindex_kernel<HDV>, dim3((unsigned)g), dim3(T), 0, s, \
                              a);                                                        \
     }

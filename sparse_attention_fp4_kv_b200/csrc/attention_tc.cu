@@ -591,11 +591,8 @@ __global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
             }
             // this CTA's part of the row's layer-l output is written
             if (NL > 1) {
-                __syncthreads();
-                if (tid == 0) {
-                    __threadfence();
-                    red_release_gpu_add(lay.row_done + bq, 1);
-                }
+                __syncthreads();  // every thread's output stores precede the release below
+                if (tid == 0) red_release_gpu_add(lay.row_done + bq, 1);
             }
             // The slot, the tiles and TMEM are free for the next item once every
             // CTA of the cluster has combined. With keep, the next use is the

@@ -842,6 +842,10 @@ __global__ void __launch_bounds__(FT_THREADS, 1) topk_fast_kernel(TopkArgs a, ui
 // bin's keys, then emission in index order (= ascending positions) through a
 // bitmap. An empty slot holds key 0, which no finite score produces.
 constexpr int PT_MAX = kPoolBlocks * kBlockTokens;                  // 16,384 pooled tokens
+// Rows of up to this many blocks take the one-kernel path (one CTA reads the
+// row in passes of TK_THREADS x TS_PER candidates; the emission bitmap of n bits
+// fits in the tie buffer); longer rows are compacted by many CTAs first.
+constexpr int64_t PT_ONE_CTA_MAX_N = TF_MAX_N;
 constexpr size_t PT_SMEM = TK_HIST * 4 + TK_MAXK * 4 + (size_t)PT_MAX * 8;  // 160 KB
 static_assert((size_t)PT_MAX * 8 >= (size_t)TK_BUF * 8, "the key array holds the tie buffer");
 
@@ -1101,7 +1105,7 @@ int launch_pool_and_tokens(const float *blk, const int32_t *n_blk, int R, int64_
     TopkArgs a{blk, nullptr, n_blk, R, nblk, P, pool};
     PoolTokArgs pa{tok, ctx_len, cap, ktop, top};
     TopkHistWs w = topk_hist_ws(ws, R, P);
-    if (nblk <= TS_MAX_N)
+    if (nblk <= PT_ONE_CTA_MAX_N)
         return launch_kernel(true, topk_row_pool_tokens_kernel, dim3(R), dim3(TK_THREADS), PT_SMEM, s,
                              a, w.hist, pa);
     const int64_t slices = (nblk + TC_SLICE - 1) / TC_SLICE;

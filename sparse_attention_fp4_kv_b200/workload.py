@@ -140,7 +140,9 @@ class DecodeWorkload:
 
     def launches_per_step(self) -> int:
         """libcsa2 kernels one step launches: the append, then per Full layer
-        the scan and one selection of the pool and its top tokens; per Reindex
+        the scan and one selection of the pool and its top tokens (a
+        compaction kernel before it for rows of more than POOL_ONE_KERNEL_MAX
+        blocks); per Reindex
         layer the rescoring and the token selection. Attention: one
         kernel per layer group (a Full or Reindex layer and the Reuse layers
         after it, at most ATTN_GROUP_MAX layers per kernel) where the
@@ -157,7 +159,8 @@ class DecodeWorkload:
         n = 1
         run = 0  # layers in the current attention launch
         for m in self.modes:
-            n += {synth.FULL: 1 + sel(nblk), synth.REINDEX: 1 + sel(pooled), synth.REUSE: 0}[m]
+            full_sel = 1 if nblk <= csa2.POOL_ONE_KERNEL_MAX else 2
+            n += {synth.FULL: 1 + full_sel, synth.REINDEX: 1 + sel(pooled), synth.REUSE: 0}[m]
             if grouped and m == synth.REUSE and 0 < run < csa2.ATTN_GROUP_MAX:
                 run += 1
             else:

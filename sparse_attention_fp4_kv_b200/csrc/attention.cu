@@ -8,210 +8,363 @@
 // as E2M1 codes with one E4M3 scale per 16 channels; dequantization
 // e2m1 * e4m3 is exact in fp32.
 //
-// General kernel: one CTA per (query, head), 16 warps when a lane holds at
-// most 2 channel pairs (C <= 128), else 8. Lane l of a warp holds
-// channel pairs l, l + 32, ... (pair i = channels 2i, 2i + 1 = one FP4 byte).
-//  1. The query's selected positions go to shared memory.
-//  2. Logits: warp w takes keys in runs of U (= 32 / NP, at least 2: as many
-//     as the registers hold) with all their loads issued before the first use;
-//     fp32 dot, shuffle reduce.
-//  3. Softmax statistics over the logits in shared memory.
-//  4. P V: warp w accumulates p_j row_j over the same keys in registers (the
-//     lane's channels), U keys per round; the warps' sums are added in shared
-//     memory.
-// Used for shapes outside the tensor-core kernels' constraints (other channel
-// and head counts, e.g. 8 heads of 128 channels).
+// General kernel (shapes outside the tensor-core kernels' constraints: other
+// channel and head counts, e.g. 8 heads of 128 channels). The keys of a query
+// are split over a cluster of NS CTAs (up to 8); each CTA serves a group of 8
+// heads, so every key row is read once per head group, and the CTAs exchange
+// their partial softmax results through distributed shared memory.
+//  1. The CTA's keys, in chunks that fit in shared memory: positions, then
+//     every row dequantized into a bf16 tile (E2M1 x E4M3 or x E8M0 has at
+//     most 6 significant bits, so bf16 holds it exactly; window rows are bf16).
+//  2. Logits: warp w takes keys w, w + 8, ...; lane l holds channel pairs
+//     l, l + 32, ... of the 8 heads' Q; the 8 dot products are reduced across
+//     the warp by a transposing butterfly (9 shuffles), lane 4h + i ends with
+//     head h's logit.
+//  3. Online softmax and P V: warp h owns head h, rescales its running output
+//     (the lane's channels, in registers) and accumulates p_j row_j.
+//  4. Combine: each CTA publishes (m, l, O) in shared memory; after a cluster
+//     barrier, CTA r combines the heads h with h % NS == r from all NS CTAs.
+// Every loop stays rolled: a call runs once per layer on an instruction cache
+// that the kernels before it have emptied.
 #include "attention.cuh"
 
 namespace csa2 {
 
-// threads of the CTA for NP channel pairs per lane
-template <int NP>
-constexpr int gen_threads() { return NP <= 2 ? 512 : 256; }
-constexpr int GEN_MAX_WARPS = 16;
-// keys per warp per round with NP channel pairs per lane
-template <int NP>
-constexpr int gen_keys_per_round() { return NP >= 16 ? 2 : 32 / NP; }
+constexpr int GEN_THREADS = 256;
+constexpr int GEN_WARPS = GEN_THREADS / 32;
+constexpr int GEN_HG = 8;                  // heads per CTA: one warp per head in steps 3-4
+constexpr int GEN_MAX_NS = 8;              // CTAs per cluster (portable cluster size)
+constexpr size_t GEN_TILE_BYTES = 96 * 1024;  // bf16 key tile per chunk
+// Dynamic shared memory the kernel is set up for: the tile plus Q/O (8 x 1024
+// fp32) and the logits and positions of the chunk (at most 41 KB more).
+constexpr size_t GEN_SMEM_LIMIT = 160 * 1024;
+static_assert(GEN_HG == GEN_WARPS, "one warp per head");
 
-// Key j of query bq (j < K: selected row, else window row j - K) as NP channel
-// pairs per lane, dequantized; valid = false for an empty selected slot.
-template <int NP>
-__device__ __forceinline__ void gen_load_key(const AttnArgs &a, int b, const int32_t *sel,
-                                             const AttnWindow &w, int j, int lane, float2 (&v)[NP],
-                                             bool &valid) {
-    const int C = a.C, npairs = C / 2;
-    if (j < a.K) {
-        const int32_t pos = sel[j];
-        valid = pos >= 0 && pos < a.cap;
-        const int64_t cell = (int64_t)b * a.cap + (valid ? pos : 0);
-        const uint8_t *row = a.kv_fp4 + cell * (C / 2);
-        const uint8_t *sfr = a.kv_sf + cell * (C / (a.mx ? 32 : 16));
-        uint32_t byte[NP];
-        float sc[NP];
+struct GenGeom {
+    int ns;   // CTAs per cluster (key splits)
+    int kpc;  // keys per CTA (the last CTA of a query may hold fewer)
+    int kch;  // keys per chunk
+};
+
+__device__ __forceinline__ uint32_t gen_cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void gen_cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+// Address of this CTA's shared variable p in the shared memory of cluster CTA r.
+__device__ __forceinline__ uint32_t gen_dsmem(const void *p, uint32_t r) {
+    uint32_t a = (uint32_t)__cvta_generic_to_shared(p), out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(a), "r"(r));
+    return out;
+}
+__device__ __forceinline__ float gen_ld_remote(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ float2 gen_ld_remote2(uint32_t addr) {
+    float2 v;
+    asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+// Dequantizes 32 channels (16 code bytes, two scales) into 16 bf16 pairs.
+__device__ __forceinline__ void gen_dequant32(uint2 lo, uint2 hi, float s0, float s1, uint4 *dst) {
+    const uint32_t w[4] = {lo.x, lo.y, hi.x, hi.y};
 #pragma unroll
-        for (int i = 0; i < NP; i++) {
-            const int p = lane + 32 * i;
-            byte[i] = p < npairs ? __ldg(row + p) : 0u;
-            sc[i] = p < npairs ? kv_group_scale(sfr, p >> 3, a.mx) : 0.0f;
+    for (int q = 0; q < 4; q++) {
+        const float sc = q < 2 ? s0 : s1;
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const uint32_t byte = (w[q] >> (8 * e)) & 0xFFu;
+            const float x = e2m1_to_f32(byte & 0xFu) * sc, y = e2m1_to_f32(byte >> 4) * sc;
+            o[e] = (__float_as_uint(x) >> 16) | (__float_as_uint(y) & 0xFFFF0000u);  // exact
         }
-#pragma unroll
-        for (int i = 0; i < NP; i++)
-            v[i] = valid ? make_float2(e2m1_to_f32(byte[i] & 0xF) * sc[i], e2m1_to_f32(byte[i] >> 4) * sc[i])
-                         : make_float2(0.0f, 0.0f);
-    } else {
-        valid = true;
-        const uint32_t *row = reinterpret_cast<const uint32_t *>(a.swa) +
-                              ((int64_t)b * a.swa_rows + w.row0 + (j - a.K)) * (C / 2);
-#pragma unroll
-        for (int i = 0; i < NP; i++) {
-            const int p = lane + 32 * i;
-            const uint32_t u = p < npairs ? __ldg(row + p) : 0u;
-            v[i] = make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
-        }
+        dst[q] = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
 
-template <int NP>
-__global__ void __launch_bounds__(gen_threads<NP>()) attn_general_kernel(AttnArgs a) {
-    constexpr int GEN_U = gen_keys_per_round<NP>();
-    constexpr int GEN_THREADS = gen_threads<NP>();
-    constexpr int GEN_WARPS = GEN_THREADS / 32;
+template <int NPL>  // channel pairs per lane (C / 64, rounded up to a power of two)
+__global__ void __launch_bounds__(GEN_THREADS) attn_general_kernel(AttnArgs a, GenGeom g) {
     grid_dep_wait();
     grid_dep_launch();
-    extern __shared__ float sm[];
-    const int C = a.C, npairs = C / 2;
-    float *lg = sm;                                    // [K + n_win] logits, then p
-    float *red = sm + a.K + a.n_win;                   // [warps][C] partial sums
-    int32_t *sel = reinterpret_cast<int32_t *>(red + GEN_WARPS * C);  // [K]
-    __shared__ float wred[GEN_MAX_WARPS];
+    extern __shared__ __align__(16) uint8_t gsm[];
+    const int C = a.C, npairs = C / 2, nch = C / 32;
+    uint32_t *tile = reinterpret_cast<uint32_t *>(gsm);                           // [kch][C/2] bf16x2
+    float *qo = reinterpret_cast<float *>(gsm + (size_t)g.kch * C * 2);          // [8][C] Q, then O
+    float *lg = qo + GEN_HG * C;                                                   // [8][kch]
+    int32_t *kpos = reinterpret_cast<int32_t *>(lg + GEN_HG * g.kch);             // [kch]
+    __shared__ float m_sh[GEN_HG], l_sh[GEN_HG];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t bq = blockIdx.x / a.Hq;
-    const int h = (int)(blockIdx.x % a.Hq);
-    const int b = (int)(bq / a.Nq);
-    const AttnWindow w = attn_window(a, b, bq);
-    const int nkeys = a.K + w.n;
-    for (int j = tid; j < a.K; j += GEN_THREADS) sel[j] = a.topk[bq * a.K + j];
-
-    // this lane's query channels
-    const uint32_t *q = reinterpret_cast<const uint32_t *>(a.q) + (bq * a.Hq + h) * (int64_t)(C / 2);
-    float2 qv[NP];
-#pragma unroll
-    for (int i = 0; i < NP; i++) {
-        const int p = lane + 32 * i;
-        const uint32_t u = p < npairs ? __ldg(q + p) : 0u;
-        qv[i] = make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
-    }
-    __syncthreads();
-
-    // ---- logits
-    for (int j0 = warp * GEN_U; j0 < nkeys; j0 += GEN_WARPS * GEN_U) {
-        float2 v[GEN_U][NP];
-        bool valid[GEN_U];
-#pragma unroll
-        for (int u = 0; u < GEN_U; u++) {
-            valid[u] = false;
-            if (j0 + u < nkeys) gen_load_key<NP>(a, b, sel, w, j0 + u, lane, v[u], valid[u]);
+    const uint32_t rank = gen_cluster_rank();
+    const int h0 = blockIdx.y * GEN_HG;
+    const int64_t rows = (int64_t)a.B * a.Nq;
+    for (int64_t bq = blockIdx.z; bq < rows; bq += gridDim.z) {
+        const int b = (int)(bq / a.Nq);
+        const AttnWindow w = attn_window(a, b, bq);
+        const int nkeys = a.K + w.n;
+        const int j_beg = (int)rank * g.kpc;
+        const int j_end = min(nkeys, j_beg + g.kpc);
+        // Q of the 8 heads as fp32 (heads beyond Hq read as zero)
+#pragma unroll 4
+        for (int i = tid; i < GEN_HG * npairs; i += GEN_THREADS) {
+            const int h = i / npairs, p = i - h * npairs;
+            uint32_t u = 0;
+            if (h0 + h < a.Hq)
+                u = __ldg(reinterpret_cast<const uint32_t *>(a.q) + (bq * a.Hq + h0 + h) * (int64_t)npairs + p);
+            qo[h * C + 2 * p] = bf16_lo(u);
+            qo[h * C + 2 * p + 1] = bf16_hi(u);
         }
+        // running softmax state of head `warp` (warp-uniform) and its output
+        float m_run = -INFINITY, l_run = 0.0f;
+        float2 acc[NPL];
 #pragma unroll
-        for (int u = 0; u < GEN_U; u++) {
-            float dot = 0.0f;
+        for (int i = 0; i < NPL; i++) acc[i] = make_float2(0.0f, 0.0f);
+        for (int c0 = j_beg; c0 < j_end; c0 += g.kch) {
+            const int kn = min(g.kch, j_end - c0);
+            __syncthreads();  // the previous chunk's tile and logits are consumed
+            // 1a. positions (-1: empty slot; window rows as -2 - row)
+            for (int j = tid; j < kn; j += GEN_THREADS) {
+                const int jj = c0 + j;
+                int32_t v;
+                if (jj < a.K) {
+                    const int32_t pos = a.topk[bq * a.K + jj];
+                    v = (pos >= 0 && pos < a.cap) ? pos : -1;
+                } else {
+                    v = -2 - (int32_t)(w.row0 + (jj - a.K));
+                }
+                kpos[j] = v;
+            }
+            __syncthreads();
+            // 1b. rows into the tile, 32 channels per item: the chunk's
+            // selected rows [0, nf), then its window rows [nf, kn)
+            const int nf = max(0, min(kn, a.K - c0));
+#pragma unroll 2
+            for (int it = tid; it < nf * nch; it += GEN_THREADS) {
+                const int j = it / nch, c32 = it - j * nch;
+                const int32_t v = kpos[j];
+                if (v < 0) continue;  // empty slot: its logit is -inf, its row never read
+                const int64_t cell = (int64_t)b * a.cap + v;
+                const uint8_t *row = a.kv_fp4 + cell * (C / 2) + 16 * c32;
+                const uint2 lo = __ldg(reinterpret_cast<const uint2 *>(row));
+                const uint2 hi = __ldg(reinterpret_cast<const uint2 *>(row + 8));
+                float s0, s1;
+                if (a.mx) {
+                    s0 = s1 = e8m0_to_f32(__ldg(a.kv_sf + cell * (C / 32) + c32));
+                } else {
+                    const uint8_t *sf = a.kv_sf + cell * (C / 16) + 2 * c32;
+                    s0 = e4m3_to_f32(__ldg(sf));
+                    s1 = e4m3_to_f32(__ldg(sf + 1));
+                }
+                gen_dequant32(lo, hi, s0, s1, reinterpret_cast<uint4 *>(tile + (size_t)j * npairs + 16 * c32));
+            }
+#pragma unroll 2
+            for (int it = nf * nch + tid; it < kn * nch; it += GEN_THREADS) {
+                const int j = it / nch, c32 = it - j * nch;
+                const int64_t wrow = -2 - kpos[j];
+                const uint4 *src = reinterpret_cast<const uint4 *>(a.swa) +
+                                   (((int64_t)b * a.swa_rows + wrow) * C * 2 + 64 * c32) / 16;
+                uint4 *dst = reinterpret_cast<uint4 *>(tile + (size_t)j * npairs + 16 * c32);
 #pragma unroll
-            for (int i = 0; i < NP; i++) dot += qv[i].x * v[u][i].x + qv[i].y * v[u][i].y;
+                for (int q = 0; q < 4; q++) dst[q] = __ldg(src + q);
+            }
+            __syncthreads();
+            // 2. logits of the 8 heads
+#pragma unroll 1
+            for (int j = warp; j < kn; j += GEN_WARPS) {
+                float d[GEN_HG];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-            if (lane == 0 && j0 + u < nkeys) lg[j0 + u] = valid[u] ? dot * a.scale : -INFINITY;
-        }
-    }
-    __syncthreads();
-
-    // ---- softmax statistics
-    float m = -INFINITY;
-    for (int j = tid; j < nkeys; j += GEN_THREADS) m = fmaxf(m, lg[j]);
+                for (int h = 0; h < GEN_HG; h++) d[h] = 0.0f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) wred[warp] = m;
-    __syncthreads();
-    m = -INFINITY;
-    for (int w2 = 0; w2 < GEN_WARPS; w2++) m = fmaxf(m, wred[w2]);
-    __syncthreads();
-    float z = 0.0f;
-    for (int j = tid; j < nkeys; j += GEN_THREADS) {
-        const float p = (lg[j] == -INFINITY) ? 0.0f : expf(lg[j] - m);
-        lg[j] = p;
-        z += p;
-    }
+                for (int i = 0; i < NPL; i++) {
+                    const int p = lane + 32 * i;
+                    if (p < npairs) {
+                        const uint32_t kw = tile[(size_t)j * npairs + p];
+                        const float kx = bf16_lo(kw), ky = bf16_hi(kw);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    if (lane == 0) wred[warp] = z;
-    __syncthreads();
-    z = 0.0f;
-    for (int w2 = 0; w2 < GEN_WARPS; w2++) z += wred[w2];
-    const float inv = z > 0.0f ? 1.0f / z : 0.0f;
-
-    // ---- P V over the same keys
-    float2 acc[NP];
+                        for (int h = 0; h < GEN_HG; h++) {
+                            const float2 qq = *reinterpret_cast<const float2 *>(qo + h * C + 2 * p);
+                            d[h] = fmaf(qq.x, kx, fmaf(qq.y, ky, d[h]));
+                        }
+                    }
+                }
+                // transposing butterfly: lanes with bit 4 keep heads 4-7, then
+                // bit 3 halves again, bit 2 once more; bits 1 and 0 finish the sum
+                const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+                float e4[4], e2[2];
 #pragma unroll
-    for (int i = 0; i < NP; i++) acc[i] = make_float2(0.0f, 0.0f);
-    for (int j0 = warp * GEN_U; j0 < nkeys; j0 += GEN_WARPS * GEN_U) {
-        float2 v[GEN_U][NP];
-        bool valid[GEN_U];
+                for (int i = 0; i < 4; i++) {
+                    const float send = b4 ? d[i] : d[i + 4];
+                    const float keep = b4 ? d[i + 4] : d[i];
+                    e4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+                }
 #pragma unroll
-        for (int u = 0; u < GEN_U; u++) {
-            valid[u] = false;
-            if (j0 + u < nkeys && lg[j0 + u] != 0.0f) gen_load_key<NP>(a, b, sel, w, j0 + u, lane, v[u], valid[u]);
-        }
+                for (int i = 0; i < 2; i++) {
+                    const float send = b3 ? e4[i] : e4[i + 2];
+                    const float keep = b3 ? e4[i + 2] : e4[i];
+                    e2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+                }
+                float e1 = (b2 ? e2[1] : e2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? e2[0] : e2[1], 4);
+                e1 += __shfl_xor_sync(0xffffffffu, e1, 2);
+                e1 += __shfl_xor_sync(0xffffffffu, e1, 1);
+                if ((lane & 3) == 0) {
+                    const int h = lane >> 2;  // = 4 b4 + 2 b3 + b2
+                    lg[h * g.kch + j] = kpos[j] == -1 ? -INFINITY : e1 * a.scale;
+                }
+            }
+            __syncthreads();
+            // 3. online softmax and P V of head `warp`
+            {
+                float *lh = lg + warp * g.kch;
+                float mc = -INFINITY;
+                for (int j = lane; j < kn; j += 32) mc = fmaxf(mc, lh[j]);
 #pragma unroll
-        for (int u = 0; u < GEN_U; u++) {
-            if (!valid[u]) continue;
-            const float p = lg[j0 + u];
+                for (int o = 16; o > 0; o >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
+                const float m_new = fmaxf(m_run, mc);
+                if (m_new != -INFINITY) {
+                    const float alpha = m_run == -INFINITY ? 0.0f : expf(m_run - m_new);
+                    float z = 0.0f;
+                    for (int j = lane; j < kn; j += 32) {
+                        const float p = lh[j] == -INFINITY ? 0.0f : expf(lh[j] - m_new);
+                        lh[j] = p;
+                        z += p;
+                    }
 #pragma unroll
-            for (int i = 0; i < NP; i++) {
-                acc[i].x += p * v[u][i].x;
-                acc[i].y += p * v[u][i].y;
+                    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+                    l_run = l_run * alpha + z;
+                    m_run = m_new;
+#pragma unroll
+                    for (int i = 0; i < NPL; i++) {
+                        acc[i].x *= alpha;
+                        acc[i].y *= alpha;
+                    }
+                    __syncwarp();
+#pragma unroll 1
+                    for (int j = 0; j < kn; j++) {
+                        const float p = lh[j];
+                        if (p == 0.0f) continue;  // warp-uniform
+#pragma unroll
+                        for (int i = 0; i < NPL; i++) {
+                            const int pp = lane + 32 * i;
+                            if (pp < npairs) {
+                                const uint32_t vw = tile[(size_t)j * npairs + pp];
+                                acc[i].x = fmaf(p, bf16_lo(vw), acc[i].x);
+                                acc[i].y = fmaf(p, bf16_hi(vw), acc[i].y);
+                            }
+                        }
+                    }
+                }
             }
         }
-    }
+        // 4. publish (m, l, O) of the 8 heads; Q is dead once every warp has
+        // passed the last chunk's logits (or there was no chunk)
+        __syncthreads();
 #pragma unroll
-    for (int i = 0; i < NP; i++) {
-        const int p = lane + 32 * i;
-        if (p < npairs) {
-            red[warp * C + 2 * p] = acc[i].x;
-            red[warp * C + 2 * p + 1] = acc[i].y;
+        for (int i = 0; i < NPL; i++) {
+            const int pp = lane + 32 * i;
+            if (pp < npairs) *reinterpret_cast<float2 *>(qo + warp * C + 2 * pp) = acc[i];
         }
-    }
-    __syncthreads();
-    float *out = a.out + (bq * a.Hq + h) * (int64_t)C;
-    for (int c = tid; c < C; c += GEN_THREADS) {
-        float sum = 0.0f;
+        if (lane == 0) {
+            m_sh[warp] = m_run;
+            l_sh[warp] = l_run;
+        }
+        gen_cluster_sync();
+        const int h = warp;
+        if (h % g.ns == (int)rank && h0 + h < a.Hq) {
+            float m_all = -INFINITY;
+            for (int r = 0; r < g.ns; r++) m_all = fmaxf(m_all, gen_ld_remote(gen_dsmem(&m_sh[h], r)));
+            float L = 0.0f;
+            float2 o[NPL];
 #pragma unroll
-        for (int w2 = 0; w2 < GEN_WARPS; w2++) sum += red[w2 * C + c];
-        out[c] = sum * inv;
+            for (int i = 0; i < NPL; i++) o[i] = make_float2(0.0f, 0.0f);
+            if (m_all != -INFINITY) {
+                for (int r = 0; r < g.ns; r++) {
+                    const float mr = gen_ld_remote(gen_dsmem(&m_sh[h], r));
+                    if (mr == -INFINITY) continue;
+                    const float e = expf(mr - m_all);
+                    L += e * gen_ld_remote(gen_dsmem(&l_sh[h], r));
+#pragma unroll
+                    for (int i = 0; i < NPL; i++) {
+                        const int pp = lane + 32 * i;
+                        if (pp < npairs) {
+                            const float2 v = gen_ld_remote2(gen_dsmem(qo + h * C + 2 * pp, r));
+                            o[i].x = fmaf(e, v.x, o[i].x);
+                            o[i].y = fmaf(e, v.y, o[i].y);
+                        }
+                    }
+                }
+            }
+            const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+            float *out = a.out + (bq * a.Hq + h0 + h) * (int64_t)C;
+#pragma unroll
+            for (int i = 0; i < NPL; i++) {
+                const int pp = lane + 32 * i;
+                if (pp < npairs)
+                    *reinterpret_cast<float2 *>(out + 2 * pp) = make_float2(o[i].x * inv, o[i].y * inv);
+            }
+        }
+        gen_cluster_sync();  // no CTA reuses or leaves its shared memory while others read it
     }
 }
 
-template <int NP>
-static int launch_general(const AttnArgs &a, size_t smem, int64_t grid, cudaStream_t s) {
+static GenGeom gen_geometry(const AttnArgs &a) {
+    const int win = a.swa_rows > 0 && a.swa && a.n_win > 0 ? (a.n_win < a.swa_rows ? a.n_win : a.swa_rows) : 0;
+    const int T = a.K + win;  // most keys of one query
+    GenGeom g;
+    g.ns = (T + 63) / 64;  // about 64 keys or more per CTA
+    if (g.ns < 1) g.ns = 1;
+    if (g.ns > GEN_MAX_NS) g.ns = GEN_MAX_NS;
+    g.kpc = T > 0 ? (T + g.ns - 1) / g.ns : 1;
+    const int fit = (int)(GEN_TILE_BYTES / ((size_t)a.C * 2));
+    g.kch = g.kpc < fit ? g.kpc : fit;
+    return g;
+}
+
+static size_t gen_smem_bytes(const AttnArgs &a, const GenGeom &g) {
+    return (size_t)g.kch * a.C * 2 + (size_t)GEN_HG * a.C * 4 + (size_t)GEN_HG * g.kch * 4 +
+           (size_t)g.kch * 4;
+}
+
+template <int NPL>
+static int launch_general(const AttnArgs &a, const GenGeom &g, size_t smem, cudaStream_t s) {
     static PerDevice smem_set;
-    if (smem > 48 * 1024 && !set_smem_limit_once(smem_set, attn_general_kernel<NP>, 227 * 1024))
-        return CSA2_ERR_CUDA;
-    return launch_kernel(a.pdl, attn_general_kernel<NP>, dim3((unsigned)grid), dim3(gen_threads<NP>()),
-                         smem, s, a);
+    if (!set_smem_limit_once(smem_set, attn_general_kernel<NPL>, GEN_SMEM_LIMIT)) return CSA2_ERR_CUDA;
+    const int64_t rows = (int64_t)a.B * a.Nq;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)g.ns, (unsigned)((a.Hq + GEN_HG - 1) / GEN_HG),
+                       (unsigned)(rows < 65535 ? rows : 65535));
+    cfg.blockDim = dim3(GEN_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)g.ns;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.pdl ? 2 : 1;
+    if (cudaLaunchKernelEx(&cfg, attn_general_kernel<NPL>, a, g) != cudaSuccess) return CSA2_ERR_CUDA;
+    return launch_status();
 }
 
 int launch_attn_general(const AttnArgs &a, cudaStream_t s) {
-    // logits [K + n_win], partial sums [warps][C], selected positions [K]
-    const int pairs_per_lane = (a.C / 2 + 31) / 32;  // 1 .. 16 (C <= 1024)
-    const int warps = pairs_per_lane <= 2 ? 16 : 8;
-    const size_t smem = sizeof(float) * ((size_t)a.K + a.n_win + (size_t)warps * a.C) +
-                        sizeof(int32_t) * (size_t)a.K;
-    if (smem > 227 * 1024) return CSA2_ERR_SHAPE;
-    const int64_t grid = (int64_t)a.B * a.Nq * a.Hq;
-    if (grid > INT32_MAX) return CSA2_ERR_SHAPE;
-    if (pairs_per_lane <= 1) return launch_general<1>(a, smem, grid, s);
-    if (pairs_per_lane <= 2) return launch_general<2>(a, smem, grid, s);
-    if (pairs_per_lane <= 4) return launch_general<4>(a, smem, grid, s);
-    if (pairs_per_lane <= 8) return launch_general<8>(a, smem, grid, s);
-    return launch_general<16>(a, smem, grid, s);
+    const GenGeom g = gen_geometry(a);
+    const size_t smem = gen_smem_bytes(a, g);
+    if (smem > GEN_SMEM_LIMIT) return CSA2_ERR_SHAPE;
+    const int npl = (a.C / 2 + 31) / 32;  // 1 .. 16 (C <= 1024)
+    if (npl <= 1) return launch_general<1>(a, g, smem, s);
+    if (npl <= 2) return launch_general<2>(a, g, smem, s);
+    if (npl <= 4) return launch_general<4>(a, g, smem, s);
+    if (npl <= 8) return launch_general<8>(a, g, smem, s);
+    return launch_general<16>(a, g, smem, s);
 }
 
 }  // namespace csa2

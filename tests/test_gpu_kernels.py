@@ -467,6 +467,30 @@ def test_sparse_attention_matches_oracle(B, Bn, ctx, C, Hq, K):
     _attention_case(B, Bn, ctx, C, Hq, K, 128, seed=ctx + C)
 
 
+# The general kernel (shapes outside the tensor-core kernels'): keys split over a
+# cluster of up to 8 CTAs, 8 heads per CTA, key rows staged in chunks of at
+# most 96 KB. Odd pair counts per lane (96 channels), a partial last head
+# group (13 heads), few keys (3 CTAs), the largest row (1024 channels: 48-key
+# chunks, 11 of them per CTA at K = 4096), no window, masked slots and causal
+# positions.
+@pytest.mark.parametrize("Bn,ctx,C,Hq,K,n_win,drop", [(2, 3000, 96, 5, 300, 128, 0),
+                                                      (2, 3000, 128, 13, 20, 128, 3),
+                                                      (1, 6000, 1024, 2, 4096, 128, 5),
+                                                      (3, 2000, 256, 8, 512, 0, 0),
+                                                      (1, 2000, 32, 1, 512, 64, 2),
+                                                      (2, 700, 128, 8, 1024, 100, 0)])
+def test_sparse_attention_general_kernel(B, Bn, ctx, C, Hq, K, n_win, drop):
+    _attention_case(B, Bn, ctx, C, Hq, K, n_win, seed=ctx + C + Hq, drop=drop)
+
+
+def test_sparse_attention_general_kernel_causal_positions(B):
+    ctx = 1300
+    q_pos = torch.tensor([[1299, 700, 129, 128, 5, 0], [1000, 1001, 64, 3, 1250, 600]],
+                         dtype=torch.int64, device=DEV)
+    _attention_case(B, 2, ctx, 128, 8, 512, 128, seed=21, q_pos=q_pos, Nq=6, drop=4)
+    _attention_case(B, 2, ctx, 128, 8, 512, 128, seed=22, q_pos=q_pos, Nq=6, mx=True)
+
+
 def test_sparse_attention_skips_negative_indices_and_short_window(B):
     _attention_case(B, 2, 2500, 512, 64, 512, 128, seed=1, drop=3)
     _attention_case(B, 1, 50, 512, 64, 512, 128, seed=2)

@@ -869,11 +869,17 @@ struct PoolTokArgs {
 // the CTA, after a barrier that follows the pool's writes.
 __device__ void pool_tokens_select(const TopkArgs &a, const PoolTokArgs &pa, int64_t r,
                                    TopkShared sh, TopkState &st) {
-    const int P = a.k, n = P * kBlockTokens;
+    const int P = a.k;
     uint64_t *keys = sh.buf;
     int64_t V = pa.ctx_len[r];
     if (V > pa.cap) V = pa.cap;
     const int32_t *pool = a.out + r * (int64_t)P;
+    // the pool is ascending and -1 padded: only its valid entries' tokens are
+    // candidates (a row shorter than the pool has fewer)
+    int npool = 0;
+    for (int i0 = 0; i0 < P; i0 += TK_THREADS)
+        npool += __syncthreads_count(i0 + (int)threadIdx.x < P && pool[i0 + threadIdx.x] >= 0);
+    const int n = npool * kBlockTokens;
     const float *tok = pa.tok + r * pa.cap;
     for (int i = threadIdx.x; i < n; i += TK_THREADS) {
         const int32_t blk = pool[i >> 3];
@@ -935,7 +941,7 @@ __device__ void pool_tokens_select(const TopkArgs &a, const PoolTokArgs &pa, int
     const uint64_t p = st.prefix, m = st.mask;
     // bitmap of the selected indices over [0, n), in the histogram's space
     uint32_t *bm = sh.hist;
-    const int nwords = n / 32;
+    const int nwords = (n + 31) / 32;
     for (int i = threadIdx.x; i < nwords; i += TK_THREADS) bm[i] = 0;
     __syncthreads();
     for (int i = threadIdx.x; i < n; i += TK_THREADS) {

@@ -59,14 +59,24 @@ struct TopkState {
 
 // Block-wide (NT threads): given hist[0..NB), find the bin d where the count
 // of keys at or above it first reaches kk (scanning from the top bin down).
+// Thread t sums the contiguous bins [t BPT, t BPT + BPT); with 4 bins per
+// thread it reads them with one 16-byte load (a warp's loads are then
+// conflict-free) and keeps them in registers for the second walk.
 template <int NT = TK_THREADS>
 __device__ void find_digit(const uint32_t *hist, int NB, int kk, TopkState &st) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int BPT = (NB + NT - 1) / NT;
     const int b0 = tid * BPT;
+    const bool quad = NB == 4 * NT;
+    uint4 q4 = make_uint4(0, 0, 0, 0);
     uint32_t local = 0;
-    for (int j = 0; j < BPT; j++)
-        if (b0 + j < NB) local += hist[b0 + j];
+    if (quad) {
+        q4 = reinterpret_cast<const uint4 *>(hist)[tid];
+        local = q4.x + q4.y + q4.z + q4.w;
+    } else {
+        for (int j = 0; j < BPT; j++)
+            if (b0 + j < NB) local += hist[b0 + j];
+    }
     // inclusive suffix sum inside the warp
     uint32_t x = local;
 #pragma unroll
@@ -85,7 +95,7 @@ __device__ void find_digit(const uint32_t *hist, int NB, int kk, TopkState &st) 
     for (int j = BPT - 1; j >= 0; j--) {
         const int bin = b0 + j;
         if (bin >= NB) continue;
-        const uint32_t h = hist[bin];
+        const uint32_t h = quad ? (j == 3 ? q4.w : j == 2 ? q4.z : j == 1 ? q4.y : q4.x) : hist[bin];
         if (above < (uint32_t)kk && above + h >= (uint32_t)kk) {
             st.digit = bin;
             st.above = above;
@@ -94,6 +104,53 @@ __device__ void find_digit(const uint32_t *hist, int NB, int kk, TopkState &st) 
         above += h;
     }
     if (tid == 0) st.total = all;
+    __syncthreads();
+}
+
+// find_digit over a producer's 4096-bin first-digit histogram row in global
+// memory, without a shared-memory copy: thread t loads its TK_HIST / NT
+// contiguous bins straight into registers (16-byte loads).
+template <int NT>
+__device__ void hist_threshold(const uint32_t *gh, int kk, TopkState &st) {
+    constexpr int BPT = TK_HIST / NT;
+    static_assert(BPT % 4 == 0 && BPT * NT == TK_HIST, "whole 16-byte groups per thread");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t hb[BPT];
+    const uint4 *hp = reinterpret_cast<const uint4 *>(gh) + (BPT / 4) * tid;
+#pragma unroll
+    for (int q = 0; q < BPT / 4; q++) {
+        const uint4 v = hp[q];
+        hb[4 * q] = v.x;
+        hb[4 * q + 1] = v.y;
+        hb[4 * q + 2] = v.z;
+        hb[4 * q + 3] = v.w;
+    }
+    uint32_t local = 0;
+#pragma unroll
+    for (int j = 0; j < BPT; j++) local += hb[j];
+    uint32_t x = local;  // inclusive suffix sum over the lanes of the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
+        if (lane + o < 32) x += y;
+    }
+    if (lane == 0) st.wsum[warp] = x;
+    __syncthreads();
+    uint32_t above = x - local, total = 0;
+    for (int w = 0; w < NT / 32; w++) {
+        total += st.wsum[w];
+        if (w > warp) above += st.wsum[w];
+    }
+#pragma unroll
+    for (int j = BPT - 1; j >= 0; j--) {
+        if (above < (uint32_t)kk && above + hb[j] >= (uint32_t)kk) {
+            st.digit = BPT * tid + j;
+            st.above = above;
+            st.match = hb[j];
+        }
+        above += hb[j];
+    }
+    if (tid == 0) st.total = total;
     __syncthreads();
 }
 
@@ -336,18 +393,6 @@ struct TopkHistWs {
     uint64_t *tie;   // [R][TK_BUF] keys
 };
 
-// Copy a 4096-bin histogram row from global to shared memory with 16-byte
-// loads issued together (one round trip), NT threads.
-template <int NT>
-__device__ __forceinline__ void load_hist(uint32_t *dst, const uint32_t *src) {
-    constexpr int PER = TK_HIST / 4 / NT;
-    uint4 v[PER];
-#pragma unroll
-    for (int u = 0; u < PER; u++) v[u] = reinterpret_cast<const uint4 *>(src)[u * NT + threadIdx.x];
-#pragma unroll
-    for (int u = 0; u < PER; u++) reinterpret_cast<uint4 *>(dst)[u * NT + threadIdx.x] = v[u];
-}
-
 // Copy n elements of T from global to shared memory, 8 loads in flight per thread.
 template <typename T>
 __device__ __forceinline__ void load_batched(T *dst, const T *src, int n) {
@@ -379,7 +424,6 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
 __global__ void __launch_bounds__(TC_THREADS) topk_compact_kernel(TopkArgs a, TopkHistWs ws) {
     grid_dep_wait();
     grid_dep_launch();
-    __shared__ uint32_t hist[TK_HIST];
     __shared__ TopkState st;
     const int64_t r = blockIdx.y;
     int64_t nv = a.n;
@@ -389,9 +433,7 @@ __global__ void __launch_bounds__(TC_THREADS) topk_compact_kernel(TopkArgs a, To
     }
     const int64_t i_beg = (int64_t)blockIdx.x * TC_SLICE;
     if (i_beg >= nv) return;
-    load_hist<TC_THREADS>(hist, ws.hist + r * TK_HIST);
-    __syncthreads();
-    find_digit<TC_THREADS>(hist, TK_HIST, a.k, st);
+    hist_threshold<TC_THREADS>(ws.hist + r * TK_HIST, a.k, st);
     const bool all = st.total <= (uint32_t)a.k;
     const uint64_t d = (uint64_t)st.digit;
     const bool vec = ((r * a.n) % 4 == 0) && aligned16(a.score) &&
@@ -546,7 +588,6 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_finish_kernel(TopkArgs a, 
     __shared__ TopkState st;
     TopkShared sh = topk_shared(smem_raw);
     const int64_t r = blockIdx.x;
-    load_hist<TK_THREADS>(sh.hist, ws.hist + r * TK_HIST);
     const int nsel0 = min(ws.cnt[2 * r], a.k);
     const int ntie = ws.cnt[2 * r + 1];
     if (threadIdx.x == 0) {
@@ -555,8 +596,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_finish_kernel(TopkArgs a, 
         st.nsel = 0;
         st.nbuf = 0;
     }
-    __syncthreads();
-    find_digit(sh.hist, TK_HIST, a.k, st);
+    hist_threshold<TK_THREADS>(ws.hist + r * TK_HIST, a.k, st);
     const bool all = st.total <= (uint32_t)a.k;
     if ((!all && ntie > TK_BUF) || a.n > TF_MAX_N) {
         __syncthreads();
@@ -594,15 +634,13 @@ __device__ void topk_row_hist_body(const TopkArgs &a, int64_t r, uint32_t *ghist
         const int64_t v = a.n_valid[r];
         nv = v < 0 ? 0 : (v < a.n ? v : a.n);
     }
-    load_hist<TK_THREADS>(sh.hist, ghist + r * TK_HIST);
     if (threadIdx.x == 0) {
         st.prefix = 0;
         st.mask = 0;
         st.nsel = 0;
         st.nbuf = 0;
     }
-    __syncthreads();
-    find_digit(sh.hist, TK_HIST, a.k, st);
+    hist_threshold<TK_THREADS>(ghist + r * TK_HIST, a.k, st);
     const bool all = st.total <= (uint32_t)a.k;
     const uint32_t d = (uint32_t)st.digit;
     const bool vec = ((r * a.n) % 4 == 0) && aligned16(a.score) &&
@@ -993,7 +1031,6 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     __shared__ TopkState st;
     TopkShared sh = pool_tokens_shared(smem_raw);
     const int64_t r = blockIdx.x;
-    load_hist<TK_THREADS>(sh.hist, ws.hist + r * TK_HIST);
     const int nsel0 = min(ws.cnt[2 * r], a.k);
     const int ntie = ws.cnt[2 * r + 1];
     if (threadIdx.x == 0) {
@@ -1002,8 +1039,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
         st.nsel = 0;
         st.nbuf = 0;
     }
-    __syncthreads();
-    find_digit(sh.hist, TK_HIST, a.k, st);
+    hist_threshold<TK_THREADS>(ws.hist + r * TK_HIST, a.k, st);
     const bool all = st.total <= (uint32_t)a.k;
     if ((!all && ntie > TK_BUF) || a.n > TF_MAX_N) {
         __syncthreads();

@@ -111,6 +111,18 @@ __global__ void __launch_bounds__(GEN_THREADS) attn_general_kernel(AttnArgs a, G
         const int nkeys = a.K + w.n;
         const int j_beg = (int)rank * g.kpc;
         const int j_end = min(nkeys, j_beg + g.kpc);
+        // positions of the first chunk (see 1a), loaded together with Q
+        const int kn0 = max(0, min(g.kch, j_end - j_beg));
+        int32_t pos0 = -1;
+        if (tid < kn0) {
+            const int jj = j_beg + tid;
+            if (jj < a.K) {
+                const int32_t pos = a.topk[bq * a.K + jj];
+                pos0 = (pos >= 0 && pos < a.cap) ? pos : -1;
+            } else {
+                pos0 = -2 - (int32_t)(w.row0 + (jj - a.K));
+            }
+        }
         // Q of the 8 heads as fp32 (heads beyond Hq read as zero)
 #pragma unroll 4
         for (int i = tid; i < GEN_HG * npairs; i += GEN_THREADS) {
@@ -129,8 +141,10 @@ __global__ void __launch_bounds__(GEN_THREADS) attn_general_kernel(AttnArgs a, G
         for (int c0 = j_beg; c0 < j_end; c0 += g.kch) {
             const int kn = min(g.kch, j_end - c0);
             __syncthreads();  // the previous chunk's tile and logits are consumed
-            // 1a. positions (-1: empty slot; window rows as -2 - row)
-            for (int j = tid; j < kn; j += GEN_THREADS) {
+            // 1a. positions (-1: empty slot; window rows as -2 - row); the first
+            // chunk's first GEN_THREADS came with Q
+            if (c0 == j_beg && tid < kn) kpos[tid] = pos0;
+            for (int j = (c0 == j_beg ? tid + GEN_THREADS : tid); j < kn; j += GEN_THREADS) {
                 const int jj = c0 + j;
                 int32_t v;
                 if (jj < a.K) {
@@ -277,18 +291,26 @@ __global__ void __launch_bounds__(GEN_THREADS) attn_general_kernel(AttnArgs a, G
         gen_cluster_sync();
         const int h = warp;
         if (h % g.ns == (int)rank && h0 + h < a.Hq) {
+            // every source's statistics with one round of remote loads
+            float mr[GEN_MAX_NS], lr[GEN_MAX_NS];
+#pragma unroll
+            for (int r = 0; r < GEN_MAX_NS; r++) {
+                mr[r] = r < g.ns ? gen_ld_remote(gen_dsmem(&m_sh[h], r)) : -INFINITY;
+                lr[r] = r < g.ns ? gen_ld_remote(gen_dsmem(&l_sh[h], r)) : 0.0f;
+            }
             float m_all = -INFINITY;
-            for (int r = 0; r < g.ns; r++) m_all = fmaxf(m_all, gen_ld_remote(gen_dsmem(&m_sh[h], r)));
+#pragma unroll
+            for (int r = 0; r < GEN_MAX_NS; r++) m_all = fmaxf(m_all, mr[r]);
             float L = 0.0f;
             float2 o[NPL];
 #pragma unroll
             for (int i = 0; i < NPL; i++) o[i] = make_float2(0.0f, 0.0f);
             if (m_all != -INFINITY) {
-                for (int r = 0; r < g.ns; r++) {
-                    const float mr = gen_ld_remote(gen_dsmem(&m_sh[h], r));
-                    if (mr == -INFINITY) continue;
-                    const float e = expf(mr - m_all);
-                    L += e * gen_ld_remote(gen_dsmem(&l_sh[h], r));
+#pragma unroll
+                for (int r = 0; r < GEN_MAX_NS; r++) {
+                    if (r >= g.ns || mr[r] == -INFINITY) continue;
+                    const float e = expf(mr[r] - m_all);
+                    L += e * lr[r];
 #pragma unroll
                     for (int i = 0; i < NPL; i++) {
                         const int pp = lane + 32 * i;

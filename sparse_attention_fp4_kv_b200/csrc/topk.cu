@@ -634,6 +634,14 @@ __device__ void topk_row_hist_body(const TopkArgs &a, int64_t r, uint32_t *ghist
         const int64_t v = a.n_valid[r];
         nv = v < 0 ? 0 : (v < a.n ? v : a.n);
     }
+    if (a.cand_pos == nullptr && nv <= a.k) {
+        // a row of at most k candidates: every index is selected, in order
+        int32_t *out = a.out + r * a.k;
+        for (int i = threadIdx.x; i < a.k; i += TK_THREADS) out[i] = i < nv ? i : -1;
+        for (int b = threadIdx.x; b < TK_HIST; b += TK_THREADS) ghist[r * TK_HIST + b] = 0;
+        if (threadIdx.x == 0) st.nsel = (int)nv;
+        return;
+    }
     if (threadIdx.x == 0) {
         st.prefix = 0;
         st.mask = 0;

@@ -163,7 +163,12 @@ __global__ void __launch_bounds__(GEN_THREADS) attn_general_kernel(AttnArgs a, G
             for (int it = tid; it < nf * nch; it += GEN_THREADS) {
                 const int j = it / nch, c32 = it - j * nch;
                 const int32_t v = kpos[j];
-                if (v < 0) continue;  // empty slot: its logit is -inf, its row never read
+                if (v < 0) {  // empty slot: logit -inf, a zero row (p = 0 times it stays 0)
+                    uint4 *dst = reinterpret_cast<uint4 *>(tile + (size_t)j * npairs + 16 * c32);
+#pragma unroll
+                    for (int q = 0; q < 4; q++) dst[q] = make_uint4(0, 0, 0, 0);
+                    continue;
+                }
                 const int64_t cell = (int64_t)b * a.cap + v;
                 const uint8_t *row = a.kv_fp4 + cell * (C / 2) + 16 * c32;
                 const uint2 lo = __ldg(reinterpret_cast<const uint2 *>(row));
@@ -190,6 +195,17 @@ __global__ void __launch_bounds__(GEN_THREADS) attn_general_kernel(AttnArgs a, G
             }
             __syncthreads();
             // 2. logits of the 8 heads
+            // with at most 2 channel pairs per lane the 8 heads' Q stay in registers
+            constexpr int QR = NPL <= 2 ? NPL : 1;
+            float2 qr[GEN_HG][QR];
+#pragma unroll
+            for (int h = 0; h < GEN_HG; h++)
+#pragma unroll
+                for (int i = 0; i < QR; i++) {
+                    const int p = lane + 32 * i;
+                    qr[h][i] = (NPL <= 2 && p < npairs) ? *reinterpret_cast<const float2 *>(qo + h * C + 2 * p)
+                                                        : make_float2(0.0f, 0.0f);
+                }
 #pragma unroll 1
             for (int j = warp; j < kn; j += GEN_WARPS) {
                 float d[GEN_HG];
@@ -203,7 +219,8 @@ __global__ void __launch_bounds__(GEN_THREADS) attn_general_kernel(AttnArgs a, G
                         const float kx = bf16_lo(kw), ky = bf16_hi(kw);
 #pragma unroll
                         for (int h = 0; h < GEN_HG; h++) {
-                            const float2 qq = *reinterpret_cast<const float2 *>(qo + h * C + 2 * p);
+                            const float2 qq = NPL <= 2 ? qr[h][i < QR ? i : 0]
+                                                       : *reinterpret_cast<const float2 *>(qo + h * C + 2 * p);
                             d[h] = fmaf(qq.x, kx, fmaf(qq.y, ky, d[h]));
                         }
                     }
@@ -259,19 +276,29 @@ __global__ void __launch_bounds__(GEN_THREADS) attn_general_kernel(AttnArgs a, G
                         acc[i].y *= alpha;
                     }
                     __syncwarp();
+                    // four keys per round, all their loads issued first (every row of
+                    // the tile is finite: empty slots hold zeros)
 #pragma unroll 1
-                    for (int j = 0; j < kn; j++) {
-                        const float p = lh[j];
-                        if (p == 0.0f) continue;  // warp-uniform
+                    for (int j0 = 0; j0 < kn; j0 += 4) {
+                        float p[4];
+                        uint32_t vw[4][NPL];
 #pragma unroll
-                        for (int i = 0; i < NPL; i++) {
-                            const int pp = lane + 32 * i;
-                            if (pp < npairs) {
-                                const uint32_t vw = tile[(size_t)j * npairs + pp];
-                                acc[i].x = fmaf(p, bf16_lo(vw), acc[i].x);
-                                acc[i].y = fmaf(p, bf16_hi(vw), acc[i].y);
+                        for (int u = 0; u < 4; u++) {
+                            const int j = j0 + u;
+                            p[u] = j < kn ? lh[j] : 0.0f;
+#pragma unroll
+                            for (int i = 0; i < NPL; i++) {
+                                const int pp = lane + 32 * i;
+                                vw[u][i] = (j < kn && pp < npairs) ? tile[(size_t)j * npairs + pp] : 0u;
                             }
                         }
+#pragma unroll
+                        for (int u = 0; u < 4; u++)
+#pragma unroll
+                            for (int i = 0; i < NPL; i++) {
+                                acc[i].x = fmaf(p[u], bf16_lo(vw[u][i]), acc[i].x);
+                                acc[i].y = fmaf(p[u], bf16_hi(vw[u][i]), acc[i].y);
+                            }
                     }
                 }
             }

@@ -913,8 +913,10 @@ struct PoolTokArgs {
 // Top-pa.k tokens of row r among the tokens of the a.k pool blocks this CTA
 // just wrote to a.out (row r, ascending block ids, -1 padded). All threads of
 // the CTA, after a barrier that follows the pool's writes.
+// identity_n >= 0: the pool is blocks 0 .. identity_n - 1 (a row of at most P
+// blocks), so it is not read back.
 __device__ void pool_tokens_select(const TopkArgs &a, const PoolTokArgs &pa, int64_t r,
-                                   TopkShared sh, TopkState &st) {
+                                   TopkShared sh, TopkState &st, int identity_n) {
     const int P = a.k;
     uint64_t *keys = sh.buf;
     int64_t V = pa.ctx_len[r];
@@ -923,12 +925,16 @@ __device__ void pool_tokens_select(const TopkArgs &a, const PoolTokArgs &pa, int
     // the pool is ascending and -1 padded: only its valid entries' tokens are
     // candidates (a row shorter than the pool has fewer)
     int npool = 0;
-    for (int i0 = 0; i0 < P; i0 += TK_THREADS)
-        npool += __syncthreads_count(i0 + (int)threadIdx.x < P && pool[i0 + threadIdx.x] >= 0);
+    if (identity_n >= 0) {
+        npool = identity_n < P ? identity_n : P;
+    } else {
+        for (int i0 = 0; i0 < P; i0 += TK_THREADS)
+            npool += __syncthreads_count(i0 + (int)threadIdx.x < P && pool[i0 + threadIdx.x] >= 0);
+    }
     const int n = npool * kBlockTokens;
     const float *tok = pa.tok + r * pa.cap;
     for (int i = threadIdx.x; i < n; i += TK_THREADS) {
-        const int32_t blk = pool[i >> 3];
+        const int32_t blk = identity_n >= 0 ? (i >> 3) : pool[i >> 3];
         const int64_t pos = 8 * (int64_t)blk + (i & 7);
         keys[i] = (blk >= 0 && pos < V) ? rank_key(tok[pos], (int32_t)pos) : 0ull;
     }
@@ -986,17 +992,21 @@ __device__ void pool_tokens_select(const TopkArgs &a, const PoolTokArgs &pa, int
     }
     const uint64_t p = st.prefix, m = st.mask;
     // bitmap of the selected indices over [0, n), in the histogram's space
+    // a warp covers 32 consecutive keys, one bitmap word: one ballot writes it
     uint32_t *bm = sh.hist;
     const int nwords = (n + 31) / 32;
-    for (int i = threadIdx.x; i < nwords; i += TK_THREADS) bm[i] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n; i += TK_THREADS) {
-        const uint64_t key = keys[i];
-        const bool take =
-            key && (all || (key >> 52) > d || (!listed && (key & m) >= p && (key >> 52) == d));
-        if (take) atomicOr(&bm[i >> 5], 1u << (i & 31));
+    for (int i0 = 0; i0 < nwords * 32; i0 += TK_THREADS) {
+        const int i = i0 + (int)threadIdx.x;
+        bool take = false;
+        if (i < n) {
+            const uint64_t key = keys[i];
+            take = key && (all || (key >> 52) > d || (!listed && (key & m) >= p && (key >> 52) == d));
+        }
+        const uint32_t word = __ballot_sync(0xffffffffu, take);
+        if ((threadIdx.x & 31) == 0 && i < nwords * 32) bm[i >> 5] = word;
     }
     if (listed) {
+        __syncthreads();  // the tie bits go on top of the words written above
         for (int i = threadIdx.x; i < st.nbuf; i += TK_THREADS) {
             const uint64_t key = ties[i];
             if ((key & m) >= p) {
@@ -1067,7 +1077,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     for (int b = threadIdx.x; b < TK_HIST; b += TK_THREADS) ws.hist[r * TK_HIST + b] = 0;
     if (threadIdx.x < 2) ws.cnt[2 * r + threadIdx.x] = 0;
     __syncthreads();
-    pool_tokens_select(a, pa, r, sh, st);
+    pool_tokens_select(a, pa, r, sh, st, -1);
 }
 
 // Pool from one pass over the row (as topk_row_hist_kernel), then the row's top
@@ -1081,7 +1091,13 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     TopkShared sh = pool_tokens_shared(smem_raw);
     topk_row_hist_body(a, blockIdx.x, ghist, sh, st);
     __syncthreads();
-    pool_tokens_select(a, pa, blockIdx.x, sh, st);
+    // a row of at most P blocks pooled all of them, in order
+    int64_t nv = a.n;
+    if (a.n_valid) {
+        const int64_t v = a.n_valid[blockIdx.x];
+        nv = v < 0 ? 0 : (v < a.n ? v : a.n);
+    }
+    pool_tokens_select(a, pa, blockIdx.x, sh, st, nv <= a.k ? (int)nv : -1);
 }
 
 }  // namespace csa2

@@ -101,8 +101,9 @@ struct Cfg {
     static constexpr int L_OFF = M_OFF + HPC * 4;    // fp32 row sum [HPC]
     static constexpr int SLOT_OFF = L_OFF + HPC * 4; // int64 source row per key slot [T]
     static constexpr int KIND_OFF = SLOT_OFF + T * 8;
-    static constexpr int BAR_OFF = (KIND_OFF + T + 15) / 16 * 16;  // [0] loads, [1] MMAs
-    static constexpr int TADDR_OFF = BAR_OFF + 16;
+    // mbarriers: [0] loads, [1] MMAs, [2] the P V MMAs of channel blocks 0-1
+    static constexpr int BAR_OFF = (KIND_OFF + T + 15) / 16 * 16;
+    static constexpr int TADDR_OFF = BAR_OFF + 24;
     static constexpr int SMEM_USED = TADDR_OFF + 16;
     static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
     static constexpr int MIN_BLOCKS = SMEM_BYTES <= 112 * 1024 ? 2 : 1;
@@ -204,6 +205,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
     int64_t *slot_src = reinterpret_cast<int64_t *>(sm + L::SLOT_OFF);
     uint8_t *slot_kind = sm + L::KIND_OFF;
     const uint32_t bar_ld = base + L::BAR_OFF, bar = base + L::BAR_OFF + 8;
+    const uint32_t bar_pv = base + L::BAR_OFF + 16;
     uint32_t *taddr_s = reinterpret_cast<uint32_t *>(sm + L::TADDR_OFF);
     // this cluster's exchange slot in the workspace
     float *xo = reinterpret_cast<float *>(a.ws) + (int64_t)blockIdx.y * L::XSLOT_FLOATS;
@@ -214,6 +216,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
     if (tid == 0) {
         mbar_init(bar_ld, 1);
         mbar_init(bar, 1);
+        mbar_init(bar_pv, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) tmem_alloc(base + L::TADDR_OFF, L::TMEM_COLS);
@@ -234,7 +237,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
     const bool row_major = !keep && L::HG == 1;
     const int64_t n_mine =
         (int64_t)blockIdx.y < items ? (items - 1 - (int64_t)blockIdx.y) / gridDim.y + 1 : 0;
-    uint32_t ld_phase = 0;
+    uint32_t ld_phase = 0, pv_phase = 0;
     bool ld_pending = false;  // (thread 0) copies issued on bar_ld and not yet waited for
     bool ok = true;
     // Q and window rows of this cluster's first item, every layer: warmed in
@@ -488,22 +491,30 @@ __global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
             // K = 80 keys): V^T is the KV tile read MN-major, [P_hi; P_lo]^T the P
             // tile read K-major; block c of 128 channels accumulates in columns
             // [2 HPC c, 2 HPC c + 2 HPC) (hi part, then lo part)
+            // Channel blocks 0-1 first, committed on their own barrier, so that
+            // warps 0-3 publish them while blocks 2-3 are multiplied.
+            const bool pv_issued = ok;  // uniform here
             if (tid == 0 && ok) {
                 tc_fence_after();
                 constexpr uint32_t id_o = idesc_bf16(128, 2 * HPC, false, true);
-#pragma unroll 1
-                for (int kk = 0; kk < T / 16; kk++) {
-                    const uint64_t pd = sdesc(base + L::P_OFF + (kk >> 2) * L::P_ATOM + (kk & 3) * 32, 16, 1024);
 #pragma unroll
-                    for (int c = 0; c < 4; c++) {
-                        const uint64_t vd =
-                            sdesc(base + L::K_OFF + 2 * c * K_CHUNK + kk * 2048, K_CHUNK, 1024);
-                        mma_bf16(tmem + 2 * HPC * c, vd, pd, id_o, kk > 0);
+                for (int c2 = 0; c2 < 2; c2++) {
+#pragma unroll 1
+                    for (int kk = 0; kk < T / 16; kk++) {
+                        const uint64_t pd =
+                            sdesc(base + L::P_OFF + (kk >> 2) * L::P_ATOM + (kk & 3) * 32, 16, 1024);
+#pragma unroll
+                        for (int c = 2 * c2; c < 2 * c2 + 2; c++) {
+                            const uint64_t vd =
+                                sdesc(base + L::K_OFF + 2 * c * K_CHUNK + kk * 2048, K_CHUNK, 1024);
+                            mma_bf16(tmem + 2 * HPC * c, vd, pd, id_o, kk > 0);
+                        }
                     }
+                    mma_commit(c2 == 0 ? bar_pv : bar);
                 }
-                mma_commit(bar);
             }
-            if (ok) ok = mbar_wait_bounded(bar, 1, WAIT_NS);
+            if (ok) ok = warp < 4 ? mbar_wait_bounded(bar_pv, pv_phase, WAIT_NS) : mbar_wait_bounded(bar, 1, WAIT_NS);
+            if (pv_issued) pv_phase ^= 1;
             tc_fence_after();
 
             // ---- publish this CTA's unnormalized O, row maxima and sums in the

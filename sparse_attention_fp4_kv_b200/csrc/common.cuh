@@ -261,6 +261,11 @@ int launch_index_full_hist(const int8_t *q_idx, const int8_t *k_idx, const float
 int launch_pool_gather_hist(const float *tok_score, const int32_t *pool, const int64_t *ctx_len,
                             int B, int P, int64_t cap, float *pool_score, int32_t *pool_pos,
                             uint32_t *hist, cudaStream_t s);
+// The decode step's first kernel: the new rows' append (kv may be NULL) and the
+// zeroing of two workspace regions (16-byte aligned, sizes multiples of 16).
+int launch_decode_step_begin(const uint16_t *kv, int B, int C, const int64_t *ctx_len, int64_t cap,
+                             uint8_t *fp4, uint8_t *sf, void *z0, size_t z0_bytes, void *z1,
+                             size_t z1_bytes, cudaStream_t s);
 int launch_reindex_hist(const int8_t *q_idx, const int8_t *k_idx, const float *k_scale,
                         const int32_t *pool, const int64_t *ctx_len, int B, int H, int D,
                         int64_t cap, int P, float *pool_score, int32_t *pool_pos, uint32_t *hist,

@@ -16,13 +16,13 @@
 
 namespace csa2 {
 
-__global__ void __launch_bounds__(256) kv_append_fp4_kernel(
-    const uint16_t *__restrict__ kv, int B, int n_new, int C, const int64_t *__restrict__ start_pos,
-    int64_t pos_offset, int64_t cap, uint8_t *__restrict__ fp4, uint8_t *__restrict__ sf) {
-    grid_dep_wait();
-    grid_dep_launch();
+// 16-channel group gid of the B x n_new new rows.
+__device__ __forceinline__ void kv_append_group(const uint16_t *__restrict__ kv, int B, int n_new,
+                                                int C, const int64_t *__restrict__ start_pos,
+                                                int64_t pos_offset, int64_t cap,
+                                                uint8_t *__restrict__ fp4, uint8_t *__restrict__ sf,
+                                                int64_t gid) {
     const int G = C / 16;
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t total = (int64_t)B * n_new * G;
     if (gid >= total) return;
     const int g = (int)(gid % G);
@@ -58,6 +58,33 @@ __global__ void __launch_bounds__(256) kv_append_fp4_kernel(
     const int64_t cell = (int64_t)b * cap + pos;
     *reinterpret_cast<uint2 *>(fp4 + cell * (C / 2) + (int64_t)g * 8) = make_uint2(lo, hi);
     sf[cell * G + g] = (uint8_t)scode;
+}
+
+__global__ void __launch_bounds__(256) kv_append_fp4_kernel(
+    const uint16_t *__restrict__ kv, int B, int n_new, int C, const int64_t *__restrict__ start_pos,
+    int64_t pos_offset, int64_t cap, uint8_t *__restrict__ fp4, uint8_t *__restrict__ sf) {
+    grid_dep_wait();
+    grid_dep_launch();
+    kv_append_group(kv, B, n_new, C, start_pos, pos_offset, cap, fp4, sf,
+                    (int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+}
+
+// First kernel of a decode step: the new token's row of every sequence (at
+// position ctx_len - 1, when kv is given) and the zeroing of the step's two
+// workspace regions that must start at zero (z0 [n0], z1 [n1] 16-byte words).
+// A kernel instead of memsets keeps the step one chain of dependent launches.
+__global__ void __launch_bounds__(256) decode_step_begin_kernel(
+    const uint16_t *__restrict__ kv, int B, int C, const int64_t *__restrict__ ctx_len, int64_t cap,
+    uint8_t *__restrict__ fp4, uint8_t *__restrict__ sf, uint4 *z0, int64_t n0, uint4 *z1, int64_t n1) {
+    grid_dep_wait();
+    grid_dep_launch();
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    if (kv)
+        for (int64_t g = gid; g < (int64_t)B * (C / 16); g += stride)
+            kv_append_group(kv, B, 1, C, ctx_len, -1, cap, fp4, sf, g);
+    for (int64_t i = gid; i < n0; i += stride) z0[i] = make_uint4(0, 0, 0, 0);
+    for (int64_t i = gid; i < n1; i += stride) z1[i] = make_uint4(0, 0, 0, 0);
 }
 
 // MXFP4 variant: one thread per 32-channel block. The shared exponent is the
@@ -122,6 +149,20 @@ int launch_kv_append(const uint16_t *kv, int B, int n_new, int C, const int64_t 
     if (blocks > INT32_MAX) return CSA2_ERR_SHAPE;
     return launch_kernel(pdl, kv_append_fp4_kernel, dim3((unsigned)blocks), dim3(threads), 0, s, kv,
                          B, n_new, C, pos_base, pos_offset, cap, fp4, sf);
+}
+
+int launch_decode_step_begin(const uint16_t *kv, int B, int C, const int64_t *ctx_len, int64_t cap,
+                             uint8_t *fp4, uint8_t *sf, void *z0, size_t z0_bytes, void *z1,
+                             size_t z1_bytes, cudaStream_t s) {
+    const int64_t n0 = (int64_t)(z0_bytes / 16), n1 = (int64_t)(z1_bytes / 16);
+    int64_t work = kv ? (int64_t)B * (C / 16) : 0;
+    if (n0 + n1 > work) work = n0 + n1;
+    int64_t blocks = (work + 256 * 4 - 1) / (256 * 4);  // about 4 items per thread
+    if (blocks < 1) blocks = 1;
+    if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
+    return launch_kernel(true, decode_step_begin_kernel, dim3((unsigned)blocks), dim3(256), 0, s, kv, B,
+                         C, ctx_len, cap, fp4, sf, static_cast<uint4 *>(z0), n0,
+                         static_cast<uint4 *>(z1), n1);
 }
 
 }  // namespace csa2

@@ -139,7 +139,8 @@ class DecodeWorkload:
         return inputs, outputs
 
     def launches_per_step(self) -> int:
-        """libcsa2 kernels one step launches: the append, then per Full layer
+        """libcsa2 kernels one step launches: the step-begin kernel (the new
+        rows' append and the zeroing of the step's counters), then per Full layer
         the scan and one selection of the pool and its top tokens (a
         compaction kernel before it for rows of more than POOL_ONE_KERNEL_MAX
         blocks); per Reindex
@@ -148,8 +149,7 @@ class DecodeWorkload:
         after it, at most ATTN_GROUP_MAX layers per kernel) where the
         tensor-core cluster kernel takes the shape, else one per layer. A
         selection is one kernel for rows of at most TOPK_SHORT_ROW candidates,
-        else two (compaction + finish). (The per-step clear of the histograms
-        and counters is a memset, not counted.)"""
+        else two (compaction + finish)."""
         def sel(n):
             return 1 if n <= csa2.TOPK_SHORT_ROW else 2
         w = self.w

@@ -321,8 +321,9 @@ int csa2_sparse_attn_decode_mxfp4(const void *q_bf16, const uint8_t *kv_fp4, con
  *         with 0 the first non-Reuse layer must be Full.
  *  softmax_scale as given (1/sqrt(C) in the pages' reading).
  *  scan_events: NULL, or two cudaEvent_t that are recorded on `stream` right
- *         before and right after the first Full layer's indexer scan (to time
- *         that kernel inside the step).
+ *         before and right after the step's first indexer kernel: the first
+ *         Full layer's scan, or, in a stack without a Full layer, the first
+ *         Reindex rescoring (to time that kernel inside the step).
  *  ws/ws_bytes: at least csa2_decode_stack_workspace_size(...) bytes; it
  *         starts with the call's error word (csa2_workspace_status), cleared
  *         by the call.

@@ -188,9 +188,16 @@ extern "C" int csa2_decode_stack(const csa2_layer *layers, int n_layers,
             if (st) return st;
             cur = L.topk;
         } else if (L.mode == CSA2_MODE_REINDEX) {
+            // timed when the stack has no Full layer before it
+            const bool timed = scan_events && !scan_timed;
+            if (timed) cudaEventRecord((cudaEvent_t)scan_events[0], (cudaStream_t)stream);
             st = launch_reindex_hist(L.q_idx, k_idx, k_scale, pool, ctx_len, B, H, D, cap,
                                      kPoolBlocks, w.pscore, w.ppos, hist_tok, s);
             if (st) return st;
+            if (timed) {
+                cudaEventRecord((cudaEvent_t)scan_events[1], (cudaStream_t)stream);
+                scan_timed = true;
+            }
             st = launch_topk_from_hist(w.pscore, w.ppos, nullptr, B, P8, kTopK, L.topk, w.sel_tok,
                                        s);
             if (st) return st;

@@ -744,22 +744,23 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_row_hist_kernel(TopkArgs a
 // threads per row holds every candidate's position, and the rank keys (score
 // order bits, inverted index) of the threshold bin's candidates, in shared
 // memory.
-//  1. The histogram row (8 bins per thread, in registers) gives the threshold
+//  1. The histogram row (4 bins per thread, in registers) gives the threshold
 //     bin d by one block-wide suffix scan.
-//  2. One pass over the candidates (32 per thread, 16-byte loads): positions
+//  2. One pass over the candidates (16 per thread, 16-byte loads): positions
 //     to shared memory; the candidates above d go straight to a bitmap over
 //     the indices, the keys of bin d to a compact tie list.
-//  3. When only part of bin d is taken, the remaining digits (10, 10, then the
-//     index bytes) are resolved over the tie list; every key is distinct, so
-//     the last digit decides.
+//  3. When only part of bin d is taken, its best keys are found over the tie
+//     list: by rank for a short list, else by the remaining digits (10, 10,
+//     then the index bytes); every key is distinct, so the last digit decides.
 //  4. Emission in index order (= position order inside the step) through a
 //     block prefix count of the bitmap words; -1 padding; the histogram row is
 //     cleared for the next producer.
-constexpr int FT_THREADS = 512;
+constexpr int FT_THREADS = 1024;
 constexpr int FT_N = 16384;
 constexpr int FT_K = 512;
-constexpr int FT_PER = FT_N / FT_THREADS;                       // 32 candidates per thread
-constexpr int FT_BPT = TK_HIST / FT_THREADS;                    // 8 histogram bins per thread
+constexpr int FT_PER = FT_N / FT_THREADS;                       // 16 candidates per thread
+constexpr int FT_BPT = TK_HIST / FT_THREADS;                    // 4 histogram bins per thread
+static_assert(FT_BPT % 4 == 0 && FT_PER % 4 == 0 && FT_N / 32 <= FT_THREADS, "fast-path shape");
 constexpr size_t FT_SMEM = (size_t)FT_N * 8 + (size_t)FT_N * 4 + (size_t)(FT_N / 32) * 4 + 1024 * 4;
 
 __global__ void __launch_bounds__(FT_THREADS, 1) topk_fast_kernel(TopkArgs a, uint32_t *ghist) {
@@ -779,13 +780,18 @@ __global__ void __launch_bounds__(FT_THREADS, 1) topk_fast_kernel(TopkArgs a, ui
         nv = v < 0 ? 0 : (v < a.n ? (int)v : (int)a.n);
     }
     const int k = a.k;
-    // ---- 1. threshold bin from the histogram row (bins [8 tid, 8 tid + 8))
+    // ---- 1. threshold bin from the histogram row (bins [FT_BPT tid, FT_BPT tid + FT_BPT))
     uint32_t hb[FT_BPT];
     {
-        const uint4 *hp = reinterpret_cast<const uint4 *>(ghist + r * TK_HIST) + 2 * tid;
-        const uint4 h0 = hp[0], h1 = hp[1];
-        hb[0] = h0.x; hb[1] = h0.y; hb[2] = h0.z; hb[3] = h0.w;
-        hb[4] = h1.x; hb[5] = h1.y; hb[6] = h1.z; hb[7] = h1.w;
+        const uint4 *hp = reinterpret_cast<const uint4 *>(ghist + r * TK_HIST) + (FT_BPT / 4) * tid;
+#pragma unroll
+        for (int q = 0; q < FT_BPT / 4; q++) {
+            const uint4 h = hp[q];
+            hb[4 * q] = h.x;
+            hb[4 * q + 1] = h.y;
+            hb[4 * q + 2] = h.z;
+            hb[4 * q + 3] = h.w;
+        }
     }
     for (int i = tid; i < FT_N / 32; i += FT_THREADS) bm[i] = 0;
     uint32_t local = 0;
@@ -820,7 +826,7 @@ __global__ void __launch_bounds__(FT_THREADS, 1) topk_fast_kernel(TopkArgs a, ui
     }
     __syncthreads();
     const int d = all ? -1 : st.digit;
-    // ---- 2. candidates (32 per thread, 16-byte loads): the positions to shared
+    // ---- 2. candidates (16 per thread, 16-byte loads): the positions to shared
     // memory, the candidates above d to the bitmap and the threshold bin's keys
     // to a compact tie list (rank key with the index, not the position, in the
     // low bits: ties go to the lower index, which inside the step is the lower
@@ -887,7 +893,7 @@ __global__ void __launch_bounds__(FT_THREADS, 1) topk_fast_kernel(TopkArgs a, ui
         __syncthreads();
     }
     // ---- 4. emission in index order: thread t owns bitmap word t
-    const uint32_t word = bm[tid];
+    const uint32_t word = tid < FT_N / 32 ? bm[tid] : 0u;
     const int c = __popc(word);
     int rank = block_excl_scan(c, st);
     int32_t *out = a.out + r * a.k;
@@ -901,9 +907,9 @@ __global__ void __launch_bounds__(FT_THREADS, 1) topk_fast_kernel(TopkArgs a, ui
     if (tid == FT_THREADS - 1) st.nsel = rank;
     // clear the histogram row for the next producer
     {
-        uint4 *hp = reinterpret_cast<uint4 *>(ghist + r * TK_HIST) + 2 * tid;
-        hp[0] = make_uint4(0, 0, 0, 0);
-        hp[1] = make_uint4(0, 0, 0, 0);
+        uint4 *hp = reinterpret_cast<uint4 *>(ghist + r * TK_HIST) + (FT_BPT / 4) * tid;
+#pragma unroll
+        for (int q = 0; q < FT_BPT / 4; q++) hp[q] = make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
     for (int i = st.nsel + tid; i < k; i += FT_THREADS) out[i] = -1;

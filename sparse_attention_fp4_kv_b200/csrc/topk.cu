@@ -951,9 +951,14 @@ struct PoolTokArgs {
 // just wrote to a.out (row r, ascending block ids, -1 padded). All threads of
 // the CTA, after a barrier that follows the pool's writes.
 // identity_n >= 0: the pool is blocks 0 .. identity_n - 1 (a row of at most P
-// blocks), so it is not read back.
+// blocks), so it is not read back. dblk >= 0: the first-digit bin of the
+// row's pa.k-th best block score. The best pa.k tokens lie in the best pa.k
+// blocks (every block ranked ahead of a token's block holds a token ranked
+// ahead of that token), so only the pooled blocks whose score reaches bin dblk
+// are candidates: a superset of those blocks, usually about a quarter of the
+// pool.
 __device__ void pool_tokens_select(const TopkArgs &a, const PoolTokArgs &pa, int64_t r,
-                                   TopkShared sh, TopkState &st, int identity_n) {
+                                   TopkShared sh, TopkState &st, int identity_n, int dblk) {
     const int P = a.k;
     uint64_t *keys = sh.buf;
     int64_t V = pa.ctx_len[r];
@@ -968,13 +973,38 @@ __device__ void pool_tokens_select(const TopkArgs &a, const PoolTokArgs &pa, int
         for (int i0 = 0; i0 < P; i0 += TK_THREADS)
             npool += __syncthreads_count(i0 + (int)threadIdx.x < P && pool[i0 + threadIdx.x] >= 0);
     }
+    // candidate blocks in pool order (ascending), in the histogram's space until
+    // their tokens are gathered
+    int32_t *cand = reinterpret_cast<int32_t *>(sh.hist);
+    const bool filtered = identity_n < 0 && dblk >= 0;
+    if (filtered) {
+        constexpr int PPT_MAX = (kPoolBlocks + TK_THREADS - 1) / TK_THREADS;
+        const int ppt = (P + TK_THREADS - 1) / TK_THREADS;  // <= PPT_MAX (P <= kPoolBlocks)
+        int32_t cb[PPT_MAX];
+        int c = 0;
+#pragma unroll
+        for (int j = 0; j < PPT_MAX; j++) {
+            const int sl = ppt * (int)threadIdx.x + j;
+            const int32_t blk = (j < ppt && sl < npool) ? pool[sl] : -1;
+            cb[j] = (blk >= 0 && (int)hist_bin(a.score[r * a.n + blk]) >= dblk) ? blk : -1;
+            c += cb[j] >= 0;
+        }
+        int off = block_excl_scan(c, st);
+#pragma unroll
+        for (int j = 0; j < PPT_MAX; j++)
+            if (cb[j] >= 0) cand[off++] = cb[j];
+        if (threadIdx.x == TK_THREADS - 1) st.nsel = off;
+        __syncthreads();
+        npool = st.nsel;
+    }
     const int n = npool * kBlockTokens;
     const float *tok = pa.tok + r * pa.cap;
     for (int i = threadIdx.x; i < n; i += TK_THREADS) {
-        const int32_t blk = identity_n >= 0 ? (i >> 3) : pool[i >> 3];
+        const int32_t blk = filtered ? cand[i >> 3] : identity_n >= 0 ? (i >> 3) : pool[i >> 3];
         const int64_t pos = 8 * (int64_t)blk + (i & 7);
         keys[i] = (blk >= 0 && pos < V) ? rank_key(tok[pos], (int32_t)pos) : 0ull;
     }
+    if (filtered) __syncthreads();  // the candidate list is read; the histogram takes its space
     for (int b = threadIdx.x; b < TK_HIST; b += TK_THREADS) sh.hist[b] = 0;
     __syncthreads();
     for (int i = threadIdx.x; i < n; i += TK_THREADS) {
@@ -1091,8 +1121,12 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     grid_dep_launch();
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ TopkState st;
+    __shared__ int dblk_s;
     TopkShared sh = pool_tokens_shared(smem_raw);
     const int64_t r = blockIdx.x;
+    // the bin of the pa.k-th best block score, for the token candidates
+    hist_threshold<TK_THREADS>(ws.hist + r * TK_HIST, pa.k, st);
+    if (threadIdx.x == 0) dblk_s = st.total <= (uint32_t)pa.k ? -1 : st.digit;
     const int nsel0 = min(ws.cnt[2 * r], a.k);
     const int ntie = ws.cnt[2 * r + 1];
     if (threadIdx.x == 0) {
@@ -1121,7 +1155,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     for (int b = threadIdx.x; b < TK_HIST; b += TK_THREADS) ws.hist[r * TK_HIST + b] = 0;
     if (threadIdx.x < 2) ws.cnt[2 * r + threadIdx.x] = 0;
     __syncthreads();
-    pool_tokens_select(a, pa, r, sh, st, -1);
+    pool_tokens_select(a, pa, r, sh, st, -1, dblk_s);
 }
 
 // Pool from one pass over the row (as topk_row_hist_kernel), then the row's top
@@ -1132,7 +1166,11 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     grid_dep_launch();
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ TopkState st;
+    __shared__ int dblk_s;
     TopkShared sh = pool_tokens_shared(smem_raw);
+    // the bin of the pa.k-th best block score, for the token candidates
+    hist_threshold<TK_THREADS>(ghist + blockIdx.x * TK_HIST, pa.k, st);
+    if (threadIdx.x == 0) dblk_s = st.total <= (uint32_t)pa.k ? -1 : st.digit;
     topk_row_hist_body(a, blockIdx.x, ghist, sh, st);
     __syncthreads();
     // a row of at most P blocks pooled all of them, in order
@@ -1141,7 +1179,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
         const int64_t v = a.n_valid[blockIdx.x];
         nv = v < 0 ? 0 : (v < a.n ? v : a.n);
     }
-    pool_tokens_select(a, pa, blockIdx.x, sh, st, nv <= a.k ? (int)nv : -1);
+    pool_tokens_select(a, pa, blockIdx.x, sh, st, nv <= a.k ? (int)nv : -1, dblk_s);
 }
 
 }  // namespace csa2

@@ -193,6 +193,22 @@ def test_pooled_top512_equals_whole_context_top512(ctx, levels):
     assert np.array_equal(r["pool"][r["pool"] >= 0], np.sort(bo[:2048]))
 
 
+@pytest.mark.parametrize("ctx,levels", [(20000, None), (33333, None), (20000, 64)])
+def test_top512_tokens_lie_in_top512_blocks(ctx, levels):
+    """Every one of the best 512 tokens lies in one of the best 512 blocks (by
+    block max desc, block asc): each block ranked ahead of a token's block holds
+    a token ranked ahead of that token. The decode selection gathers only the
+    pooled blocks that reach the 512th block's histogram bin, a superset of
+    those blocks."""
+    q, k, s = _indexer_case(ctx, seed=ctx + 1, levels=levels)
+    r = oracle.full_layer(q, k, s, ctx)
+    blk = r["blk_score"]
+    bo = np.lexsort((np.arange(blk.size), -blk.astype(np.float64)))
+    best = set(bo[:512].tolist())
+    tv = r["top"][r["top"] >= 0]
+    assert set((tv // 8).tolist()) <= best
+
+
 def test_reindex_subset_of_pool_and_identity_with_full_query():
     ctx = 30000
     q, k, s = _indexer_case(ctx, seed=9)

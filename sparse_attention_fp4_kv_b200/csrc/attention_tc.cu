@@ -230,11 +230,12 @@ __global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
     // A cluster with at most one item keeps its dequantized selected rows for
     // every layer. With 64 heads per cluster a cluster owns whole rows, so it
     // takes its rows one after another and runs all layers of a row before the
-    // next (row_major): one gather per row and no wait on other clusters.
-    // Otherwise (several head groups per row, more items than clusters) the
-    // cluster walks its items layer by layer and gathers per item and layer.
+    // next (row_major): one gather per row, and layer l + 1 of the row follows
+    // layer l through the cluster barrier, not the per-row counters. Otherwise
+    // (several head groups per row, more items than clusters) the cluster
+    // walks its items layer by layer and gathers per item and layer.
     const bool keep = (int64_t)gridDim.y >= items;
-    const bool row_major = !keep && L::HG == 1;
+    const bool row_major = L::HG == 1;
     const int64_t n_mine =
         (int64_t)blockIdx.y < items ? (items - 1 - (int64_t)blockIdx.y) / gridDim.y + 1 : 0;
     uint32_t ld_phase = 0, pv_phase = 0;
@@ -601,17 +602,18 @@ __global__ void __launch_bounds__(THREADS, Cfg<HPC>::MIN_BLOCKS)
                 }
             }
             // this CTA's part of the row's layer-l output is written
-            if (NL > 1) {
+            if (NL > 1 && !row_major) {
                 __syncthreads();  // every thread's output stores precede the release below
                 if (tid == 0) red_release_gpu_add(lay.row_done + bq, 1);
             }
             // The slot, the tiles and TMEM are free for the next item once every
-            // CTA of the cluster has combined. With keep, the next use is the
-            // next layer of the same row, which first waits until every CTA of
-            // the row has written this layer's output (after its combine); after
-            // the last item of the last layer nothing is shared any more.
+            // CTA of the cluster has combined. With keep and several clusters per
+            // row, the next use is the next layer of the same row, which first
+            // waits until every CTA of the row has written this layer's output
+            // (after its combine); after the last item of the last layer nothing
+            // is shared any more.
             const bool last = step == n_mine * NL - 1;
-            if (!keep && !last) cluster_sync();
+            if ((!keep || row_major) && !last) cluster_sync();
         }
     }
     if (!ok) {
@@ -726,7 +728,9 @@ static int launch_tc(const AttnArgs &a, const void *const *q, const void *const 
     lay.n = n;
     lay.row_done = row_done;
     lay.row_base = row_base;
-    if (adds) *adds = n > 1 ? n * L::HG * tc::CL : 0;
+    // clusters that own whole rows follow their layers through the cluster
+    // barrier and leave the per-row counters alone
+    if (adds) *adds = (n > 1 && L::HG > 1) ? n * L::HG * tc::CL : 0;
     for (int i = 0; i < n; i++) {
         lay.q[i] = q[i];
         lay.swa[i] = swa[i];

@@ -88,8 +88,11 @@ __device__ void fs_find_digit(const uint32_t *hist, int NB, int kk, FsState &st)
 // T = 0 (take = 0) when all candidates are selected. Returns the number
 // selected. The digits start below the leading bits that all candidate keys
 // share (an OR / AND reduction), 12 bits first, then 10 at a time.
+// With k2 > 0 (k2 <= k), C2 also receives a key value that every one of the
+// best k2 keys reaches, from the first digit's histogram: the keys >= C2 are a
+// superset of the best k2 (the rest of their first-digit bin included).
 __device__ int fs_select(const uint32_t *keys, int n, int k, uint32_t *hist, FsState &st,
-                         uint32_t &T, int &take) {
+                         uint32_t &T, int &take, int k2, uint32_t &C2) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t kor = 0, kand = 0xFFFFFFFFu, cnt = 0;
     for (int i = tid; i < n; i += FS_THREADS) {
@@ -120,6 +123,7 @@ __device__ int fs_select(const uint32_t *keys, int n, int k, uint32_t *hist, FsS
         kand &= st.wand[w];
         cnt += st.wn[w];
     }
+    C2 = 1u;  // every candidate (key 0 is no candidate)
     if (cnt <= (uint32_t)k) {
         T = 0;
         take = 0;
@@ -130,6 +134,7 @@ __device__ int fs_select(const uint32_t *keys, int n, int k, uint32_t *hist, FsS
     if (L == 32) {
         T = kand;
         take = k;
+        C2 = kand;
         return k;
     }
     int shift = 32 - L > 12 ? 32 - L - 12 : 0;
@@ -148,6 +153,13 @@ __device__ int fs_select(const uint32_t *keys, int n, int k, uint32_t *hist, FsS
                 atomicAdd(&hist[hpad((int)((key >> shift) & mask))], 1u);
         }
         __syncthreads();
+        if (k2 > 0 && pshift == 32 - L) {
+            // first digit: the bin of the k2-th best key (all keys share the
+            // top L bits, so the bin's lowest key value bounds the best k2)
+            fs_find_digit(hist, (int)mask + 1, k2, st);
+            const uint32_t c = ((prefix << nbits) | (uint32_t)st.digit) << shift;
+            C2 = c ? c : 1u;
+        }
         fs_find_digit(hist, (int)mask + 1, kk, st);
         prefix = (prefix << nbits) | (uint32_t)st.digit;
         kk -= (int)st.above;
@@ -204,7 +216,7 @@ __device__ void fs_emit(KeyF key_of, int n, uint32_t T, int take, FsState &st, F
     __syncthreads();
 }
 
-__global__ void __launch_bounds__(FS_THREADS) full_select_kernel(
+__global__ void __launch_bounds__(FS_THREADS, 3) full_select_kernel(
     const float *__restrict__ blk, const int32_t *__restrict__ n_blk, const float *__restrict__ tok,
     const int64_t *ctx_len, const int64_t *q_pos, int B, int Nq, int64_t cap, int P, int K,
     int32_t *__restrict__ pool, int32_t *__restrict__ top) {
@@ -243,9 +255,9 @@ __global__ void __launch_bounds__(FS_THREADS) full_select_kernel(
         }
     }
     __syncthreads();
-    uint32_t T;
+    uint32_t T, C2;
     int take;
-    const int npool = fs_select(keys, nb, P, hist, st, T, take);
+    const int npool = fs_select(keys, nb, P, hist, st, T, take, K < P ? K : 0, C2);
     fs_emit([&](int i) { return keys[i]; }, nb, T, take, st, [&](int slot, int i) { pool_s[slot] = i; });
     int32_t *prow = pool + row * P;
     for (int s = tid; s < P; s += FS_THREADS) {
@@ -254,15 +266,27 @@ __global__ void __launch_bounds__(FS_THREADS) full_select_kernel(
     }
     __syncthreads();
 
-    // ---- 2. the best min(K, P) blocks, found inside the pool (ascending)
+    // ---- 2. blocks whose tokens are candidates (ascending): the pooled blocks
+    // whose key reaches C2, a superset of the best K blocks, when their tokens
+    // fit the key array; else exactly the best K blocks
     const int32_t *kblk = pool_s;
     int nkb = npool;
     if (K < npool) {
-        fs_select(keys, nb, K, hist, st, T, take);
-        fs_emit([&](int s) { return keys[pool_s[s]]; }, npool, T, take, st,
-                [&](int slot, int s) { kblk_s[slot] = pool_s[s]; });
+        int n_c2 = 0;
+        for (int s0 = 0; s0 < npool; s0 += FS_THREADS)
+            n_c2 += __syncthreads_count(s0 + tid < npool && keys[pool_s[s0 + tid]] >= C2);
+        if (8 * (int64_t)n_c2 <= nkeys) {
+            fs_emit([&](int s) { return keys[pool_s[s]]; }, npool, C2 - 1u, 0, st,
+                    [&](int slot, int s) { kblk_s[slot] = pool_s[s]; });
+            nkb = n_c2;
+        } else {
+            uint32_t unused;
+            fs_select(keys, nb, K, hist, st, T, take, 0, unused);
+            fs_emit([&](int s) { return keys[pool_s[s]]; }, npool, T, take, st,
+                    [&](int slot, int s) { kblk_s[slot] = pool_s[s]; });
+            nkb = K;
+        }
         kblk = kblk_s;
-        nkb = K;
     }
 
     // ---- 3. their token scores in position order, then the best K tokens
@@ -286,7 +310,8 @@ __global__ void __launch_bounds__(FS_THREADS) full_select_kernel(
         }
     }
     __syncthreads();
-    const int ntop = fs_select(keys, n2, K, hist, st, T, take);
+    uint32_t unused;
+    const int ntop = fs_select(keys, n2, K, hist, st, T, take, 0, unused);
     int32_t *trow_out = top + row * K;
     fs_emit([&](int i) { return keys[i]; }, n2, T, take, st,
             [&](int slot, int i) { trow_out[slot] = 8 * kblk[i >> 3] + (i & 7); });

@@ -268,7 +268,8 @@ int csa2_index_reindex(const int8_t *q_idx, const int8_t *k_idx, const float *k_
  *  C % 32 == 0, 32 <= C <= 1024; 1 <= Hq <= 256; 0 <= K <= 4096; 0 <= n_win <= 4096.
  *  ws/ws_bytes: at least csa2_sparse_attn_workspace_size(...) bytes (0 for
  *           shapes whose kernel has no bounded wait and no scratch: then ws
- *           may be NULL). It starts with the call's error word (read with
+ *           may be NULL), 16-byte aligned (CSA2_ERR_ALIGN otherwise; device
+ *           allocations are). It starts with the call's error word (read with
  *           csa2_workspace_status); the rest is the kernels' exchange space.
  * ------------------------------------------------------------------------ */
 size_t csa2_sparse_attn_workspace_size(int B, int Nq, int Hq, int C, int K, int n_win);
@@ -324,9 +325,10 @@ int csa2_sparse_attn_decode_mxfp4(const void *q_bf16, const uint8_t *kv_fp4, con
  *         before and right after the step's first indexer kernel: the first
  *         Full layer's scan, or, in a stack without a Full layer, the first
  *         Reindex rescoring (to time that kernel inside the step).
- *  ws/ws_bytes: at least csa2_decode_stack_workspace_size(...) bytes; it
- *         starts with the call's error word (csa2_workspace_status), cleared
- *         by the call.
+ *  ws/ws_bytes: at least csa2_decode_stack_workspace_size(...) bytes,
+ *         16-byte aligned (CSA2_ERR_ALIGN otherwise; device allocations
+ *         are); it starts with the call's error word (csa2_workspace_status),
+ *         cleared by the call.
  *  Errors: CSA2_ERR_RANGE if a Reuse layer has no preceding Full/Reindex
  *  layer or a Reindex layer has no pool; nothing is launched then.
  * ------------------------------------------------------------------------ */

@@ -123,6 +123,9 @@ extern "C" int csa2_decode_stack(const csa2_layer *layers, int n_layers,
     if (kv_new_bf16 && !aligned(kv_new_bf16, 16)) return CSA2_ERR_ALIGN;
     const StackWs w = stack_layout(ws, B, Hq, C, cap);
     if (!ws || ws_bytes < w.total) return CSA2_ERR_WORKSPACE;
+    // the kernels read the workspace's histograms, lists and exchange slots
+    // with 16-byte accesses
+    if (!aligned(ws, 16)) return CSA2_ERR_ALIGN;
     // host-side schedule check before anything is launched
     bool have_pool = pool_ready != 0, have_idx = false;
     for (int l = 0; l < n_layers; l++) {
@@ -150,22 +153,10 @@ extern "C" int csa2_decode_stack(const csa2_layer *layers, int n_layers,
     // The append of the new rows, and the error word, the selection histograms
     // and counters and the attention layer counters set to zero (every
     // finishing top-k kernel also leaves its rows clear for the next
-    // producer): one kernel, or the append and two memsets when the workspace
-    // is not 16-byte aligned.
-    if (aligned(ws, 16)) {
-        st = launch_decode_step_begin((const uint16_t *)kv_new_bf16, B, C, ctx_len, cap, kv_fp4, kv_sf,
-                                      w.err, w.zero_bytes, w.sel_tok, w.hist_bytes, s);
-        if (st) return st;
-    } else {
-        if (kv_new_bf16) {
-            st = launch_kv_append((const uint16_t *)kv_new_bf16, B, 1, C, ctx_len, -1, cap, kv_fp4,
-                                  kv_sf, s, true);
-            if (st) return st;
-        }
-        if (cudaMemsetAsync(w.err, 0, w.zero_bytes, s) != cudaSuccess ||
-            cudaMemsetAsync(w.sel_tok, 0, w.hist_bytes, s) != cudaSuccess)
-            return CSA2_ERR_CUDA;
-    }
+    // producer), in one kernel.
+    st = launch_decode_step_begin((const uint16_t *)kv_new_bf16, B, C, ctx_len, cap, kv_fp4, kv_sf,
+                                  w.err, w.zero_bytes, w.sel_tok, w.hist_bytes, s);
+    if (st) return st;
     uint32_t *hist_blk = topk_hist_ptr_of(w.sel_blk);
     uint32_t *hist_tok = topk_hist_ptr_of(w.sel_tok);
     int row_base = 0;  // value of every per-row layer counter before the next group

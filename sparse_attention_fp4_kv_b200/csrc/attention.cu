@@ -471,6 +471,7 @@ int attn_call(AttnArgs a, size_t ws_bytes, cudaStream_t s) {
     const size_t need = attn_workspace_bytes(a.B, a.Nq, a.Hq, a.C, a.K, a.n_win);
     if (need == 0) return attn_checked_launch(a, ws_bytes, s);
     if (a.ws == nullptr || ws_bytes < need) return CSA2_ERR_WORKSPACE;
+    if (!aligned(a.ws, 16)) return CSA2_ERR_ALIGN;  // 16-byte accesses to the exchange slots
     a.err = static_cast<int *>(a.ws);
     if (cudaMemsetAsync(a.err, 0, sizeof(int), s) != cudaSuccess) return CSA2_ERR_CUDA;
     a.ws = static_cast<char *>(a.ws) + kErrWordBytes;

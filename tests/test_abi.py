@@ -73,6 +73,11 @@ def test_host_validation_codes():
                                      None) == -2
     # alignment
     assert L.csa2_kv_append_fp4(odd, 1, 1, 512, good, 10, good, good, None) == -3
+    need = L.csa2_sparse_attn_workspace_size(1, 1, 64, 512, 512, 128)
+    assert need > 0
+    assert L.csa2_sparse_attn_decode(good, good, good, 1000, good, 512, good, good, 128, None, 128,
+                                     1, 1, 64, 512, ctypes.c_float(0.04), good, odd, need + 64,
+                                     None) == -3
     assert L.csa2_index_full(odd, good, good, good, None, 1, 1, 16, 128, 10, None, good, None,
                              None) == -3
     # empty work is a no-op
@@ -114,6 +119,10 @@ def test_decode_stack_schedule_checks():
     small = list(args)
     small[-2] = ws_need - 1
     assert B.lib.csa2_decode_stack(layers, 2, None, *small) == -5
+    # workspace not 16-byte aligned: rejected before anything is launched
+    odd = list(args)
+    odd[-3] = P(4096 + 8)
+    assert B.lib.csa2_decode_stack(layers, 2, None, *odd) == -3
     # unknown mode
     layers[1] = B.csa2_layer(7, good, good, good, good, good)
     assert B.lib.csa2_decode_stack(layers, 2, None, *args) == -4

@@ -154,6 +154,54 @@ __device__ void hist_threshold(const uint32_t *gh, int kk, TopkState &st) {
     __syncthreads();
 }
 
+// hist_threshold for rank k1 (into st) and, from the same registers, the bin
+// of rank k2 into *d2 (-1 when the row holds at most k2 keys): one read of the
+// histogram row for both.
+template <int NT>
+__device__ void hist_threshold2(const uint32_t *gh, int k1, int k2, TopkState &st, int *d2) {
+    constexpr int BPT = TK_HIST / NT;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t hb[BPT];
+    const uint4 *hp = reinterpret_cast<const uint4 *>(gh) + (BPT / 4) * tid;
+#pragma unroll
+    for (int q = 0; q < BPT / 4; q++) {
+        const uint4 v = hp[q];
+        hb[4 * q] = v.x;
+        hb[4 * q + 1] = v.y;
+        hb[4 * q + 2] = v.z;
+        hb[4 * q + 3] = v.w;
+    }
+    uint32_t local = 0;
+#pragma unroll
+    for (int j = 0; j < BPT; j++) local += hb[j];
+    uint32_t x = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
+        if (lane + o < 32) x += y;
+    }
+    if (lane == 0) st.wsum[warp] = x;
+    if (tid == 0) *d2 = -1;
+    __syncthreads();
+    uint32_t above = x - local, total = 0;
+    for (int w = 0; w < NT / 32; w++) {
+        total += st.wsum[w];
+        if (w > warp) above += st.wsum[w];
+    }
+#pragma unroll
+    for (int j = BPT - 1; j >= 0; j--) {
+        if (above < (uint32_t)k1 && above + hb[j] >= (uint32_t)k1) {
+            st.digit = BPT * tid + j;
+            st.above = above;
+            st.match = hb[j];
+        }
+        if (total > (uint32_t)k2 && above < (uint32_t)k2 && above + hb[j] >= (uint32_t)k2) *d2 = BPT * tid + j;
+        above += hb[j];
+    }
+    if (tid == 0) st.total = total;
+    __syncthreads();
+}
+
 // Candidate i of row r from global memory; false if it is not a candidate.
 __device__ __forceinline__ bool load_cand(const TopkArgs &a, int64_t r, int64_t i, uint64_t &key) {
     const int32_t pos = a.cand_pos ? a.cand_pos[r * a.n + i] : (int32_t)i;
@@ -1124,9 +1172,6 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     __shared__ int dblk_s;
     TopkShared sh = pool_tokens_shared(smem_raw);
     const int64_t r = blockIdx.x;
-    // the bin of the pa.k-th best block score, for the token candidates
-    hist_threshold<TK_THREADS>(ws.hist + r * TK_HIST, pa.k, st);
-    if (threadIdx.x == 0) dblk_s = st.total <= (uint32_t)pa.k ? -1 : st.digit;
     const int nsel0 = min(ws.cnt[2 * r], a.k);
     const int ntie = ws.cnt[2 * r + 1];
     if (threadIdx.x == 0) {
@@ -1135,7 +1180,9 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
         st.nsel = 0;
         st.nbuf = 0;
     }
-    hist_threshold<TK_THREADS>(ws.hist + r * TK_HIST, a.k, st);
+    // the pool's threshold bin, and the bin of the pa.k-th best block score for
+    // the token candidates, from one read of the histogram
+    hist_threshold2<TK_THREADS>(ws.hist + r * TK_HIST, a.k, pa.k, st, &dblk_s);
     const bool all = st.total <= (uint32_t)a.k;
     if ((!all && ntie > TK_BUF) || a.n > TF_MAX_N) {
         __syncthreads();

@@ -23,9 +23,6 @@ N_WIN = 128
 # Rows of at most this many candidates are selected by one single-CTA kernel
 # inside the decode step; longer rows take a compaction and a finishing kernel.
 TOPK_SHORT_ROW = 65536
-# The decode Full layer's pool and top-512 run as one kernel per row for rows of
-# up to this many blocks (a compaction kernel first for longer rows).
-POOL_ONE_KERNEL_MAX = 65536
 # csa2_full_select holds a row of block scores (and of pooled token scores) in
 # shared memory: at most this many of each.
 FULL_SELECT_MAX = 16384

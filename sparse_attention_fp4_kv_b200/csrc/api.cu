@@ -80,7 +80,7 @@ StackWs stack_layout(void *base, int B, int Hq, int C, int64_t cap) {
     off += up(topk_hist_ws_bytes(B, kPoolBlocks));
     w.sel_tok = p + off;
     off += up(topk_hist_ws_bytes(B, kTopK));
-    w.hist_bytes = up((size_t)B * kHistBins * 4) + up((size_t)B * 2 * 4);
+    w.hist_bytes = topk_hist_zero_bytes(B);
     w.zero_bytes = kErrWordBytes + up(sizeof(int) * (size_t)B) + w.hist_bytes;
     w.tok = reinterpret_cast<float *>(p + off);
     off += up(sizeof(float) * (size_t)B * cap);

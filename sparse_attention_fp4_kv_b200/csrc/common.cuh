@@ -242,10 +242,13 @@ constexpr int kHistBins = 4096;
 __device__ __forceinline__ uint32_t hist_bin(float score) { return f32_order_key(score) >> 20; }
 
 // Histogram-fed top-k (topk.cu): the workspace starts with hist[R][4096] and
-// two counters per row, all zero before the producer runs. This launcher and
+// four counters per row, all zero before the producer runs. This launcher and
 // the three score producers below serve the decode step only and launch with
 // programmatic stream serialization.
 size_t topk_hist_ws_bytes(int R, int k);
+// The leading bytes of such a workspace (histogram rows and per-row counters)
+// that must be zero before a producer adds to it.
+size_t topk_hist_zero_bytes(int R);
 // Pool and top tokens of the decode Full layer in one selection (topk.cu).
 int launch_pool_and_tokens(const float *blk, const int32_t *n_blk, int R, int64_t nblk, int P,
                            int32_t *pool, void *ws, const float *tok, const int64_t *ctx_len,

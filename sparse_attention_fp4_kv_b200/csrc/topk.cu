@@ -436,7 +436,7 @@ constexpr int64_t TF_MAX_N = (int64_t)TK_BUF * 2 * 32;  // bitmap capacity of th
 
 struct TopkHistWs {
     uint32_t *hist;  // [R][4096]
-    int *cnt;        // [R][2]: selected, ties
+    int *cnt;        // [R][4]: selected, ties, CTAs done (fused compaction), unused
     int32_t *sel;    // [R][k] candidate indices
     uint64_t *tie;   // [R][TK_BUF] keys
 };
@@ -524,8 +524,8 @@ __global__ void __launch_bounds__(TC_THREADS) topk_compact_kernel(TopkArgs a, To
             ts += a1;
             tt += a2;
         }
-        cbase[0] = ts ? atomicAdd(ws.cnt + 2 * r, ts) : 0;
-        cbase[1] = tt ? atomicAdd(ws.cnt + 2 * r + 1, tt) : 0;
+        cbase[0] = ts ? atomicAdd(ws.cnt + 4 * r, ts) : 0;
+        cbase[1] = tt ? atomicAdd(ws.cnt + 4 * r + 1, tt) : 0;
     }
     __syncthreads();
     int bs = cbase[0] + wsel[warp] + is - ns;
@@ -661,8 +661,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_finish_kernel(TopkArgs a, 
     __shared__ TopkState st;
     TopkShared sh = topk_shared(smem_raw);
     const int64_t r = blockIdx.x;
-    const int nsel0 = min(ws.cnt[2 * r], a.k);
-    const int ntie = ws.cnt[2 * r + 1];
+    const int nsel0 = min(ws.cnt[4 * r], a.k);
+    const int ntie = ws.cnt[4 * r + 1];
     if (threadIdx.x == 0) {
         st.prefix = 0;
         st.mask = 0;
@@ -687,7 +687,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_finish_kernel(TopkArgs a, 
     // leave the histogram and counters of this row clear for the next producer
     __syncthreads();
     for (int b = threadIdx.x; b < TK_HIST; b += TK_THREADS) ws.hist[r * TK_HIST + b] = 0;
-    if (threadIdx.x < 2) ws.cnt[2 * r + threadIdx.x] = 0;
+    if (threadIdx.x < 3) ws.cnt[4 * r + threadIdx.x] = 0;
 }
 
 // Rows of at most TS_MAX_N candidates skip the global lists: one CTA per row
@@ -1161,19 +1161,13 @@ __device__ void pool_tokens_select(const TopkArgs &a, const PoolTokArgs &pa, int
     for (int i = st.nsel + threadIdx.x; i < pa.k; i += TK_THREADS) out[i] = -1;
 }
 
-// Pool from the compacted global lists (as topk_finish_kernel), then the row's
-// top tokens among the pooled tokens.
-__global__ void __launch_bounds__(TK_THREADS, 1)
-    topk_finish_pool_tokens_kernel(TopkArgs a, TopkHistWs ws, PoolTokArgs pa) {
-    grid_dep_wait();
-    grid_dep_launch();
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    __shared__ TopkState st;
-    __shared__ int dblk_s;
-    TopkShared sh = pool_tokens_shared(smem_raw);
-    const int64_t r = blockIdx.x;
-    const int nsel0 = min(ws.cnt[2 * r], a.k);
-    const int ntie = ws.cnt[2 * r + 1];
+// Pool of row r from the compacted global lists (as topk_finish_kernel), then
+// the row's top tokens among the pooled tokens. All threads of a CTA of
+// TK_THREADS; the lists and counters of the row are complete and visible.
+__device__ void finish_pool_tokens_row(const TopkArgs &a, const TopkHistWs &ws, const PoolTokArgs &pa,
+                                       int64_t r, TopkShared sh, TopkState &st, int &dblk_s) {
+    const int nsel0 = min(ws.cnt[4 * r], a.k);
+    const int ntie = ws.cnt[4 * r + 1];
     if (threadIdx.x == 0) {
         st.prefix = 0;
         st.mask = 0;
@@ -1200,9 +1194,94 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     // leave the histogram and counters of this row clear for the next producer
     __syncthreads();
     for (int b = threadIdx.x; b < TK_HIST; b += TK_THREADS) ws.hist[r * TK_HIST + b] = 0;
-    if (threadIdx.x < 2) ws.cnt[2 * r + threadIdx.x] = 0;
+    if (threadIdx.x < 3) ws.cnt[4 * r + threadIdx.x] = 0;
     __syncthreads();
     pool_tokens_select(a, pa, r, sh, st, -1, dblk_s);
+}
+
+// Rows longer than PT_ONE_CTA_MAX_N blocks in one launch: CTA (x, r) compacts
+// blocks [x TK_THREADS 4, ...) of row r into the row's global lists (the
+// indices above the threshold bin and the bin's keys, slots by one global
+// atomic per list per CTA), then takes a ticket; the last CTA of the row
+// finishes the pool and selects the row's top tokens. The ticket is a release /
+// acquire pair (fences around the atomic), so no CTA waits on another.
+constexpr int TC2_SLICE = TK_THREADS * 4;  // candidates per CTA, one 16-byte load per thread
+
+__global__ void __launch_bounds__(TK_THREADS, 1)
+    topk_compact_pool_tokens_kernel(TopkArgs a, TopkHistWs ws, PoolTokArgs pa) {
+    grid_dep_wait();
+    grid_dep_launch();
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __shared__ TopkState st;
+    __shared__ int dblk_s, last_s, wsel[TK_THREADS / 32], wtie[TK_THREADS / 32], cbase[2];
+    const int64_t r = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int64_t nv = a.n;
+    if (a.n_valid) {
+        const int64_t v = a.n_valid[r];
+        nv = v < 0 ? 0 : (v < a.n ? v : a.n);
+    }
+    const int64_t i_beg = (int64_t)blockIdx.x * TC2_SLICE;
+    if (i_beg < nv) {  // uniform over the CTA
+        hist_threshold<TK_THREADS>(ws.hist + r * TK_HIST, a.k, st);
+        const bool all = st.total <= (uint32_t)a.k;
+        const uint64_t d = (uint64_t)st.digit;
+        const bool vec = ((r * a.n) % 4 == 0) && aligned16(a.score) &&
+                         (a.cand_pos == nullptr || aligned16(a.cand_pos));
+        const int64_t i0 = i_beg + 4 * (int64_t)threadIdx.x;
+        uint64_t pk[4];
+        bool ok[4];
+        load_cand4(a, r, i0, nv, vec, pk, ok);
+        uint32_t selm = 0, tiem = 0;
+#pragma unroll
+        for (int v = 0; v < 4; v++) {
+            const uint64_t bin = pk[v] >> 52;
+            if (ok[v] && (all || bin > d)) selm |= 1u << v;
+            else if (ok[v] && bin == d) tiem |= 1u << v;
+        }
+        const int ns = __popc(selm), nt = __popc(tiem);
+        const int is = warp_incl_scan(ns), it = warp_incl_scan(nt);
+        if (lane == 31) {
+            wsel[warp] = is;
+            wtie[warp] = it;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int ts = 0, tt = 0;
+            for (int w = 0; w < TK_THREADS / 32; w++) {
+                const int a1 = wsel[w], a2 = wtie[w];
+                wsel[w] = ts;
+                wtie[w] = tt;
+                ts += a1;
+                tt += a2;
+            }
+            cbase[0] = ts ? atomicAdd(ws.cnt + 4 * r, ts) : 0;
+            cbase[1] = tt ? atomicAdd(ws.cnt + 4 * r + 1, tt) : 0;
+        }
+        __syncthreads();
+        int bs = cbase[0] + wsel[warp] + is - ns;
+        int bt = cbase[1] + wtie[warp] + it - nt;
+#pragma unroll
+        for (int v = 0; v < 4; v++) {
+            if (selm & (1u << v)) {
+                if (bs < a.k) ws.sel[r * a.k + bs] = (int32_t)(i0 + v);
+                bs++;
+            } else if (tiem & (1u << v)) {
+                // index-keyed: the ordered score bits above the inverted index
+                if (bt < TK_BUF)
+                    ws.tie[r * TK_BUF + bt] = (pk[v] & 0xFFFFFFFF00000000ull) | (uint32_t)~(uint32_t)(i0 + v);
+                bt++;
+            }
+        }
+    }
+    // this CTA's list entries are written: take the row's ticket
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last_s = atomicAdd(ws.cnt + 4 * r + 2, 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (!last_s) return;
+    __threadfence();  // every other CTA's entries of this row are visible
+    finish_pool_tokens_row(a, ws, pa, r, pool_tokens_shared(smem_raw), st, dblk_s);
 }
 
 // Pool from one pass over the row (as topk_row_hist_kernel), then the row's top
@@ -1237,8 +1316,14 @@ namespace csa2 {
 
 size_t topk_hist_ws_bytes(int R, int k) {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-    return up((size_t)R * TK_HIST * 4) + up((size_t)R * 2 * 4) + up((size_t)R * k * 4) +
-           up((size_t)R * TK_BUF * 8);
+    return topk_hist_zero_bytes(R) + up((size_t)R * k * 4) + up((size_t)R * TK_BUF * 8);
+}
+
+// The leading bytes of a selection workspace that must be zero before a
+// producer fills it: the histogram rows and the counters.
+size_t topk_hist_zero_bytes(int R) {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    return up((size_t)R * TK_HIST * 4) + up((size_t)R * 4 * 4);
 }
 
 static TopkHistWs topk_hist_ws(void *base, int R, int k) {
@@ -1248,7 +1333,7 @@ static TopkHistWs topk_hist_ws(void *base, int R, int k) {
     w.hist = reinterpret_cast<uint32_t *>(p);
     p += up((size_t)R * TK_HIST * 4);
     w.cnt = reinterpret_cast<int *>(p);
-    p += up((size_t)R * 2 * 4);
+    p += up((size_t)R * 4 * 4);
     w.sel = reinterpret_cast<int32_t *>(p);
     p += up((size_t)R * k * 4);
     w.tie = reinterpret_cast<uint64_t *>(p);
@@ -1287,15 +1372,16 @@ int launch_topk_from_hist(const float *score, const int32_t *cand_pos, const int
 
 // The decode Full layer's pool (k = P blocks of the block scores blk, whose
 // histogram the scan filled) and the top ktop tokens among the pooled tokens
-// (token scores tok [R][cap]): written to pool and top. One kernel per row, or
-// compaction + one kernel per row for rows longer than TS_MAX_N blocks.
+// (token scores tok [R][cap]): written to pool and top. One CTA per row, or for
+// rows longer than PT_ONE_CTA_MAX_N blocks a compaction over many CTAs per row
+// whose last CTA finishes the row: one launch either way.
 int launch_pool_and_tokens(const float *blk, const int32_t *n_blk, int R, int64_t nblk, int P,
                            int32_t *pool, void *ws, const float *tok, const int64_t *ctx_len,
                            int64_t cap, int ktop, int32_t *top, cudaStream_t s) {
     if (R == 0) return CSA2_OK;
     if (R > 65535 || P * kBlockTokens > PT_MAX || ktop > TK_MAXK) return CSA2_ERR_SHAPE;
     static PerDevice smem_set[2];
-    if (!set_smem_limit_once(smem_set[0], topk_finish_pool_tokens_kernel, PT_SMEM) ||
+    if (!set_smem_limit_once(smem_set[0], topk_compact_pool_tokens_kernel, PT_SMEM) ||
         !set_smem_limit_once(smem_set[1], topk_row_pool_tokens_kernel, PT_SMEM))
         return CSA2_ERR_CUDA;
     TopkArgs a{blk, nullptr, n_blk, R, nblk, P, pool};
@@ -1304,12 +1390,10 @@ int launch_pool_and_tokens(const float *blk, const int32_t *n_blk, int R, int64_
     if (nblk <= PT_ONE_CTA_MAX_N)
         return launch_kernel(true, topk_row_pool_tokens_kernel, dim3(R), dim3(TK_THREADS), PT_SMEM, s,
                              a, w.hist, pa);
-    const int64_t slices = (nblk + TC_SLICE - 1) / TC_SLICE;
-    const int st = launch_kernel(true, topk_compact_kernel, dim3((unsigned)slices, (unsigned)R),
-                                 dim3(TC_THREADS), 0, s, a, w);
-    if (st) return st;
-    return launch_kernel(true, topk_finish_pool_tokens_kernel, dim3(R), dim3(TK_THREADS), PT_SMEM, s, a,
-                         w, pa);
+    const int64_t slices = (nblk + TC2_SLICE - 1) / TC2_SLICE;
+    if (slices > 65535) return CSA2_ERR_SHAPE;
+    return launch_kernel(true, topk_compact_pool_tokens_kernel, dim3((unsigned)slices, (unsigned)R),
+                         dim3(TK_THREADS), PT_SMEM, s, a, w, pa);
 }
 
 }  // namespace csa2

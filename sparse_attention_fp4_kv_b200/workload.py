@@ -141,9 +141,7 @@ class DecodeWorkload:
     def launches_per_step(self) -> int:
         """libcsa2 kernels one step launches: the step-begin kernel (the new
         rows' append and the zeroing of the step's counters), then per Full layer
-        the scan and one selection of the pool and its top tokens (a
-        compaction kernel before it for rows of more than POOL_ONE_KERNEL_MAX
-        blocks); per Reindex
+        the scan and one selection of the pool and its top tokens; per Reindex
         layer the rescoring and the token selection. Attention: one
         kernel per layer group (a Full or Reindex layer and the Reuse layers
         after it, at most ATTN_GROUP_MAX layers per kernel) where the
@@ -153,14 +151,12 @@ class DecodeWorkload:
         def sel(n):
             return 1 if n <= csa2.TOPK_SHORT_ROW else 2
         w = self.w
-        nblk = (self.kv_fp4.shape[1] + 7) // 8
         pooled = csa2.POOL_BLOCKS * csa2.BLOCK_TOKENS
         grouped = w.C == 512 and w.Hq == 64 and w.B < csa2.ATTN_ROWS_MIN
         n = 1
         run = 0  # layers in the current attention launch
         for m in self.modes:
-            full_sel = 1 if nblk <= csa2.POOL_ONE_KERNEL_MAX else 2
-            n += {synth.FULL: 1 + full_sel, synth.REINDEX: 1 + sel(pooled), synth.REUSE: 0}[m]
+            n += {synth.FULL: 2, synth.REINDEX: 1 + sel(pooled), synth.REUSE: 0}[m]
             if grouped and m == synth.REUSE and 0 < run < csa2.ATTN_GROUP_MAX:
                 run += 1
             else:

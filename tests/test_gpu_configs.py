@@ -116,11 +116,45 @@ def test_stack_tie_heavy_keys(levels):
     _free()
 
 
+@pytest.mark.parametrize("levels", [0, 1])
+def test_stack_ragged_long_rows(levels):
+    """Sequences of 532,000, 300,001 and 9 tokens in one step over a
+    532,000-token cache: the pool selection takes its many-CTA form (rows of
+    more than 65,536 blocks), whose CTAs past a short row's end only take the
+    row's ticket, and whose last CTA per row finishes the row. levels=1 makes
+    every indexer score zero, so the pool's threshold bin holds the whole row
+    (more ties than the compacted tie list holds)."""
+    ctxs = [532000, 300001, 9]
+    wl = _workload("decoder_stack20_b4_ctx1m", B=3, ctx=ctxs[0], modes=[synth.FULL, synth.REUSE])
+    if levels:
+        wl.k_idx.zero_()
+    rows = wl.swa_rows
+    for b, c in enumerate(ctxs):
+        wl.ctx_len[b] = c
+        wl.swa_pos0[b] = c - rows  # the window's last row is position c - 1
+        wl.kv_bf16[b, c - 1] = wl.kv_new[b]  # the step appends the new token at c - 1
+    wl.step()
+    torch.cuda.synchronize()
+    for b, c in enumerate(ctxs):
+        kn, sn = wl.k_idx[b].cpu().numpy(), wl.k_scale[b].cpu().numpy()
+        r = oracle.full_layer(wl.q_idx[0][b, 0].cpu().numpy(), kn, sn, c)
+        assert np.array_equal(wl.pool[b].cpu().numpy(), r["pool"]), f"pool b={b}"
+        assert np.array_equal(wl.topk[0][b].cpu().numpy(), r["top"]), f"top-512 b={b}"
+        kvb = bf16_np(wl.kv_bf16[b, :c])
+        for l in range(2):
+            ref = oracle.sparse_attention(bf16_np(wl.q[l][b, 0]), lambda P: kvb[P], r["top"],
+                                          bf16_np(wl.swa[l][b]), c - 1, c - rows, wl.scale)
+            assert_attn_close(wl.out[l][b, 0].cpu().numpy(), ref, f"attention b={b} l={l}")
+    del wl
+    _free()
+
+
 @pytest.mark.parametrize("ctx", [30000, 600000])
 def test_launches_per_step_matches_profiler(ctx):
     """The kernel count the benchmark reports equals the libcsa2 kernels the
     CUDA profiler sees in one step (600K tokens: the pool selection's rows are
-    long enough to take two kernels)."""
+    long enough to take the many-CTA compaction whose last CTA per row
+    finishes it)."""
     wl = _workload("decoder_stack20_b4_ctx1m", B=1, ctx=ctx)
     wl.step()
     torch.cuda.synchronize()

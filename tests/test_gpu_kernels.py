@@ -424,7 +424,10 @@ def test_reindex_bitexact(B):
 
 
 # ----------------------------------------------------------------------------- a8 attention
-def _attention_case(B, Bn, ctx, C, Hq, K, n_win, seed, q_pos=None, Nq=1, drop=0, mx=False):
+def _attention_case(B, Bn, ctx, C, Hq, K, n_win, seed, q_pos=None, Nq=1, drop=0, mx=False,
+                    q_mul=None):
+    """q_mul [Hq]: factors applied to Q per head (then rounded to bf16, the
+    values both sides see)."""
     w = synth.scaled(synth.WORKLOADS["decoder_group1_b8_ctx128k"], B=Bn, ctx=ctx, C=C, Hq=Hq,
                      seed=seed)
     kv = torch.stack([synth.main_kv_bf16(w, b, 0, ctx, DEV) for b in range(Bn)])
@@ -432,6 +435,8 @@ def _attention_case(B, Bn, ctx, C, Hq, K, n_win, seed, q_pos=None, Nq=1, drop=0,
     sf = torch.empty((Bn, ctx, C // (32 if mx else 16)), dtype=torch.uint8, device=DEV)
     B.csa2_kv_append_fp4(kv, torch.zeros(Bn, dtype=torch.int64, device=DEV), fp4, sf, mx=mx)
     q = synth.main_q(w, 0, Nq, DEV)
+    if q_mul is not None:
+        q = (q.float() * q_mul.to(DEV).view(1, 1, Hq, 1)).to(torch.bfloat16)
     g = torch.Generator(device=DEV).manual_seed(seed)
     kk = min(K, ctx)
     top = torch.stack([torch.stack([torch.randperm(ctx, generator=g, device=DEV)[:kk].sort().values
@@ -520,6 +525,15 @@ def test_sparse_attention_head_groups(B, Bn, Nq, drop, n_win):
                                                 (3, 8, 576, 64, 7)])
 def test_sparse_attention_one_cta_per_row(B, Bn, Nq, K, n_win, drop):
     _attention_case(B, Bn, 3000, 512, 64, K, n_win, seed=7 * Bn + K + n_win, Nq=Nq, drop=drop)
+
+
+def test_sparse_attention_one_cta_per_row_q_magnitudes(B):
+    """Heads whose Q lies anywhere from 2^-60 to 2^66 times N(0, 1): softmax from
+    uniform to one-hot, on the per-row kernel (40-row calls) and the split-key
+    clusters (one row)."""
+    mul = torch.tensor([2.0 ** e for e in range(-60, 68, 2)], dtype=torch.float32)
+    _attention_case(B, 2, 3000, 512, 64, 512, 128, seed=13, Nq=40, q_mul=mul)
+    _attention_case(B, 1, 3000, 512, 64, 512, 128, seed=14, drop=5, q_mul=mul)
 
 
 def test_sparse_attention_one_cta_per_row_causal_positions(B):

@@ -75,6 +75,8 @@ def _free():
 @pytest.mark.parametrize("name,kw", [
     ("decoder_stack20_b4_ctx1m", dict(B=3, ctx=20003)),
     ("decoder_stack20_b4_ctx1m", dict(B=2, ctx=16389)),
+    # an indexer of 4 x 64 channels (the rescoring's generic row shapes)
+    ("decoder_stack20_b4_ctx1m", dict(B=2, ctx=20003, H_idx=4, D_idx=64)),
     ("decoder_group1_b8_ctx128k", dict(B=5, ctx=3001)),
     ("decoder_group1_b8_ctx128k", dict(B=1, ctx=100)),
     ("reindex_group_b32_ctx256k", dict(B=3, ctx=50001)),

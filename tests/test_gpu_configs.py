@@ -80,6 +80,9 @@ def _free():
     ("decoder_group1_b8_ctx128k", dict(B=5, ctx=3001)),
     ("decoder_group1_b8_ctx128k", dict(B=1, ctx=100)),
     ("reindex_group_b32_ctx256k", dict(B=3, ctx=50001)),
+    # pools of 38 and 2 blocks: every pooled token is selected (fewer than 512)
+    ("reindex_group_b32_ctx256k", dict(B=2, ctx=300)),
+    ("reindex_group_b32_ctx256k", dict(B=1, ctx=9)),
     # more rows than resident clusters: clusters take whole rows (64 heads) one
     # after another and run every layer of a row before the next
     ("reindex_group_b32_ctx256k", dict(B=20, ctx=9001)),
@@ -147,6 +150,17 @@ def test_stack_ragged_long_rows(levels):
             ref = oracle.sparse_attention(bf16_np(wl.q[l][b, 0]), lambda P: kvb[P], r["top"],
                                           bf16_np(wl.swa[l][b]), c - 1, c - rows, wl.scale)
             assert_attn_close(wl.out[l][b, 0].cpu().numpy(), ref, f"attention b={b} l={l}")
+    del wl
+    _free()
+
+
+@pytest.mark.parametrize("ctx", [524288, 524296])
+def test_stack_pool_path_boundary(ctx):
+    """The Full layer's pool selection at the edge of its two forms: 65,536
+    blocks (the largest row one CTA selects) and 65,537 blocks (the many-CTA
+    compaction, whose last slice holds one block)."""
+    wl = _workload("decoder_stack20_b4_ctx1m", B=1, ctx=ctx, modes=[synth.FULL, synth.REUSE])
+    _check(wl, [0])
     del wl
     _free()
 

@@ -407,7 +407,13 @@ void orc_attention(const uint16_t *q, int Hq, int C, const double *kv, int64_t n
 {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int h = 0; h < Hq; h++) {
-        double *logit = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+        if (n == 0) {
+            /* no key: no softmax; the output is defined as zero */
+            for (int c = 0; c < C; c++)
+                out[h * C + c] = 0.0;
+            continue;
+        }
+        double *logit = (double *)malloc(sizeof(double) * (size_t)n);
         double mx = -INFINITY;
         for (int64_t j = 0; j < n; j++) {
             double dot = 0.0;

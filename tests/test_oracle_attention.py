@@ -49,6 +49,20 @@ def test_attention_closed_forms():
                                rtol=1e-12, atol=1e-14)
 
 
+def test_attention_without_keys_is_zero():
+    """A query that attends no key (every index masked, no window row) has no
+    softmax; its output is zero by definition, and the oracle's sparse path
+    reaches that case from masked indices and an empty window."""
+    qb = _bf16_bits(torch.randn(4, 32, generator=torch.Generator().manual_seed(3)))
+    out = oracle.attention(qb, np.zeros((0, 32)), 0.3)
+    assert out.shape == (4, 32) and np.array_equal(out, np.zeros((4, 32)))
+    rows = np.zeros((10, 32), np.uint16)
+    swa = np.zeros((128, 32), np.uint16)
+    out = oracle.sparse_attention(qb, lambda p: rows[p], -np.ones(8, np.int32), swa, 500, 373, 0.3,
+                                  n_win=0)
+    assert np.array_equal(out, np.zeros((4, 32)))
+
+
 def test_window_rows():
     assert oracle.window_rows(999, 872, 128).tolist() == list(range(128))
     assert oracle.window_rows(99, 0, 100).tolist() == list(range(100))

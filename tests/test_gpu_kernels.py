@@ -501,6 +501,18 @@ def test_sparse_attention_skips_negative_indices_and_short_window(B):
     _attention_case(B, 1, 50, 512, 64, 512, 128, seed=2)
 
 
+def test_sparse_attention_window_only_and_no_keys(B):
+    """K = 0: the window rows alone, on the split-key clusters, the per-row
+    kernel and the general kernel; then every index masked and no window: no
+    key at all, a zero output."""
+    _attention_case(B, 2, 1000, 512, 64, 0, 128, seed=41)
+    _attention_case(B, 1, 1000, 512, 64, 0, 128, seed=42, Nq=64)
+    _attention_case(B, 2, 1000, 128, 8, 0, 100, seed=43)
+    _attention_case(B, 2, 1000, 512, 64, 512, 0, seed=44, drop=1)
+    _attention_case(B, 1, 1000, 512, 64, 512, 0, seed=45, Nq=64, drop=1)
+    _attention_case(B, 2, 1000, 128, 8, 100, 0, seed=46, drop=1)
+
+
 def test_sparse_attention_prefill_positions(B):
     ctx = 1200
     q_pos = torch.tensor([[1199, 1100, 600, 130]], dtype=torch.int64, device=DEV)

@@ -96,6 +96,16 @@ def test_scaled_stack(name, kw):
     _free()
 
 
+def test_stack_with_64_sequences_takes_the_per_row_attention():
+    """64 sequences: the stack's attention runs one launch per layer on the
+    one-CTA-per-row kernel (the cluster kernel serves fewer rows); a Full group
+    and a Reindex group, every ninth sequence checked."""
+    wl = _workload("decoder_stack20_b4_ctx1m", B=64, ctx=2001, modes=list(synth.DECODER_MODES[:8]))
+    _check(wl, range(0, 64, 9))
+    del wl
+    _free()
+
+
 def test_stack_reuse_run_longer_than_one_attention_launch():
     """A Full layer followed by 10 Reuse layers: the attention of the first 8
     layers runs as one launch and the last 3 as a second launch led by a Reuse
